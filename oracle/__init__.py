@@ -1,0 +1,174 @@
+"""ctypes binding of the CPU oracle (oracle/moe_oracle.c).
+
+TEST INFRASTRUCTURE ONLY: the tests, the package entry's smoke check and the bench's CPU baseline
+leg are the only callers. The CUDA product path never imports this package, and this package never
+imports the product. Inputs are numpy arrays (float32 for tensors that are bf16 or fp32 on the GPU:
+bf16 values are exact in float32); results come back as float64 / int32 numpy arrays.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "moe_oracle.c")
+_OUT = os.path.join(_HERE, "_build", "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (-O2, OpenMP, strict IEEE: no fast-math)."""
+    if force or not os.path.exists(_OUT) or os.path.getmtime(_OUT) < os.path.getmtime(_SRC):
+        os.makedirs(os.path.dirname(_OUT), exist_ok=True)
+        tmp = _OUT + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared",
+                               "-Wall", "-Wextra", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _OUT)
+    return _OUT
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        _lib = ctypes.CDLL(build())
+        L = _lib
+        P = ctypes.c_void_p
+        i64, i32 = ctypes.c_int64, ctypes.c_int32
+        L.oracle_num_threads.restype = ctypes.c_int
+        L.oracle_router_logits.argtypes = [P, P, P, i64, i32, P, i64, P, P]
+        L.oracle_topk_softmax.argtypes = [P, i64, i32, i32, P, P]
+        L.oracle_weights_for.argtypes = [P, P, i64, i32, i32, P]
+        L.oracle_sparse_map.argtypes = [P, i64, i32, P, P, P, P]
+        L.oracle_sparse_map.restype = ctypes.c_int
+        L.oracle_expert_hidden.argtypes = [P, P, P, i64, i64, i32, i32, P]
+        L.oracle_mlp_forward.argtypes = [P, P, P, P, P, P, i64, i64, i32, i32, P, i64, P, P, P, P]
+        L.oracle_scatter_linear.argtypes = [P, P, i64, i64, i64, i32, i32, P, P, P, ctypes.c_int,
+                                            ctypes.c_int, P]
+    return _lib
+
+
+def _f32(a):
+    if a is None:
+        return None
+    if hasattr(a, "detach"):  # torch tensor
+        a = a.detach().to("cpu").float().numpy()
+    return np.ascontiguousarray(a, dtype=np.float32)
+
+
+def _i32(a):
+    if a is None:
+        return None
+    if hasattr(a, "detach"):
+        a = a.detach().to("cpu").numpy()
+    return np.ascontiguousarray(a, dtype=np.int32)
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def num_threads() -> int:
+    return lib().oracle_num_threads()
+
+
+def router_logits(x, w_gate, bias=None, tokens=None):
+    """fp64 logits [n, E] and magnitude sums sum_d |x_d W[d,e]| [n, E] for the listed tokens."""
+    x, w_gate, bias = _f32(x), _f32(w_gate), _f32(bias)
+    S, D = x.shape
+    E = w_gate.shape[1]
+    tokens = np.arange(S, dtype=np.int32) if tokens is None else _i32(tokens)
+    n = tokens.shape[0]
+    logits = np.zeros((n, E), dtype=np.float64)
+    absdot = np.zeros((n, E), dtype=np.float64)
+    lib().oracle_router_logits(_p(x), _p(w_gate), _p(bias), D, E, _p(tokens), n, _p(logits),
+                               _p(absdot))
+    return logits, absdot
+
+
+def topk_softmax(logits, k):
+    logits = np.ascontiguousarray(logits, dtype=np.float64)
+    n, E = logits.shape
+    te = np.zeros((n, k), dtype=np.int32)
+    tw = np.zeros((n, k), dtype=np.float64)
+    lib().oracle_topk_softmax(_p(logits), n, E, k, _p(te), _p(tw))
+    return te, tw
+
+
+def weights_for(logits, top_experts):
+    logits = np.ascontiguousarray(logits, dtype=np.float64)
+    te = _i32(top_experts)
+    n, E = logits.shape
+    k = te.shape[1]
+    tw = np.zeros((n, k), dtype=np.float64)
+    lib().oracle_weights_for(_p(logits), _p(te), n, E, k, _p(tw))
+    return tw
+
+
+def route(x, w_gate, k, bias=None):
+    logits, _ = router_logits(x, w_gate, bias)
+    return topk_softmax(logits, k)
+
+
+def sparse_map(top_experts, E):
+    """Returns (counts [E], offsets [E+1], sparse_rows [R], sorted_rows [R]) or raises ValueError
+    on an expert id outside [0, E)."""
+    te = _i32(top_experts).reshape(-1)
+    R = te.shape[0]
+    counts = np.zeros(E, dtype=np.int32)
+    offsets = np.zeros(E + 1, dtype=np.int32)
+    sparse_rows = np.zeros(R, dtype=np.int32)
+    sorted_rows = np.zeros(R, dtype=np.int32)
+    rc = lib().oracle_sparse_map(_p(te), R, E, _p(counts), _p(offsets), _p(sparse_rows),
+                                 _p(sorted_rows))
+    if rc != 0:
+        raise ValueError("expert id outside [0, E)")
+    return counts, offsets, sparse_rows, sorted_rows
+
+
+def expert_hidden(x, w_gate_e, w_up, token, expert):
+    x, wge, wu = _f32(x), _f32(w_gate_e), _f32(w_up)
+    D = x.shape[1]
+    F = wge.shape[2]
+    h = np.zeros(F, dtype=np.float64)
+    lib().oracle_expert_hidden(_p(x), _p(wge), _p(wu), D, F, int(token), int(expert), _p(h))
+    return h
+
+
+def mlp_forward(x, w_gate, w_gate_e, w_up, w_down, k, bias=None, tokens=None,
+                given_top_experts=None):
+    """fp64 y [n, D] for the listed tokens (all tokens by default), plus the oracle's (or the
+    given) top experts [n, k] and weights [n, k]."""
+    x, w_gate, bias = _f32(x), _f32(w_gate), _f32(bias)
+    wge, wu, wd = _f32(w_gate_e), _f32(w_up), _f32(w_down)
+    S, D = x.shape
+    E = w_gate.shape[1]
+    F = wge.shape[2]
+    tokens = np.arange(S, dtype=np.int32) if tokens is None else _i32(tokens)
+    given = _i32(given_top_experts)
+    n = tokens.shape[0]
+    out = np.zeros((n, D), dtype=np.float64)
+    te = np.zeros((n, k), dtype=np.int32)
+    tw = np.zeros((n, k), dtype=np.float64)
+    lib().oracle_mlp_forward(_p(x), _p(w_gate), _p(bias), _p(wge), _p(wu), _p(wd), D, F, E, k,
+                             _p(tokens), n, _p(given), _p(out), _p(te), _p(tw))
+    return out, te, tw
+
+
+def scatter_linear(X, W, k, sorted_rows, offsets, gates=None, gather_in=True, scatter_out=True,
+                   S=None):
+    """ParallelLinear(X, W, I, G) in fp64: grouped rows [R, Dout] or the token-order sum [S, Dout]."""
+    X, W, gates = _f32(X), _f32(W), _f32(gates)
+    sorted_rows, offsets = _i32(sorted_rows), _i32(offsets)
+    E, Din, Dout = W.shape
+    if S is None:
+        S = X.shape[0] if gather_in else (sorted_rows.shape[0] // k)
+    P = int(offsets[E])
+    rows = S if scatter_out else max(P, 0)
+    Y = np.zeros((rows, Dout), dtype=np.float64)
+    lib().oracle_scatter_linear(_p(X), _p(W), S, Din, Dout, E, k, _p(sorted_rows), _p(offsets),
+                                _p(gates.reshape(-1) if gates is not None else None),
+                                int(bool(gather_in)), int(bool(scatter_out)), _p(Y))
+    return Y

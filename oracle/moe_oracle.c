@@ -1,0 +1,278 @@
+/*
+ * CPU oracle for the dropless sparse-MoE expert-MLP forward.
+ *
+ * TEST INFRASTRUCTURE ONLY. Only the tests, the package entry's smoke check and the bench's CPU
+ * baseline leg may load this library. It shares no code, header, table or helper with the CUDA
+ * library; neither includes or loads the other.
+ *
+ * Every function is the plain definition of one step, in fp64, with inputs given as float32
+ * arrays (bf16 inputs are exactly representable in float32). Loops are written in the order of
+ * the definitions; the only liberties are the loop nesting of the dot products (a d-outer /
+ * f-inner order that walks the [D,F] weights contiguously; each output is still summed over
+ * d = 0..D-1 in ascending order) and OpenMP parallelism over independent tokens or slots.
+ *
+ * Sources (page title, then section / equation):
+ *  - "ScatterMoE Guide: Fast Fused Kernels for Sparse MoE LLMs"
+ *      "1. The Dynamic Routing Imbalance Dilemma", router equation H(X) = Softmax(TopK(X W_gate, k))
+ *      "1. The Anatomy of ParallelLinear", ParallelLinear(X, W, I, G) with W in R^{E x Din x Dout}
+ *      "2. Grouped Coordinate Indexing Without Padding", Histogram(e) and Offsets(e) equations
+ *      "The ParallelLinear Core Abstraction" figure, Steps 1-3 (gather, tile GEMM, gate + scatter)
+ *      "3. Assembling the ScatterMoE FFN Block" (SwiGLU: silu(gate) * up, gate half first)
+ *  - "Add scalable sparse map kernel for large MoE models (128+ experts)"
+ *      "Pass 1: Histogram with Atomics", "Pass 2: Two Assignment Variants",
+ *      "4. Correctness Validation" (unique rows, rows inside their expert's range, counts,
+ *      non-overlapping ranges, determinism)
+ *
+ * Readings taken where the pages are silent or inconsistent (all listed in the design notes):
+ *  - softmax over the k selected logits (weights sum to 1); the guide's code takes the full
+ *    softmax, then top-k, then renormalises, which is the same in exact arithmetic;
+ *  - top-k order: logits descending, equal logits -> smaller expert id first;
+ *  - slot order inside an expert follows the flat route index i = s*k + j (a stable sort), which is
+ *    the one deterministic result the map tests demand;
+ *  - the optional logit bias is added to the logits before selection and softmax;
+ *  - weights are used as x * W[e] with W[e] of shape [Din, Dout].
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* Router logits l[s,e] = sum_d x[s,d] * W_gate[d,e] (+ bias[e]), and the magnitude sum
+ * a[s,e] = sum_d |x[s,d] * W_gate[d,e]| that bounds the rounding error of any float evaluation of
+ * the same dot product. W_gate is [D,E]. Computed for the listed tokens only. */
+static void logits_one(const float *xs, const float *w_gate, const float *bias, int64_t D,
+                       int32_t E, double *l, double *a) {
+    for (int32_t e = 0; e < E; ++e) {
+        l[e] = 0.0;
+        if (a) a[e] = 0.0;
+    }
+    for (int64_t d = 0; d < D; ++d) {
+        const double xv = (double)xs[d];
+        const float *wrow = w_gate + d * E;
+        for (int32_t e = 0; e < E; ++e) {
+            const double p = xv * (double)wrow[e];
+            l[e] += p;
+            if (a) a[e] += fabs(p);
+        }
+    }
+    if (bias)
+        for (int32_t e = 0; e < E; ++e) l[e] += (double)bias[e];
+}
+
+void oracle_router_logits(const float *x, const float *w_gate, const float *bias, int64_t D,
+                          int32_t E, const int32_t *tokens, int64_t n_tokens, double *logits,
+                          double *absdot) {
+    #pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < n_tokens; ++t)
+        logits_one(x + (int64_t)tokens[t] * D, w_gate, bias, D, E, logits + t * E,
+                   absdot ? absdot + t * E : NULL);
+}
+
+/* Top-k selection and softmax over the selected logits for one token.
+ * J_0..J_{k-1}: the k largest logits, in descending order; on equal logits the smaller expert id
+ * ranks first. Selection is k passes of "best not yet taken"; the strict '>' keeps the smaller id
+ * on ties. Weights w_j = exp(l_{J_j} - l_{J_0}) / sum_j' exp(l_{J_j'} - l_{J_0}). */
+static void topk_one(const double *l, int32_t E, int32_t k, int32_t *J, double *w) {
+    for (int32_t j = 0; j < k; ++j) {
+        int32_t best = -1;
+        for (int32_t e = 0; e < E; ++e) {
+            int taken = 0;
+            for (int32_t q = 0; q < j; ++q)
+                if (J[q] == e) taken = 1;
+            if (taken) continue;
+            if (best < 0 || l[e] > l[best]) best = e;
+        }
+        J[j] = best;
+    }
+    const double m = l[J[0]];
+    double den = 0.0;
+    for (int32_t j = 0; j < k; ++j) den += exp(l[J[j]] - m);
+    for (int32_t j = 0; j < k; ++j) w[j] = exp(l[J[j]] - m) / den;
+}
+
+void oracle_topk_softmax(const double *logits, int64_t n_tokens, int32_t E, int32_t k,
+                         int32_t *top_experts, double *top_weights) {
+    #pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < n_tokens; ++t)
+        topk_one(logits + t * E, E, k, top_experts + t * k, top_weights + t * k);
+}
+
+/* Softmax weights for a given (externally chosen) expert list J of each token, in J's order. */
+void oracle_weights_for(const double *logits, const int32_t *top_experts, int64_t n_tokens,
+                        int32_t E, int32_t k, double *top_weights) {
+    for (int64_t t = 0; t < n_tokens; ++t) {
+        const double *l = logits + t * E;
+        const int32_t *J = top_experts + t * k;
+        double m = l[J[0]];
+        for (int32_t j = 1; j < k; ++j)
+            if (l[J[j]] > m) m = l[J[j]];
+        double den = 0.0;
+        for (int32_t j = 0; j < k; ++j) den += exp(l[J[j]] - m);
+        for (int32_t j = 0; j < k; ++j) top_weights[t * k + j] = exp(l[J[j]] - m) / den;
+    }
+}
+
+/* Sparse map over the flat route list i = 0..R-1 (i = s*k + j), expert(i) = top_experts[i]:
+ *   counts[e]       = #{i : expert(i) = e}                             (Histogram(e))
+ *   offsets[e]      = sum_{e' < e} counts[e'],  offsets[E] = R          (Offsets(e))
+ *   sparse_rows[i]  = offsets[expert(i)] + #{i' < i : expert(i') = expert(i)}   (stable slot)
+ *   sorted_rows[p]  = the i with sparse_rows[i] = p                    (expert-sorted route list)
+ * A sequential counting sort. Returns 0, or -1 (and writes nothing) if an id is outside [0, E). */
+int oracle_sparse_map(const int32_t *top_experts, int64_t R, int32_t E, int32_t *counts,
+                      int32_t *offsets, int32_t *sparse_rows, int32_t *sorted_rows) {
+    for (int64_t i = 0; i < R; ++i)
+        if (top_experts[i] < 0 || top_experts[i] >= E) return -1;
+    for (int32_t e = 0; e < E; ++e) counts[e] = 0;
+    for (int64_t i = 0; i < R; ++i) counts[top_experts[i]] += 1;
+    offsets[0] = 0;
+    for (int32_t e = 0; e < E; ++e) offsets[e + 1] = offsets[e] + counts[e];
+    int32_t *next = (int32_t *)malloc(sizeof(int32_t) * (size_t)(E > 0 ? E : 1));
+    for (int32_t e = 0; e < E; ++e) next[e] = offsets[e];
+    for (int64_t i = 0; i < R; ++i) {
+        const int32_t e = top_experts[i];
+        sparse_rows[i] = next[e];
+        sorted_rows[next[e]] = (int32_t)i;
+        next[e] += 1;
+    }
+    free(next);
+    return 0;
+}
+
+static double silu(double z) { return z / (1.0 + exp(-z)); }
+
+/* Expert hidden row h = silu(v . W_gate_e[e]) * (v . W_up[e]), W_gate_e[e], W_up[e] of shape [D,F]
+ * (the gate half is the one passed through SiLU). */
+static void expert_hidden(const float *v, const float *wge, const float *wu, int64_t D, int64_t F,
+                          double *g, double *u, double *h) {
+    for (int64_t f = 0; f < F; ++f) {
+        g[f] = 0.0;
+        u[f] = 0.0;
+    }
+    for (int64_t d = 0; d < D; ++d) {
+        const double vd = (double)v[d];
+        const float *gr = wge + d * F;
+        const float *ur = wu + d * F;
+        for (int64_t f = 0; f < F; ++f) {
+            g[f] += vd * (double)gr[f];
+            u[f] += vd * (double)ur[f];
+        }
+    }
+    for (int64_t f = 0; f < F; ++f) h[f] = silu(g[f]) * u[f];
+}
+
+void oracle_expert_hidden(const float *x, const float *w_gate_e, const float *w_up, int64_t D,
+                          int64_t F, int32_t token, int32_t expert, double *h) {
+    double *g = (double *)malloc(sizeof(double) * (size_t)F);
+    double *u = (double *)malloc(sizeof(double) * (size_t)F);
+    expert_hidden(x + (int64_t)token * D, w_gate_e + (int64_t)expert * D * F,
+                  w_up + (int64_t)expert * D * F, D, F, g, u, h);
+    free(g);
+    free(u);
+}
+
+/* Forward for the listed tokens: y[s] = sum_j w_j * FFN_{J_j}(x[s]) with
+ * FFN_e(v) = (silu(v W_gate_e[e]) * (v W_up[e])) W_down[e], W_down[e] of shape [F,D].
+ * If given_top_experts ([S,k], indexed by token) is non-null, its experts replace the oracle's
+ * own selection and the weights are the softmax of the fp64 logits over that list.
+ * Outputs: out [n_tokens, D]; top_experts_out / top_weights_out [n_tokens, k] (nullable). */
+void oracle_mlp_forward(const float *x, const float *w_gate, const float *bias,
+                        const float *w_gate_e, const float *w_up, const float *w_down, int64_t D,
+                        int64_t F, int32_t E, int32_t k, const int32_t *tokens, int64_t n_tokens,
+                        const int32_t *given_top_experts, double *out, int32_t *top_experts_out,
+                        double *top_weights_out) {
+    #pragma omp parallel
+    {
+        double *l = (double *)malloc(sizeof(double) * (size_t)E);
+        double *g = (double *)malloc(sizeof(double) * (size_t)F);
+        double *u = (double *)malloc(sizeof(double) * (size_t)F);
+        double *h = (double *)malloc(sizeof(double) * (size_t)F);
+        int32_t J[64];
+        double w[64];
+        #pragma omp for schedule(dynamic, 1)
+        for (int64_t t = 0; t < n_tokens; ++t) {
+            const int32_t s = tokens[t];
+            logits_one(x + (int64_t)s * D, w_gate, bias, D, E, l, NULL);
+            if (given_top_experts) {
+                for (int32_t j = 0; j < k; ++j) J[j] = given_top_experts[(int64_t)s * k + j];
+                oracle_weights_for(l, J, 1, E, k, w);
+            } else {
+                topk_one(l, E, k, J, w);
+            }
+            double *y = out + t * D;
+            for (int64_t d = 0; d < D; ++d) y[d] = 0.0;
+            const float *v = x + (int64_t)s * D;
+            for (int32_t j = 0; j < k; ++j) {
+                const int64_t e = J[j];
+                expert_hidden(v, w_gate_e + e * D * F, w_up + e * D * F, D, F, g, u, h);
+                const float *wd = w_down + e * F * D;
+                for (int64_t f = 0; f < F; ++f) {
+                    const double c = w[j] * h[f];
+                    const float *row = wd + f * D;
+                    for (int64_t d = 0; d < D; ++d) y[d] += c * (double)row[d];
+                }
+            }
+            if (top_experts_out)
+                for (int32_t j = 0; j < k; ++j) top_experts_out[t * k + j] = J[j];
+            if (top_weights_out)
+                for (int32_t j = 0; j < k; ++j) top_weights_out[t * k + j] = w[j];
+        }
+        free(l);
+        free(g);
+        free(u);
+        free(h);
+    }
+}
+
+/* ParallelLinear(X, W, I, G): for every slot p of expert e (offsets[e] <= p < offsets[e+1]) with
+ * route i = sorted_rows[p] and token s = i / k:
+ *   v_p = src_p . W[e],  src_p = X[s] if gather_in else X[p],  W of shape [E, Din, Dout];
+ *   c_p = gates[i] * v_p if gates is non-null, else v_p;
+ *   scatter_out: Y[s] += c_p  (Y [S, Dout], zeroed here; slot contributions added in slot order)
+ *   else:        Y[p]  = c_p  (Y [R, Dout], expert-grouped rows).   */
+void oracle_scatter_linear(const float *X, const float *W, int64_t S, int64_t Din, int64_t Dout,
+                           int32_t E, int32_t k, const int32_t *sorted_rows,
+                           const int32_t *offsets, const float *gates, int gather_in,
+                           int scatter_out, double *Y) {
+    const int64_t P = offsets[E];
+    double *grouped = (double *)calloc((size_t)(P > 0 ? P : 1) * (size_t)Dout, sizeof(double));
+    #pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t p = 0; p < P; ++p) {
+        int32_t e = 0;
+        while (e < E && !(offsets[e] <= p && p < offsets[e + 1])) ++e;
+        const int64_t i = sorted_rows[p];
+        const int64_t s = i / k;
+        const float *src = X + (gather_in ? s : p) * Din;
+        const float *We = W + (int64_t)e * Din * Dout;
+        double *v = grouped + p * Dout;
+        for (int64_t d = 0; d < Din; ++d) {
+            const double xv = (double)src[d];
+            const float *wr = We + d * Dout;
+            for (int64_t n = 0; n < Dout; ++n) v[n] += xv * (double)wr[n];
+        }
+        if (gates) {
+            const double g = (double)gates[i];
+            for (int64_t n = 0; n < Dout; ++n) v[n] *= g;
+        }
+    }
+    if (scatter_out) {
+        memset(Y, 0, sizeof(double) * (size_t)S * (size_t)Dout);
+        for (int64_t p = 0; p < P; ++p) {
+            const int64_t s = sorted_rows[p] / k;
+            for (int64_t n = 0; n < Dout; ++n) Y[s * Dout + n] += grouped[p * Dout + n];
+        }
+    } else {
+        memcpy(Y, grouped, sizeof(double) * (size_t)P * (size_t)Dout);
+    }
+    free(grouped);
+}
