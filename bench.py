@@ -1,0 +1,378 @@
+"""Benchmark of the dropless MoE expert-MLP forward on B200 (one JSON line on stdout).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one whole forward (zero out, route, sparse map, GEMM1, GEMM2) through the C ABI over one
+batch of seeded synthetic inputs. Default workload: the Mixtral-8x7B-shaped prefill layer
+(S=4096, D=4096, F=14336, E=8, top-2, bf16). With N > 1 (launched by torch.distributed.run) every
+rank runs its own replica on its own batch (weak scaling, no data-path collective); the timed
+region is bracketed by a barrier and device synchronisation, and the max over ranks is reported.
+`--impl reference` times the CPU oracle instead (rank 0 only), on a bounded token sample.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import moe_workloads as W  # noqa: E402
+
+METRIC = "MoE-layer fwd tokens/s and TFLOP/s (bf16) as % of B200 peak; sparse-map GB/s"
+NOMINAL_TFLOPS = {"bf16": 2250.0, "f32": 1125.0}   # dense bf16; tf32 for fp32 inputs
+NOMINAL_HBM_GBS = 8000.0
+
+
+def flops_of(w: W.Workload) -> dict:
+    R = w.R
+    return {
+        "router": 2.0 * w.S * w.D * w.E,
+        "gemm1": 4.0 * R * w.D * w.F,
+        "gemm2": 2.0 * R * w.F * w.D,
+    }
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return p, "measured"
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, \
+            "fallback"
+
+
+def recorded_traffic(kernel_key: str):
+    """DRAM bytes per launch of `kernel_key` from the committed ncu summary, if the kernel source
+    is unchanged since it was captured (the summary records the source hash)."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.md")
+    src = os.path.join(ROOT, "sparse_mixture_experts_02_b200", "csrc", "grouped_gemm.cu")
+    try:
+        text = open(path).read()
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    except OSError:
+        return None
+    m = re.search(r"^\|\s*" + re.escape(kernel_key) + r"\s*\|\s*([0-9]+)\s*\|\s*([0-9a-f]+)\s*\|",
+                  text, re.M)
+    if not m or m.group(2) != sha:
+        return None
+    return int(m.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.file = None
+
+    def __enter__(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.file, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or self.file is None:
+            return None
+        self.file.flush()
+        rows = []
+        with open(self.file.name) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+                except ValueError:
+                    continue
+        os.unlink(self.file.name)
+        if not rows:
+            return None
+        mx = max(r[1] for r in rows)
+        loaded = [r for r in rows if r[0] > 0.5 * mx] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[2])
+                          if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": mx,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def run_oracle_sample(w, inp_cpu, n_tokens, seed=0):
+    """Times the CPU oracle on n_tokens tokens of the workload; returns (seconds, tokens, cores)."""
+    import numpy as np
+
+    import oracle
+    toks = np.random.default_rng(seed).choice(w.S, size=min(n_tokens, w.S),
+                                              replace=False).astype(np.int32)
+    t0 = time.perf_counter()
+    oracle.mlp_forward(inp_cpu["x"], inp_cpu["w_gate"], inp_cpu["w_gate_e"], inp_cpu["w_up"],
+                       inp_cpu["w_down"], w.k, bias=inp_cpu["logit_bias"], tokens=toks)
+    return time.perf_counter() - t0, len(toks), oracle.num_threads()
+
+
+def host_inputs(inp):
+    return {k: (v.float().cpu().numpy() if v is not None else None) for k, v in inp.items()}
+
+
+def calibrate_oracle(w, inp_cpu, budget_s):
+    """Number of tokens the oracle covers in about budget_s seconds (one token probes the rate)."""
+    t1, _, _ = run_oracle_sample(w, inp_cpu, 1, seed=123)
+    return max(1, min(w.S, int(budget_s / max(t1, 1e-6))))
+
+
+def dist_setup():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return ws, rank, local
+
+
+def bench_reference(args, w, ws, rank):
+    """The oracle on the host cores: each step a bounded token sample of the workload."""
+    if rank != 0:
+        return None
+    inp = W.make_inputs(w, device="cuda" if torch.cuda.is_available() else "cpu")
+    inp_cpu = host_inputs(inp)
+    del inp
+    # each step a bounded sample: the whole warm-up + timed run stays near 150 s of oracle work
+    step_s = args.ref_step_s or min(4.0, max(0.2, 150.0 / (args.steps + args.warmup)))
+    per_step = calibrate_oracle(w, inp_cpu, step_s)
+    for i in range(args.warmup):
+        run_oracle_sample(w, inp_cpu, per_step, seed=1000 + i)
+    t_total, n_total, cores = 0.0, 0, 1
+    for i in range(args.steps):
+        t, n, cores = run_oracle_sample(w, inp_cpu, per_step, seed=i)
+        t_total += t
+        n_total += n
+    value = n_total / t_total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * t_total / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, **{k: getattr(w, k) for k in "SDFEk"},
+                   "input_dtype": w.dtype},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{per_step} seeded tokens of {w.S} per step"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    return line
+
+
+def bench_ours(args, w, ws, rank, local):
+    import sparse_mixture_experts_02_b200 as moe
+
+    dev = torch.device("cuda", local)
+    seed = rank  # every rank its own batch; rank 0 is the N=1 workload
+    inp = W.make_inputs(w, device=dev, seed=seed)
+    wsp = moe.ForwardWorkspace(w.S, w.D, w.F, w.E, w.k, inp["x"].dtype, dev)
+    out = torch.empty((w.S, w.D), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(events=None):
+        if events is not None:
+            moe.profile_events(events)
+        moe.mlp_forward(inp["x"], inp["w_gate"], inp["w_gate_e"], inp["w_up"], inp["w_down"],
+                        w.k, logit_bias=inp["logit_bias"], out=out, ws=wsp)
+
+    for _ in range(args.warmup):
+        step()
+    moe.check_device_status(wsp)
+    launches_per_step = moe.last_launch_count()
+
+    # events for the per-stage breakdown, 5 per step, created and recorded once up front
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    for row in evs:
+        for e in row:
+            e.record(stream)
+    torch.cuda.synchronize(dev)
+
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        if ws > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize(dev)
+        t0.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+        if ws > 1:
+            torch.distributed.barrier()
+    ms_total = t0.elapsed_time(t1)
+    moe.check_device_status(wsp)
+    if ws > 1:
+        t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_total = float(t.item())
+    stage = {"zero+route": [], "sparse_map": [], "gemm1": [], "gemm2": []}
+    for row in evs:
+        stage["zero+route"].append(row[0].elapsed_time(row[1]))
+        stage["sparse_map"].append(row[1].elapsed_time(row[2]))
+        stage["gemm1"].append(row[2].elapsed_time(row[3]))
+        stage["gemm2"].append(row[3].elapsed_time(row[4]))
+    stage_ms = {k: sum(v) / len(v) for k, v in stage.items()}
+
+    # end to end: pinned host x in, host out back, inside the timed region
+    x_host = inp["x"].cpu().pin_memory()
+    out_host = torch.empty((w.S, w.D), dtype=torch.float32).pin_memory()
+    x_dev = torch.empty_like(inp["x"])
+
+    def e2e_step():
+        x_dev.copy_(x_host, non_blocking=True)
+        moe.mlp_forward(x_dev, inp["w_gate"], inp["w_gate_e"], inp["w_up"], inp["w_down"], w.k,
+                        logit_bias=inp["logit_bias"], out=out, ws=wsp)
+        out_host.copy_(out, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    if ws > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1)
+    if ws > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    counts = wsp.view("expert_counts").cpu()
+    hist = {"max": int(counts.max()), "min": int(counts.min()),
+            "empty": int((counts == 0).sum()), "mean": float(counts.float().mean())}
+
+    if rank != 0:
+        return None
+
+    fl = flops_of(w)
+    flop_step = sum(fl.values())
+    s_per_step = ms_total / 1000.0 / args.steps
+    tokens_per_s = w.S * ws / s_per_step
+    tflops = flop_step / s_per_step / 1e12
+    pk, pk_kind = peaks()
+    dt = w.dtype
+    ratio = 1.0 if dt == "bf16" else NOMINAL_TFLOPS["f32"] / NOMINAL_TFLOPS["bf16"]
+    peak_burst = pk["bf16_tflops"] * ratio
+    peak_sust = pk["bf16_tflops_sustained"] * ratio
+    map_bytes = w.R * 4 + 2 * w.R * 4 + (2 * w.E + 1) * 4
+    g1_tflops = fl["gemm1"] / (stage_ms["gemm1"] / 1000.0) / 1e12
+    key = f"gemm1_gateup_swiglu@{w.name}"
+    line = {
+        "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": dt, "data": "synthetic",
+        "config": {"workload": w.name, **{k: getattr(w, k) for k in "SDFEk"},
+                   "router": w.router_std, "zipf_s": w.zipf_s, "seed": "rank",
+                   "parallelism": f"replicas{ws}",
+                   "l2": "inputs larger than L2 (all expert weights streamed every step)"},
+        "tflops": tflops,
+        "tflops_frac": {"of_measured_sustained": tflops / peak_sust,
+                        "of_measured_burst": tflops / peak_burst,
+                        "of_nominal": tflops / NOMINAL_TFLOPS[dt], "peaks": pk_kind},
+        "stage_ms": stage_ms,
+        "sparse_map_gbs": map_bytes / (stage_ms["sparse_map"] / 1000.0) / 1e9,
+        "expert_hist": hist,
+        "roofline": {"kernel": "gemm1_gateup_swiglu", "bound": "tensor", "achieved": g1_tflops,
+                     "peak": peak_sust, "unit": "TFLOP/s", "frac": g1_tflops / peak_sust,
+                     "peak_kind": f"{pk_kind} sustained bf16"
+                                  + ("" if dt == "bf16" else " x tf32/bf16 nominal ratio"),
+                     "traffic": recorded_traffic(key)},
+        "e2e": {"value": w.S * ws / (e2e_ms / 1000.0 / args.steps), "unit": "tokens/s",
+                "h2d_bytes_per_step": w.S * w.D * inp["x"].element_size(),
+                "d2h_bytes_per_step": w.S * w.D * 4},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+    }
+    if ws == 1 and not args.no_cpu_baseline:
+        inp_cpu = host_inputs(inp)
+        n = calibrate_oracle(w, inp_cpu, args.cpu_budget_s)
+        t, ntok, cores = run_oracle_sample(w, inp_cpu, n)
+        line["cpu_baseline"] = {"value": ntok / t, "unit": "tokens/s", "cores": cores,
+                                "kind": "oracle",
+                                "sample": f"{ntok} seeded tokens of {w.S} ({t:.1f} s)"}
+    return line
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="mixtral_prefill", choices=list(W.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget-s", type=float, default=15.0)
+    ap.add_argument("--ref-step-s", type=float, default=None)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    w = W.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        # the oracle runs on rank 0's host cores only; other ranks have nothing to do
+        ws = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        if rank == 0:
+            line = bench_reference(args, w, ws, rank)
+            print(json.dumps(line), flush=True)
+        return
+    ws, rank, local = dist_setup()
+    try:
+        line = bench_ours(args, w, ws, rank, local)
+        if rank == 0 and line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if ws > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

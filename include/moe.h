@@ -1,0 +1,184 @@
+/*
+ * moe.h — C ABI of the B200 (sm_100a) dropless sparse-MoE expert-MLP forward.
+ *
+ * The operation, as the pages state it:
+ *  - router: H(X) = Softmax(TopK(X W_gate, k))
+ *      ("ScatterMoE Guide: Fast Fused Kernels for Sparse MoE LLMs",
+ *       "1. The Dynamic Routing Imbalance Dilemma", router equation);
+ *  - sparse map: Histogram(e), Offsets(e) and an expert-sorted route index I
+ *      (same page, "2. Grouped Coordinate Indexing Without Padding"; and "Add scalable sparse map
+ *       kernel for large MoE models (128+ experts)", "Pass 1", "Pass 2" and "Usage");
+ *  - ParallelLinear(X, W, I, G): gather rows on load, multiply by W[expert], scale by the router
+ *    weight and scatter-add into token order (ScatterMoE guide, "1. The Anatomy of ParallelLinear"
+ *    and "The ParallelLinear Core Abstraction" figure, Steps 1-3);
+ *  - SwiGLU expert MLP y = sum_j w_j (silu(x W_gate_e[e_j]) * (x W_up[e_j])) W_down[e_j]
+ *    (ScatterMoE guide, "3. Assembling the ScatterMoE FFN Block"; fused gate+up as in the
+ *     abstract of "Cross-Platform Fused MoE Dispatch in Triton").
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers owned by the caller, row-major and contiguous.
+ *    Tensors read by the tensor cores (x, weights, X, Y, out) must be 16-byte aligned; int32 and
+ *    float32 side arrays must be 4-byte aligned. The library never allocates device memory in
+ *    these calls: scratch space comes from the caller's workspace `ws` (size from
+ *    moe_workspace_size, alignment 256 bytes).
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy default stream) and
+ *    never synchronise the host. Argument errors are detected on the host and returned before any
+ *    launch. Errors the device detects (an expert id outside [0,E), a bounded wait that ran out)
+ *    set a status word inside `ws`; moe_check_device_status() synchronises the stream and reports
+ *    it. Every call that takes `ws` clears that word first.
+ *  - Return value: MOE_OK (0) or a negative moe_status; moe_last_error() gives a message for the
+ *    last failing call on the calling host thread.
+ *  - Limits checked on the host: 1 <= k <= min(E, 8); E <= 256; 0 <= S and S*k < 2^31;
+ *    D, F, Din, Dout multiples of 8 and > 0; all dims < 2^31.
+ *  - Floating point: bf16 inputs multiply on the tensor cores with fp32 accumulation; fp32 inputs
+ *    multiply as tf32 with fp32 accumulation; the router accumulates in fp32 on the CUDA cores.
+ *    Scatter outputs are fp32 and use fp32 atomic adds, so their last bits may differ between
+ *    runs. The sparse map is exact and deterministic.
+ *  - Requires a device of compute capability 10.0 (B200, sm_100a); other devices get
+ *    MOE_ERR_UNSUPPORTED.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *moe_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = -1,    /* null / misaligned pointer, bad size or limit */
+    MOE_ERR_UNSUPPORTED = -2,    /* device is not sm_100, or dtype not supported */
+    MOE_ERR_WORKSPACE = -3,      /* ws is null, misaligned or smaller than moe_workspace_size */
+    MOE_ERR_CUDA = -4,           /* a CUDA runtime / driver call failed */
+    MOE_ERR_BAD_EXPERT_ID = -5,  /* device saw an expert id outside [0, E) */
+    MOE_ERR_DEVICE_TIMEOUT = -6  /* a bounded device-side wait ran out; the kernel returned */
+} moe_status;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+
+/*
+ * Router: per token s, logits l = x[s] . W_gate (+ logit_bias), then the k largest logits in
+ * descending order (equal logits: smaller expert id first) and their softmax weights
+ * w_j = exp(l_{e_j} - l_{e_0}) / sum_j' exp(l_{e_j'} - l_{e_0}).
+ *   x           [S, D]  dt        token activations
+ *   w_gate      [D, E]  dt        router weight (x . W_gate, E contiguous)
+ *   logit_bias  [E]     float32   nullable; added to the logits before selection and softmax
+ *   top_experts [S, k]  int32     out
+ *   top_weights [S, k]  float32   out
+ * Cites: ScatterMoE guide, "1. The Dynamic Routing Imbalance Dilemma" (router equation) and
+ * "3. Assembling the ScatterMoE FFN Block" (softmax, top-k, renormalise).
+ */
+int moe_route_topk(const void *x, const void *w_gate, const float *logit_bias, int64_t S,
+                   int64_t D, int32_t E, int32_t k, moe_dtype dt, int32_t *top_experts,
+                   float *top_weights, moe_stream_t stream);
+
+/*
+ * Sparse map of the flat route list i = s*k + j, expert(i) = top_experts[i]:
+ *   expert_counts  [E]    int32  out  Histogram(e) = #{i : expert(i) = e}
+ *   expert_offsets [E+1]  int32  out  Offsets(e) = sum_{e'<e} Histogram(e'); offsets[E] = S*k.
+ *                                     expert_offsets[1..E] are the "expert_ends" of the Fast-LLM
+ *                                     API; with zero padding the "pad begins" equal the ends.
+ *   sparse_rows    [S*k]  int32  out  slot of route i: offsets[e] + #{i' < i : expert(i') = e}
+ *   sorted_rows    [S*k]  int32  out  inverse permutation: sorted_rows[sparse_rows[i]] = i
+ * Slots inside an expert follow increasing i (stable), so the result is unique and bit-exact.
+ * An id outside [0,E) is not counted, gets sparse_rows[i] = -1, and sets MOE_ERR_BAD_EXPERT_ID in
+ * the device status.  ws: moe_workspace_size("sparse_map", S, 0, 0, E, k, dt) bytes.
+ * Cites: ScatterMoE guide, "2. Grouped Coordinate Indexing Without Padding"; "Add scalable sparse
+ * map kernel for large MoE models (128+ experts)", "Pass 1: Histogram with Atomics", "Pass 2: Two
+ * Assignment Variants", "4. Correctness Validation" and "Usage".
+ */
+int moe_sparse_map(const int32_t *top_experts, int64_t S, int32_t k, int32_t E,
+                   int32_t *expert_counts, int32_t *expert_offsets, int32_t *sparse_rows,
+                   int32_t *sorted_rows, void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * ParallelLinear(X, W, I, G): for each slot p of expert e (offsets[e] <= p < offsets[e+1]),
+ * route i = sorted_rows[p], token s = i / k:
+ *   v_p = src_p . W[e]   with src_p = X[s] (gather_in = 1, X is [S, Din] in token order)
+ *                        or   src_p = X[p] (gather_in = 0, X is [S*k, Din] in slot order)
+ *   c_p = top_weights[i] * v_p   (top_weights nullable: no scaling)
+ *   scatter_out = 1: Y[s] += c_p  (Y is [S, Dout] float32; the caller zeroes it first)
+ *   scatter_out = 0: Y[p]  = c_p  (Y is [S*k, Dout] in dt, slot order)
+ *   W [E, Din, Dout] dt; sorted_rows [S*k], expert_offsets [E+1] as from moe_sparse_map.
+ * ws: moe_workspace_size("scatter_linear", ...) bytes (holds the device status word).
+ * Cites: ScatterMoE guide, "1. The Anatomy of ParallelLinear", "The ParallelLinear Core
+ * Abstraction" figure (Steps 1-3) and "2. Grouped Coordinate Indexing Without Padding" (tiles of
+ * an expert's rows, last tile masked, no padding in memory).
+ */
+int moe_scatter_linear(const void *X, const void *W, int64_t S, int64_t Din, int64_t Dout,
+                       int32_t E, int32_t k, const int32_t *sorted_rows,
+                       const int32_t *expert_offsets, const float *top_weights, int gather_in,
+                       int scatter_out, moe_dtype dt, void *Y, void *ws, size_t ws_bytes,
+                       moe_stream_t stream);
+
+/*
+ * Whole MoE expert-MLP forward:
+ *   out[s] = sum_j w_j * ( silu(x[s] W_gate_e[e_j]) * (x[s] W_up[e_j]) ) W_down[e_j]
+ * with (e_j, w_j) from moe_route_topk. Steps on `stream`: zero out, route, sparse map, GEMM1
+ * (gathered x rows, fused gate+up, SwiGLU in registers, h in slot order), GEMM2 (h rows,
+ * W_down, router weight, scatter-add into out). No host synchronisation.
+ *   x [S,D], w_gate [D,E], w_gate_e [E,D,F], w_up [E,D,F], w_down [E,F,D]: dt
+ *   logit_bias [E] float32 nullable;  out [S,D] float32 (overwritten).
+ *   ws: moe_workspace_size("mlp_forward", S, D, F, E, k, dt) bytes; after the call it holds the
+ *   routing (see moe_workspace_view) until the next call that uses it.
+ * Cites: ScatterMoE guide, "3. Assembling the ScatterMoE FFN Block" and "Enter ScatterMoE" pipeline
+ * figure; fused gate+up from the abstract of "Cross-Platform Fused MoE Dispatch in Triton".
+ */
+int moe_mlp_forward(const void *x, const void *w_gate, const float *logit_bias,
+                    const void *w_gate_e, const void *w_up, const void *w_down, int64_t S,
+                    int64_t D, int64_t F, int32_t E, int32_t k, moe_dtype dt, float *out, void *ws,
+                    size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Workspace bytes for op = "sparse_map", "scatter_linear" or "mlp_forward" (unused sizes may be
+ * 0). Returns 0 for an unknown op or sizes outside the limits.
+ */
+size_t moe_workspace_size(const char *op, int64_t S, int64_t D, int64_t F, int32_t E, int32_t k,
+                          moe_dtype dt);
+
+/*
+ * Byte offsets inside an "mlp_forward" workspace of the intermediate results the forward leaves
+ * there (for inspection and tests): which = "top_experts" [S*k] int32, "top_weights" [S*k] f32,
+ * "expert_counts" [E], "expert_offsets" [E+1], "sparse_rows" [S*k], "sorted_rows" [S*k] int32,
+ * "h" [S*k, F] (bf16 for bf16, f32 for f32). Returns -1 for an unknown name.
+ */
+int64_t moe_workspace_view(const char *which, int64_t S, int64_t D, int64_t F, int32_t E,
+                           int32_t k, moe_dtype dt);
+
+/* Message for the last failing call on this host thread ("" if none). */
+const char *moe_last_error(void);
+
+/*
+ * Synchronises `stream`, reads the status word in `ws` and returns MOE_OK,
+ * MOE_ERR_BAD_EXPERT_ID or MOE_ERR_DEVICE_TIMEOUT (or MOE_ERR_CUDA). Off the hot path.
+ */
+int moe_check_device_status(void *ws, moe_stream_t stream);
+
+/*
+ * Optional per-stage timing of moe_mlp_forward on the calling host thread: when `events` holds
+ * n >= 5 cudaEvent_t handles, the next moe_mlp_forward records them on its stream at: start,
+ * after route, after the sparse map, after GEMM1, after GEMM2; then the registration clears.
+ * Pass n = 0 to clear. Returns MOE_OK or MOE_ERR_INVALID_ARG.
+ */
+int moe_profile_events(void *const *events, int n);
+
+/*
+ * Self-test of the bounded device wait: launches one block that waits on a barrier nothing
+ * arrives at, with a limit of `limit_ns` nanoseconds (1 .. 10^9), then returns. The status word in
+ * `ws` then reads MOE_ERR_DEVICE_TIMEOUT through moe_check_device_status. ws >= 256 bytes.
+ */
+int moe_debug_wait_timeout(int64_t limit_ns, void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Number of kernels the last successful call on this host thread launched. */
+int moe_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

@@ -1,0 +1,279 @@
+"""Python binding of the B200 dropless sparse-MoE expert-MLP library (libmoe_b200.so).
+
+This module only marshals arguments: it checks tensor shapes, dtypes and devices, allocates the
+outputs and the workspace with torch (device memory and streams are torch's), and calls the C ABI
+declared in include/moe.h on the current CUDA stream. Every step of the computation runs in the
+library's CUDA kernels; there is no CPU or PyTorch fallback. If the compiled library is missing
+the import raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "_lib", "libmoe_b200.so")
+
+MOE_F32, MOE_BF16 = 0, 1
+STATUS_NAMES = {0: "MOE_OK", -1: "MOE_ERR_INVALID_ARG", -2: "MOE_ERR_UNSUPPORTED",
+                -3: "MOE_ERR_WORKSPACE", -4: "MOE_ERR_CUDA", -5: "MOE_ERR_BAD_EXPERT_ID",
+                -6: "MOE_ERR_DEVICE_TIMEOUT"}
+
+EXPORTS = ["moe_route_topk", "moe_sparse_map", "moe_scatter_linear", "moe_mlp_forward",
+           "moe_workspace_size", "moe_workspace_view", "moe_last_error",
+           "moe_check_device_status", "moe_profile_events", "moe_debug_wait_timeout",
+           "moe_last_launch_count"]
+
+
+class MoeError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"{STATUS_NAMES.get(code, code)}: {msg}")
+        self.code = code
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m sparse_mixture_experts_02_b200.build`"
+            " (the library has no fallback path)")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, i64, i32, c_int = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int
+    lib.moe_route_topk.argtypes = [P, P, P, i64, i64, i32, i32, c_int, P, P, P]
+    lib.moe_sparse_map.argtypes = [P, i64, i32, i32, P, P, P, P, P, ctypes.c_size_t, P]
+    lib.moe_scatter_linear.argtypes = [P, P, i64, i64, i64, i32, i32, P, P, P, c_int, c_int,
+                                       c_int, P, P, ctypes.c_size_t, P]
+    lib.moe_mlp_forward.argtypes = [P, P, P, P, P, P, i64, i64, i64, i32, i32, c_int, P, P,
+                                    ctypes.c_size_t, P]
+    lib.moe_workspace_size.argtypes = [ctypes.c_char_p, i64, i64, i64, i32, i32, c_int]
+    lib.moe_workspace_size.restype = ctypes.c_size_t
+    lib.moe_workspace_view.argtypes = [ctypes.c_char_p, i64, i64, i64, i32, i32, c_int]
+    lib.moe_workspace_view.restype = ctypes.c_int64
+    lib.moe_last_error.restype = ctypes.c_char_p
+    lib.moe_check_device_status.argtypes = [P, P]
+    lib.moe_profile_events.argtypes = [P, c_int]
+    lib.moe_debug_wait_timeout.argtypes = [i64, P, ctypes.c_size_t, P]
+    for name in ("moe_route_topk", "moe_sparse_map", "moe_scatter_linear", "moe_mlp_forward",
+                 "moe_check_device_status", "moe_profile_events", "moe_debug_wait_timeout",
+                 "moe_last_launch_count"):
+        getattr(lib, name).restype = c_int
+    return lib
+
+
+lib = _load()
+
+
+def _check(rc: int):
+    if rc != 0:
+        raise MoeError(rc, lib.moe_last_error().decode())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return MOE_BF16
+    if t.dtype == torch.float32:
+        return MOE_F32
+    raise TypeError(f"unsupported dtype {t.dtype} (bf16 or float32)")
+
+
+def _req(t, name, dtype=None, dim=None, device=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if dim is not None and t.dim() != dim:
+        raise ValueError(f"{name} must have {dim} dims, got {tuple(t.shape)}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
+def workspace_size(op: str, S: int, D: int, F: int, E: int, k: int, dtype) -> int:
+    code = dtype if isinstance(dtype, int) else (MOE_BF16 if dtype == torch.bfloat16 else MOE_F32)
+    return int(lib.moe_workspace_size(op.encode(), S, D, F, E, k, code))
+
+
+def workspace_view(which: str, S: int, D: int, F: int, E: int, k: int, dtype) -> int:
+    code = dtype if isinstance(dtype, int) else (MOE_BF16 if dtype == torch.bfloat16 else MOE_F32)
+    return int(lib.moe_workspace_view(which.encode(), S, D, F, E, k, code))
+
+
+def alloc_workspace(nbytes: int, device) -> torch.Tensor:
+    # torch's caching allocator returns 512-byte aligned blocks
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+def route_topk(x: torch.Tensor, w_gate: torch.Tensor, k: int,
+               logit_bias: Optional[torch.Tensor] = None):
+    """Top-k experts [S,k] int32 and softmax weights [S,k] float32 (moe_route_topk)."""
+    _req(x, "x", dim=2)
+    _req(w_gate, "w_gate", dtype=x.dtype, dim=2, device=x.device)
+    S, D = x.shape
+    E = w_gate.shape[1]
+    if w_gate.shape[0] != D:
+        raise ValueError("w_gate must be [D, E]")
+    if logit_bias is not None:
+        _req(logit_bias, "logit_bias", dtype=torch.float32, dim=1, device=x.device)
+    te = torch.empty((S, k), dtype=torch.int32, device=x.device)
+    tw = torch.empty((S, k), dtype=torch.float32, device=x.device)
+    _check(lib.moe_route_topk(_ptr(x), _ptr(w_gate), _ptr(logit_bias), S, D, E, k,
+                              _dtype_code(x), _ptr(te), _ptr(tw), _stream(x.device)))
+    return te, tw
+
+
+def sparse_map(top_experts: torch.Tensor, E: int, ws: Optional[torch.Tensor] = None):
+    """(counts [E], offsets [E+1], sparse_rows [S*k], sorted_rows [S*k]) int32 (moe_sparse_map)."""
+    _req(top_experts, "top_experts", dtype=torch.int32, dim=2)
+    S, k = top_experts.shape
+    dev = top_experts.device
+    need = workspace_size("sparse_map", S, 0, 0, E, k, MOE_BF16)
+    if need == 0:
+        raise ValueError("sizes outside the library's limits")
+    if ws is None:
+        ws = alloc_workspace(need, dev)
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    sparse_rows = torch.empty(S * k, dtype=torch.int32, device=dev)
+    sorted_rows = torch.empty(S * k, dtype=torch.int32, device=dev)
+    _check(lib.moe_sparse_map(_ptr(top_experts), S, k, E, _ptr(counts), _ptr(offsets),
+                              _ptr(sparse_rows), _ptr(sorted_rows), _ptr(ws), ws.numel(),
+                              _stream(dev)))
+    return counts, offsets, sparse_rows, sorted_rows
+
+
+def scatter_linear(X: torch.Tensor, W: torch.Tensor, k: int, sorted_rows: torch.Tensor,
+                   expert_offsets: torch.Tensor, gates: Optional[torch.Tensor] = None,
+                   gather_in: bool = True, scatter_out: bool = True, S: Optional[int] = None,
+                   out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None):
+    """ParallelLinear(X, W, I, G) (moe_scatter_linear). Returns Y: [S, Dout] float32 when
+    scatter_out (accumulated into `out` if given, else into a fresh zero tensor), otherwise
+    [S*k, Dout] in X's dtype."""
+    _req(X, "X", dim=2)
+    _req(W, "W", dtype=X.dtype, dim=3, device=X.device)
+    _req(sorted_rows, "sorted_rows", dtype=torch.int32, dim=1, device=X.device)
+    _req(expert_offsets, "expert_offsets", dtype=torch.int32, dim=1, device=X.device)
+    E, Din, Dout = W.shape
+    if X.shape[1] != Din:
+        raise ValueError("X and W disagree on Din")
+    R = sorted_rows.shape[0]
+    if S is None:
+        S = X.shape[0] if gather_in else R // k
+    if S * k != R:
+        raise ValueError("sorted_rows must hold S*k entries")
+    if not gather_in and X.shape[0] != R:
+        raise ValueError("grouped X must have S*k rows")
+    if gates is not None:
+        _req(gates, "gates", dtype=torch.float32, device=X.device)
+        if gates.numel() != R:
+            raise ValueError("gates must hold S*k entries")
+    dev = X.device
+    if scatter_out:
+        Y = torch.zeros((S, Dout), dtype=torch.float32, device=dev) if out is None else out
+        _req(Y, "out", dtype=torch.float32, dim=2, device=dev)
+    else:
+        Y = torch.empty((R, Dout), dtype=X.dtype, device=dev) if out is None else out
+        _req(Y, "out", dtype=X.dtype, dim=2, device=dev)
+    if ws is None:
+        ws = alloc_workspace(workspace_size("scatter_linear", S, Din, Dout, E, k, X.dtype), dev)
+    _check(lib.moe_scatter_linear(_ptr(X), _ptr(W), S, Din, Dout, E, k, _ptr(sorted_rows),
+                                  _ptr(expert_offsets), _ptr(gates), int(bool(gather_in)),
+                                  int(bool(scatter_out)), _dtype_code(X), _ptr(Y), _ptr(ws),
+                                  ws.numel(), _stream(dev)))
+    return Y
+
+
+class ForwardWorkspace:
+    """A workspace for mlp_forward plus typed views of what the forward leaves in it."""
+
+    def __init__(self, S, D, F, E, k, dtype, device):
+        self.shape = (S, D, F, E, k)
+        self.dtype = dtype
+        code = _dtype_code(torch.empty(0, dtype=dtype))
+        self.code = code
+        n = workspace_size("mlp_forward", S, D, F, E, k, code)
+        if n == 0:
+            raise ValueError("sizes outside the library's limits")
+        self.buf = alloc_workspace(n, device)
+
+    def view(self, which: str) -> torch.Tensor:
+        S, D, F, E, k = self.shape
+        off = workspace_view(which, S, D, F, E, k, self.code)
+        if off < 0:
+            raise KeyError(which)
+        R = S * k
+        n, dt, shape = {
+            "top_experts": (R, torch.int32, (S, k)),
+            "top_weights": (R, torch.float32, (S, k)),
+            "expert_counts": (E, torch.int32, (E,)),
+            "expert_offsets": (E + 1, torch.int32, (E + 1,)),
+            "sparse_rows": (R, torch.int32, (R,)),
+            "sorted_rows": (R, torch.int32, (R,)),
+            "h": (R * F, self.dtype, (R, F)),
+        }[which]
+        nbytes = n * torch.empty(0, dtype=dt).element_size()
+        return self.buf[off:off + nbytes].view(dt).view(shape)
+
+
+def mlp_forward(x: torch.Tensor, w_gate: torch.Tensor, w_gate_e: torch.Tensor,
+                w_up: torch.Tensor, w_down: torch.Tensor, k: int,
+                logit_bias: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                ws: Optional[ForwardWorkspace] = None) -> torch.Tensor:
+    """The whole MoE expert-MLP forward (moe_mlp_forward); returns out [S, D] float32."""
+    _req(x, "x", dim=2)
+    dev = x.device
+    for t, n, d in ((w_gate, "w_gate", 2), (w_gate_e, "w_gate_e", 3), (w_up, "w_up", 3),
+                    (w_down, "w_down", 3)):
+        _req(t, n, dtype=x.dtype, dim=d, device=dev)
+    S, D = x.shape
+    E = w_gate.shape[1]
+    F = w_gate_e.shape[2]
+    if w_gate.shape[0] != D or tuple(w_gate_e.shape) != (E, D, F) or \
+            tuple(w_up.shape) != (E, D, F) or tuple(w_down.shape) != (E, F, D):
+        raise ValueError("expected w_gate [D,E], w_gate_e/w_up [E,D,F], w_down [E,F,D]")
+    if logit_bias is not None:
+        _req(logit_bias, "logit_bias", dtype=torch.float32, dim=1, device=dev)
+    if out is None:
+        out = torch.empty((S, D), dtype=torch.float32, device=dev)
+    _req(out, "out", dtype=torch.float32, dim=2, device=dev)
+    if ws is None:
+        ws = ForwardWorkspace(S, D, F, E, k, x.dtype, dev)
+    _check(lib.moe_mlp_forward(_ptr(x), _ptr(w_gate), _ptr(logit_bias), _ptr(w_gate_e),
+                               _ptr(w_up), _ptr(w_down), S, D, F, E, k, _dtype_code(x),
+                               _ptr(out), _ptr(ws.buf), ws.buf.numel(), _stream(dev)))
+    return out
+
+
+def check_device_status(ws: torch.Tensor):
+    """Synchronises and raises MoeError if the device flagged a bad expert id or a timeout."""
+    buf = ws.buf if isinstance(ws, ForwardWorkspace) else ws
+    _check(lib.moe_check_device_status(_ptr(buf), _stream(buf.device)))
+
+
+def profile_events(events):
+    """Registers torch.cuda.Event objects (>= 5) for the next mlp_forward on this thread."""
+    if not events:
+        _check(lib.moe_profile_events(None, 0))
+        return
+    arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    _check(lib.moe_profile_events(arr, len(events)))
+
+
+def debug_wait_timeout(limit_ns: int, ws: torch.Tensor):
+    _check(lib.moe_debug_wait_timeout(limit_ns, _ptr(ws), ws.numel(), _stream(ws.device)))
+
+
+def last_launch_count() -> int:
+    return int(lib.moe_last_launch_count())

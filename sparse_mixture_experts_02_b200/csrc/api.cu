@@ -1,0 +1,407 @@
+// C ABI of the MoE library: argument checks, workspace layout, launch order, status reporting.
+// Every public call validates on the host, then enqueues kernels on the caller's stream; nothing
+// here synchronises except moe_check_device_status.
+#include "moe_internal.cuh"
+
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+
+namespace moe {
+
+static thread_local char g_err[512] = "";
+static thread_local int g_launches = 0;
+static thread_local void *g_prof_events[8] = {};
+static thread_local int g_prof_n = 0;
+
+int set_error(int code, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof(g_err), fmt, ap);
+    va_end(ap);
+    return code;
+}
+
+int num_sms() {
+    int dev = 0, n = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n > 0 ? n : 1;
+}
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Supported device: compute capability 10.0 (checked once per device).
+int check_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return set_error(MOE_ERR_CUDA, "cudaGetDevice failed");
+    static std::mutex mu;
+    static int known[64] = {0};  // 0 unknown, 1 ok, -1 unsupported
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev < 0 || dev >= 64) return set_error(MOE_ERR_UNSUPPORTED, "device index %d", dev);
+    if (known[dev] == 0) {
+        int major = 0, minor = 0;
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+        known[dev] = (major == 10 && minor == 0) ? 1 : -1;
+    }
+    if (known[dev] < 0)
+        return set_error(MOE_ERR_UNSUPPORTED, "this library is built for sm_100a (B200) only");
+    return MOE_OK;
+}
+
+int check_launch(const char *what) {
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return set_error(MOE_ERR_CUDA, "%s launch: %s", what, cudaGetErrorString(e));
+    return MOE_OK;
+}
+
+int check_dims(int64_t S, int32_t E, int32_t k) {
+    if (S < 0) return set_error(MOE_ERR_INVALID_ARG, "S must be >= 0 (got %lld)", (long long)S);
+    if (E < 1 || E > 256) return set_error(MOE_ERR_INVALID_ARG, "E must be in [1, 256] (got %d)", E);
+    if (k < 1 || k > 8 || k > E)
+        return set_error(MOE_ERR_INVALID_ARG, "k must be in [1, min(E, 8)] (got k=%d, E=%d)", k, E);
+    if (S * (int64_t)k >= (int64_t(1) << 31))
+        return set_error(MOE_ERR_INVALID_ARG, "S*k must be < 2^31");
+    return MOE_OK;
+}
+
+int check_feat(const char *name, int64_t v) {
+    if (v <= 0 || v % 8 != 0 || v >= (int64_t(1) << 31))
+        return set_error(MOE_ERR_INVALID_ARG, "%s must be a positive multiple of 8 below 2^31 (got %lld)",
+                         name, (long long)v);
+    return MOE_OK;
+}
+
+int check_ptr(const char *name, const void *p, size_t align, bool nullable = false) {
+    if (p == nullptr) {
+        if (nullable) return MOE_OK;
+        return set_error(MOE_ERR_INVALID_ARG, "%s is null", name);
+    }
+    if (!aligned(p, align)) return set_error(MOE_ERR_INVALID_ARG, "%s is not %zu-byte aligned", name, align);
+    return MOE_OK;
+}
+
+int check_dtype(moe_dtype dt) {
+    if (dt != MOE_F32 && dt != MOE_BF16) return set_error(MOE_ERR_UNSUPPORTED, "unknown dtype %d", (int)dt);
+    return MOE_OK;
+}
+
+size_t esize(moe_dtype dt) { return dt == MOE_BF16 ? 2 : 4; }
+
+// ---- workspace layout ------------------------------------------------------------------------
+struct MlpLayout {
+    size_t status, top_e, top_w, counts, offsets, sparse_rows, sorted_rows, scratch, h, total;
+};
+
+MlpLayout mlp_layout(int64_t S, int64_t F, int32_t E, int32_t k, moe_dtype dt) {
+    const int64_t R = S * k;
+    MlpLayout L;
+    size_t o = 0;
+    L.status = o; o += kStatusBytes;
+    L.top_e = o; o = align_up(o + sizeof(int32_t) * (size_t)R);
+    L.top_w = o; o = align_up(o + sizeof(float) * (size_t)R);
+    L.counts = o; o = align_up(o + sizeof(int32_t) * (size_t)E);
+    L.offsets = o; o = align_up(o + sizeof(int32_t) * (size_t)(E + 1));
+    L.sparse_rows = o; o = align_up(o + sizeof(int32_t) * (size_t)R);
+    L.sorted_rows = o; o = align_up(o + sizeof(int32_t) * (size_t)R);
+    L.scratch = o; o = align_up(o + map_scratch_bytes(R, E));
+    L.h = o; o = align_up(o + esize(dt) * (size_t)R * (size_t)F);
+    L.total = o;
+    return L;
+}
+
+size_t map_ws_bytes(int64_t S, int32_t E, int32_t k) {
+    return kStatusBytes + align_up(map_scratch_bytes(S * k, E));
+}
+
+int check_ws(void *ws, size_t ws_bytes, size_t need) {
+    if (ws == nullptr) return set_error(MOE_ERR_WORKSPACE, "workspace is null");
+    if (!aligned(ws, kAlign)) return set_error(MOE_ERR_WORKSPACE, "workspace is not 256-byte aligned");
+    if (ws_bytes < need)
+        return set_error(MOE_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", ws_bytes, need);
+    return MOE_OK;
+}
+
+template <class T>
+T *at(void *ws, size_t off) {
+    return reinterpret_cast<T *>(static_cast<uint8_t *>(ws) + off);
+}
+
+void record_prof(int idx, cudaStream_t s) {
+    if (g_prof_n > idx && g_prof_events[idx] != nullptr)
+        cudaEventRecord(static_cast<cudaEvent_t>(g_prof_events[idx]), s);
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+const char *moe_last_error(void) { return g_err; }
+
+int moe_last_launch_count(void) { return g_launches; }
+
+int moe_profile_events(void *const *events, int n) {
+    if (n < 0 || n > 8 || (n > 0 && events == nullptr))
+        return set_error(MOE_ERR_INVALID_ARG, "profile events: n must be in [0, 8]");
+    g_prof_n = n;
+    for (int i = 0; i < n; ++i) g_prof_events[i] = events[i];
+    return MOE_OK;
+}
+
+size_t moe_workspace_size(const char *op, int64_t S, int64_t D, int64_t F, int32_t E, int32_t k,
+                          moe_dtype dt) {
+    (void)D;
+    if (op == nullptr || S < 0 || E < 1 || E > 256 || k < 1 || k > 8 || k > E) return 0;
+    if (S * (int64_t)k >= (int64_t(1) << 31)) return 0;
+    if (strcmp(op, "sparse_map") == 0) return map_ws_bytes(S, E, k);
+    if (strcmp(op, "scatter_linear") == 0) return kStatusBytes;
+    if (strcmp(op, "mlp_forward") == 0) {
+        if (F <= 0 || (dt != MOE_F32 && dt != MOE_BF16)) return 0;
+        return mlp_layout(S, F, E, k, dt).total;
+    }
+    return 0;
+}
+
+int64_t moe_workspace_view(const char *which, int64_t S, int64_t D, int64_t F, int32_t E,
+                           int32_t k, moe_dtype dt) {
+    (void)D;
+    if (which == nullptr) return -1;
+    const MlpLayout L = mlp_layout(S, F, E, k, dt);
+    if (!strcmp(which, "top_experts")) return (int64_t)L.top_e;
+    if (!strcmp(which, "top_weights")) return (int64_t)L.top_w;
+    if (!strcmp(which, "expert_counts")) return (int64_t)L.counts;
+    if (!strcmp(which, "expert_offsets")) return (int64_t)L.offsets;
+    if (!strcmp(which, "sparse_rows")) return (int64_t)L.sparse_rows;
+    if (!strcmp(which, "sorted_rows")) return (int64_t)L.sorted_rows;
+    if (!strcmp(which, "h")) return (int64_t)L.h;
+    return -1;
+}
+
+int moe_route_topk(const void *x, const void *w_gate, const float *logit_bias, int64_t S,
+                   int64_t D, int32_t E, int32_t k, moe_dtype dt, int32_t *top_experts,
+                   float *top_weights, moe_stream_t stream) {
+    g_launches = 0;
+    int rc;
+    if ((rc = check_dtype(dt)) || (rc = check_dims(S, E, k)) || (rc = check_feat("D", D))) return rc;
+    const size_t eb = esize(dt);
+    if ((rc = check_ptr("x", x, eb)) || (rc = check_ptr("w_gate", w_gate, eb)) ||
+        (rc = check_ptr("logit_bias", logit_bias, 4, true)) ||
+        (rc = check_ptr("top_experts", top_experts, 4)) ||
+        (rc = check_ptr("top_weights", top_weights, 4)))
+        return rc;
+    if ((rc = check_device())) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    g_launches += launch_route(x, w_gate, logit_bias, S, D, E, k, dt == MOE_BF16, top_experts,
+                               top_weights, s);
+    return check_launch("route");
+}
+
+int moe_sparse_map(const int32_t *top_experts, int64_t S, int32_t k, int32_t E,
+                   int32_t *expert_counts, int32_t *expert_offsets, int32_t *sparse_rows,
+                   int32_t *sorted_rows, void *ws, size_t ws_bytes, moe_stream_t stream) {
+    g_launches = 0;
+    int rc;
+    if ((rc = check_dims(S, E, k))) return rc;
+    const int64_t R = S * k;
+    if ((rc = check_ptr("top_experts", top_experts, 4, R == 0)) ||
+        (rc = check_ptr("expert_counts", expert_counts, 4)) ||
+        (rc = check_ptr("expert_offsets", expert_offsets, 4)) ||
+        (rc = check_ptr("sparse_rows", sparse_rows, 4, R == 0)) ||
+        (rc = check_ptr("sorted_rows", sorted_rows, 4, R == 0)))
+        return rc;
+    if ((rc = check_ws(ws, ws_bytes, map_ws_bytes(S, E, k)))) return rc;
+    if ((rc = check_device())) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    unsigned *status = at<unsigned>(ws, 0);
+    if (cudaMemsetAsync(status, 0, sizeof(unsigned), s) != cudaSuccess)
+        return set_error(MOE_ERR_CUDA, "cudaMemsetAsync of the status word failed");
+    int n = 0;
+    launch_sparse_map(top_experts, R, E, expert_counts, expert_offsets, sparse_rows, sorted_rows,
+                      at<int32_t>(ws, kStatusBytes), status, s, &n);
+    g_launches = n;
+    return check_launch("sparse_map");
+}
+
+int moe_scatter_linear(const void *X, const void *W, int64_t S, int64_t Din, int64_t Dout,
+                       int32_t E, int32_t k, const int32_t *sorted_rows,
+                       const int32_t *expert_offsets, const float *top_weights, int gather_in,
+                       int scatter_out, moe_dtype dt, void *Y, void *ws, size_t ws_bytes,
+                       moe_stream_t stream) {
+    g_launches = 0;
+    int rc;
+    if ((rc = check_dtype(dt)) || (rc = check_dims(S, E, k)) || (rc = check_feat("Din", Din)) ||
+        (rc = check_feat("Dout", Dout)))
+        return rc;
+    const int64_t R = S * k;
+    if ((rc = check_ptr("X", X, 16, R == 0)) || (rc = check_ptr("W", W, 16)) ||
+        (rc = check_ptr("sorted_rows", sorted_rows, 4, R == 0)) ||
+        (rc = check_ptr("expert_offsets", expert_offsets, 4)) ||
+        (rc = check_ptr("top_weights", top_weights, 4, true)) || (rc = check_ptr("Y", Y, 16, R == 0)))
+        return rc;
+    if ((rc = check_ws(ws, ws_bytes, kStatusBytes))) return rc;
+    if ((rc = check_device())) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    unsigned *status = at<unsigned>(ws, 0);
+    if (cudaMemsetAsync(status, 0, sizeof(unsigned), s) != cudaSuccess)
+        return set_error(MOE_ERR_CUDA, "cudaMemsetAsync of the status word failed");
+    if (R == 0) return MOE_OK;
+    GemmArgs a{};
+    a.A = X;
+    a.a_rows = gather_in ? S : R;
+    a.B0 = W;
+    a.B1 = nullptr;
+    a.offsets = expert_offsets;
+    a.sorted_rows = sorted_rows;
+    a.gates = top_weights;
+    a.out = Y;
+    a.S = S;
+    a.R = R;
+    a.E = E;
+    a.k = k;
+    a.K = Din;
+    a.N = Dout;
+    a.bf16 = dt == MOE_BF16;
+    a.gather = gather_in != 0;
+    a.glu = false;
+    a.scatter = scatter_out != 0;
+    a.status = status;
+    a.wait_limit_ns = kWaitLimitNs;
+    if ((rc = launch_grouped_gemm(a, s))) return rc;
+    g_launches = 1;
+    return check_launch("scatter_linear");
+}
+
+int moe_mlp_forward(const void *x, const void *w_gate, const float *logit_bias,
+                    const void *w_gate_e, const void *w_up, const void *w_down, int64_t S,
+                    int64_t D, int64_t F, int32_t E, int32_t k, moe_dtype dt, float *out, void *ws,
+                    size_t ws_bytes, moe_stream_t stream) {
+    g_launches = 0;
+    int rc;
+    if ((rc = check_dtype(dt)) || (rc = check_dims(S, E, k)) || (rc = check_feat("D", D)) ||
+        (rc = check_feat("F", F)))
+        return rc;
+    if ((rc = check_ptr("x", x, 16, S == 0)) || (rc = check_ptr("w_gate", w_gate, 16)) ||
+        (rc = check_ptr("logit_bias", logit_bias, 4, true)) ||
+        (rc = check_ptr("w_gate_e", w_gate_e, 16)) || (rc = check_ptr("w_up", w_up, 16)) ||
+        (rc = check_ptr("w_down", w_down, 16)) || (rc = check_ptr("out", out, 16, S == 0)))
+        return rc;
+    const MlpLayout L = mlp_layout(S, F, E, k, dt);
+    if ((rc = check_ws(ws, ws_bytes, L.total))) return rc;
+    if ((rc = check_device())) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int64_t R = S * k;
+    unsigned *status = at<unsigned>(ws, L.status);
+    int32_t *top_e = at<int32_t>(ws, L.top_e);
+    float *top_w = at<float>(ws, L.top_w);
+    int32_t *counts = at<int32_t>(ws, L.counts);
+    int32_t *offsets = at<int32_t>(ws, L.offsets);
+    int32_t *sparse_rows = at<int32_t>(ws, L.sparse_rows);
+    int32_t *sorted_rows = at<int32_t>(ws, L.sorted_rows);
+    void *h = at<void>(ws, L.h);
+    int n = 0;
+
+    record_prof(0, s);
+    n += launch_zero_f32(out, S * D, status, s);
+    if ((rc = check_launch("zero"))) return rc;
+    n += launch_route(x, w_gate, logit_bias, S, D, E, k, dt == MOE_BF16, top_e, top_w, s);
+    if ((rc = check_launch("route"))) return rc;
+    record_prof(1, s);
+    launch_sparse_map(top_e, R, E, counts, offsets, sparse_rows, sorted_rows,
+                      at<int32_t>(ws, L.scratch), status, s, &n);
+    if ((rc = check_launch("sparse_map"))) return rc;
+    record_prof(2, s);
+    if (R > 0) {
+        GemmArgs a{};
+        a.A = x;
+        a.a_rows = S;
+        a.B0 = w_gate_e;
+        a.B1 = w_up;
+        a.offsets = offsets;
+        a.sorted_rows = sorted_rows;
+        a.gates = nullptr;
+        a.out = h;
+        a.S = S;
+        a.R = R;
+        a.E = E;
+        a.k = k;
+        a.K = D;
+        a.N = F;
+        a.bf16 = dt == MOE_BF16;
+        a.gather = true;
+        a.glu = true;
+        a.scatter = false;
+        a.status = status;
+        a.wait_limit_ns = kWaitLimitNs;
+        if ((rc = launch_grouped_gemm(a, s))) return rc;
+        if ((rc = check_launch("gemm1"))) return rc;
+        ++n;
+        record_prof(3, s);
+        GemmArgs b = a;
+        b.A = h;
+        b.a_rows = R;
+        b.B0 = w_down;
+        b.B1 = nullptr;
+        b.gates = top_w;
+        b.out = out;
+        b.K = F;
+        b.N = D;
+        b.gather = false;
+        b.glu = false;
+        b.scatter = true;
+        if ((rc = launch_grouped_gemm(b, s))) return rc;
+        if ((rc = check_launch("gemm2"))) return rc;
+        ++n;
+        record_prof(4, s);
+    } else {
+        record_prof(3, s);
+        record_prof(4, s);
+    }
+    g_prof_n = 0;
+    g_launches = n;
+    return MOE_OK;
+}
+
+int moe_check_device_status(void *ws, moe_stream_t stream) {
+    if (ws == nullptr) return set_error(MOE_ERR_WORKSPACE, "workspace is null");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return set_error(MOE_ERR_CUDA, "stream: %s", cudaGetErrorString(e));
+    unsigned v = 0;
+    e = cudaMemcpy(&v, ws, sizeof(v), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return set_error(MOE_ERR_CUDA, "status read: %s", cudaGetErrorString(e));
+    if (v & kStatusTimeout)
+        return set_error(MOE_ERR_DEVICE_TIMEOUT, "a device wait ran out (kernel id %u)", (v >> 8) & 0xFFu);
+    if (v & kStatusBadExpert)
+        return set_error(MOE_ERR_BAD_EXPERT_ID, "an expert id outside [0, E) was seen");
+    return MOE_OK;
+}
+
+int moe_debug_wait_timeout(int64_t limit_ns, void *ws, size_t ws_bytes, moe_stream_t stream) {
+    g_launches = 0;
+    int rc;
+    if (limit_ns < 1 || limit_ns > 1000000000LL)
+        return set_error(MOE_ERR_INVALID_ARG, "limit_ns must be in [1, 1e9]");
+    if ((rc = check_ws(ws, ws_bytes, kStatusBytes))) return rc;
+    if ((rc = check_device())) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    unsigned *status = at<unsigned>(ws, 0);
+    if (cudaMemsetAsync(status, 0, sizeof(unsigned), s) != cudaSuccess)
+        return set_error(MOE_ERR_CUDA, "cudaMemsetAsync of the status word failed");
+    launch_debug_wait(limit_ns, status, s);
+    g_launches = 1;
+    return check_launch("debug_wait");
+}
+
+}  // extern "C"

@@ -1,0 +1,543 @@
+// Scattered grouped GEMM on the sm_100a tensor cores (tcgen05 + TMEM + TMA), one kernel for
+// every form of ParallelLinear(X, W, I, G) the library needs:
+//
+//   GEMM1 of the MoE MLP:   gathered x rows, W_gate_e and W_up side by side in one MMA (N = 256:
+//                           128 gate columns + the same 128 up columns), SwiGLU in registers,
+//                           h rows stored in slot (expert-grouped) order;
+//   GEMM2 of the MoE MLP:   contiguous h rows, W_down, router-weight scaling, fp32 vector
+//                           atomic scatter-add into token order;
+//   moe_scatter_linear:     any of gather / contiguous input x scatter / grouped output.
+//
+// Sources: ScatterMoE guide ("ScatterMoE Guide: Fast Fused Kernels for Sparse MoE LLMs"),
+// "The ParallelLinear Core Abstraction" figure (Step 1 indexed gather, Step 2 tile GEMM against
+// W[expert], Step 3 gate scaling and scatter-add), "2. Grouped Coordinate Indexing Without
+// Padding" (ceil(N_e / B_M) tiles per expert, the last one masked, no padding in memory) and
+// "3. Assembling the ScatterMoE FFN Block" (SwiGLU, gate half first); the fused gate+up
+// mainloop follows the abstract of "Cross-Platform Fused MoE Dispatch in Triton"; the per-tile
+// expert id follows "Inside the Flash-MoE Kernel: Fused Tile-Level Dispatch".
+//
+// Design (B200): persistent, one CTA per SM, 6 warps:
+//   warp 0      TMA producer. B tiles by 3-D tensor map (N, K, expert). A tiles either by a
+//               2-D box (contiguous rows) or, for gathered rows, by tile::gather4: each of the
+//               32 lanes fetches 4 token rows, so one stage's 128 rows need no [S*k, D] copy.
+//   warp 1      TMEM owner (512 columns = two 128 x 256 fp32 accumulators) and MMA issuer
+//               (one thread): 4 x tcgen05.mma (M=128, N=256, K=32 bytes) per 128-byte K stage.
+//   warps 2-5   epilogue: tcgen05.ld of the accumulator (thread = tile row), then SwiGLU + bf16
+//               store, or gate * acc and red.global.add.v4.f32 into out[token].
+// Stages: 4 x (A 16 KB + B 32 KB), 128-byte swizzle; A is K-major, B (weights, N contiguous)
+// is MN-major. Two accumulators let the epilogue of tile i overlap the mainloop of tile i+1.
+// Tile schedule: every CTA derives it from expert_offsets on the device (no host sync):
+// tiles are ordered expert-major, then N tile, then M tile, so the CTAs running at one time
+// share expert weight tiles and gathered rows through L2. Waits are bounded (see mbar_wait).
+#include "moe_internal.cuh"
+
+#include <stdio.h>
+#include <mutex>
+
+namespace moe {
+namespace {
+
+constexpr int BM = 128;                 // rows per tile (TMEM lanes)
+constexpr int BN = 256;                 // MMA N = accumulator columns
+constexpr int STAGES = 4;
+constexpr int KBYTES = 128;             // bytes of K per stage (one 128-byte swizzle row)
+constexpr int A_BYTES = BM * KBYTES;    // 16 KB
+constexpr int B_BYTES = BN * KBYTES;    // 32 KB (BN columns x (128 / eb) K rows x eb)
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int MAX_E = 256;
+constexpr int THREADS = 192;
+constexpr uint32_t TMEM_COLS = 512;
+
+struct SmemTail {
+    uint64_t full[STAGES];
+    uint64_t empty[STAGES];
+    uint64_t tfull[2];
+    uint64_t tempty[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+    int32_t off[MAX_E + 1];
+    int32_t tstart[MAX_E + 1];
+};
+constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + sizeof(SmemTail);
+
+struct KParams {
+    const int32_t *offsets;
+    const int32_t *sorted_rows;
+    const float *gates;
+    void *out;
+    int32_t E, k;
+    int32_t N;        // output columns
+    int32_t num_kb;   // K stages
+    int32_t n_tiles;  // N tiles
+    int64_t S, R;     // bounds of scatter rows (tokens) and grouped rows (slots)
+    unsigned *status;
+    int64_t wait_limit_ns;
+};
+
+struct TileInfo {
+    int e, row_begin, rows, n_idx;
+};
+
+__device__ __forceinline__ TileInfo decode_tile(int t, const SmemTail &st, int E, int n_tiles) {
+    int lo = 0, hi = E;  // tstart[lo] <= t < tstart[hi]
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (st.tstart[mid] <= t) lo = mid;
+        else hi = mid;
+    }
+    TileInfo ti;
+    ti.e = lo;
+    const int local = t - st.tstart[lo];
+    const int cnt = st.off[lo + 1] - st.off[lo];
+    const int mt = (cnt + BM - 1) / BM;
+    ti.n_idx = local / mt;
+    const int m = local - ti.n_idx * mt;
+    ti.row_begin = st.off[lo] + m * BM;
+    ti.rows = min(BM, st.off[lo + 1] - ti.row_begin);
+    (void)n_tiles;
+    return ti;
+}
+
+__device__ __forceinline__ float silu_f(float z) { return z / (1.0f + __expf(-z)); }
+
+template <bool BF16, bool GATHER, bool GLU, bool SCATTER>
+__global__ void __launch_bounds__(THREADS, 1)
+grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                    const __grid_constant__ CUtensorMap tmB0,
+                    const __grid_constant__ CUtensorMap tmB1, const KParams p) {
+    constexpr int EB = BF16 ? 2 : 4;          // input element bytes
+    constexpr int BK = KBYTES / EB;           // K elements per stage
+    constexpr int CW = KBYTES / EB;           // N elements per 128-byte B chunk
+    constexpr int NCH = BN / CW;              // B chunks per stage
+    constexpr int CHUNK = BK * KBYTES;        // bytes of one B chunk
+    constexpr int B_KSTEP = (32 / EB) * KBYTES;  // bytes of B per MMA K step (32 bytes of K)
+    constexpr int OUT_COLS = GLU ? BN / 2 : BN;  // output columns per tile
+    constexpr uint32_t IDESC = dev::idesc_f32acc(BF16, BM, BN, true);
+    static_assert(NCH * CHUNK == B_BYTES, "B stage size");
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    SmemTail &st = *reinterpret_cast<SmemTail *>(smem + (size_t)STAGES * STAGE_BYTES);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int E = p.E;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            dev::mbar_init(&st.full[s], 1);
+            dev::mbar_init(&st.empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            dev::mbar_init(&st.tfull[b], 1);
+            dev::mbar_init(&st.tempty[b], 4);
+        }
+        dev::mbar_init(&st.drain, 1);
+        st.abort = 0;
+        dev::fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        dev::prefetch_tmap(&tmA);
+        dev::prefetch_tmap(&tmB0);
+        if (GLU) dev::prefetch_tmap(&tmB1);
+    }
+    if (warp == 1) {
+        dev::tmem_alloc(&st.tmem_base, TMEM_COLS);
+        dev::tmem_relinquish();
+        dev::tc_fence_before();
+    }
+    for (int e = threadIdx.x; e <= E; e += THREADS) st.off[e] = __ldg(p.offsets + e);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int run = 0;
+        for (int e = 0; e < E; ++e) {
+            st.tstart[e] = run;
+            const int mt = (st.off[e + 1] - st.off[e] + BM - 1) / BM;
+            run += mt * p.n_tiles;
+        }
+        st.tstart[E] = run;
+    }
+    __syncthreads();
+    dev::tc_fence_after();
+    const uint32_t tmem_base = st.tmem_base;
+    const int total = st.tstart[E];
+    volatile int *abort = &st.abort;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------------ TMA producer
+        uint32_t s = 0, ph = 0;
+        uint32_t issued = 0, last_par = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+            const TileInfo ti = decode_tile(t, st, E, p.n_tiles);
+            int32_t rr[4] = {0, 0, 0, 0};
+            if (GATHER) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int r = lane * 4 + j;
+                    const int pr = ti.row_begin + min(r, ti.rows - 1);
+                    rr[j] = __ldg(p.sorted_rows + pr) / p.k;
+                }
+            }
+            const int n0 = ti.n_idx * OUT_COLS;
+            for (int kb = 0; kb < p.num_kb; ++kb) {
+                bool w = true;
+                if (lane == 0)
+                    w = dev::mbar_wait(&st.empty[s], ph ^ 1u, abort, p.status, p.wait_limit_ns,
+                                       kKernelGemm);
+                w = __shfl_sync(0xffffffffu, w, 0);
+                if (!w) {
+                    ok = false;
+                    break;
+                }
+                uint8_t *sA = smem + (size_t)s * STAGE_BYTES;
+                uint8_t *sB = sA + A_BYTES;
+                if (lane == 0) dev::mbar_arrive_expect_tx(&st.full[s], STAGE_BYTES);
+                __syncwarp();
+                const int kc = kb * BK;
+                if (GATHER) {
+                    dev::tma_gather4(sA + lane * 4 * KBYTES, &tmA, &st.full[s], kc, rr[0], rr[1],
+                                     rr[2], rr[3]);
+                } else if (lane == 0) {
+                    dev::tma_load_2d(sA, &tmA, &st.full[s], kc, ti.row_begin);
+                }
+                if (lane == 0) {
+#pragma unroll
+                    for (int c = 0; c < NCH; ++c) {
+                        if (GLU) {
+                            const int half = NCH / 2;
+                            const CUtensorMap *m = c < half ? &tmB0 : &tmB1;
+                            dev::tma_load_3d(sB + c * CHUNK, m, &st.full[s],
+                                             n0 + (c % half) * CW, kc, ti.e);
+                        } else {
+                            dev::tma_load_3d(sB + c * CHUNK, &tmB0, &st.full[s], n0 + c * CW, kc,
+                                             ti.e);
+                        }
+                    }
+                }
+                issued |= 1u << s;
+                last_par = (last_par & ~(1u << s)) | (ph << s);
+                if (++s == STAGES) {
+                    s = 0;
+                    ph ^= 1u;
+                }
+            }
+        }
+        // teardown: every load this warp issued must land before the CTA may exit
+        if (lane == 0) {
+            for (int s2 = 0; s2 < STAGES; ++s2)
+                if (issued & (1u << s2))
+                    dev::mbar_wait(&st.full[s2], (last_par >> s2) & 1u, nullptr, p.status,
+                                   kDrainLimitNs, kKernelGemm);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            uint32_t s = 0, ph = 0;
+            int it = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++it) {
+                const uint32_t b = it & 1, aph = (it >> 1) & 1;
+                if (!dev::mbar_wait(&st.tempty[b], aph ^ 1u, abort, p.status, p.wait_limit_ns,
+                                    kKernelGemm))
+                    break;
+                dev::tc_fence_after();
+                const uint32_t d_tmem = tmem_base + b * BN;
+                for (int kb = 0; kb < p.num_kb; ++kb) {
+                    if (!dev::mbar_wait(&st.full[s], ph, abort, p.status, p.wait_limit_ns,
+                                        kKernelGemm)) {
+                        ok = false;
+                        break;
+                    }
+                    dev::tc_fence_after();
+                    const uint32_t sA = dev::smem_u32(smem + (size_t)s * STAGE_BYTES);
+                    const uint32_t sB = sA + A_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < KBYTES / 32; ++kk) {
+                        const uint64_t ad = dev::sdesc_sw128(sA + kk * 32, 16, 1024);
+                        const uint64_t bd = dev::sdesc_sw128(sB + kk * B_KSTEP, CHUNK, 1024);
+                        if (BF16) dev::mma_bf16(d_tmem, ad, bd, IDESC, (kb | kk) != 0);
+                        else dev::mma_tf32(d_tmem, ad, bd, IDESC, (kb | kk) != 0);
+                    }
+                    dev::mma_commit(&st.empty[s]);
+                    if (++s == STAGES) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                dev::mma_commit(&st.tfull[b]);
+            }
+            // teardown: all issued MMAs complete before TMEM is released
+            dev::mma_commit(&st.drain);
+            dev::mbar_wait(&st.drain, 0, nullptr, p.status, kDrainLimitNs, kKernelGemm);
+            dev::tc_fence_before();
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------------ epilogue
+        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        const int r = q * 32 + lane;
+        int it = 0;
+        for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
+            const TileInfo ti = decode_tile(t, st, E, p.n_tiles);
+            const uint32_t b = it & 1, aph = (it >> 1) & 1;
+            bool w = true;
+            if (lane == 0)
+                w = dev::mbar_wait(&st.tfull[b], aph, abort, p.status, p.wait_limit_ns,
+                                   kKernelGemm);
+            w = __shfl_sync(0xffffffffu, w, 0);
+            if (!w) break;
+            dev::tc_fence_after();
+            const int prow = ti.row_begin + r;
+            bool valid = r < ti.rows && prow >= 0 && prow < p.R;
+            int64_t orow = prow;
+            float g = 1.0f;
+            if (valid && (SCATTER || p.gates != nullptr)) {
+                const int i = __ldg(p.sorted_rows + prow);
+                if (SCATTER) orow = i / p.k;
+                if (p.gates != nullptr && i >= 0 && i < p.R) g = __ldg(p.gates + i);
+                // a slot whose route is outside [0, R) is skipped rather than written anywhere
+                if (i < 0 || i >= p.R) valid = false;
+            }
+            const int n0 = ti.n_idx * OUT_COLS;
+            const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + b * BN;
+            if (GLU) {
+#pragma unroll 1
+                for (int c = 0; c < OUT_COLS / 32; ++c) {
+                    uint32_t gv[32], uv[32];
+                    dev::tmem_ld32(tbase + c * 32, gv);
+                    dev::tmem_ld32(tbase + OUT_COLS + c * 32, uv);
+                    dev::tmem_ld_wait();
+                    const int col0 = n0 + c * 32;
+                    if (valid && col0 < p.N) {
+                        float hv[32];
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            hv[j] = g * silu_f(__uint_as_float(gv[j])) * __uint_as_float(uv[j]);
+                        if (BF16) {
+                            __nv_bfloat16 *dst =
+                                reinterpret_cast<__nv_bfloat16 *>(p.out) + orow * p.N + col0;
+#pragma unroll
+                            for (int v = 0; v < 4; ++v) {
+                                if (col0 + v * 8 < p.N) {
+                                    uint4 pk;
+                                    uint32_t *pw = reinterpret_cast<uint32_t *>(&pk);
+#pragma unroll
+                                    for (int j = 0; j < 4; ++j) {
+                                        __nv_bfloat162 t2 = __floats2bfloat162_rn(
+                                            hv[v * 8 + 2 * j], hv[v * 8 + 2 * j + 1]);
+                                        pw[j] = *reinterpret_cast<uint32_t *>(&t2);
+                                    }
+                                    *reinterpret_cast<uint4 *>(dst + v * 8) = pk;
+                                }
+                            }
+                        } else {
+                            float *dst = reinterpret_cast<float *>(p.out) + orow * p.N + col0;
+#pragma unroll
+                            for (int v = 0; v < 8; ++v)
+                                if (col0 + v * 4 < p.N)
+                                    *reinterpret_cast<float4 *>(dst + v * 4) = make_float4(
+                                        hv[v * 4], hv[v * 4 + 1], hv[v * 4 + 2], hv[v * 4 + 3]);
+                        }
+                    }
+                }
+            } else {
+#pragma unroll 1
+                for (int c = 0; c < OUT_COLS / 32; ++c) {
+                    uint32_t av[32];
+                    dev::tmem_ld32(tbase + c * 32, av);
+                    dev::tmem_ld_wait();
+                    const int col0 = n0 + c * 32;
+                    if (valid && col0 < p.N) {
+                        if (SCATTER) {
+                            float *dst = reinterpret_cast<float *>(p.out) + orow * p.N + col0;
+#pragma unroll
+                            for (int v = 0; v < 8; ++v)
+                                if (col0 + v * 4 < p.N)
+                                    dev::red_add_v4(dst + v * 4, g * __uint_as_float(av[v * 4]),
+                                                    g * __uint_as_float(av[v * 4 + 1]),
+                                                    g * __uint_as_float(av[v * 4 + 2]),
+                                                    g * __uint_as_float(av[v * 4 + 3]));
+                        } else if (BF16) {
+                            __nv_bfloat16 *dst =
+                                reinterpret_cast<__nv_bfloat16 *>(p.out) + orow * p.N + col0;
+#pragma unroll
+                            for (int v = 0; v < 4; ++v) {
+                                if (col0 + v * 8 < p.N) {
+                                    uint4 pk;
+                                    uint32_t *pw = reinterpret_cast<uint32_t *>(&pk);
+#pragma unroll
+                                    for (int j = 0; j < 4; ++j) {
+                                        __nv_bfloat162 t2 = __floats2bfloat162_rn(
+                                            g * __uint_as_float(av[v * 8 + 2 * j]),
+                                            g * __uint_as_float(av[v * 8 + 2 * j + 1]));
+                                        pw[j] = *reinterpret_cast<uint32_t *>(&t2);
+                                    }
+                                    *reinterpret_cast<uint4 *>(dst + v * 8) = pk;
+                                }
+                            }
+                        } else {
+                            float *dst = reinterpret_cast<float *>(p.out) + orow * p.N + col0;
+#pragma unroll
+                            for (int v = 0; v < 8; ++v)
+                                if (col0 + v * 4 < p.N)
+                                    *reinterpret_cast<float4 *>(dst + v * 4) =
+                                        make_float4(g * __uint_as_float(av[v * 4]),
+                                                    g * __uint_as_float(av[v * 4 + 1]),
+                                                    g * __uint_as_float(av[v * 4 + 2]),
+                                                    g * __uint_as_float(av[v * 4 + 3]));
+                        }
+                    }
+                }
+            }
+            dev::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) dev::mbar_arrive(&st.tempty[b]);
+        }
+    }
+
+    __syncthreads();
+    if (warp == 1) {
+        dev::tc_fence_after();
+        dev::tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+__global__ void debug_wait_kernel(int64_t limit_ns, unsigned *status) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        dev::mbar_init(&bar, 1);  // nothing ever arrives
+        abort_flag = 0;
+        dev::fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0)
+        dev::mbar_wait(&bar, 0, &abort_flag, status, limit_ns, kKernelDebugWait);
+}
+
+// ---- host side: tensor maps -------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+int encode(CUtensorMap *m, bool bf16, int rank, const void *base, const uint64_t *dims,
+           const uint64_t *strides_bytes, const uint32_t *box) {
+    EncodeTiledFn fn = get_encode();
+    if (!fn) return set_error(MOE_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+    cuuint64_t gd[3], gs[2];
+    cuuint32_t bx[3], es[3] = {1, 1, 1};
+    for (int i = 0; i < rank; ++i) {
+        gd[i] = dims[i];
+        bx[i] = box[i];
+    }
+    for (int i = 0; i < rank - 1; ++i) gs[i] = strides_bytes[i];
+    const CUresult r = fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                          (cuuint32_t)rank, const_cast<void *>(base), gd, gs, bx, es,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return set_error(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return MOE_OK;
+}
+
+template <bool BF16, bool GATHER, bool GLU, bool SCATTER>
+int launch_t(const GemmArgs &a, cudaStream_t s) {
+    constexpr int EB = BF16 ? 2 : 4;
+    constexpr int BK = KBYTES / EB;
+    constexpr int CW = KBYTES / EB;
+    auto kern = grouped_gemm_kernel<BF16, GATHER, GLU, SCATTER>;
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [&] {
+        attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)SMEM_BYTES);
+    });
+    if (attr_err != cudaSuccess)
+        return set_error(MOE_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(attr_err));
+
+    CUtensorMap mA, mB0, mB1;
+    {
+        const uint64_t dims[2] = {(uint64_t)a.K, (uint64_t)a.a_rows};
+        const uint64_t str[1] = {(uint64_t)a.K * EB};
+        const uint32_t box[2] = {(uint32_t)BK, GATHER ? 1u : (uint32_t)BM};
+        int rc = encode(&mA, BF16, 2, a.A, dims, str, box);
+        if (rc) return rc;
+    }
+    {
+        const uint64_t dims[3] = {(uint64_t)a.N, (uint64_t)a.K, (uint64_t)a.E};
+        const uint64_t str[2] = {(uint64_t)a.N * EB, (uint64_t)a.N * a.K * EB};
+        const uint32_t box[3] = {(uint32_t)CW, (uint32_t)BK, 1u};
+        int rc = encode(&mB0, BF16, 3, a.B0, dims, str, box);
+        if (rc) return rc;
+        if (GLU) {
+            rc = encode(&mB1, BF16, 3, a.B1, dims, str, box);
+            if (rc) return rc;
+        } else {
+            mB1 = mB0;
+        }
+    }
+    KParams kp;
+    kp.offsets = a.offsets;
+    kp.sorted_rows = a.sorted_rows;
+    kp.gates = a.gates;
+    kp.out = a.out;
+    kp.E = a.E;
+    kp.k = a.k;
+    kp.N = (int32_t)a.N;
+    kp.num_kb = (int32_t)((a.K * EB + KBYTES - 1) / KBYTES);
+    constexpr int OUT_COLS = GLU ? BN / 2 : BN;
+    kp.n_tiles = (int32_t)((a.N + OUT_COLS - 1) / OUT_COLS);
+    kp.S = a.S;
+    kp.R = a.R;
+    kp.status = a.status;
+    kp.wait_limit_ns = a.wait_limit_ns;
+    kern<<<num_sms(), THREADS, SMEM_BYTES, s>>>(mA, mB0, mB1, kp);
+    return MOE_OK;
+}
+
+}  // namespace
+
+int launch_grouped_gemm(const GemmArgs &a, cudaStream_t s) {
+    // instantiated forms: (gather, glu, scatter) in {(1,1,0), (0,0,1), (1,0,0), (1,0,1),
+    // (0,0,0)} x {bf16, f32}
+#define MOE_DISPATCH(BF, G, L, SC)                                                          \
+    if (a.bf16 == BF && a.gather == G && a.glu == L && a.scatter == SC)                     \
+        return launch_t<BF, G, L, SC>(a, s);
+    MOE_DISPATCH(true, true, true, false)
+    MOE_DISPATCH(true, false, false, true)
+    MOE_DISPATCH(true, true, false, false)
+    MOE_DISPATCH(true, true, false, true)
+    MOE_DISPATCH(true, false, false, false)
+    MOE_DISPATCH(false, true, true, false)
+    MOE_DISPATCH(false, false, false, true)
+    MOE_DISPATCH(false, true, false, false)
+    MOE_DISPATCH(false, true, false, true)
+    MOE_DISPATCH(false, false, false, false)
+#undef MOE_DISPATCH
+    return set_error(MOE_ERR_UNSUPPORTED, "grouped GEMM form not built");
+}
+
+int launch_debug_wait(int64_t limit_ns, unsigned *status, cudaStream_t s) {
+    debug_wait_kernel<<<1, 32, 0, s>>>(limit_ns, status);
+    return MOE_OK;
+}
+
+}  // namespace moe

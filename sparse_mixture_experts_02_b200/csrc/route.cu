@@ -1,0 +1,196 @@
+// Router: logits = x . W_gate (+ bias), top-k in descending order (ties: smaller expert id),
+// softmax over the k selected logits.
+//
+// ScatterMoE guide ("ScatterMoE Guide: Fast Fused Kernels for Sparse MoE LLMs"),
+// "1. The Dynamic Routing Imbalance Dilemma": H(X) = Softmax(TopK(X W_gate, k)).
+//
+// Layout: one warp owns kTokPerWarp tokens; lane l owns experts e = l + 32 j (j < NJ), so the
+// W_gate row loads are coalesced and the logits of a token end up spread over the warp, where the
+// top-k is a k-round warp arg-max. x rows are staged through shared memory (fp32) in chunks of 64
+// columns, read back as float4 broadcasts. Accumulation is fp32 FMA in ascending d.
+#include "moe_internal.cuh"
+
+#include <math.h>
+
+namespace moe {
+namespace {
+
+constexpr int kTokPerWarp = 8;
+constexpr int kWarps = 8;
+constexpr int kChunk = 64;
+
+template <bool BF16>
+__device__ __forceinline__ float ld_elem(const void *p, int64_t i) {
+    if constexpr (BF16) {
+        return __bfloat162float(__ldg(reinterpret_cast<const __nv_bfloat16 *>(p) + i));
+    } else {
+        return __ldg(reinterpret_cast<const float *>(p) + i);
+    }
+}
+
+// (value, index) is better than (v2, i2): larger value, or equal value and smaller index.
+__device__ __forceinline__ bool better(float v, int i, float v2, int i2) {
+    return (v > v2) || (v == v2 && i < i2);
+}
+
+template <int NJ, bool BF16>
+__global__ void __launch_bounds__(kWarps * 32)
+route_kernel(const void *__restrict__ x, const void *__restrict__ w_gate,
+             const float *__restrict__ bias, int64_t S, int64_t D, int32_t E, int32_t k,
+             int32_t *__restrict__ top_e, float *__restrict__ top_w) {
+    __shared__ __align__(16) float xs[kWarps][kTokPerWarp][kChunk];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t tok0 = ((int64_t)blockIdx.x * kWarps + warp) * kTokPerWarp;
+    if (tok0 >= S) return;
+
+    float acc[kTokPerWarp][NJ];
+#pragma unroll
+    for (int t = 0; t < kTokPerWarp; ++t)
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) acc[t][j] = 0.f;
+
+    for (int64_t d0 = 0; d0 < D; d0 += kChunk) {
+        // stage x[tok0 + t][d0 : d0 + 64] as fp32; lane l holds columns 2l, 2l+1
+#pragma unroll
+        for (int t = 0; t < kTokPerWarp; ++t) {
+            const int64_t s = tok0 + t;
+            const int64_t c = d0 + 2 * lane;
+            float a = 0.f, b = 0.f;
+            if (s < S) {
+                if (c < D) a = ld_elem<BF16>(x, s * D + c);
+                if (c + 1 < D) b = ld_elem<BF16>(x, s * D + c + 1);
+            }
+            xs[warp][t][2 * lane] = a;
+            xs[warp][t][2 * lane + 1] = b;
+        }
+        __syncwarp();
+        const int nd = (D - d0 < kChunk) ? (int)(D - d0) : kChunk;
+        for (int d = 0; d < nd; d += 4) {
+            float4 xv[kTokPerWarp];
+#pragma unroll
+            for (int t = 0; t < kTokPerWarp; ++t)
+                xv[t] = *reinterpret_cast<const float4 *>(&xs[warp][t][d]);
+#pragma unroll
+            for (int dd = 0; dd < 4; ++dd) {
+                if (d + dd >= nd) break;
+                const int64_t row = (d0 + d + dd) * (int64_t)E;
+                float w[NJ];
+#pragma unroll
+                for (int j = 0; j < NJ; ++j) {
+                    const int e = lane + 32 * j;
+                    w[j] = (e < E) ? ld_elem<BF16>(w_gate, row + e) : 0.f;
+                }
+#pragma unroll
+                for (int t = 0; t < kTokPerWarp; ++t) {
+                    const float xd = dd == 0 ? xv[t].x : dd == 1 ? xv[t].y : dd == 2 ? xv[t].z
+                                                                                   : xv[t].w;
+#pragma unroll
+                    for (int j = 0; j < NJ; ++j) acc[t][j] = fmaf(xd, w[j], acc[t][j]);
+                }
+            }
+        }
+        __syncwarp();
+    }
+
+    // top-k per token: k rounds of a warp arg-max over the lanes' untaken experts
+#pragma unroll
+    for (int t = 0; t < kTokPerWarp; ++t) {
+        const int64_t s = tok0 + t;
+        if (s >= S) break;
+        float v[NJ];
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) {
+            const int e = lane + 32 * j;
+            float l = acc[t][j];
+            if (e < E && bias != nullptr) l += __ldg(bias + e);
+            if (e >= E || isnan(l)) l = -INFINITY;
+            v[j] = l;
+        }
+        unsigned taken = 0;
+        float sel_v[8];
+        int sel_i[8];
+        for (int r = 0; r < k; ++r) {
+            float bv = -INFINITY;
+            int bi = 0x7fffffff;
+#pragma unroll
+            for (int j = 0; j < NJ; ++j) {
+                const int e = lane + 32 * j;
+                if (e < E && !(taken & (1u << j)) && better(v[j], e, bv, bi)) {
+                    bv = v[j];
+                    bi = e;
+                }
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+                const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+                if (better(ov, oi, bv, bi)) {
+                    bv = ov;
+                    bi = oi;
+                }
+            }
+            if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+            sel_v[r] = bv;
+            sel_i[r] = bi;
+        }
+        if (lane == 0) {
+            const float m = sel_v[0];
+            float den = 0.f;
+            for (int r = 0; r < k; ++r) den += expf(sel_v[r] - m);
+            for (int r = 0; r < k; ++r) {
+                top_e[s * k + r] = sel_i[r];
+                top_w[s * k + r] = expf(sel_v[r] - m) / den;
+            }
+        }
+    }
+}
+
+__global__ void zero_kernel(float4 *__restrict__ p, int64_t n4, float *__restrict__ tail,
+                            int tail_n, unsigned *status) {
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += stride)
+        p[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (blockIdx.x == 0 && threadIdx.x < tail_n) tail[threadIdx.x] = 0.f;
+    if (blockIdx.x == 0 && threadIdx.x == 0 && status != nullptr) *status = 0u;
+}
+
+template <int NJ>
+int launch_route_nj(const void *x, const void *w_gate, const float *bias, int64_t S, int64_t D,
+                    int32_t E, int32_t k, bool bf16, int32_t *top_e, float *top_w,
+                    cudaStream_t s) {
+    const int64_t per_block = (int64_t)kWarps * kTokPerWarp;
+    const int64_t blocks = (S + per_block - 1) / per_block;
+    if (blocks == 0) return 0;
+    if (bf16)
+        route_kernel<NJ, true><<<(unsigned)blocks, kWarps * 32, 0, s>>>(x, w_gate, bias, S, D, E,
+                                                                        k, top_e, top_w);
+    else
+        route_kernel<NJ, false><<<(unsigned)blocks, kWarps * 32, 0, s>>>(x, w_gate, bias, S, D,
+                                                                         E, k, top_e, top_w);
+    return 1;
+}
+
+}  // namespace
+
+int launch_route(const void *x, const void *w_gate, const float *bias, int64_t S, int64_t D,
+                 int32_t E, int32_t k, bool bf16, int32_t *top_e, float *top_w, cudaStream_t s) {
+    if (E <= 32) return launch_route_nj<1>(x, w_gate, bias, S, D, E, k, bf16, top_e, top_w, s);
+    if (E <= 64) return launch_route_nj<2>(x, w_gate, bias, S, D, E, k, bf16, top_e, top_w, s);
+    if (E <= 128) return launch_route_nj<4>(x, w_gate, bias, S, D, E, k, bf16, top_e, top_w, s);
+    return launch_route_nj<8>(x, w_gate, bias, S, D, E, k, bf16, top_e, top_w, s);
+}
+
+int launch_zero_f32(float *p, int64_t n, unsigned *status, cudaStream_t s) {
+    // p is 16-byte aligned (checked by the caller); n4 float4 stores plus a < 4 element tail
+    const int64_t n4 = n / 4;
+    const int tail = (int)(n - n4 * 4);
+    int64_t blocks = (n4 + 255) / 256;
+    const int64_t cap = (int64_t)num_sms() * 8;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    zero_kernel<<<(unsigned)blocks, 256, 0, s>>>(reinterpret_cast<float4 *>(p), n4, p + n4 * 4,
+                                                  tail, status);
+    return 1;
+}
+
+}  // namespace moe

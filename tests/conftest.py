@@ -25,3 +25,19 @@ def oracle_lib():
     import oracle
     oracle.lib()
     return oracle
+
+
+def pytest_collection_modifyitems(config, items):
+    if gpu_available():
+        return
+    skip = pytest.mark.skip(reason="no CUDA device in this process")
+    for item in items:
+        if "gpu" in item.keywords:
+            item.add_marker(skip)
+
+
+@pytest.fixture(scope="session")
+def moe():
+    """The CUDA library binding; on a GPU machine a missing library is an error, never a skip."""
+    import sparse_mixture_experts_02_b200 as m
+    return m

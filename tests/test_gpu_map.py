@@ -1,0 +1,105 @@
+"""Sparse map on the GPU against the oracle's counting sort: bit-exact on every output, plus the
+invariants of "4. Correctness Validation" in "Add scalable sparse map kernel for large MoE models
+(128+ experts)" (unique rows, rows inside their expert's range, histogram counts, non-overlapping
+ranges, deterministic across runs), over that page's expert-count grid and the route counts of
+every workload."""
+import numpy as np
+import pytest
+import torch
+
+import moe_workloads as W
+from test_oracle_pins import check_map_invariants
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(moe, te_cpu, E):
+    te = te_cpu.to("cuda")
+    out = moe.sparse_map(te, E)
+    torch.cuda.synchronize()
+    return [o.cpu().numpy() for o in out]
+
+
+def _compare(oracle_lib, moe, te_cpu, E):
+    got = _run(moe, te_cpu, E)
+    ref = oracle_lib.sparse_map(te_cpu.numpy(), E)
+    for name, a, b in zip(("counts", "offsets", "sparse_rows", "sorted_rows"), got, ref):
+        assert np.array_equal(a, b), f"{name} differs at {np.nonzero(a != b)[0][:10]}"
+    check_map_invariants(te_cpu.numpy(), E, *got)
+    return got
+
+
+@pytest.mark.parametrize("E", [4, 8, 16, 32, 64, 96, 128, 256])
+@pytest.mark.parametrize("mode", ["uniform", "zipf"])
+def test_map_expert_grid(oracle_lib, moe, E, mode):
+    k = min(4, E)
+    te = W.make_top_experts(3001, k, E, seed=E + 7, mode=mode)
+    _compare(oracle_lib, moe, te, E)
+
+
+@pytest.mark.parametrize("name", list(W.WORKLOADS))
+def test_map_workload_sizes(oracle_lib, moe, name):
+    w = W.WORKLOADS[name]
+    mode = "zipf" if w.zipf_s > 0 else "uniform"
+    te = W.make_top_experts(w.S, w.k, w.E, seed=1, mode=mode)
+    _compare(oracle_lib, moe, te, w.E)
+
+
+def test_map_deterministic(oracle_lib, moe):
+    te = W.make_top_experts(40000, 6, 64, seed=3, mode="zipf")
+    first = _compare(oracle_lib, moe, te, 64)
+    for _ in range(3):
+        again = _run(moe, te, 64)
+        for a, b in zip(first, again):
+            assert np.array_equal(a, b)
+
+
+@pytest.mark.parametrize("S,k,E", [(1, 1, 1), (1, 3, 7), (511, 1, 5), (512, 1, 5), (513, 1, 5),
+                                   (70000, 2, 3)])
+def test_map_edges(oracle_lib, moe, S, k, E):
+    te = W.make_top_experts(S, k, E, seed=S, mode="any")
+    _compare(oracle_lib, moe, te, E)
+
+
+def test_map_all_one_expert_and_empty(oracle_lib, moe):
+    te = W.make_top_experts(5000, 4, 32, mode="one")
+    counts, offsets, _, _ = _compare(oracle_lib, moe, te, 32)
+    assert counts[0] == 20000 and counts[1:].sum() == 0
+    # S = 0: counts and offsets all zero
+    got = _run(moe, torch.zeros((0, 2), dtype=torch.int32), 6)
+    assert got[0].tolist() == [0] * 6 and got[1].tolist() == [0] * 7
+
+
+def test_map_large_route_count(oracle_lib, moe):
+    te = W.make_top_experts(1 << 18, 8, 256, seed=9, mode="zipf")  # 2^21 routes
+    _compare(oracle_lib, moe, te, 256)
+
+
+def test_map_bad_expert_id_is_reported(moe):
+    te = W.make_top_experts(100, 2, 8, seed=2).clone()
+    te[17, 1] = 8
+    te[50, 0] = -3
+    tg = te.to("cuda")
+    need = moe.workspace_size("sparse_map", 100, 0, 0, 8, 2, 1)
+    ws = moe.alloc_workspace(need, tg.device)
+    counts = torch.empty(8, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(9, dtype=torch.int32, device="cuda")
+    sp = torch.empty(200, dtype=torch.int32, device="cuda")
+    so = torch.empty(200, dtype=torch.int32, device="cuda")
+    import ctypes
+    rc = moe.lib.moe_sparse_map(ctypes.c_void_p(tg.data_ptr()), 100, 2, 8,
+                                ctypes.c_void_p(counts.data_ptr()),
+                                ctypes.c_void_p(offsets.data_ptr()), ctypes.c_void_p(sp.data_ptr()),
+                                ctypes.c_void_p(so.data_ptr()), ctypes.c_void_p(ws.data_ptr()),
+                                ws.numel(), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert rc == 0
+    with pytest.raises(moe.MoeError) as ei:
+        moe.check_device_status(ws)
+    assert ei.value.code == -5
+    # the valid routes are still mapped, the bad ones get -1
+    spn = sp.cpu().numpy()
+    assert spn[17 * 2 + 1] == -1 and spn[50 * 2] == -1
+    assert counts.sum().item() == 198
+    # the status clears on the next call
+    moe.sparse_map(W.make_top_experts(100, 2, 8, seed=2).to("cuda"), 8, ws=ws)
+    moe.check_device_status(ws)

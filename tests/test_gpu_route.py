@@ -1,0 +1,69 @@
+"""Router on the GPU against the oracle: top-k experts equal except at justified near-ties (the
+fp32 rounding bound on the oracle's fp64 logits), weights within fp32 rounding of the oracle's
+softmax over the GPU's own choice.
+
+Source: "ScatterMoE Guide: Fast Fused Kernels for Sparse MoE LLMs", "1. The Dynamic Routing
+Imbalance Dilemma" (H(X) = Softmax(TopK(X W_gate, k))).
+"""
+import numpy as np
+import pytest
+import torch
+
+import moe_workloads as W
+from parity import check_routing
+
+pytestmark = pytest.mark.gpu
+
+
+def _route_and_check(oracle_lib, moe, inp, k, tokens=None, max_diff_frac=0.01):
+    x, wg, bias = inp["x"], inp["w_gate"], inp["logit_bias"]
+    S, D = x.shape
+    te, tw = moe.route_topk(x.cuda(), wg.cuda(), k, None if bias is None else bias.cuda())
+    torch.cuda.synchronize()
+    te, tw = te.cpu().numpy(), tw.cpu().numpy()
+    if tokens is None:
+        tokens = np.arange(S, dtype=np.int32)
+    logits, absdot = oracle_lib.router_logits(x, wg, bias, tokens=tokens)
+    ote, otw = oracle_lib.topk_softmax(logits, k)
+    diff = check_routing(te[tokens], ote, logits, absdot, D)
+    assert diff <= max(1, int(max_diff_frac * len(tokens)))
+    # weights: the oracle's softmax over the GPU's experts, in the GPU's order
+    ow = oracle_lib.weights_for(logits, te[tokens])
+    assert np.max(np.abs(tw[tokens] - ow)) < 1e-5
+    assert np.allclose(tw.sum(axis=1), 1.0, atol=2e-6)
+    assert np.all(np.diff(tw, axis=1) <= 1e-7)
+    return te, tw
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("E,k", [(1, 1), (5, 2), (8, 2), (32, 8), (33, 3), (64, 6), (96, 4),
+                                 (128, 4), (200, 8), (256, 8)])
+def test_route_small(oracle_lib, moe, dtype, E, k):
+    w = W.custom("r", S=300, D=136, F=8, E=E, k=k, dtype=dtype, router_std="1/sqrt(D)")
+    _route_and_check(oracle_lib, moe, W.make_inputs(w, seed=E * 31 + k), k)
+
+
+def test_route_bias_zipf(oracle_lib, moe):
+    w = W.custom("z", S=2000, D=256, F=8, E=64, k=6, router_std="1/sqrt(D)", zipf_s=1.2)
+    te, _ = _route_and_check(oracle_lib, moe, W.make_inputs(w), 6)
+    counts = np.bincount(te.reshape(-1), minlength=64)
+    assert counts.max() > 4 * counts.mean()   # the bias produces the skew
+
+
+def test_route_exact_ties_pick_lower_id(moe):
+    # x = 0: every logit is 0 (a tie everywhere), so the experts are 0..k-1 with weight 1/k
+    x = torch.zeros(70, 64, dtype=torch.bfloat16, device="cuda")
+    wg = torch.randn(64, 12, device="cuda").to(torch.bfloat16)
+    te, tw = moe.route_topk(x, wg, 3)
+    assert torch.equal(te.cpu(), torch.tensor([[0, 1, 2]] * 70, dtype=torch.int32))
+    assert torch.allclose(tw.cpu(), torch.full((70, 3), 1 / 3))
+
+
+@pytest.mark.parametrize("name", ["mixtral_prefill", "e128", "zipf64"])
+def test_route_full_workloads(oracle_lib, moe, name):
+    w = W.WORKLOADS[name]
+    inp = W.make_inputs(w, device="cuda")
+    cpu = {k: (v.cpu() if v is not None else None) for k, v in inp.items()
+           if k in ("x", "w_gate", "logit_bias")}
+    toks = np.random.default_rng(0).choice(w.S, size=2048, replace=False).astype(np.int32)
+    _route_and_check(oracle_lib, moe, cpu, w.k, tokens=np.sort(toks))
