@@ -347,7 +347,8 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="mixtral_prefill", choices=list(W.WORKLOADS))
+    ap.add_argument("--workload", default="mixtral_prefill",
+                    choices=list(W.WORKLOADS) + list(W.PROFILE_WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
@@ -355,7 +356,7 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    w = W.WORKLOADS[args.workload]
+    w = {**W.WORKLOADS, **W.PROFILE_WORKLOADS}[args.workload]
     if args.impl == "reference":
         # the oracle runs on rank 0's host cores only; other ranks have nothing to do
         ws = int(os.environ.get("WORLD_SIZE", "1"))

@@ -62,6 +62,13 @@ WORKLOADS = {
                        router_std="1/sqrt(D)", zipf_s=1.2),
 }
 
+# A smaller prefill-shaped case for detailed profiler captures (1.4 GB of weights, 4 M tiles per
+# expert): same kernels and regime as the Mixtral prefill layer, a fraction of its size.
+PROFILE_WORKLOADS = {
+    "prefill_profile": Workload("prefill_profile", S=2048, D=4096, F=7168, E=8, k=2,
+                                dtype="bf16", router_std="0.02"),
+}
+
 
 def custom(name, S, D, F, E, k, dtype="bf16", router_std="0.02", zipf_s=0.0) -> Workload:
     return Workload(name, S=S, D=D, F=F, E=E, k=k, dtype=dtype, router_std=router_std,

@@ -196,15 +196,20 @@ int moe_route_topk(const void *x, const void *w_gate, const float *logit_bias, i
     int rc;
     if ((rc = check_dtype(dt)) || (rc = check_dims(S, E, k)) || (rc = check_feat("D", D))) return rc;
     const size_t eb = esize(dt);
-    if ((rc = check_ptr("x", x, eb)) || (rc = check_ptr("w_gate", w_gate, eb)) ||
+    (void)eb;
+    if ((rc = check_ptr("x", x, 16)) || (rc = check_ptr("w_gate", w_gate, 16)) ||
         (rc = check_ptr("logit_bias", logit_bias, 4, true)) ||
         (rc = check_ptr("top_experts", top_experts, 4)) ||
         (rc = check_ptr("top_weights", top_weights, 4)))
         return rc;
     if ((rc = check_device())) return rc;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    g_launches += launch_route(x, w_gate, logit_bias, S, D, E, k, dt == MOE_BF16, top_experts,
-                               top_weights, s);
+    // no workspace in this call: a device-side wait timeout of the tensor-core router is not
+    // reported here (moe_mlp_forward reports it through its workspace)
+    const int n = launch_route(x, w_gate, logit_bias, S, D, E, k, dt == MOE_BF16, top_experts,
+                               top_weights, nullptr, s);
+    if (n < 0) return MOE_ERR_CUDA;
+    g_launches = n;
     return check_launch("route");
 }
 
@@ -315,7 +320,12 @@ int moe_mlp_forward(const void *x, const void *w_gate, const float *logit_bias,
     record_prof(0, s);
     n += launch_zero_f32(out, S * D, status, s);
     if ((rc = check_launch("zero"))) return rc;
-    n += launch_route(x, w_gate, logit_bias, S, D, E, k, dt == MOE_BF16, top_e, top_w, s);
+    {
+        const int nr = launch_route(x, w_gate, logit_bias, S, D, E, k, dt == MOE_BF16, top_e,
+                                    top_w, status, s);
+        if (nr < 0) return MOE_ERR_CUDA;
+        n += nr;
+    }
     if ((rc = check_launch("route"))) return rc;
     record_prof(1, s);
     launch_sparse_map(top_e, R, E, counts, offsets, sparse_rows, sorted_rows,

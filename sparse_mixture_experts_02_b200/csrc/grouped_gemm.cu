@@ -17,9 +17,13 @@
 // expert id follows "Inside the Flash-MoE Kernel: Fused Tile-Level Dispatch".
 //
 // Design (B200): persistent, one CTA per SM, 6 warps:
-//   warp 0      TMA producer. B tiles by 3-D tensor map (N, K, expert). A tiles either by a
-//               2-D box (contiguous rows) or, for gathered rows, by tile::gather4: each of the
-//               32 lanes fetches 4 token rows, so one stage's 128 rows need no [S*k, D] copy.
+//   warp 0      TMA producer: B tiles by 3-D tensor map (N, K, expert); contiguous A tiles
+//               (slot-ordered rows) by a 2-D box.
+//   warps 6-9   (gathered A only) row gatherers: 128 threads copy the stage's 128 token rows
+//               (row = x[sorted_rows[p] / k]) with 16-byte cp.async straight into the 128-byte
+//               swizzled layout, so no [S*k, D] copy of x ever exists. (TMA tile::gather4 was
+//               measured at ~7x the cost per row of a box load here, leaving the tensor pipe
+//               80% idle; the LSU path keeps the gather off the TMA unit.)
 //   warp 1      TMEM owner (512 columns = two 128 x 256 fp32 accumulators) and MMA issuer
 //               (one thread): 4 x tcgen05.mma (M=128, N=256, K=32 bytes) per 128-byte K stage.
 //   warps 2-5   epilogue: tcgen05.ld of the accumulator (thread = tile row), then SwiGLU + bf16
@@ -45,7 +49,8 @@ constexpr int A_BYTES = BM * KBYTES;    // 16 KB
 constexpr int B_BYTES = BN * KBYTES;    // 32 KB (BN columns x (128 / eb) K rows x eb)
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int MAX_E = 256;
-constexpr int THREADS = 192;
+constexpr int THREADS = 192;            // producer, MMA, 4 epilogue warps
+constexpr int GATHER_THREADS = 128;     // extra warps 6-9 for gathered A
 constexpr uint32_t TMEM_COLS = 512;
 
 struct SmemTail {
@@ -62,6 +67,8 @@ struct SmemTail {
 constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + sizeof(SmemTail);
 
 struct KParams {
+    const void *A;    // gathered mode: x [S, K] (rows fetched by the gather warps)
+    int64_t K;
     const int32_t *offsets;
     const int32_t *sorted_rows;
     const float *gates;
@@ -71,6 +78,11 @@ struct KParams {
     int32_t num_kb;   // K stages
     int32_t n_tiles;  // N tiles
     int64_t S, R;     // bounds of scatter rows (tokens) and grouped rows (slots)
+    // router mode: logit bias [E] (nullable), outputs [S, k]
+    const float *bias;
+    int32_t *top_e;
+    float *top_w;
+    int32_t b_chunks; // B chunks loaded per stage (router: ceil(E / chunk width))
     unsigned *status;
     int64_t wait_limit_ns;
 };
@@ -101,8 +113,8 @@ __device__ __forceinline__ TileInfo decode_tile(int t, const SmemTail &st, int E
 
 __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + __expf(-z)); }
 
-template <bool BF16, bool GATHER, bool GLU, bool SCATTER>
-__global__ void __launch_bounds__(THREADS, 1)
+template <bool BF16, bool GATHER, bool GLU, bool SCATTER, bool ROUTER>
+__global__ void __launch_bounds__(GATHER ? THREADS + GATHER_THREADS : THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     const __grid_constant__ CUtensorMap tmB0,
                     const __grid_constant__ CUtensorMap tmB1, const KParams p) {
@@ -114,6 +126,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     constexpr int B_KSTEP = (32 / EB) * KBYTES;  // bytes of B per MMA K step (32 bytes of K)
     constexpr int OUT_COLS = GLU ? BN / 2 : BN;  // output columns per tile
     constexpr uint32_t IDESC = dev::idesc_f32acc(BF16, BM, BN, true);
+    // B (weights, N contiguous) is MN-major: 128-byte swizzle for bf16 (8-row atoms of 1024 B);
+    // tf32 needs the 32-byte-unit variant (4-row atoms of 512 B).
+    constexpr uint32_t B_LAYOUT = BF16 ? dev::kLayoutSw128 : dev::kLayoutSw128Base32;
+    constexpr uint32_t B_SBO = BF16 ? 1024 : 512;
     static_assert(NCH * CHUNK == B_BYTES, "B stage size");
 
     extern __shared__ uint8_t smem_raw[];
@@ -126,7 +142,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            dev::mbar_init(&st.full[s], 1);
+            // full: the TMA thread's expect_tx arrival (+ one cp.async arrival per gatherer)
+            dev::mbar_init(&st.full[s], GATHER ? 1 + GATHER_THREADS : 1);
             dev::mbar_init(&st.empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -147,21 +164,36 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         dev::tmem_relinquish();
         dev::tc_fence_before();
     }
-    for (int e = threadIdx.x; e <= E; e += THREADS) st.off[e] = __ldg(p.offsets + e);
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        int run = 0;
-        for (int e = 0; e < E; ++e) {
-            st.tstart[e] = run;
-            const int mt = (st.off[e + 1] - st.off[e] + BM - 1) / BM;
-            run += mt * p.n_tiles;
+    if constexpr (ROUTER) {
+        // one "expert" holding all S rows: tiles are the 128-token blocks of x
+        if (threadIdx.x == 0) {
+            st.off[0] = 0;
+            st.off[1] = (int32_t)p.S;
+            st.tstart[0] = 0;
+            st.tstart[1] = (int32_t)((p.S + BM - 1) / BM);
         }
-        st.tstart[E] = run;
+        __syncthreads();
+    } else {
+        for (int e = threadIdx.x; e <= E; e += blockDim.x) st.off[e] = __ldg(p.offsets + e);
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            int run = 0;
+            for (int e = 0; e < E; ++e) {
+                st.tstart[e] = run;
+                const int mt = (st.off[e + 1] - st.off[e] + BM - 1) / BM;
+                run += mt * p.n_tiles;
+            }
+            st.tstart[E] = run;
+        }
+        __syncthreads();
     }
-    __syncthreads();
     dev::tc_fence_after();
     const uint32_t tmem_base = st.tmem_base;
-    const int total = st.tstart[E];
+    const int E_sched = ROUTER ? 1 : E;
+    const int total = st.tstart[E_sched];
+    const int nch = ROUTER ? p.b_chunks : NCH;
+    const uint32_t stage_tx = (uint32_t)((GATHER ? 0 : A_BYTES) + nch * CHUNK);
+    const uint32_t idesc = ROUTER ? dev::idesc_f32acc(BF16, BM, (uint32_t)(nch * CW), true) : IDESC;
     volatile int *abort = &st.abort;
 
     if (warp == 0) {
@@ -170,16 +202,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         uint32_t issued = 0, last_par = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-            const TileInfo ti = decode_tile(t, st, E, p.n_tiles);
-            int32_t rr[4] = {0, 0, 0, 0};
-            if (GATHER) {
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int r = lane * 4 + j;
-                    const int pr = ti.row_begin + min(r, ti.rows - 1);
-                    rr[j] = __ldg(p.sorted_rows + pr) / p.k;
-                }
-            }
+            const TileInfo ti = decode_tile(t, st, E_sched, p.n_tiles);
             const int n0 = ti.n_idx * OUT_COLS;
             for (int kb = 0; kb < p.num_kb; ++kb) {
                 bool w = true;
@@ -193,18 +216,14 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                 }
                 uint8_t *sA = smem + (size_t)s * STAGE_BYTES;
                 uint8_t *sB = sA + A_BYTES;
-                if (lane == 0) dev::mbar_arrive_expect_tx(&st.full[s], STAGE_BYTES);
+                if (lane == 0) dev::mbar_arrive_expect_tx(&st.full[s], stage_tx);
                 __syncwarp();
                 const int kc = kb * BK;
-                if (GATHER) {
-                    dev::tma_gather4(sA + lane * 4 * KBYTES, &tmA, &st.full[s], kc, rr[0], rr[1],
-                                     rr[2], rr[3]);
-                } else if (lane == 0) {
-                    dev::tma_load_2d(sA, &tmA, &st.full[s], kc, ti.row_begin);
-                }
+                if (!GATHER && lane == 0) dev::tma_load_2d(sA, &tmA, &st.full[s], kc, ti.row_begin);
                 if (lane == 0) {
 #pragma unroll
                     for (int c = 0; c < NCH; ++c) {
+                        if (c >= nch) break;
                         if (GLU) {
                             const int half = NCH / 2;
                             const CUtensorMap *m = c < half ? &tmB0 : &tmB1;
@@ -252,14 +271,16 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         break;
                     }
                     dev::tc_fence_after();
+                    if (GATHER) dev::fence_proxy_async_smem();  // cp.async rows -> tensor core
                     const uint32_t sA = dev::smem_u32(smem + (size_t)s * STAGE_BYTES);
                     const uint32_t sB = sA + A_BYTES;
 #pragma unroll
                     for (int kk = 0; kk < KBYTES / 32; ++kk) {
-                        const uint64_t ad = dev::sdesc_sw128(sA + kk * 32, 16, 1024);
-                        const uint64_t bd = dev::sdesc_sw128(sB + kk * B_KSTEP, CHUNK, 1024);
-                        if (BF16) dev::mma_bf16(d_tmem, ad, bd, IDESC, (kb | kk) != 0);
-                        else dev::mma_tf32(d_tmem, ad, bd, IDESC, (kb | kk) != 0);
+                        const uint64_t ad =
+                            dev::sdesc(sA + kk * 32, 16, 1024, dev::kLayoutSw128);
+                        const uint64_t bd = dev::sdesc(sB + kk * B_KSTEP, CHUNK, B_SBO, B_LAYOUT);
+                        if (BF16) dev::mma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0);
+                        else dev::mma_tf32(d_tmem, ad, bd, idesc, (kb | kk) != 0);
                     }
                     dev::mma_commit(&st.empty[s]);
                     if (++s == STAGES) {
@@ -276,13 +297,61 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             dev::tc_fence_before();
         }
         __syncwarp();
+    } else if (GATHER && warp >= THREADS / 32) {
+        // ------------------------------------------------------------------ row gatherers
+        // thread -> 8 rows of the 128-row stage (rows gw*32 + 4i + lane/8) and one 16-byte chunk
+        // (lane % 8) of each row's 128 bytes, so a warp instruction covers 4 whole rows.
+        const int gw = warp - THREADS / 32;
+        const int chunk = lane & 7;
+        const int rsub = lane >> 3;
+        const int64_t row_bytes = (int64_t)p.K * EB;
+        const uint8_t *xa = reinterpret_cast<const uint8_t *>(p.A);
+        uint32_t s = 0, ph = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+            const TileInfo ti = decode_tile(t, st, E_sched, p.n_tiles);
+            const uint8_t *src[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int r = gw * 32 + i * 4 + rsub;
+                const int pr = ti.row_begin + min(r, ti.rows - 1);  // tail rows repeat a valid row
+                const int64_t tok = __ldg(p.sorted_rows + pr) / p.k;
+                src[i] = xa + tok * row_bytes;
+            }
+            for (int kb = 0; kb < p.num_kb; ++kb) {
+                bool w = true;
+                if (lane == 0)
+                    w = dev::mbar_wait(&st.empty[s], ph ^ 1u, abort, p.status, p.wait_limit_ns,
+                                       kKernelGemm);
+                w = __shfl_sync(0xffffffffu, w, 0);
+                if (!w) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t sA = dev::smem_u32(smem + (size_t)s * STAGE_BYTES);
+                const int64_t cb = (int64_t)kb * KBYTES + chunk * 16;
+                const uint32_t nbytes = cb < row_bytes ? 16u : 0u;  // zero-fill past K
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int r = gw * 32 + i * 4 + rsub;
+                    const uint32_t dst = sA + r * KBYTES + ((chunk ^ (r & 7)) << 4);
+                    dev::cp_async16(dst, nbytes ? src[i] + cb : src[i], nbytes);
+                }
+                dev::cp_async_arrive_noinc(&st.full[s]);
+                if (++s == STAGES) {
+                    s = 0;
+                    ph ^= 1u;
+                }
+            }
+        }
+        dev::cp_async_wait_all();
     } else {
         // ------------------------------------------------------------------ epilogue
         const int q = warp & 3;  // TMEM lane quarter this warp may access
         const int r = q * 32 + lane;
         int it = 0;
         for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
-            const TileInfo ti = decode_tile(t, st, E, p.n_tiles);
+            const TileInfo ti = decode_tile(t, st, E_sched, p.n_tiles);
             const uint32_t b = it & 1, aph = (it >> 1) & 1;
             bool w = true;
             if (lane == 0)
@@ -304,7 +373,56 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             }
             const int n0 = ti.n_idx * OUT_COLS;
             const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + b * BN;
-            if (GLU) {
+            if constexpr (ROUTER) {
+                // thread = token row: running top-8 of (logit + bias) over the E columns, in
+                // increasing expert order; ties keep the smaller expert id first
+                float tv[8];
+                int tix[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    tv[j] = -INFINITY;
+                    tix[j] = 0x7fffffff;
+                }
+                for (int c = 0; c * 32 < E; ++c) {
+                    uint32_t av[32];
+                    dev::tmem_ld32(tbase + c * 32, av);
+                    dev::tmem_ld_wait();
+#pragma unroll 4
+                    for (int j = 0; j < 32; ++j) {
+                        int e = c * 32 + j;
+                        if (e >= E) break;
+                        float v = __uint_as_float(av[j]);
+                        if (p.bias != nullptr) v += __ldg(p.bias + e);
+                        if (isnan(v)) v = -INFINITY;
+#pragma unroll
+                        for (int q2 = 0; q2 < 8; ++q2) {
+                            if (v > tv[q2] || (v == tv[q2] && e < tix[q2])) {
+                                const float tf = tv[q2];
+                                const int ti2 = tix[q2];
+                                tv[q2] = v;
+                                tix[q2] = e;
+                                v = tf;
+                                e = ti2;
+                            }
+                        }
+                    }
+                }
+                if (r < ti.rows) {
+                    const int64_t srow = ti.row_begin + r;
+                    const float m = tv[0];
+                    float den = 0.f;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        if (j < p.k) den += expf(tv[j] - m);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        if (j < p.k) {
+                            p.top_e[srow * p.k + j] = tix[j];
+                            p.top_w[srow * p.k + j] = expf(tv[j] - m) / den;
+                        }
+                    }
+                }
+            } else if (GLU) {
 #pragma unroll 1
                 for (int c = 0; c < OUT_COLS / 32; ++c) {
                     uint32_t gv[32], uv[32];
@@ -440,7 +558,8 @@ EncodeTiledFn get_encode() {
 }
 
 int encode(CUtensorMap *m, bool bf16, int rank, const void *base, const uint64_t *dims,
-           const uint64_t *strides_bytes, const uint32_t *box) {
+           const uint64_t *strides_bytes, const uint32_t *box,
+           CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
     EncodeTiledFn fn = get_encode();
     if (!fn) return set_error(MOE_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
     cuuint64_t gd[3], gs[2];
@@ -452,18 +571,18 @@ int encode(CUtensorMap *m, bool bf16, int rank, const void *base, const uint64_t
     for (int i = 0; i < rank - 1; ++i) gs[i] = strides_bytes[i];
     const CUresult r = fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
                           (cuuint32_t)rank, const_cast<void *>(base), gd, gs, bx, es,
-                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return set_error(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
     return MOE_OK;
 }
 
-template <bool BF16, bool GATHER, bool GLU, bool SCATTER>
+template <bool BF16, bool GATHER, bool GLU, bool SCATTER, bool ROUTER = false>
 int launch_t(const GemmArgs &a, cudaStream_t s) {
     constexpr int EB = BF16 ? 2 : 4;
     constexpr int BK = KBYTES / EB;
     constexpr int CW = KBYTES / EB;
-    auto kern = grouped_gemm_kernel<BF16, GATHER, GLU, SCATTER>;
+    auto kern = grouped_gemm_kernel<BF16, GATHER, GLU, SCATTER, ROUTER>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [&] {
@@ -482,19 +601,23 @@ int launch_t(const GemmArgs &a, cudaStream_t s) {
         if (rc) return rc;
     }
     {
-        const uint64_t dims[3] = {(uint64_t)a.N, (uint64_t)a.K, (uint64_t)a.E};
+        const uint64_t dims[3] = {(uint64_t)a.N, (uint64_t)a.K, ROUTER ? 1u : (uint64_t)a.E};
         const uint64_t str[2] = {(uint64_t)a.N * EB, (uint64_t)a.N * a.K * EB};
         const uint32_t box[3] = {(uint32_t)CW, (uint32_t)BK, 1u};
-        int rc = encode(&mB0, BF16, 3, a.B0, dims, str, box);
+        const CUtensorMapSwizzle swz =
+            BF16 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B;
+        int rc = encode(&mB0, BF16, 3, a.B0, dims, str, box, swz);
         if (rc) return rc;
         if (GLU) {
-            rc = encode(&mB1, BF16, 3, a.B1, dims, str, box);
+            rc = encode(&mB1, BF16, 3, a.B1, dims, str, box, swz);
             if (rc) return rc;
         } else {
             mB1 = mB0;
         }
     }
     KParams kp;
+    kp.A = a.A;
+    kp.K = a.K;
     kp.offsets = a.offsets;
     kp.sorted_rows = a.sorted_rows;
     kp.gates = a.gates;
@@ -507,9 +630,14 @@ int launch_t(const GemmArgs &a, cudaStream_t s) {
     kp.n_tiles = (int32_t)((a.N + OUT_COLS - 1) / OUT_COLS);
     kp.S = a.S;
     kp.R = a.R;
+    kp.bias = a.bias;
+    kp.top_e = a.top_e;
+    kp.top_w = a.top_w;
+    kp.b_chunks = (int32_t)((a.N + CW - 1) / CW);
     kp.status = a.status;
     kp.wait_limit_ns = a.wait_limit_ns;
-    kern<<<num_sms(), THREADS, SMEM_BYTES, s>>>(mA, mB0, mB1, kp);
+    kern<<<num_sms(), GATHER ? THREADS + GATHER_THREADS : THREADS, SMEM_BYTES, s>>>(mA, mB0, mB1,
+                                                                                  kp);
     return MOE_OK;
 }
 
@@ -533,6 +661,30 @@ int launch_grouped_gemm(const GemmArgs &a, cudaStream_t s) {
     MOE_DISPATCH(false, false, false, false)
 #undef MOE_DISPATCH
     return set_error(MOE_ERR_UNSUPPORTED, "grouped GEMM form not built");
+}
+
+int launch_route_tc(const void *x, const void *w_gate, const float *bias, int64_t S, int64_t D,
+                    int32_t E, int32_t k, int32_t *top_e, float *top_w, unsigned *status,
+                    cudaStream_t s) {
+    GemmArgs a{};
+    a.A = x;
+    a.a_rows = S;
+    a.B0 = w_gate;  // [D, E] viewed as one expert of a [1, K=D, N=E] weight
+    a.B1 = nullptr;
+    a.S = S;
+    a.R = S;
+    a.E = E;
+    a.k = k;
+    a.K = D;
+    a.N = E;
+    a.bf16 = true;
+    a.bias = bias;
+    a.top_e = top_e;
+    a.top_w = top_w;
+    a.status = status;
+    a.wait_limit_ns = kWaitLimitNs;
+    // the B map spans one "expert" of [D, E]
+    return launch_t<true, false, false, false, true>(a, s);
 }
 
 int launch_debug_wait(int64_t limit_ns, unsigned *status, cudaStream_t s) {

@@ -31,8 +31,10 @@ constexpr int64_t kDrainLimitNs = 1000000000LL;
 
 // ---- host-side launchers (defined in the .cu files) -----------------------------------------
 int launch_zero_f32(float *p, int64_t n, unsigned *status, cudaStream_t s);
+// Returns the number of kernels launched (0 or 1), or -1 after set_error.
 int launch_route(const void *x, const void *w_gate, const float *bias, int64_t S, int64_t D,
-                 int32_t E, int32_t k, bool bf16, int32_t *top_e, float *top_w, cudaStream_t s);
+                 int32_t E, int32_t k, bool bf16, int32_t *top_e, float *top_w, unsigned *status,
+                 cudaStream_t s);
 size_t map_scratch_bytes(int64_t R, int32_t E);
 int launch_sparse_map(const int32_t *top_e, int64_t R, int32_t E, int32_t *counts,
                       int32_t *offsets, int32_t *sparse_rows, int32_t *sorted_rows,
@@ -51,11 +53,19 @@ struct GemmArgs {
     int32_t E, k;
     int64_t K, N;
     bool bf16, gather, glu, scatter;
+    const float *bias;      // router mode only
+    int32_t *top_e;
+    float *top_w;
     unsigned *status;
     int64_t wait_limit_ns;
 };
 int launch_grouped_gemm(const GemmArgs &a, cudaStream_t s);
 int launch_debug_wait(int64_t limit_ns, unsigned *status, cudaStream_t s);
+// Router on the tensor cores (bf16, E % 8 == 0): logits of 128-token tiles in TMEM, top-k and
+// softmax in the epilogue.
+int launch_route_tc(const void *x, const void *w_gate, const float *bias, int64_t S, int64_t D,
+                    int32_t E, int32_t k, int32_t *top_e, float *top_w, unsigned *status,
+                    cudaStream_t s);
 
 // error message plumbing (api.cu)
 int set_error(int code, const char *fmt, ...);
@@ -149,16 +159,26 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, u
         "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
         : "memory");
 }
-// Four rows r0..r3 (each one box of the 2-D map, box height 1) into 4 consecutive box slots.
-__device__ __forceinline__ void tma_gather4(void *dst, const CUtensorMap *map, uint64_t *bar,
-                                            int32_t col, int32_t r0, int32_t r1, int32_t r2,
-                                            int32_t r3) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(col), "r"(r0), "r"(r1),
-        "r"(r2), "r"(r3)
-        : "memory");
+// ---- cp.async (LSU path) ------------------------------------------------------------------------
+// 16 bytes global -> shared, bypassing L1; src_bytes = 0 writes zeros (K tail).
+__device__ __forceinline__ void cp_async16(uint32_t dst_smem, const void *src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst_smem), "l"(src),
+                 "r"(src_bytes)
+                 : "memory");
+}
+// One arrival on `bar` once every cp.async this thread issued so far has landed (the barrier's
+// expected count must include it: .noinc does not raise the pending count).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.wait_all;" ::: "memory");
+}
+// Orders this thread's view of generic-proxy shared-memory writes before its later async-proxy
+// (tensor core) reads.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
@@ -229,14 +249,20 @@ __device__ __forceinline__ void tmem_ld_wait() {
 
 // ---- shared-memory matrix descriptors (tcgen05 format) -----------------------------------------
 // bits [0,14) start>>4, [16,30) LBO>>4, [32,46) SBO>>4, [46,48) version = 1,
-// [49,52) base offset = 0, [52] LBO mode = 0, [61,64) layout: 2 = 128-byte swizzle.
-__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+// [49,52) base offset = 0, [52] LBO mode = 0, [61,64) layout type:
+//   2 = 128-byte swizzle (16-byte units, 8-row / 1024-byte atom),
+//   1 = 128-byte swizzle with 32-byte units (4-row / 512-byte atom); the only swizzled layout
+//       the tensor cores accept for an MN-major tf32 operand.
+constexpr uint32_t kLayoutSw128 = 2;
+constexpr uint32_t kLayoutSw128Base32 = 1;
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo,
+                                          uint32_t layout) {
     uint64_t d = 0;
     d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
     d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
     d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
     d |= (uint64_t)1 << 46;
-    d |= (uint64_t)2 << 61;
+    d |= (uint64_t)(layout & 7u) << 61;
     return d;
 }
 

@@ -173,7 +173,16 @@ int launch_route_nj(const void *x, const void *w_gate, const float *bias, int64_
 }  // namespace
 
 int launch_route(const void *x, const void *w_gate, const float *bias, int64_t S, int64_t D,
-                 int32_t E, int32_t k, bool bf16, int32_t *top_e, float *top_w, cudaStream_t s) {
+                 int32_t E, int32_t k, bool bf16, int32_t *top_e, float *top_w, unsigned *status,
+                 cudaStream_t s) {
+    if (S == 0) return 0;
+    // bf16 with E a multiple of 8 (16-byte W_gate rows for TMA): tensor-core router.
+    // Otherwise (fp32 inputs, or odd E): exact fp32 FMA accumulation on the CUDA cores.
+    if (bf16 && E % 8 == 0) {
+        if (launch_route_tc(x, w_gate, bias, S, D, E, k, top_e, top_w, status, s) != MOE_OK)
+            return -1;
+        return 1;
+    }
     if (E <= 32) return launch_route_nj<1>(x, w_gate, bias, S, D, E, k, bf16, top_e, top_w, s);
     if (E <= 64) return launch_route_nj<2>(x, w_gate, bias, S, D, E, k, bf16, top_e, top_w, s);
     if (E <= 128) return launch_route_nj<4>(x, w_gate, bias, S, D, E, k, bf16, top_e, top_w, s);
