@@ -3,8 +3,9 @@
 This module only marshals arguments: it checks tensor shapes, dtypes and devices, allocates the
 outputs and the workspace with torch (device memory and streams are torch's), and calls the C ABI
 declared in include/moe.h on the current CUDA stream. Every step of the computation runs in the
-library's CUDA kernels; there is no CPU or PyTorch fallback. If the compiled library is missing
-the import raises.
+library's CUDA kernels; there is no CPU or PyTorch fallback. The compiled library is loaded on
+first use (so that the build module can be imported before it exists); if it is missing, that
+first use raises ImportError.
 """
 from __future__ import annotations
 
@@ -62,12 +63,25 @@ def _load():
     return lib
 
 
-lib = _load()
+_LIB = None
+
+
+def _lib():
+    global _LIB
+    if _LIB is None:
+        _LIB = _load()
+    return _LIB
+
+
+def __getattr__(name):
+    if name == "lib":
+        return _lib()
+    raise AttributeError(name)
 
 
 def _check(rc: int):
     if rc != 0:
-        raise MoeError(rc, lib.moe_last_error().decode())
+        raise MoeError(rc, _lib().moe_last_error().decode())
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -103,12 +117,12 @@ def _req(t, name, dtype=None, dim=None, device=None):
 
 def workspace_size(op: str, S: int, D: int, F: int, E: int, k: int, dtype) -> int:
     code = dtype if isinstance(dtype, int) else (MOE_BF16 if dtype == torch.bfloat16 else MOE_F32)
-    return int(lib.moe_workspace_size(op.encode(), S, D, F, E, k, code))
+    return int(_lib().moe_workspace_size(op.encode(), S, D, F, E, k, code))
 
 
 def workspace_view(which: str, S: int, D: int, F: int, E: int, k: int, dtype) -> int:
     code = dtype if isinstance(dtype, int) else (MOE_BF16 if dtype == torch.bfloat16 else MOE_F32)
-    return int(lib.moe_workspace_view(which.encode(), S, D, F, E, k, code))
+    return int(_lib().moe_workspace_view(which.encode(), S, D, F, E, k, code))
 
 
 def alloc_workspace(nbytes: int, device) -> torch.Tensor:
@@ -129,7 +143,7 @@ def route_topk(x: torch.Tensor, w_gate: torch.Tensor, k: int,
         _req(logit_bias, "logit_bias", dtype=torch.float32, dim=1, device=x.device)
     te = torch.empty((S, k), dtype=torch.int32, device=x.device)
     tw = torch.empty((S, k), dtype=torch.float32, device=x.device)
-    _check(lib.moe_route_topk(_ptr(x), _ptr(w_gate), _ptr(logit_bias), S, D, E, k,
+    _check(_lib().moe_route_topk(_ptr(x), _ptr(w_gate), _ptr(logit_bias), S, D, E, k,
                               _dtype_code(x), _ptr(te), _ptr(tw), _stream(x.device)))
     return te, tw
 
@@ -148,7 +162,7 @@ def sparse_map(top_experts: torch.Tensor, E: int, ws: Optional[torch.Tensor] = N
     offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
     sparse_rows = torch.empty(S * k, dtype=torch.int32, device=dev)
     sorted_rows = torch.empty(S * k, dtype=torch.int32, device=dev)
-    _check(lib.moe_sparse_map(_ptr(top_experts), S, k, E, _ptr(counts), _ptr(offsets),
+    _check(_lib().moe_sparse_map(_ptr(top_experts), S, k, E, _ptr(counts), _ptr(offsets),
                               _ptr(sparse_rows), _ptr(sorted_rows), _ptr(ws), ws.numel(),
                               _stream(dev)))
     return counts, offsets, sparse_rows, sorted_rows
@@ -188,7 +202,7 @@ def scatter_linear(X: torch.Tensor, W: torch.Tensor, k: int, sorted_rows: torch.
         _req(Y, "out", dtype=X.dtype, dim=2, device=dev)
     if ws is None:
         ws = alloc_workspace(workspace_size("scatter_linear", S, Din, Dout, E, k, X.dtype), dev)
-    _check(lib.moe_scatter_linear(_ptr(X), _ptr(W), S, Din, Dout, E, k, _ptr(sorted_rows),
+    _check(_lib().moe_scatter_linear(_ptr(X), _ptr(W), S, Din, Dout, E, k, _ptr(sorted_rows),
                                   _ptr(expert_offsets), _ptr(gates), int(bool(gather_in)),
                                   int(bool(scatter_out)), _dtype_code(X), _ptr(Y), _ptr(ws),
                                   ws.numel(), _stream(dev)))
@@ -250,7 +264,7 @@ def mlp_forward(x: torch.Tensor, w_gate: torch.Tensor, w_gate_e: torch.Tensor,
     _req(out, "out", dtype=torch.float32, dim=2, device=dev)
     if ws is None:
         ws = ForwardWorkspace(S, D, F, E, k, x.dtype, dev)
-    _check(lib.moe_mlp_forward(_ptr(x), _ptr(w_gate), _ptr(logit_bias), _ptr(w_gate_e),
+    _check(_lib().moe_mlp_forward(_ptr(x), _ptr(w_gate), _ptr(logit_bias), _ptr(w_gate_e),
                                _ptr(w_up), _ptr(w_down), S, D, F, E, k, _dtype_code(x),
                                _ptr(out), _ptr(ws.buf), ws.buf.numel(), _stream(dev)))
     return out
@@ -259,21 +273,21 @@ def mlp_forward(x: torch.Tensor, w_gate: torch.Tensor, w_gate_e: torch.Tensor,
 def check_device_status(ws: torch.Tensor):
     """Synchronises and raises MoeError if the device flagged a bad expert id or a timeout."""
     buf = ws.buf if isinstance(ws, ForwardWorkspace) else ws
-    _check(lib.moe_check_device_status(_ptr(buf), _stream(buf.device)))
+    _check(_lib().moe_check_device_status(_ptr(buf), _stream(buf.device)))
 
 
 def profile_events(events):
     """Registers torch.cuda.Event objects (>= 5) for the next mlp_forward on this thread."""
     if not events:
-        _check(lib.moe_profile_events(None, 0))
+        _check(_lib().moe_profile_events(None, 0))
         return
     arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
-    _check(lib.moe_profile_events(arr, len(events)))
+    _check(_lib().moe_profile_events(arr, len(events)))
 
 
 def debug_wait_timeout(limit_ns: int, ws: torch.Tensor):
-    _check(lib.moe_debug_wait_timeout(limit_ns, _ptr(ws), ws.numel(), _stream(ws.device)))
+    _check(_lib().moe_debug_wait_timeout(limit_ns, _ptr(ws), ws.numel(), _stream(ws.device)))
 
 
 def last_launch_count() -> int:
-    return int(lib.moe_last_launch_count())
+    return int(_lib().moe_last_launch_count())
