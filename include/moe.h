@@ -97,6 +97,27 @@ int moe_sparse_map(const int32_t *top_experts, int64_t S, int32_t k, int32_t E,
                    int32_t *sorted_rows, void *ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * Sparse map without any workspace: the same outputs as moe_sparse_map (bit-identical), for
+ * callers that can pass their input and output buffers but cannot obtain extra device memory at
+ * call time, such as plugin-style interfaces that hand over only fixed input/output bindings, or
+ * runtimes that keep all device memory in their own pool, where a cudaMalloc for scratch would
+ * fail or stall the device. The pages have no counterpart of this entry point.
+ * The scratch is a fixed array inside the library: 1 MiB of counters plus a 256-byte status area,
+ * held on every device that loads the library until the process exits. Sizes must satisfy
+ * ceil(S*k / 512) * E * 4 <= 1 MiB (for example S*k <= 524288 routes at E = 256); larger sizes
+ * are rejected with MOE_ERR_INVALID_ARG before any launch. The call allocates nothing.
+ * The first call on a device looks up the array's device address (with that device current);
+ * make that first call before any stream capture. All calls share the array, which keeps the
+ * last call's contents; calls whose kernels overlap on the GPU (e.g. on two streams) race on it
+ * and must be serialised by the caller. An expert id outside [0,E) is not counted and gets
+ * sparse_rows[i] = -1; this call reports no device status, so such ids show as
+ * expert_offsets[E] < S*k.
+ */
+int moe_sparse_map_noalloc(const int32_t *top_experts, int64_t S, int32_t k, int32_t E,
+                           int32_t *expert_counts, int32_t *expert_offsets, int32_t *sparse_rows,
+                           int32_t *sorted_rows, moe_stream_t stream);
+
+/*
  * ParallelLinear(X, W, I, G): for each slot p of expert e (offsets[e] <= p < offsets[e+1]),
  * route i = sorted_rows[p], token s = i / k:
  *   v_p = src_p . W[e]   with src_p = X[s] (gather_in = 1, X is [S, Din] in token order)

@@ -23,7 +23,8 @@ STATUS_NAMES = {0: "MOE_OK", -1: "MOE_ERR_INVALID_ARG", -2: "MOE_ERR_UNSUPPORTED
                 -3: "MOE_ERR_WORKSPACE", -4: "MOE_ERR_CUDA", -5: "MOE_ERR_BAD_EXPERT_ID",
                 -6: "MOE_ERR_DEVICE_TIMEOUT"}
 
-EXPORTS = ["moe_route_topk", "moe_sparse_map", "moe_scatter_linear", "moe_mlp_forward",
+EXPORTS = ["moe_route_topk", "moe_sparse_map", "moe_sparse_map_noalloc", "moe_scatter_linear",
+           "moe_mlp_forward",
            "moe_workspace_size", "moe_workspace_view", "moe_last_error",
            "moe_check_device_status", "moe_profile_events", "moe_debug_wait_timeout",
            "moe_last_launch_count"]
@@ -44,6 +45,7 @@ def _load():
     P, i64, i32, c_int = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int
     lib.moe_route_topk.argtypes = [P, P, P, i64, i64, i32, i32, c_int, P, P, P]
     lib.moe_sparse_map.argtypes = [P, i64, i32, i32, P, P, P, P, P, ctypes.c_size_t, P]
+    lib.moe_sparse_map_noalloc.argtypes = [P, i64, i32, i32, P, P, P, P, P]
     lib.moe_scatter_linear.argtypes = [P, P, i64, i64, i64, i32, i32, P, P, P, c_int, c_int,
                                        c_int, P, P, ctypes.c_size_t, P]
     lib.moe_mlp_forward.argtypes = [P, P, P, P, P, P, i64, i64, i64, i32, i32, c_int, P, P,
@@ -56,7 +58,8 @@ def _load():
     lib.moe_check_device_status.argtypes = [P, P]
     lib.moe_profile_events.argtypes = [P, c_int]
     lib.moe_debug_wait_timeout.argtypes = [i64, P, ctypes.c_size_t, P]
-    for name in ("moe_route_topk", "moe_sparse_map", "moe_scatter_linear", "moe_mlp_forward",
+    for name in ("moe_route_topk", "moe_sparse_map", "moe_sparse_map_noalloc",
+                 "moe_scatter_linear", "moe_mlp_forward",
                  "moe_check_device_status", "moe_profile_events", "moe_debug_wait_timeout",
                  "moe_last_launch_count"):
         getattr(lib, name).restype = c_int
