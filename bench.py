@@ -148,9 +148,13 @@ def host_inputs(inp):
 
 
 def calibrate_oracle(w, inp_cpu, budget_s):
-    """Number of tokens the oracle covers in about budget_s seconds (one token probes the rate)."""
-    t1, _, _ = run_oracle_sample(w, inp_cpu, 1, seed=123)
-    return max(1, min(w.S, int(budget_s / max(t1, 1e-6))))
+    """Number of tokens the oracle covers in about budget_s seconds, from a probe that keeps
+    every host thread busy (one token per thread; its time is the per-wave cost)."""
+    import oracle
+    n_probe = max(1, min(w.S, oracle.num_threads()))
+    t, n, _ = run_oracle_sample(w, inp_cpu, n_probe, seed=123)
+    per_token = max(t, 1e-6) / n
+    return max(1, min(w.S, int(budget_s / per_token)))
 
 
 def dist_setup():

@@ -4,6 +4,7 @@
 #include "moe_internal.cuh"
 
 #include <stdarg.h>
+#include <stdlib.h>
 #include <stdio.h>
 #include <string.h>
 
@@ -22,6 +23,15 @@ int set_error(int code, const char *fmt, ...) {
     vsnprintf(g_err, sizeof(g_err), fmt, ap);
     va_end(ap);
     return code;
+}
+
+bool prefer_2sm(int64_t R, int32_t E, bool gather) {
+    const char *env = getenv("MOE_GEMM_2SM");
+    if (env != nullptr && (env[0] == '0' || env[0] == '1')) return env[0] == '1';
+    // Pair tiles pay off on contiguous (slot-ordered) A when experts are long enough that the
+    // 256-row tiles waste little. With gathered A the pair kernel measured slower than one CTA
+    // (its cp.async row gather could not keep the pair MMA fed), so gathered GEMMs stay on one CTA.
+    return !gather && E > 0 && R / E >= 384;
 }
 
 int num_sms() {
@@ -283,7 +293,8 @@ int moe_scatter_linear(const void *X, const void *W, int64_t S, int64_t Din, int
     a.scatter = scatter_out != 0;
     a.status = status;
     a.wait_limit_ns = kWaitLimitNs;
-    if ((rc = launch_grouped_gemm(a, s))) return rc;
+    if ((rc = prefer_2sm(R, E, a.gather) ? launch_grouped_gemm_2sm(a, s) : launch_grouped_gemm(a, s)))
+        return rc;
     g_launches = 1;
     return check_launch("scatter_linear");
 }
@@ -354,7 +365,8 @@ int moe_mlp_forward(const void *x, const void *w_gate, const float *logit_bias,
         a.scatter = false;
         a.status = status;
         a.wait_limit_ns = kWaitLimitNs;
-        if ((rc = launch_grouped_gemm(a, s))) return rc;
+        if ((rc = prefer_2sm(R, E, true) ? launch_grouped_gemm_2sm(a, s) : launch_grouped_gemm(a, s)))
+            return rc;
         if ((rc = check_launch("gemm1"))) return rc;
         ++n;
         record_prof(3, s);
@@ -370,7 +382,8 @@ int moe_mlp_forward(const void *x, const void *w_gate, const float *logit_bias,
         b.gather = false;
         b.glu = false;
         b.scatter = true;
-        if ((rc = launch_grouped_gemm(b, s))) return rc;
+        if ((rc = prefer_2sm(R, E, false) ? launch_grouped_gemm_2sm(b, s) : launch_grouped_gemm(b, s)))
+            return rc;
         if ((rc = check_launch("gemm2"))) return rc;
         ++n;
         record_prof(4, s);

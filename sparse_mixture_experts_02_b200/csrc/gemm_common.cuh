@@ -1,0 +1,203 @@
+// Pieces shared by the one-CTA and the two-CTA (cta_group::2) grouped GEMM kernels: tile
+// constants, kernel parameters, the device-side tile schedule and the per-row epilogue.
+#pragma once
+
+#include "moe_internal.cuh"
+
+namespace moe {
+namespace gemm {
+
+constexpr int BM = 128;                 // rows per tile (TMEM lanes)
+constexpr int BN = 256;                 // MMA N = accumulator columns
+constexpr int STAGES = 4;
+constexpr int KBYTES = 128;             // bytes of K per stage (one 128-byte swizzle row)
+constexpr int A_BYTES = BM * KBYTES;    // 16 KB
+constexpr int B_BYTES = BN * KBYTES;    // 32 KB (BN columns x (128 / eb) K rows x eb)
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int MAX_E = 256;
+constexpr int THREADS = 192;            // producer, MMA, 4 epilogue warps
+constexpr int GATHER_THREADS = 128;     // extra warps 6-9 for gathered A
+constexpr uint32_t TMEM_COLS = 512;
+
+// Shared-memory bookkeeping of the one-CTA kernel (after its STAGES operand stages).
+struct SmemTail {
+    uint64_t full[STAGES];
+    uint64_t empty[STAGES];
+    uint64_t tfull[2];
+    uint64_t tempty[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+    int32_t off[MAX_E + 1];
+    int32_t tstart[MAX_E + 1];
+};
+constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + sizeof(SmemTail);
+
+struct KParams {
+    const void *A;    // gathered mode: x [S, K] (rows fetched by the gather warps)
+    int64_t K;
+    const int32_t *offsets;
+    const int32_t *sorted_rows;
+    const float *gates;
+    void *out;
+    int32_t E, k;
+    int32_t N;        // output columns
+    int32_t num_kb;   // K stages
+    int32_t n_tiles;  // N tiles
+    int64_t S, R;     // bounds of scatter rows (tokens) and grouped rows (slots)
+    // router mode: logit bias [E] (nullable), outputs [S, k]
+    const float *bias;
+    int32_t *top_e;
+    float *top_w;
+    int32_t b_chunks; // B chunks loaded per stage (router: ceil(E / chunk width))
+    unsigned *status;
+    int64_t wait_limit_ns;
+};
+
+struct TileInfo {
+    int e, row_begin, rows, n_idx;
+};
+
+// Device-side tile schedule. Expert e owns ceil(N_e / TM) M tiles of TM rows (the last one
+// partial, none for an empty expert) times n_tiles N tiles; tstart[e] is the exclusive prefix of
+// those counts over experts. Tiles are numbered expert-major, then N tile, then M tile, so the
+// CTAs that run at the same time share one expert's weight tiles and gathered rows in L2.
+template <int TM>
+__device__ __forceinline__ void build_schedule(const int32_t *off, int32_t *tstart, int E,
+                                               int n_tiles) {
+    int run = 0;
+    for (int e = 0; e < E; ++e) {
+        tstart[e] = run;
+        run += ((off[e + 1] - off[e] + TM - 1) / TM) * n_tiles;
+    }
+    tstart[E] = run;
+}
+
+template <int TM>
+__device__ __forceinline__ TileInfo decode_tile(int t, const int32_t *off, const int32_t *tstart,
+                                                int E) {
+    int lo = 0, hi = E;  // tstart[lo] <= t < tstart[hi]
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (tstart[mid] <= t) lo = mid;
+        else hi = mid;
+    }
+    TileInfo ti;
+    ti.e = lo;
+    const int local = t - tstart[lo];
+    const int cnt = off[lo + 1] - off[lo];
+    const int mt = (cnt + TM - 1) / TM;
+    ti.n_idx = local / mt;
+    const int m = local - ti.n_idx * mt;
+    ti.row_begin = off[lo] + m * TM;
+    ti.rows = min(TM, off[lo + 1] - ti.row_begin);
+    return ti;
+}
+
+__device__ __forceinline__ float silu_f(float z) { return z / (1.0f + __expf(-z)); }
+
+
+// Epilogue of one accumulator row (the calling thread's TMEM lane) of a 128 x 256 tile:
+//   GLU:      h = silu(acc[:, c]) * acc[:, 128 + c] (* g), rounded to the output dtype, stored
+//             at out[orow, n0 + c] for the 128 output columns c;
+//   SCATTER:  out[orow, n0 + c] += g * acc[:, c] with fp32 vector atomics (256 columns);
+//   else:     out[orow, n0 + c] = g * acc[:, c] in the output dtype (256 columns).
+// Columns at or past N are skipped (N is a multiple of 8). `valid` is false for rows past the
+// tile's end; every lane still takes part in the warp-wide TMEM loads.
+template <bool BF16, bool GLU, bool SCATTER>
+__device__ __forceinline__ void epilogue_row(const KParams &p, uint32_t tbase, bool valid,
+                                             int64_t orow, float g, int n0) {
+    constexpr int OUT_COLS = GLU ? BN / 2 : BN;
+    if constexpr (GLU) {
+#pragma unroll 1
+        for (int c = 0; c < OUT_COLS / 32; ++c) {
+            uint32_t gv[32], uv[32];
+            dev::tmem_ld32(tbase + c * 32, gv);
+            dev::tmem_ld32(tbase + OUT_COLS + c * 32, uv);
+            dev::tmem_ld_wait();
+            const int col0 = n0 + c * 32;
+            if (valid && col0 < p.N) {
+                float hv[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    hv[j] = g * silu_f(__uint_as_float(gv[j])) * __uint_as_float(uv[j]);
+                if (BF16) {
+                    __nv_bfloat16 *dst =
+                        reinterpret_cast<__nv_bfloat16 *>(p.out) + orow * p.N + col0;
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) {
+                        if (col0 + v * 8 < p.N) {
+                            uint4 pk;
+                            uint32_t *pw = reinterpret_cast<uint32_t *>(&pk);
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                __nv_bfloat162 t2 = __floats2bfloat162_rn(
+                                    hv[v * 8 + 2 * j], hv[v * 8 + 2 * j + 1]);
+                                pw[j] = *reinterpret_cast<uint32_t *>(&t2);
+                            }
+                            *reinterpret_cast<uint4 *>(dst + v * 8) = pk;
+                        }
+                    }
+                } else {
+                    float *dst = reinterpret_cast<float *>(p.out) + orow * p.N + col0;
+#pragma unroll
+                    for (int v = 0; v < 8; ++v)
+                        if (col0 + v * 4 < p.N)
+                            *reinterpret_cast<float4 *>(dst + v * 4) = make_float4(
+                                hv[v * 4], hv[v * 4 + 1], hv[v * 4 + 2], hv[v * 4 + 3]);
+                }
+            }
+        }
+    } else {
+#pragma unroll 1
+        for (int c = 0; c < OUT_COLS / 32; ++c) {
+            uint32_t av[32];
+            dev::tmem_ld32(tbase + c * 32, av);
+            dev::tmem_ld_wait();
+            const int col0 = n0 + c * 32;
+            if (valid && col0 < p.N) {
+                if (SCATTER) {
+                    float *dst = reinterpret_cast<float *>(p.out) + orow * p.N + col0;
+#pragma unroll
+                    for (int v = 0; v < 8; ++v)
+                        if (col0 + v * 4 < p.N)
+                            dev::red_add_v4(dst + v * 4, g * __uint_as_float(av[v * 4]),
+                                            g * __uint_as_float(av[v * 4 + 1]),
+                                            g * __uint_as_float(av[v * 4 + 2]),
+                                            g * __uint_as_float(av[v * 4 + 3]));
+                } else if (BF16) {
+                    __nv_bfloat16 *dst =
+                        reinterpret_cast<__nv_bfloat16 *>(p.out) + orow * p.N + col0;
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) {
+                        if (col0 + v * 8 < p.N) {
+                            uint4 pk;
+                            uint32_t *pw = reinterpret_cast<uint32_t *>(&pk);
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                __nv_bfloat162 t2 = __floats2bfloat162_rn(
+                                    g * __uint_as_float(av[v * 8 + 2 * j]),
+                                    g * __uint_as_float(av[v * 8 + 2 * j + 1]));
+                                pw[j] = *reinterpret_cast<uint32_t *>(&t2);
+                            }
+                            *reinterpret_cast<uint4 *>(dst + v * 8) = pk;
+                        }
+                    }
+                } else {
+                    float *dst = reinterpret_cast<float *>(p.out) + orow * p.N + col0;
+#pragma unroll
+                    for (int v = 0; v < 8; ++v)
+                        if (col0 + v * 4 < p.N)
+                            *reinterpret_cast<float4 *>(dst + v * 4) =
+                                make_float4(g * __uint_as_float(av[v * 4]),
+                                            g * __uint_as_float(av[v * 4 + 1]),
+                                            g * __uint_as_float(av[v * 4 + 2]),
+                                            g * __uint_as_float(av[v * 4 + 3]));
+                }
+            }
+        }
+    }
+}
+
+}  // namespace gemm
+}  // namespace moe

@@ -33,7 +33,7 @@
 // Tile schedule: every CTA derives it from expert_offsets on the device (no host sync):
 // tiles are ordered expert-major, then N tile, then M tile, so the CTAs running at one time
 // share expert weight tiles and gathered rows through L2. Waits are bounded (see mbar_wait).
-#include "moe_internal.cuh"
+#include "gemm_common.cuh"
 
 #include <stdio.h>
 #include <mutex>
@@ -41,77 +41,7 @@
 namespace moe {
 namespace {
 
-constexpr int BM = 128;                 // rows per tile (TMEM lanes)
-constexpr int BN = 256;                 // MMA N = accumulator columns
-constexpr int STAGES = 4;
-constexpr int KBYTES = 128;             // bytes of K per stage (one 128-byte swizzle row)
-constexpr int A_BYTES = BM * KBYTES;    // 16 KB
-constexpr int B_BYTES = BN * KBYTES;    // 32 KB (BN columns x (128 / eb) K rows x eb)
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int MAX_E = 256;
-constexpr int THREADS = 192;            // producer, MMA, 4 epilogue warps
-constexpr int GATHER_THREADS = 128;     // extra warps 6-9 for gathered A
-constexpr uint32_t TMEM_COLS = 512;
-
-struct SmemTail {
-    uint64_t full[STAGES];
-    uint64_t empty[STAGES];
-    uint64_t tfull[2];
-    uint64_t tempty[2];
-    uint64_t drain;
-    uint32_t tmem_base;
-    int abort;
-    int32_t off[MAX_E + 1];
-    int32_t tstart[MAX_E + 1];
-};
-constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + sizeof(SmemTail);
-
-struct KParams {
-    const void *A;    // gathered mode: x [S, K] (rows fetched by the gather warps)
-    int64_t K;
-    const int32_t *offsets;
-    const int32_t *sorted_rows;
-    const float *gates;
-    void *out;
-    int32_t E, k;
-    int32_t N;        // output columns
-    int32_t num_kb;   // K stages
-    int32_t n_tiles;  // N tiles
-    int64_t S, R;     // bounds of scatter rows (tokens) and grouped rows (slots)
-    // router mode: logit bias [E] (nullable), outputs [S, k]
-    const float *bias;
-    int32_t *top_e;
-    float *top_w;
-    int32_t b_chunks; // B chunks loaded per stage (router: ceil(E / chunk width))
-    unsigned *status;
-    int64_t wait_limit_ns;
-};
-
-struct TileInfo {
-    int e, row_begin, rows, n_idx;
-};
-
-__device__ __forceinline__ TileInfo decode_tile(int t, const SmemTail &st, int E, int n_tiles) {
-    int lo = 0, hi = E;  // tstart[lo] <= t < tstart[hi]
-    while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (st.tstart[mid] <= t) lo = mid;
-        else hi = mid;
-    }
-    TileInfo ti;
-    ti.e = lo;
-    const int local = t - st.tstart[lo];
-    const int cnt = st.off[lo + 1] - st.off[lo];
-    const int mt = (cnt + BM - 1) / BM;
-    ti.n_idx = local / mt;
-    const int m = local - ti.n_idx * mt;
-    ti.row_begin = st.off[lo] + m * BM;
-    ti.rows = min(BM, st.off[lo + 1] - ti.row_begin);
-    (void)n_tiles;
-    return ti;
-}
-
-__device__ __forceinline__ float silu_f(float z) { return z / (1.0f + __expf(-z)); }
+using namespace gemm;
 
 template <bool BF16, bool GATHER, bool GLU, bool SCATTER, bool ROUTER>
 __global__ void __launch_bounds__(GATHER ? THREADS + GATHER_THREADS : THREADS, 1)
@@ -176,15 +106,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     } else {
         for (int e = threadIdx.x; e <= E; e += blockDim.x) st.off[e] = __ldg(p.offsets + e);
         __syncthreads();
-        if (threadIdx.x == 0) {
-            int run = 0;
-            for (int e = 0; e < E; ++e) {
-                st.tstart[e] = run;
-                const int mt = (st.off[e + 1] - st.off[e] + BM - 1) / BM;
-                run += mt * p.n_tiles;
-            }
-            st.tstart[E] = run;
-        }
+        if (threadIdx.x == 0) build_schedule<BM>(st.off, st.tstart, E, p.n_tiles);
         __syncthreads();
     }
     dev::tc_fence_after();
@@ -202,7 +124,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         uint32_t issued = 0, last_par = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-            const TileInfo ti = decode_tile(t, st, E_sched, p.n_tiles);
+            const TileInfo ti = decode_tile<BM>(t, st.off, st.tstart, E_sched);
             const int n0 = ti.n_idx * OUT_COLS;
             for (int kb = 0; kb < p.num_kb; ++kb) {
                 bool w = true;
@@ -309,7 +231,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         uint32_t s = 0, ph = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-            const TileInfo ti = decode_tile(t, st, E_sched, p.n_tiles);
+            const TileInfo ti = decode_tile<BM>(t, st.off, st.tstart, E_sched);
             const uint8_t *src[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
@@ -351,7 +273,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         const int r = q * 32 + lane;
         int it = 0;
         for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
-            const TileInfo ti = decode_tile(t, st, E_sched, p.n_tiles);
+            const TileInfo ti = decode_tile<BM>(t, st.off, st.tstart, E_sched);
             const uint32_t b = it & 1, aph = (it >> 1) & 1;
             bool w = true;
             if (lane == 0)
@@ -422,94 +344,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         }
                     }
                 }
-            } else if (GLU) {
-#pragma unroll 1
-                for (int c = 0; c < OUT_COLS / 32; ++c) {
-                    uint32_t gv[32], uv[32];
-                    dev::tmem_ld32(tbase + c * 32, gv);
-                    dev::tmem_ld32(tbase + OUT_COLS + c * 32, uv);
-                    dev::tmem_ld_wait();
-                    const int col0 = n0 + c * 32;
-                    if (valid && col0 < p.N) {
-                        float hv[32];
-#pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            hv[j] = g * silu_f(__uint_as_float(gv[j])) * __uint_as_float(uv[j]);
-                        if (BF16) {
-                            __nv_bfloat16 *dst =
-                                reinterpret_cast<__nv_bfloat16 *>(p.out) + orow * p.N + col0;
-#pragma unroll
-                            for (int v = 0; v < 4; ++v) {
-                                if (col0 + v * 8 < p.N) {
-                                    uint4 pk;
-                                    uint32_t *pw = reinterpret_cast<uint32_t *>(&pk);
-#pragma unroll
-                                    for (int j = 0; j < 4; ++j) {
-                                        __nv_bfloat162 t2 = __floats2bfloat162_rn(
-                                            hv[v * 8 + 2 * j], hv[v * 8 + 2 * j + 1]);
-                                        pw[j] = *reinterpret_cast<uint32_t *>(&t2);
-                                    }
-                                    *reinterpret_cast<uint4 *>(dst + v * 8) = pk;
-                                }
-                            }
-                        } else {
-                            float *dst = reinterpret_cast<float *>(p.out) + orow * p.N + col0;
-#pragma unroll
-                            for (int v = 0; v < 8; ++v)
-                                if (col0 + v * 4 < p.N)
-                                    *reinterpret_cast<float4 *>(dst + v * 4) = make_float4(
-                                        hv[v * 4], hv[v * 4 + 1], hv[v * 4 + 2], hv[v * 4 + 3]);
-                        }
-                    }
-                }
             } else {
-#pragma unroll 1
-                for (int c = 0; c < OUT_COLS / 32; ++c) {
-                    uint32_t av[32];
-                    dev::tmem_ld32(tbase + c * 32, av);
-                    dev::tmem_ld_wait();
-                    const int col0 = n0 + c * 32;
-                    if (valid && col0 < p.N) {
-                        if (SCATTER) {
-                            float *dst = reinterpret_cast<float *>(p.out) + orow * p.N + col0;
-#pragma unroll
-                            for (int v = 0; v < 8; ++v)
-                                if (col0 + v * 4 < p.N)
-                                    dev::red_add_v4(dst + v * 4, g * __uint_as_float(av[v * 4]),
-                                                    g * __uint_as_float(av[v * 4 + 1]),
-                                                    g * __uint_as_float(av[v * 4 + 2]),
-                                                    g * __uint_as_float(av[v * 4 + 3]));
-                        } else if (BF16) {
-                            __nv_bfloat16 *dst =
-                                reinterpret_cast<__nv_bfloat16 *>(p.out) + orow * p.N + col0;
-#pragma unroll
-                            for (int v = 0; v < 4; ++v) {
-                                if (col0 + v * 8 < p.N) {
-                                    uint4 pk;
-                                    uint32_t *pw = reinterpret_cast<uint32_t *>(&pk);
-#pragma unroll
-                                    for (int j = 0; j < 4; ++j) {
-                                        __nv_bfloat162 t2 = __floats2bfloat162_rn(
-                                            g * __uint_as_float(av[v * 8 + 2 * j]),
-                                            g * __uint_as_float(av[v * 8 + 2 * j + 1]));
-                                        pw[j] = *reinterpret_cast<uint32_t *>(&t2);
-                                    }
-                                    *reinterpret_cast<uint4 *>(dst + v * 8) = pk;
-                                }
-                            }
-                        } else {
-                            float *dst = reinterpret_cast<float *>(p.out) + orow * p.N + col0;
-#pragma unroll
-                            for (int v = 0; v < 8; ++v)
-                                if (col0 + v * 4 < p.N)
-                                    *reinterpret_cast<float4 *>(dst + v * 4) =
-                                        make_float4(g * __uint_as_float(av[v * 4]),
-                                                    g * __uint_as_float(av[v * 4 + 1]),
-                                                    g * __uint_as_float(av[v * 4 + 2]),
-                                                    g * __uint_as_float(av[v * 4 + 3]));
-                        }
-                    }
-                }
+                epilogue_row<BF16, GLU, SCATTER>(p, tbase, valid, orow, g, n0);
             }
             dev::tc_fence_before();
             __syncwarp();
@@ -538,6 +374,8 @@ __global__ void debug_wait_kernel(int64_t limit_ns, unsigned *status) {
 }
 
 // ---- host side: tensor maps -------------------------------------------------------------------
+}  // namespace
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -557,9 +395,8 @@ EncodeTiledFn get_encode() {
     return fn;
 }
 
-int encode(CUtensorMap *m, bool bf16, int rank, const void *base, const uint64_t *dims,
-           const uint64_t *strides_bytes, const uint32_t *box,
-           CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
+int encode_tmap(CUtensorMap *m, bool bf16, int rank, const void *base, const uint64_t *dims,
+                const uint64_t *strides_bytes, const uint32_t *box, CUtensorMapSwizzle swz) {
     EncodeTiledFn fn = get_encode();
     if (!fn) return set_error(MOE_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
     cuuint64_t gd[3], gs[2];
@@ -576,6 +413,8 @@ int encode(CUtensorMap *m, bool bf16, int rank, const void *base, const uint64_t
     if (r != CUDA_SUCCESS) return set_error(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
     return MOE_OK;
 }
+
+namespace {
 
 template <bool BF16, bool GATHER, bool GLU, bool SCATTER, bool ROUTER = false>
 int launch_t(const GemmArgs &a, cudaStream_t s) {
@@ -597,7 +436,7 @@ int launch_t(const GemmArgs &a, cudaStream_t s) {
         const uint64_t dims[2] = {(uint64_t)a.K, (uint64_t)a.a_rows};
         const uint64_t str[1] = {(uint64_t)a.K * EB};
         const uint32_t box[2] = {(uint32_t)BK, GATHER ? 1u : (uint32_t)BM};
-        int rc = encode(&mA, BF16, 2, a.A, dims, str, box);
+        int rc = encode_tmap(&mA, BF16, 2, a.A, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
         if (rc) return rc;
     }
     {
@@ -606,10 +445,10 @@ int launch_t(const GemmArgs &a, cudaStream_t s) {
         const uint32_t box[3] = {(uint32_t)CW, (uint32_t)BK, 1u};
         const CUtensorMapSwizzle swz =
             BF16 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B;
-        int rc = encode(&mB0, BF16, 3, a.B0, dims, str, box, swz);
+        int rc = encode_tmap(&mB0, BF16, 3, a.B0, dims, str, box, swz);
         if (rc) return rc;
         if (GLU) {
-            rc = encode(&mB1, BF16, 3, a.B1, dims, str, box, swz);
+            rc = encode_tmap(&mB1, BF16, 3, a.B1, dims, str, box, swz);
             if (rc) return rc;
         } else {
             mB1 = mB0;

@@ -85,8 +85,10 @@ def _check_case(oracle_lib, moe, w, inp_gpu, tokens, h_rows=64):
     return out, v, mx, rf
 
 
+@pytest.mark.parametrize("cta", ["0", "1"])
 @pytest.mark.parametrize("name", list(SMALL))
-def test_mlp_small_all_tokens(oracle_lib, moe, name):
+def test_mlp_small_all_tokens(oracle_lib, moe, monkeypatch, name, cta):
+    monkeypatch.setenv("MOE_GEMM_2SM", cta)  # one-CTA and CTA-pair grouped GEMMs
     w = SMALL[name]
     inp = {k: (t.cuda() if t is not None else None) for k, t in W.make_inputs(w).items()}
     _check_case(oracle_lib, moe, w, inp, np.arange(w.S, dtype=np.int32))

@@ -35,12 +35,20 @@ SHAPES = [
 ]
 
 
+@pytest.fixture(params=["cta1", "cta2"])
+def gemm_kernel(request, monkeypatch):
+    """Runs a test once on the one-CTA grouped GEMM and once on the CTA-pair (cta_group::2)
+    kernel; the library reads MOE_GEMM_2SM at every launch."""
+    monkeypatch.setenv("MOE_GEMM_2SM", "1" if request.param == "cta2" else "0")
+    return request.param
+
+
 @pytest.mark.parametrize("shape", SHAPES)
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 @pytest.mark.parametrize("gather_in,scatter_out", [(True, True), (False, True), (True, False),
                                                    (False, False)])
 @pytest.mark.parametrize("gated", [True, False])
-def test_scatter_linear(oracle_lib, moe, shape, dtype, gather_in, scatter_out, gated):
+def test_scatter_linear(oracle_lib, moe, gemm_kernel, shape, dtype, gather_in, scatter_out, gated):
     S, k, E, Din, Dout, mode = shape
     tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
     gen = torch.Generator().manual_seed(S + E + Din)
@@ -65,7 +73,7 @@ def test_scatter_linear(oracle_lib, moe, shape, dtype, gather_in, scatter_out, g
     assert np.abs(got - ref).max() / scale < 10 * _tol(dtype, scatter_out)
 
 
-def test_scatter_linear_accumulates_into_out(oracle_lib, moe):
+def test_scatter_linear_accumulates_into_out(oracle_lib, moe, gemm_kernel):
     S, k, E, Din, Dout = 200, 2, 4, 64, 64
     te = W.make_top_experts(S, k, E, seed=4)
     _, offsets, _, sorted_rows = oracle_lib.sparse_map(te.numpy(), E)
@@ -79,7 +87,7 @@ def test_scatter_linear_accumulates_into_out(oracle_lib, moe):
     assert rel_frob(Y.cpu().numpy() - 3.0, ref) < 2e-5
 
 
-def test_scatter_linear_all_routes_one_expert(oracle_lib, moe):
+def test_scatter_linear_all_routes_one_expert(oracle_lib, moe, gemm_kernel):
     # every route on expert 2 of 4: three empty experts and one long run of M tiles
     S, k, E, Din, Dout = 1100, 1, 4, 128, 256
     te = torch.full((S, k), 2, dtype=torch.int32)
