@@ -54,14 +54,23 @@ def peaks():
             "fallback"
 
 
+def gemm_source_hash() -> str:
+    """Hash of the sources that define the grouped GEMM kernels (a recorded DRAM traffic figure is
+    only reported while they are unchanged)."""
+    h = hashlib.sha256()
+    for name in ("grouped_gemm.cu", "grouped_gemm_2sm.cu", "gemm_common.cuh", "moe_internal.cuh"):
+        with open(os.path.join(ROOT, "sparse_mixture_experts_02_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
 def recorded_traffic(kernel_key: str):
     """DRAM bytes per launch of `kernel_key` from the committed ncu summary, if the kernel source
     is unchanged since it was captured (the summary records the source hash)."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.md")
-    src = os.path.join(ROOT, "sparse_mixture_experts_02_b200", "csrc", "grouped_gemm.cu")
     try:
         text = open(path).read()
-        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        sha = gemm_source_hash()
     except OSError:
         return None
     m = re.search(r"^\|\s*" + re.escape(kernel_key) + r"\s*\|\s*([0-9]+)\s*\|\s*([0-9a-f]+)\s*\|",

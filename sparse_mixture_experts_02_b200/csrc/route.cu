@@ -145,6 +145,105 @@ route_kernel(const void *__restrict__ x, const void *__restrict__ w_gate,
     }
 }
 
+// Router for small batches and few experts (E <= 64): one block per token, so even a decode
+// batch spreads over every SM. Thread t accumulates, in fp32 and ascending d within its slice,
+// the E partial dot products of d in {8t .. 8t+7} + 1024 j; the block then sums the partials
+// (fixed order: warp butterfly, then the four warps in order) and one warp takes the top-k.
+template <int NE, bool BF16>
+__global__ void __launch_bounds__(128)
+route_small_kernel(const void *__restrict__ x, const void *__restrict__ w_gate,
+                   const float *__restrict__ bias, int64_t D, int32_t E, int32_t k,
+                   int32_t *__restrict__ top_e, float *__restrict__ top_w) {
+    __shared__ float part[4][NE];
+    const int64_t s = blockIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    float acc[NE];
+#pragma unroll
+    for (int e = 0; e < NE; ++e) acc[e] = 0.f;
+    for (int64_t d0 = (int64_t)tid * 8; d0 < D; d0 += 1024) {
+        float xv[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) xv[j] = ld_elem<BF16>(x, s * D + d0 + j);  // D % 8 == 0
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int64_t row = (d0 + j) * (int64_t)E;
+#pragma unroll
+            for (int e = 0; e < NE; ++e)
+                if (e < E) acc[e] = fmaf(xv[j], ld_elem<BF16>(w_gate, row + e), acc[e]);
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < NE; ++e) {
+        float v = acc[e];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+        if (lane == 0) part[warp][e] = v;
+    }
+    __syncthreads();
+    if (warp != 0) return;
+    // lane l owns experts l and l + 32
+    float v[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int e = lane + 32 * h;
+        float l = -INFINITY;
+        if (e < E && e < NE) {
+            l = ((part[0][e] + part[1][e]) + part[2][e]) + part[3][e];
+            if (bias != nullptr) l += __ldg(bias + e);
+            if (isnan(l)) l = -INFINITY;
+        }
+        v[h] = l;
+    }
+    unsigned taken = 0;
+    float sel_v[8];
+    int sel_i[8];
+    for (int r = 0; r < k; ++r) {
+        float bv = -INFINITY;
+        int bi = 0x7fffffff;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int e = lane + 32 * h;
+            if (e < E && !(taken & (1u << h)) && better(v[h], e, bv, bi)) {
+                bv = v[h];
+                bi = e;
+            }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+            const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+            if (better(ov, oi, bv, bi)) {
+                bv = ov;
+                bi = oi;
+            }
+        }
+        if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+        sel_v[r] = bv;
+        sel_i[r] = bi;
+    }
+    if (lane == 0) {
+        const float m = sel_v[0];
+        float den = 0.f;
+        for (int r = 0; r < k; ++r) den += expf(sel_v[r] - m);
+        for (int r = 0; r < k; ++r) {
+            top_e[s * k + r] = sel_i[r];
+            top_w[s * k + r] = expf(sel_v[r] - m) / den;
+        }
+    }
+}
+
+template <int NE>
+void launch_route_small_ne(const void *x, const void *w_gate, const float *bias, int64_t S,
+                           int64_t D, int32_t E, int32_t k, bool bf16, int32_t *top_e,
+                           float *top_w, cudaStream_t s) {
+    if (bf16)
+        route_small_kernel<NE, true><<<(unsigned)S, 128, 0, s>>>(x, w_gate, bias, D, E, k, top_e,
+                                                                 top_w);
+    else
+        route_small_kernel<NE, false><<<(unsigned)S, 128, 0, s>>>(x, w_gate, bias, D, E, k,
+                                                                  top_e, top_w);
+}
+
 __global__ void zero_kernel(float4 *__restrict__ p, int64_t n4, float *__restrict__ tail,
                             int tail_n, unsigned *status) {
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
@@ -176,6 +275,15 @@ int launch_route(const void *x, const void *w_gate, const float *bias, int64_t S
                  int32_t E, int32_t k, bool bf16, int32_t *top_e, float *top_w, unsigned *status,
                  cudaStream_t s) {
     if (S == 0) return 0;
+    // Few experts and a batch too small to fill the SMs with 128-token tensor-core tiles (or fp32
+    // inputs): one block per token on the CUDA cores, exact fp32 accumulation.
+    if (E <= 64 && (S <= 2048 || !bf16) && S < (int64_t(1) << 31)) {
+        if (E <= 8) launch_route_small_ne<8>(x, w_gate, bias, S, D, E, k, bf16, top_e, top_w, s);
+        else if (E <= 16) launch_route_small_ne<16>(x, w_gate, bias, S, D, E, k, bf16, top_e, top_w, s);
+        else if (E <= 32) launch_route_small_ne<32>(x, w_gate, bias, S, D, E, k, bf16, top_e, top_w, s);
+        else launch_route_small_ne<64>(x, w_gate, bias, S, D, E, k, bf16, top_e, top_w, s);
+        return 1;
+    }
     // bf16 with E a multiple of 8 (16-byte W_gate rows for TMA): tensor-core router.
     // Otherwise (fp32 inputs, or odd E): exact fp32 FMA accumulation on the CUDA cores.
     if (bf16 && E % 8 == 0) {

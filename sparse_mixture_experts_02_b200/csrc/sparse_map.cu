@@ -142,6 +142,85 @@ map_assign_kernel(const int32_t *__restrict__ te, int64_t R, int32_t E, int64_t 
     }
 }
 
+// The whole map in one block when the routes fit 32 units (R <= 16384): warp w counts unit w
+// into cnt[w][e]; the per-expert exclusive prefix over the 32 warps plus the expert offset turns
+// cnt into bases; the warps walk their units again and assign stable slots. Same results as the
+// three-kernel path, one launch instead of three (the decode and Mixtral-prefill route counts).
+constexpr int kSmallUnits = 32;
+__global__ void __launch_bounds__(kSmallUnits * 32)
+map_small_kernel(const int32_t *__restrict__ te, int64_t R, int32_t E,
+                 int32_t *__restrict__ counts, int32_t *__restrict__ offsets,
+                 int32_t *__restrict__ sparse_rows, int32_t *__restrict__ sorted_rows,
+                 unsigned *status) {
+    __shared__ int32_t cnt[kSmallUnits][kMaxE];
+    __shared__ int32_t eoff[kMaxE];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int e = lane; e < E; e += 32) cnt[warp][e] = 0;
+    __syncwarp();
+    const int64_t base = (int64_t)warp * kUnit;
+    bool bad = false;
+    for (int it = 0; it < kIters; ++it) {
+        const int64_t i = base + it * 32 + lane;
+        int e = -1;
+        if (i < R) {
+            e = __ldg(te + i);
+            if (e < 0 || e >= E) {
+                bad = true;
+                e = -1;
+            }
+        }
+        const unsigned peers = __match_any_sync(0xffffffffu, e);
+        if (e >= 0 && lane == __ffs(peers) - 1) cnt[warp][e] += __popc(peers);
+        __syncwarp();
+    }
+    if (bad) atomicOr(status, kStatusBadExpert);
+    __syncthreads();
+    // per expert: exclusive prefix over the warps (in place) and the total
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int32_t run = 0;
+        for (int w = 0; w < kSmallUnits; ++w) {
+            const int32_t c = cnt[w][e];
+            cnt[w][e] = run;
+            run += c;
+        }
+        eoff[e] = run;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int32_t run = 0;
+        for (int e = 0; e < E; ++e) {
+            const int32_t c = eoff[e];
+            counts[e] = c;
+            offsets[e] = run;
+            eoff[e] = run;
+            run += c;
+        }
+        offsets[E] = run;
+    }
+    __syncthreads();
+    for (int e = lane; e < E; e += 32) cnt[warp][e] += eoff[e];
+    __syncwarp();
+    const unsigned lower = (1u << lane) - 1u;
+    for (int it = 0; it < kIters; ++it) {
+        const int64_t i = base + it * 32 + lane;
+        int e = -1;
+        if (i < R) {
+            e = __ldg(te + i);
+            if (e < 0 || e >= E) e = -1;
+        }
+        const unsigned peers = __match_any_sync(0xffffffffu, e);
+        int32_t slot = -1;
+        if (e >= 0) slot = cnt[warp][e] + __popc(peers & lower);
+        __syncwarp();
+        if (e >= 0 && lane == __ffs(peers) - 1) cnt[warp][e] += __popc(peers);
+        __syncwarp();
+        if (i < R) {
+            sparse_rows[i] = slot;
+            if (slot >= 0) sorted_rows[slot] = (int32_t)i;
+        }
+    }
+}
+
 }  // namespace
 
 size_t map_scratch_bytes(int64_t R, int32_t E) {
@@ -155,6 +234,12 @@ int launch_sparse_map(const int32_t *te, int64_t R, int32_t E, int32_t *counts, 
     const int64_t units = (R + kUnit - 1) / kUnit;
     const int64_t blocks = (units + kWarpsPerBlock - 1) / kWarpsPerBlock;
     int n = 0;
+    if (units <= kSmallUnits) {
+        map_small_kernel<<<1, kSmallUnits * 32, 0, s>>>(te, R, E, counts, offsets, sparse_rows,
+                                                         sorted_rows, status);
+        if (n_launch) *n_launch += 1;
+        return 0;
+    }
     if (blocks > 0) {
         map_count_kernel<<<(unsigned)blocks, kWarpsPerBlock * 32, 0, s>>>(te, R, E, units,
                                                                           scratch, status);

@@ -43,5 +43,10 @@ def test_launch_counts(moe):
     w = W.custom("cnt", S=100, D=64, F=64, E=4, k=2)
     inp = {k: (v.cuda() if v is not None else None) for k, v in W.make_inputs(w).items()}
     moe.mlp_forward(inp["x"], inp["w_gate"], inp["w_gate_e"], inp["w_up"], inp["w_down"], w.k)
+    # zero, route, one-block map (S*k <= 16384 routes), GEMM1, GEMM2
+    assert moe.last_launch_count() == 5
+    w = W.custom("cnt2", S=9000, D=64, F=64, E=4, k=2)
+    inp = {k: (v.cuda() if v is not None else None) for k, v in W.make_inputs(w).items()}
+    moe.mlp_forward(inp["x"], inp["w_gate"], inp["w_gate_e"], inp["w_up"], inp["w_down"], w.k)
     # zero, route, map count / scan / assign, GEMM1, GEMM2
     assert moe.last_launch_count() == 7
