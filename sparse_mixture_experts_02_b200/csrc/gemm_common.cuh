@@ -30,6 +30,7 @@ struct SmemTail {
     int abort;
     int32_t off[MAX_E + 1];
     int32_t tstart[MAX_E + 1];
+    float stage[4][32 * 33];  // per epilogue warp: 32 rows x 32 columns (+1 pad) of one chunk
 };
 constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + sizeof(SmemTail);
 
@@ -100,14 +101,45 @@ __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + __expf(-z)
 // Epilogue of one accumulator row (the calling thread's TMEM lane) of a 128 x 256 tile:
 //   GLU:      h = silu(acc[:, c]) * acc[:, 128 + c] (* g), rounded to the output dtype, stored
 //             at out[orow, n0 + c] for the 128 output columns c;
-//   SCATTER:  out[orow, n0 + c] += g * acc[:, c] with fp32 vector atomics (256 columns);
+//   SCATTER:  out[orow, n0 + c] += g * acc[:, c] with fp32 vector atomics (256 columns),
+//             through the warp's `stage` buffer (32 x 33 floats of shared memory);
 //   else:     out[orow, n0 + c] = g * acc[:, c] in the output dtype (256 columns).
 // Columns at or past N are skipped (N is a multiple of 8). `valid` is false for rows past the
-// tile's end; every lane still takes part in the warp-wide TMEM loads.
+// tile's end; every lane of the warp calls this together (warp-wide TMEM loads and shuffles).
 template <bool BF16, bool GLU, bool SCATTER>
 __device__ __forceinline__ void epilogue_row(const KParams &p, uint32_t tbase, bool valid,
-                                             int64_t orow, float g, int n0) {
+                                             int64_t orow, float g, int n0, float *stage) {
     constexpr int OUT_COLS = GLU ? BN / 2 : BN;
+    if constexpr (SCATTER && !GLU) {
+        // The warp's 32 rows x 32 columns of each chunk go through shared memory (row stride
+        // 33 floats: conflict-free both ways), so that each red.global.add.v4.f32 instruction
+        // covers 4 rows x 128 contiguous bytes of out instead of 16 bytes in each of 32 rows.
+        const int lane = threadIdx.x & 31;
+        const int rsub = lane >> 3, cc = (lane & 7) * 4;
+#pragma unroll 1
+        for (int c = 0; c < OUT_COLS / 32; ++c) {
+            uint32_t av[32];
+            dev::tmem_ld32(tbase + c * 32, av);
+            dev::tmem_ld_wait();
+            const int col0 = n0 + c * 32;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) stage[lane * 33 + j] = g * __uint_as_float(av[j]);
+            __syncwarp();
+#pragma unroll
+            for (int pass = 0; pass < 8; ++pass) {
+                const int rr = pass * 4 + rsub;
+                const bool rv = __shfl_sync(0xffffffffu, valid, rr);
+                const long long ro = __shfl_sync(0xffffffffu, (long long)orow, rr);
+                if (rv && col0 + cc < p.N) {
+                    const float *sv = stage + rr * 33 + cc;
+                    dev::red_add_v4(reinterpret_cast<float *>(p.out) + ro * p.N + col0 + cc,
+                                    sv[0], sv[1], sv[2], sv[3]);
+                }
+            }
+            __syncwarp();
+        }
+        return;
+    }
     if constexpr (GLU) {
 #pragma unroll 1
         for (int c = 0; c < OUT_COLS / 32; ++c) {
@@ -156,16 +188,7 @@ __device__ __forceinline__ void epilogue_row(const KParams &p, uint32_t tbase, b
             dev::tmem_ld_wait();
             const int col0 = n0 + c * 32;
             if (valid && col0 < p.N) {
-                if (SCATTER) {
-                    float *dst = reinterpret_cast<float *>(p.out) + orow * p.N + col0;
-#pragma unroll
-                    for (int v = 0; v < 8; ++v)
-                        if (col0 + v * 4 < p.N)
-                            dev::red_add_v4(dst + v * 4, g * __uint_as_float(av[v * 4]),
-                                            g * __uint_as_float(av[v * 4 + 1]),
-                                            g * __uint_as_float(av[v * 4 + 2]),
-                                            g * __uint_as_float(av[v * 4 + 3]));
-                } else if (BF16) {
+                if (BF16) {
                     __nv_bfloat16 *dst =
                         reinterpret_cast<__nv_bfloat16 *>(p.out) + orow * p.N + col0;
 #pragma unroll

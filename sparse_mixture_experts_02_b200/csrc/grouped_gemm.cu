@@ -56,6 +56,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     constexpr int B_KSTEP = (32 / EB) * KBYTES;  // bytes of B per MMA K step (32 bytes of K)
     constexpr int OUT_COLS = GLU ? BN / 2 : BN;  // output columns per tile
     constexpr uint32_t IDESC = dev::idesc_f32acc(BF16, BM, BN, true);
+    // A tile with at most 64 rows (an expert's short last tile) runs an M=64 MMA: half the tensor
+    // work; its accumulator rows 16j + i (i < 16) sit in TMEM lanes 32j + i.
+    constexpr uint32_t IDESC64 = dev::idesc_f32acc(BF16, 64, BN, true);
     // B (weights, N contiguous) is MN-major: 128-byte swizzle for bf16 (8-row atoms of 1024 B);
     // tf32 needs the 32-byte-unit variant (4-row atoms of 512 B).
     constexpr uint32_t B_LAYOUT = BF16 ? dev::kLayoutSw128 : dev::kLayoutSw128Base32;
@@ -186,6 +189,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     break;
                 dev::tc_fence_after();
                 const uint32_t d_tmem = tmem_base + b * BN;
+                uint32_t tile_idesc = idesc;
+                if (!ROUTER && decode_tile<BM>(t, st.off, st.tstart, E_sched).rows <= 64)
+                    tile_idesc = IDESC64;
                 for (int kb = 0; kb < p.num_kb; ++kb) {
                     if (!dev::mbar_wait(&st.full[s], ph, abort, p.status, p.wait_limit_ns,
                                         kKernelGemm)) {
@@ -201,8 +207,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const uint64_t ad =
                             dev::sdesc(sA + kk * 32, 16, 1024, dev::kLayoutSw128);
                         const uint64_t bd = dev::sdesc(sB + kk * B_KSTEP, CHUNK, B_SBO, B_LAYOUT);
-                        if (BF16) dev::mma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0);
-                        else dev::mma_tf32(d_tmem, ad, bd, idesc, (kb | kk) != 0);
+                        if (BF16) dev::mma_bf16(d_tmem, ad, bd, tile_idesc, (kb | kk) != 0);
+                        else dev::mma_tf32(d_tmem, ad, bd, tile_idesc, (kb | kk) != 0);
                     }
                     dev::mma_commit(&st.empty[s]);
                     if (++s == STAGES) {
@@ -232,6 +238,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         bool ok = true;
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
             const TileInfo ti = decode_tile<BM>(t, st.off, st.tstart, E_sched);
+            const bool half = ti.rows <= 64;  // M=64 tile: the MMA reads rows 0-63 only
             const uint8_t *src[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
@@ -257,7 +264,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                 for (int i = 0; i < 8; ++i) {
                     const int r = gw * 32 + i * 4 + rsub;
                     const uint32_t dst = sA + r * KBYTES + ((chunk ^ (r & 7)) << 4);
-                    dev::cp_async16(dst, nbytes ? src[i] + cb : src[i], nbytes);
+                    if (r < 64 || !half) dev::cp_async16(dst, nbytes ? src[i] + cb : src[i], nbytes);
                 }
                 dev::cp_async_arrive_noinc(&st.full[s]);
                 if (++s == STAGES) {
@@ -270,7 +277,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     } else {
         // ------------------------------------------------------------------ epilogue
         const int q = warp & 3;  // TMEM lane quarter this warp may access
-        const int r = q * 32 + lane;
+        const int r_full = q * 32 + lane;
+        const int r_half = lane < 16 ? q * 16 + lane : BM;  // M=64 layout; BM = no row
         int it = 0;
         for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
             const TileInfo ti = decode_tile<BM>(t, st.off, st.tstart, E_sched);
@@ -282,6 +290,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             w = __shfl_sync(0xffffffffu, w, 0);
             if (!w) break;
             dev::tc_fence_after();
+            const int r = (!ROUTER && ti.rows <= 64) ? r_half : r_full;
             const int prow = ti.row_begin + r;
             bool valid = r < ti.rows && prow >= 0 && prow < p.R;
             int64_t orow = prow;
@@ -345,7 +354,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     }
                 }
             } else {
-                epilogue_row<BF16, GLU, SCATTER>(p, tbase, valid, orow, g, n0);
+                epilogue_row<BF16, GLU, SCATTER>(p, tbase, valid, orow, g, n0, st.stage[q]);
             }
             dev::tc_fence_before();
             __syncwarp();

@@ -48,6 +48,7 @@ struct Smem2 {
     int abort;
     int32_t off[MAX_E + 1];
     int32_t tstart[MAX_E + 1];
+    float stage[4][32 * 33];  // scatter epilogue staging, one buffer per epilogue warp
 };
 constexpr size_t SMEM2_BYTES = 1024 + (size_t)ST2 * STAGE2_BYTES + sizeof(Smem2);
 
@@ -315,7 +316,7 @@ grouped_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
             }
             const int n0 = ti.n_idx * OUT_COLS;
             const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + b * BN;
-            epilogue_row<BF16, GLU, SCATTER>(p, tbase, valid, orow, g, n0);
+            epilogue_row<BF16, GLU, SCATTER>(p, tbase, valid, orow, g, n0, st.stage[q]);
             dev::tc_fence_before();
             __syncwarp();
             if (lane == 0) dev::mbar_arrive_cluster(tempty0_base + b * (uint32_t)sizeof(uint64_t));

@@ -39,6 +39,8 @@ map_count_kernel(const int32_t *__restrict__ te, int64_t R, int32_t E, int64_t u
     __syncwarp();
     bool bad = false;
     const int64_t base = u * kUnit;
+    int ev[kIters];
+#pragma unroll
     for (int it = 0; it < kIters; ++it) {
         const int64_t i = base + it * 32 + lane;
         int e = -1;
@@ -49,6 +51,11 @@ map_count_kernel(const int32_t *__restrict__ te, int64_t R, int32_t E, int64_t u
                 e = -1;
             }
         }
+        ev[it] = e;
+    }
+#pragma unroll
+    for (int it = 0; it < kIters; ++it) {
+        const int e = ev[it];
         const unsigned peers = __match_any_sync(0xffffffffu, e);
         const int leader = __ffs(peers) - 1;
         if (e >= 0 && lane == leader) cnt[warp][e] += __popc(peers);
@@ -122,6 +129,8 @@ map_assign_kernel(const int32_t *__restrict__ te, int64_t R, int32_t E, int64_t 
     __syncwarp();
     const unsigned lower = (1u << lane) - 1u;
     const int64_t base = u * kUnit;
+    int ev[kIters];
+#pragma unroll
     for (int it = 0; it < kIters; ++it) {
         const int64_t i = base + it * 32 + lane;
         int e = -1;
@@ -129,6 +138,12 @@ map_assign_kernel(const int32_t *__restrict__ te, int64_t R, int32_t E, int64_t 
             e = __ldg(te + i);
             if (e < 0 || e >= E) e = -1;
         }
+        ev[it] = e;
+    }
+#pragma unroll
+    for (int it = 0; it < kIters; ++it) {
+        const int64_t i = base + it * 32 + lane;
+        const int e = ev[it];
         const unsigned peers = __match_any_sync(0xffffffffu, e);
         int32_t slot = -1;
         if (e >= 0) slot = cnt[warp][e] + __popc(peers & lower);
@@ -158,7 +173,10 @@ map_small_kernel(const int32_t *__restrict__ te, int64_t R, int32_t E,
     for (int e = lane; e < E; e += 32) cnt[warp][e] = 0;
     __syncwarp();
     const int64_t base = (int64_t)warp * kUnit;
+    // all of this lane's routes at once: kIters independent loads instead of a dependent chain
+    int ev[kIters];
     bool bad = false;
+#pragma unroll
     for (int it = 0; it < kIters; ++it) {
         const int64_t i = base + it * 32 + lane;
         int e = -1;
@@ -169,6 +187,11 @@ map_small_kernel(const int32_t *__restrict__ te, int64_t R, int32_t E,
                 e = -1;
             }
         }
+        ev[it] = e;
+    }
+#pragma unroll
+    for (int it = 0; it < kIters; ++it) {
+        const int e = ev[it];
         const unsigned peers = __match_any_sync(0xffffffffu, e);
         if (e >= 0 && lane == __ffs(peers) - 1) cnt[warp][e] += __popc(peers);
         __syncwarp();
@@ -201,13 +224,10 @@ map_small_kernel(const int32_t *__restrict__ te, int64_t R, int32_t E,
     for (int e = lane; e < E; e += 32) cnt[warp][e] += eoff[e];
     __syncwarp();
     const unsigned lower = (1u << lane) - 1u;
+#pragma unroll
     for (int it = 0; it < kIters; ++it) {
         const int64_t i = base + it * 32 + lane;
-        int e = -1;
-        if (i < R) {
-            e = __ldg(te + i);
-            if (e < 0 || e >= E) e = -1;
-        }
+        const int e = ev[it];
         const unsigned peers = __match_any_sync(0xffffffffu, e);
         int32_t slot = -1;
         if (e >= 0) slot = cnt[warp][e] + __popc(peers & lower);
