@@ -329,8 +329,13 @@ int moe_mlp_forward(const void *x, const void *w_gate, const float *logit_bias,
     int n = 0;
 
     record_prof(0, s);
-    n += launch_zero_f32(out, S * D, status, s);
-    if ((rc = check_launch("zero"))) return rc;
+    // The router clears the status word (its first kernel); GEMM1's epilogue warps zero `out`
+    // while they wait for their first tile. With no routes there is no GEMM: a small kernel does
+    // both.
+    if (R == 0) {
+        n += launch_zero_f32(out, S * D, status, s);
+        if ((rc = check_launch("zero"))) return rc;
+    }
     {
         const int nr = launch_route(x, w_gate, logit_bias, S, D, E, k, dt == MOE_BF16, top_e,
                                     top_w, status, s);
@@ -363,6 +368,8 @@ int moe_mlp_forward(const void *x, const void *w_gate, const float *logit_bias,
         a.gather = true;
         a.glu = true;
         a.scatter = false;
+        a.zero_ptr = out;   // zeroed by GEMM1's epilogue warps before GEMM2 adds into it
+        a.zero_n = S * D;
         a.status = status;
         a.wait_limit_ns = kWaitLimitNs;
         if ((rc = prefer_2sm(R, E, true) ? launch_grouped_gemm_2sm(a, s) : launch_grouped_gemm(a, s)))
@@ -371,6 +378,8 @@ int moe_mlp_forward(const void *x, const void *w_gate, const float *logit_bias,
         ++n;
         record_prof(3, s);
         GemmArgs b = a;
+        b.zero_ptr = nullptr;
+        b.zero_n = 0;
         b.A = h;
         b.a_rows = R;
         b.B0 = w_down;

@@ -10,6 +10,8 @@ namespace gemm {
 constexpr int BM = 128;                 // rows per tile (TMEM lanes)
 constexpr int BN = 256;                 // MMA N = accumulator columns
 constexpr int STAGES = 4;
+constexpr int MAX_STAGES = 8;           // router mode: up to 8 smaller stages in the same space
+constexpr size_t STAGE_AREA = (size_t)STAGES * (128 * 128 + 256 * 128);
 constexpr int KBYTES = 128;             // bytes of K per stage (one 128-byte swizzle row)
 constexpr int A_BYTES = BM * KBYTES;    // 16 KB
 constexpr int B_BYTES = BN * KBYTES;    // 32 KB (BN columns x (128 / eb) K rows x eb)
@@ -21,8 +23,8 @@ constexpr uint32_t TMEM_COLS = 512;
 
 // Shared-memory bookkeeping of the one-CTA kernel (after its STAGES operand stages).
 struct SmemTail {
-    uint64_t full[STAGES];
-    uint64_t empty[STAGES];
+    uint64_t full[MAX_STAGES];
+    uint64_t empty[MAX_STAGES];
     uint64_t tfull[2];
     uint64_t tempty[2];
     uint64_t drain;
@@ -32,7 +34,7 @@ struct SmemTail {
     int32_t tstart[MAX_E + 1];
     float stage[4][32 * 33];  // per epilogue warp: 32 rows x 32 columns (+1 pad) of one chunk
 };
-constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + sizeof(SmemTail);
+constexpr size_t SMEM_BYTES = 1024 + STAGE_AREA + sizeof(SmemTail);
 
 struct KParams {
     const void *A;    // gathered mode: x [S, K] (rows fetched by the gather warps)
@@ -51,6 +53,11 @@ struct KParams {
     int32_t *top_e;
     float *top_w;
     int32_t b_chunks; // B chunks loaded per stage (router: ceil(E / chunk width))
+    int32_t stages;   // router mode: pipeline depth and stage size (bytes, multiple of 1024)
+    int32_t stage_bytes;
+    // optional side job of the epilogue warps before their first tile: zero zero_n4 float4s
+    float4 *zero_ptr;
+    int64_t zero_n4;
     unsigned *status;
     int64_t wait_limit_ns;
 };
@@ -106,6 +113,16 @@ __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + __expf(-z)
 //   else:     out[orow, n0 + c] = g * acc[:, c] in the output dtype (256 columns).
 // Columns at or past N are skipped (N is a multiple of 8). `valid` is false for rows past the
 // tile's end; every lane of the warp calls this together (warp-wide TMEM loads and shuffles).
+// The epilogue warps are idle until the first accumulator of the CTA is ready; the MoE forward
+// has them zero its fp32 output there (GEMM2 scatter-adds into it only after GEMM1 has ended).
+__device__ __forceinline__ void zero_side_job(const KParams &p, int epi_thread, int epi_threads) {
+    if (p.zero_ptr == nullptr) return;
+    const int64_t stride = (int64_t)gridDim.x * epi_threads;
+    const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int64_t i = (int64_t)blockIdx.x * epi_threads + epi_thread; i < p.zero_n4; i += stride)
+        p.zero_ptr[i] = z;
+}
+
 template <bool BF16, bool GLU, bool SCATTER>
 __device__ __forceinline__ void epilogue_row(const KParams &p, uint32_t tbase, bool valid,
                                              int64_t orow, float g, int n0, float *stage) {

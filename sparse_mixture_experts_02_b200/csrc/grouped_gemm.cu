@@ -68,13 +68,18 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    SmemTail &st = *reinterpret_cast<SmemTail *>(smem + (size_t)STAGES * STAGE_BYTES);
+    SmemTail &st = *reinterpret_cast<SmemTail *>(smem + STAGE_AREA);
+    // the router's B is only ceil(E/64) chunks: it runs more, smaller stages in the same space
+    const int nst = ROUTER ? p.stages : STAGES;
+    const size_t sbytes = ROUTER ? (size_t)p.stage_bytes : (size_t)STAGE_BYTES;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int E = p.E;
+    // the router is the forward's first kernel: it clears the status word
+    if (ROUTER && blockIdx.x == 0 && threadIdx.x == 0 && p.status != nullptr) *p.status = 0u;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
+        for (int s = 0; s < nst; ++s) {
             // full: the TMA thread's expect_tx arrival (+ one cp.async arrival per gatherer)
             dev::mbar_init(&st.full[s], GATHER ? 1 + GATHER_THREADS : 1);
             dev::mbar_init(&st.empty[s], 1);
@@ -139,7 +144,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     ok = false;
                     break;
                 }
-                uint8_t *sA = smem + (size_t)s * STAGE_BYTES;
+                uint8_t *sA = smem + (size_t)s * sbytes;
                 uint8_t *sB = sA + A_BYTES;
                 if (lane == 0) dev::mbar_arrive_expect_tx(&st.full[s], stage_tx);
                 __syncwarp();
@@ -162,7 +167,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                 }
                 issued |= 1u << s;
                 last_par = (last_par & ~(1u << s)) | (ph << s);
-                if (++s == STAGES) {
+                if (++s == (uint32_t)nst) {
                     s = 0;
                     ph ^= 1u;
                 }
@@ -170,7 +175,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         }
         // teardown: every load this warp issued must land before the CTA may exit
         if (lane == 0) {
-            for (int s2 = 0; s2 < STAGES; ++s2)
+            for (int s2 = 0; s2 < nst; ++s2)
                 if (issued & (1u << s2))
                     dev::mbar_wait(&st.full[s2], (last_par >> s2) & 1u, nullptr, p.status,
                                    kDrainLimitNs, kKernelGemm);
@@ -200,7 +205,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     }
                     dev::tc_fence_after();
                     if (GATHER) dev::fence_proxy_async_smem();  // cp.async rows -> tensor core
-                    const uint32_t sA = dev::smem_u32(smem + (size_t)s * STAGE_BYTES);
+                    const uint32_t sA = dev::smem_u32(smem + (size_t)s * sbytes);
                     const uint32_t sB = sA + A_BYTES;
 #pragma unroll
                     for (int kk = 0; kk < KBYTES / 32; ++kk) {
@@ -211,7 +216,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         else dev::mma_tf32(d_tmem, ad, bd, tile_idesc, (kb | kk) != 0);
                     }
                     dev::mma_commit(&st.empty[s]);
-                    if (++s == STAGES) {
+                    if (++s == (uint32_t)nst) {
                         s = 0;
                         ph ^= 1u;
                     }
@@ -257,7 +262,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     ok = false;
                     break;
                 }
-                const uint32_t sA = dev::smem_u32(smem + (size_t)s * STAGE_BYTES);
+                const uint32_t sA = dev::smem_u32(smem + (size_t)s * sbytes);
                 const int64_t cb = (int64_t)kb * KBYTES + chunk * 16;
                 const uint32_t nbytes = cb < row_bytes ? 16u : 0u;  // zero-fill past K
 #pragma unroll
@@ -267,7 +272,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     if (r < 64 || !half) dev::cp_async16(dst, nbytes ? src[i] + cb : src[i], nbytes);
                 }
                 dev::cp_async_arrive_noinc(&st.full[s]);
-                if (++s == STAGES) {
+                if (++s == (uint32_t)nst) {
                     s = 0;
                     ph ^= 1u;
                 }
@@ -276,6 +281,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         dev::cp_async_wait_all();
     } else {
         // ------------------------------------------------------------------ epilogue
+        zero_side_job(p, threadIdx.x - 64, 128);
         const int q = warp & 3;  // TMEM lane quarter this warp may access
         const int r_full = q * 32 + lane;
         const int r_half = lane < 16 ? q * 16 + lane : BM;  // M=64 layout; BM = no row
@@ -482,6 +488,16 @@ int launch_t(const GemmArgs &a, cudaStream_t s) {
     kp.top_e = a.top_e;
     kp.top_w = a.top_w;
     kp.b_chunks = (int32_t)((a.N + CW - 1) / CW);
+    if (ROUTER) {
+        kp.stage_bytes = A_BYTES + kp.b_chunks * BK * KBYTES;
+        kp.stages = (int32_t)(STAGE_AREA / (size_t)kp.stage_bytes);
+        if (kp.stages > MAX_STAGES) kp.stages = MAX_STAGES;
+    } else {
+        kp.stage_bytes = STAGE_BYTES;
+        kp.stages = STAGES;
+    }
+    kp.zero_ptr = reinterpret_cast<float4 *>(a.zero_ptr);
+    kp.zero_n4 = a.zero_n / 4;
     kp.status = a.status;
     kp.wait_limit_ns = a.wait_limit_ns;
     kern<<<num_sms(), GATHER ? THREADS + GATHER_THREADS : THREADS, SMEM_BYTES, s>>>(mA, mB0, mB1,

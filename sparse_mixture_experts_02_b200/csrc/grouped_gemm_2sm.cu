@@ -289,6 +289,7 @@ grouped_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
         dev::cp_async_wait_all();
     } else {
         // ------------------------------------------------------------------ epilogue
+        zero_side_job(p, threadIdx.x - 64, 128);
         const int q = warp & 3;
         const int r = q * 32 + lane;
         const uint32_t tempty0_base = dev::mapa_shared(dev::smem_u32(&st.tempty[0]), 0);
@@ -383,6 +384,8 @@ int launch_2sm_t(const GemmArgs &a, cudaStream_t s, int n_pairs) {
     kp.n_tiles = (int32_t)((a.N + OUT_COLS - 1) / OUT_COLS);
     kp.S = a.S;
     kp.R = a.R;
+    kp.zero_ptr = reinterpret_cast<float4 *>(a.zero_ptr);
+    kp.zero_n4 = a.zero_n / 4;
     kp.status = a.status;
     kp.wait_limit_ns = a.wait_limit_ns;
     kern<<<2 * n_pairs, GATHER ? THREADS + GATHER_THREADS : THREADS, SMEM2_BYTES, s>>>(mA, mB0,

@@ -56,6 +56,8 @@ struct GemmArgs {
     const float *bias;      // router mode only
     int32_t *top_e;
     float *top_w;
+    float *zero_ptr;        // nullable: fp32 buffer (16-byte aligned) the epilogue warps zero
+    int64_t zero_n;         // its length (a multiple of 4)
     unsigned *status;
     int64_t wait_limit_ns;
 };

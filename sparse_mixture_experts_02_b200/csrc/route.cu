@@ -37,8 +37,9 @@ template <int NJ, bool BF16>
 __global__ void __launch_bounds__(kWarps * 32)
 route_kernel(const void *__restrict__ x, const void *__restrict__ w_gate,
              const float *__restrict__ bias, int64_t S, int64_t D, int32_t E, int32_t k,
-             int32_t *__restrict__ top_e, float *__restrict__ top_w) {
+             int32_t *__restrict__ top_e, float *__restrict__ top_w, unsigned *status) {
     __shared__ __align__(16) float xs[kWarps][kTokPerWarp][kChunk];
+    if (status != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *status = 0u;  // first kernel
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t tok0 = ((int64_t)blockIdx.x * kWarps + warp) * kTokPerWarp;
     if (tok0 >= S) return;
@@ -153,8 +154,9 @@ template <int NE, bool BF16>
 __global__ void __launch_bounds__(128)
 route_small_kernel(const void *__restrict__ x, const void *__restrict__ w_gate,
                    const float *__restrict__ bias, int64_t D, int32_t E, int32_t k,
-                   int32_t *__restrict__ top_e, float *__restrict__ top_w) {
+                   int32_t *__restrict__ top_e, float *__restrict__ top_w, unsigned *status) {
     __shared__ float part[4][NE];
+    if (status != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *status = 0u;  // first kernel
     const int64_t s = blockIdx.x;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     float acc[NE];
@@ -162,14 +164,47 @@ route_small_kernel(const void *__restrict__ x, const void *__restrict__ w_gate,
     for (int e = 0; e < NE; ++e) acc[e] = 0.f;
     for (int64_t d0 = (int64_t)tid * 8; d0 < D; d0 += 1024) {
         float xv[8];
+        if constexpr (BF16) {
+            // 8 consecutive bf16 of x in one 16-byte load (D % 8 == 0, rows 16-byte aligned)
+            const uint4 q = __ldg(reinterpret_cast<const uint4 *>(
+                reinterpret_cast<const __nv_bfloat16 *>(x) + s * D + d0));
+            const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&q);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) xv[j] = ld_elem<BF16>(x, s * D + d0 + j);  // D % 8 == 0
+            for (int j = 0; j < 4; ++j) {
+                const float2 f = __bfloat1622float2(h2[j]);
+                xv[2 * j] = f.x;
+                xv[2 * j + 1] = f.y;
+            }
+        } else {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int64_t row = (d0 + j) * (int64_t)E;
+            for (int j = 0; j < 8; ++j) xv[j] = ld_elem<BF16>(x, s * D + d0 + j);
+        }
+        if (BF16 && NE == E) {  // E in {8, 16, 32, 64}: whole 16-byte row pieces
+            // rows d0 .. d0+7 of W_gate are 8*E contiguous bf16: E 16-byte loads
 #pragma unroll
-            for (int e = 0; e < NE; ++e)
-                if (e < E) acc[e] = fmaf(xv[j], ld_elem<BF16>(w_gate, row + e), acc[e]);
+            for (int j = 0; j < 8; ++j) {
+                const uint4 *wr = reinterpret_cast<const uint4 *>(
+                    reinterpret_cast<const __nv_bfloat16 *>(w_gate) + (d0 + j) * (int64_t)E);
+#pragma unroll
+                for (int c = 0; c < NE / 8; ++c) {
+                    const uint4 q = __ldg(wr + c);
+                    const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&q);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const float2 f = __bfloat1622float2(h2[u]);
+                        acc[c * 8 + 2 * u] = fmaf(xv[j], f.x, acc[c * 8 + 2 * u]);
+                        acc[c * 8 + 2 * u + 1] = fmaf(xv[j], f.y, acc[c * 8 + 2 * u + 1]);
+                    }
+                }
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int64_t row = (d0 + j) * (int64_t)E;
+#pragma unroll
+                for (int e = 0; e < NE; ++e)
+                    if (e < E) acc[e] = fmaf(xv[j], ld_elem<BF16>(w_gate, row + e), acc[e]);
+            }
         }
     }
 #pragma unroll
@@ -235,13 +270,13 @@ route_small_kernel(const void *__restrict__ x, const void *__restrict__ w_gate,
 template <int NE>
 void launch_route_small_ne(const void *x, const void *w_gate, const float *bias, int64_t S,
                            int64_t D, int32_t E, int32_t k, bool bf16, int32_t *top_e,
-                           float *top_w, cudaStream_t s) {
+                           float *top_w, unsigned *status, cudaStream_t s) {
     if (bf16)
         route_small_kernel<NE, true><<<(unsigned)S, 128, 0, s>>>(x, w_gate, bias, D, E, k, top_e,
-                                                                 top_w);
+                                                                 top_w, status);
     else
         route_small_kernel<NE, false><<<(unsigned)S, 128, 0, s>>>(x, w_gate, bias, D, E, k,
-                                                                  top_e, top_w);
+                                                                  top_e, top_w, status);
 }
 
 __global__ void zero_kernel(float4 *__restrict__ p, int64_t n4, float *__restrict__ tail,
@@ -256,16 +291,17 @@ __global__ void zero_kernel(float4 *__restrict__ p, int64_t n4, float *__restric
 template <int NJ>
 int launch_route_nj(const void *x, const void *w_gate, const float *bias, int64_t S, int64_t D,
                     int32_t E, int32_t k, bool bf16, int32_t *top_e, float *top_w,
-                    cudaStream_t s) {
+                    unsigned *status, cudaStream_t s) {
     const int64_t per_block = (int64_t)kWarps * kTokPerWarp;
     const int64_t blocks = (S + per_block - 1) / per_block;
     if (blocks == 0) return 0;
     if (bf16)
         route_kernel<NJ, true><<<(unsigned)blocks, kWarps * 32, 0, s>>>(x, w_gate, bias, S, D, E,
-                                                                        k, top_e, top_w);
+                                                                        k, top_e, top_w, status);
     else
         route_kernel<NJ, false><<<(unsigned)blocks, kWarps * 32, 0, s>>>(x, w_gate, bias, S, D,
-                                                                         E, k, top_e, top_w);
+                                                                         E, k, top_e, top_w,
+                                                                         status);
     return 1;
 }
 
@@ -278,10 +314,10 @@ int launch_route(const void *x, const void *w_gate, const float *bias, int64_t S
     // Few experts and a batch too small to fill the SMs with 128-token tensor-core tiles (or fp32
     // inputs): one block per token on the CUDA cores, exact fp32 accumulation.
     if (E <= 64 && (S <= 2048 || !bf16) && S < (int64_t(1) << 31)) {
-        if (E <= 8) launch_route_small_ne<8>(x, w_gate, bias, S, D, E, k, bf16, top_e, top_w, s);
-        else if (E <= 16) launch_route_small_ne<16>(x, w_gate, bias, S, D, E, k, bf16, top_e, top_w, s);
-        else if (E <= 32) launch_route_small_ne<32>(x, w_gate, bias, S, D, E, k, bf16, top_e, top_w, s);
-        else launch_route_small_ne<64>(x, w_gate, bias, S, D, E, k, bf16, top_e, top_w, s);
+        if (E <= 8) launch_route_small_ne<8>(x, w_gate, bias, S, D, E, k, bf16, top_e, top_w, status, s);
+        else if (E <= 16) launch_route_small_ne<16>(x, w_gate, bias, S, D, E, k, bf16, top_e, top_w, status, s);
+        else if (E <= 32) launch_route_small_ne<32>(x, w_gate, bias, S, D, E, k, bf16, top_e, top_w, status, s);
+        else launch_route_small_ne<64>(x, w_gate, bias, S, D, E, k, bf16, top_e, top_w, status, s);
         return 1;
     }
     // bf16 with E a multiple of 8 (16-byte W_gate rows for TMA): tensor-core router.
@@ -291,10 +327,10 @@ int launch_route(const void *x, const void *w_gate, const float *bias, int64_t S
             return -1;
         return 1;
     }
-    if (E <= 32) return launch_route_nj<1>(x, w_gate, bias, S, D, E, k, bf16, top_e, top_w, s);
-    if (E <= 64) return launch_route_nj<2>(x, w_gate, bias, S, D, E, k, bf16, top_e, top_w, s);
-    if (E <= 128) return launch_route_nj<4>(x, w_gate, bias, S, D, E, k, bf16, top_e, top_w, s);
-    return launch_route_nj<8>(x, w_gate, bias, S, D, E, k, bf16, top_e, top_w, s);
+    if (E <= 32) return launch_route_nj<1>(x, w_gate, bias, S, D, E, k, bf16, top_e, top_w, status, s);
+    if (E <= 64) return launch_route_nj<2>(x, w_gate, bias, S, D, E, k, bf16, top_e, top_w, status, s);
+    if (E <= 128) return launch_route_nj<4>(x, w_gate, bias, S, D, E, k, bf16, top_e, top_w, status, s);
+    return launch_route_nj<8>(x, w_gate, bias, S, D, E, k, bf16, top_e, top_w, status, s);
 }
 
 int launch_zero_f32(float *p, int64_t n, unsigned *status, cudaStream_t s) {

@@ -43,10 +43,22 @@ def test_launch_counts(moe):
     w = W.custom("cnt", S=100, D=64, F=64, E=4, k=2)
     inp = {k: (v.cuda() if v is not None else None) for k, v in W.make_inputs(w).items()}
     moe.mlp_forward(inp["x"], inp["w_gate"], inp["w_gate_e"], inp["w_up"], inp["w_down"], w.k)
-    # zero, route, one-block map (S*k <= 16384 routes), GEMM1, GEMM2
-    assert moe.last_launch_count() == 5
+    # route, one-block map (S*k <= 16384 routes), GEMM1 (also zeroes out), GEMM2
+    assert moe.last_launch_count() == 4
     w = W.custom("cnt2", S=9000, D=64, F=64, E=4, k=2)
     inp = {k: (v.cuda() if v is not None else None) for k, v in W.make_inputs(w).items()}
     moe.mlp_forward(inp["x"], inp["w_gate"], inp["w_gate_e"], inp["w_up"], inp["w_down"], w.k)
-    # zero, route, map count / scan / assign, GEMM1, GEMM2
-    assert moe.last_launch_count() == 7
+    # route, map count / scan / assign, GEMM1, GEMM2
+    assert moe.last_launch_count() == 6
+
+
+@pytest.mark.parametrize("S,E", [(100, 4), (3000, 64), (600, 96)])
+def test_forward_clears_a_stale_status(moe, S, E):
+    # the forward's first kernel (whichever router runs) clears the status word in the workspace
+    w = W.custom("stale", S=S, D=64, F=64, E=E, k=2, router_std="1/sqrt(D)")
+    inp = {k: (v.cuda() if v is not None else None) for k, v in W.make_inputs(w).items()}
+    wsf = moe.ForwardWorkspace(w.S, w.D, w.F, w.E, w.k, torch.bfloat16, torch.device("cuda"))
+    wsf.buf[:4].view(torch.int32).fill_(2)  # a timeout flag left over from an earlier call
+    moe.mlp_forward(inp["x"], inp["w_gate"], inp["w_gate_e"], inp["w_up"], inp["w_down"], w.k,
+                    ws=wsf)
+    moe.check_device_status(wsf)
