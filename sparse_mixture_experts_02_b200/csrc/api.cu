@@ -25,13 +25,13 @@ int set_error(int code, const char *fmt, ...) {
     return code;
 }
 
-bool prefer_2sm(int64_t R, int32_t E, bool gather) {
+bool prefer_2sm(int64_t R, int32_t E) {
     const char *env = getenv("MOE_GEMM_2SM");
     if (env != nullptr && (env[0] == '0' || env[0] == '1')) return env[0] == '1';
-    // Pair tiles pay off on contiguous (slot-ordered) A when experts are long enough that the
-    // 256-row tiles waste little. With gathered A the pair kernel measured slower than one CTA
-    // (its cp.async row gather could not keep the pair MMA fed), so gathered GEMMs stay on one CTA.
-    return !gather && E > 0 && R / E >= 384;
+    // Pair tiles pay off, for gathered and slot-ordered A alike, when experts are long enough
+    // that the 256-row tiles waste little (measured: ~1024 and ~1536 rows an expert gain 5-7% on
+    // a forward; ~256 rows an expert lose 5%, ~32 lose 25%).
+    return E > 0 && R / E >= 384;
 }
 
 int num_sms() {
@@ -293,7 +293,7 @@ int moe_scatter_linear(const void *X, const void *W, int64_t S, int64_t Din, int
     a.scatter = scatter_out != 0;
     a.status = status;
     a.wait_limit_ns = kWaitLimitNs;
-    if ((rc = prefer_2sm(R, E, a.gather) ? launch_grouped_gemm_2sm(a, s) : launch_grouped_gemm(a, s)))
+    if ((rc = prefer_2sm(R, E) ? launch_grouped_gemm_2sm(a, s) : launch_grouped_gemm(a, s)))
         return rc;
     g_launches = 1;
     return check_launch("scatter_linear");
@@ -372,7 +372,7 @@ int moe_mlp_forward(const void *x, const void *w_gate, const float *logit_bias,
         a.zero_n = S * D;
         a.status = status;
         a.wait_limit_ns = kWaitLimitNs;
-        if ((rc = prefer_2sm(R, E, true) ? launch_grouped_gemm_2sm(a, s) : launch_grouped_gemm(a, s)))
+        if ((rc = prefer_2sm(R, E) ? launch_grouped_gemm_2sm(a, s) : launch_grouped_gemm(a, s)))
             return rc;
         if ((rc = check_launch("gemm1"))) return rc;
         ++n;
@@ -391,7 +391,7 @@ int moe_mlp_forward(const void *x, const void *w_gate, const float *logit_bias,
         b.gather = false;
         b.glu = false;
         b.scatter = true;
-        if ((rc = prefer_2sm(R, E, false) ? launch_grouped_gemm_2sm(b, s) : launch_grouped_gemm(b, s)))
+        if ((rc = prefer_2sm(R, E) ? launch_grouped_gemm_2sm(b, s) : launch_grouped_gemm(b, s)))
             return rc;
         if ((rc = check_launch("gemm2"))) return rc;
         ++n;

@@ -239,19 +239,42 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         const int rsub = lane >> 3;
         const int64_t row_bytes = (int64_t)p.K * EB;
         const uint8_t *xa = reinterpret_cast<const uint8_t *>(p.A);
-        uint32_t s = 0, ph = 0;
-        bool ok = true;
-        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        // sorted_rows entries of this thread's 8 rows of tile t (tail rows repeat a valid row)
+        auto fetch_rows = [&](int t, int *ent) {
             const TileInfo ti = decode_tile<BM>(t, st.off, st.tstart, E_sched);
-            const bool half = ti.rows <= 64;  // M=64 tile: the MMA reads rows 0-63 only
-            const uint8_t *src[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 const int r = gw * 32 + i * 4 + rsub;
-                const int pr = ti.row_begin + min(r, ti.rows - 1);  // tail rows repeat a valid row
-                const int64_t tok = __ldg(p.sorted_rows + pr) / p.k;
-                src[i] = xa + tok * row_bytes;
+                ent[i] = __ldg(p.sorted_rows + ti.row_begin + min(r, ti.rows - 1));
             }
+        };
+        // x row pointers of tile t from its entries; returns whether it is an M=64 tile (the
+        // MMA then reads rows 0-63 only)
+        auto row_ptrs = [&](int t, const int *ent, const uint8_t **src) {
+            const TileInfo ti = decode_tile<BM>(t, st.off, st.tstart, E_sched);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) src[i] = xa + (int64_t)(ent[i] / p.k) * row_bytes;
+            return ti.rows <= 64;
+        };
+        // Shared memory is saturated by the tensor core, so a tile's schedule lookups, index
+        // loads and divisions take ~2 us: the next tile's pointers are formed after the current
+        // tile's second stage is issued, and its entries are loaded a tile earlier still, so
+        // nothing but a register swap sits between two tiles' copies.
+        const int t0 = blockIdx.x, tstep = gridDim.x;
+        int ent[8];
+        const uint8_t *src[8], *nsrc[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) src[i] = nsrc[i] = xa;
+        bool half = false, nhalf = false;
+        if (t0 < total) {
+            fetch_rows(t0, ent);
+            half = row_ptrs(t0, ent, src);
+            if (t0 + tstep < total) fetch_rows(t0 + tstep, ent);
+        }
+        const int prep_kb = min(1, p.num_kb - 1);
+        uint32_t s = 0, ph = 0;
+        bool ok = true;
+        for (int t = t0; t < total && ok; t += tstep) {
             for (int kb = 0; kb < p.num_kb; ++kb) {
                 bool w = true;
                 if (lane == 0)
@@ -272,11 +295,18 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     if (r < 64 || !half) dev::cp_async16(dst, nbytes ? src[i] + cb : src[i], nbytes);
                 }
                 dev::cp_async_arrive_noinc(&st.full[s]);
+                if (kb == prep_kb && t + tstep < total) {
+                    nhalf = row_ptrs(t + tstep, ent, nsrc);
+                    if (t + 2 * tstep < total) fetch_rows(t + 2 * tstep, ent);
+                }
                 if (++s == (uint32_t)nst) {
                     s = 0;
                     ph ^= 1u;
                 }
             }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) src[i] = nsrc[i];
+            half = nhalf;
         }
         dev::cp_async_wait_all();
     } else {

@@ -17,10 +17,12 @@
 //   warps 2-5   epilogue of this CTA's 128 accumulator rows (shared code with the one-CTA kernel).
 //   warps 6-9   (gathered A) cp.async row gatherers of this CTA's 128 rows; their completion is
 //               counted asynchronously (cp.async.mbarrier.arrive.noinc) on a CTA-local barrier.
-//               In the odd CTA, warp 1 relays each completed stage to the leader's full barrier
-//               (a cluster-scope release by a thread with no copies of its own in flight: a
-//               release by the copying threads themselves would wait for their newer stages'
-//               copies too and serialise the pipeline).
+//   warp 10     (gathered A) relay: waits for each stage's gathered rows of this CTA, makes them
+//               visible to the async proxy and arrives on the leader's full barrier, so the MMA
+//               issuer waits on one barrier per stage and runs no fence, as with TMA-loaded A.
+//               The relay is a thread with no copies of its own in flight, and its arrive is
+//               relaxed: a cluster-scope release there measured ~0.5 us a stage, longer than a
+//               stage of MMAs, and the proxy fence in the issuer halved the MMA rate.
 #include "gemm_common.cuh"
 
 #include <mutex>
@@ -36,9 +38,11 @@ constexpr int A2_BYTES = 128 * KBYTES;
 constexpr int B2_BYTES = 128 * KBYTES;  // this CTA's 128 columns of B
 constexpr int STAGE2_BYTES = A2_BYTES + B2_BYTES;
 constexpr uint16_t kPairMask = 0x3;
+constexpr int RELAY_WARP = (THREADS + GATHER_THREADS) / 32;
+constexpr int GATHER_BLOCK = THREADS + GATHER_THREADS + 32;  // threads of a gathered-A CTA
 
 struct Smem2 {
-    uint64_t full[ST2];    // leader: one phase per stage = both CTAs' TMA bytes (+ odd CTA relay)
+    uint64_t full[ST2];    // leader: one phase per stage = both CTAs' TMA bytes (+ both relays)
     uint64_t afull[ST2];   // both CTAs: this CTA's gathered rows of the stage landed
     uint64_t empty[ST2];   // both CTAs: the pair MMAs of the stage are done
     uint64_t tfull[2];     // both CTAs: accumulator b complete
@@ -54,7 +58,7 @@ constexpr size_t SMEM2_BYTES = 1024 + (size_t)ST2 * STAGE2_BYTES + sizeof(Smem2)
 
 template <bool BF16, bool GATHER, bool GLU, bool SCATTER>
 __global__ void __cluster_dims__(2, 1, 1)
-__launch_bounds__(GATHER ? THREADS + GATHER_THREADS : THREADS, 1)
+__launch_bounds__(GATHER ? GATHER_BLOCK : THREADS, 1)
 grouped_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB0,
                         const __grid_constant__ CUtensorMap tmB1, const KParams p) {
@@ -83,7 +87,7 @@ grouped_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < ST2; ++s) {
-            dev::mbar_init(&st.full[s], GATHER ? 2 : 1);
+            dev::mbar_init(&st.full[s], GATHER ? 3 : 1);
             dev::mbar_init(&st.afull[s], GATHER_THREADS);
             dev::mbar_init(&st.empty[s], 1);
         }
@@ -185,14 +189,11 @@ grouped_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
                 const uint32_t d_tmem = tmem_base + b * BN;
                 for (int kb = 0; kb < p.num_kb; ++kb) {
                     if (!dev::mbar_wait_cluster(&st.full[s], ph, abort, p.status, p.wait_limit_ns,
-                                                kKernelGemm) ||
-                        (GATHER && !dev::mbar_wait(&st.afull[s], ph, abort, p.status,
-                                                   p.wait_limit_ns, kKernelGemm))) {
+                                                kKernelGemm)) {
                         ok = false;
                         break;
                     }
                     dev::tc_fence_after();
-                    if (GATHER) dev::fence_proxy_async_cluster();  // cp.async rows -> tensor core
                     const uint32_t sA = dev::smem_u32(smem + (size_t)s * STAGE2_BYTES);
                     const uint32_t sB = sA + A2_BYTES;
 #pragma unroll
@@ -216,8 +217,11 @@ grouped_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
             dev::mma_commit_cg2_mc(&st.drain, 0x1);
             dev::mbar_wait_cluster(&st.drain, 0, nullptr, p.status, kDrainLimitNs, kKernelGemm);
             dev::tc_fence_before();
-        } else if (GATHER && !leader && lane == 0) {
-            // relay: this CTA's gathered rows of each stage -> the leader's full barrier
+        }
+        __syncwarp();
+    } else if (GATHER && warp == RELAY_WARP) {
+        // ------------------------------------------------------------------ relay (both CTAs)
+        if (lane == 0) {
             uint32_t s = 0, ph = 0;
             bool ok = true;
             for (int t = pair; t < total && ok; t += npairs) {
@@ -227,8 +231,9 @@ grouped_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
                         ok = false;
                         break;
                     }
-                    dev::fence_proxy_async_smem();
-                    dev::mbar_arrive_cluster(dev::mapa_shared(dev::smem_u32(&st.full[s]), 0));
+                    dev::fence_proxy_async_smem();  // cp.async rows -> tensor core
+                    dev::mbar_arrive_relaxed_cluster(
+                        dev::mapa_shared(dev::smem_u32(&st.full[s]), 0));
                     if (++s == ST2) {
                         s = 0;
                         ph ^= 1u;
@@ -244,22 +249,44 @@ grouped_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
         const int rsub = lane >> 3;
         const int64_t row_bytes = (int64_t)p.K * EB;
         const uint8_t *xa = reinterpret_cast<const uint8_t *>(p.A);
-        uint32_t s = 0, ph = 0;
-        bool ok = true;
-        for (int t = pair; t < total && ok; t += npairs) {
+        // sorted_rows entries of this thread's 8 rows of tile t (tail rows repeat a valid row)
+        auto fetch_rows = [&](int t, int *ent) {
             const TileInfo ti = decode_tile<TM2>(t, st.off, st.tstart, E);
             const int rbeg = ti.row_begin + 128 * (int)rank;
             const int rows = min(128, ti.rows - 128 * (int)rank);  // may be <= 0
-            const uint8_t *src[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 const int r = gw * 32 + i * 4 + rsub;
-                src[i] = xa;
-                if (rows > 0) {
-                    const int pr = rbeg + min(r, rows - 1);  // tail rows repeat a valid row
-                    src[i] = xa + (int64_t)(__ldg(p.sorted_rows + pr) / p.k) * row_bytes;
-                }
+                ent[i] = rows > 0 ? __ldg(p.sorted_rows + rbeg + min(r, rows - 1)) : 0;
             }
+        };
+        // x row pointers of tile t from its entries; returns this CTA's rows of it (may be <= 0)
+        auto row_ptrs = [&](int t, const int *ent, const uint8_t **src) {
+            const TileInfo ti = decode_tile<TM2>(t, st.off, st.tstart, E);
+            const int rows = min(128, ti.rows - 128 * (int)rank);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                src[i] = rows > 0 ? xa + (int64_t)(ent[i] / p.k) * row_bytes : xa;
+            return rows;
+        };
+        // Shared memory is saturated by the tensor core, so a tile's schedule lookups, index
+        // loads and divisions take ~2 us: the next tile's pointers are formed after the current
+        // tile's second stage is issued, and its entries are loaded a tile earlier still, so
+        // nothing but a register swap sits between two tiles' copies.
+        int ent[8];
+        const uint8_t *src[8], *nsrc[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) src[i] = nsrc[i] = xa;
+        int rows = 0, nrows = 0;
+        if (pair < total) {
+            fetch_rows(pair, ent);
+            rows = row_ptrs(pair, ent, src);
+            if (pair + npairs < total) fetch_rows(pair + npairs, ent);
+        }
+        const int prep_kb = min(1, p.num_kb - 1);
+        uint32_t s = 0, ph = 0;
+        bool ok = true;
+        for (int t = pair; t < total && ok; t += npairs) {
             for (int kb = 0; kb < p.num_kb; ++kb) {
                 bool w = true;
                 if (lane == 0)
@@ -280,11 +307,18 @@ grouped_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
                     dev::cp_async16(dst, nbytes ? src[i] + cb : xa, nbytes);
                 }
                 dev::cp_async_arrive_noinc(&st.afull[s]);
+                if (kb == prep_kb && t + npairs < total) {
+                    nrows = row_ptrs(t + npairs, ent, nsrc);
+                    if (t + 2 * npairs < total) fetch_rows(t + 2 * npairs, ent);
+                }
                 if (++s == ST2) {
                     s = 0;
                     ph ^= 1u;
                 }
             }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) src[i] = nsrc[i];
+            rows = nrows;
         }
         dev::cp_async_wait_all();
     } else {
@@ -388,8 +422,7 @@ int launch_2sm_t(const GemmArgs &a, cudaStream_t s, int n_pairs) {
     kp.zero_n4 = a.zero_n / 4;
     kp.status = a.status;
     kp.wait_limit_ns = a.wait_limit_ns;
-    kern<<<2 * n_pairs, GATHER ? THREADS + GATHER_THREADS : THREADS, SMEM2_BYTES, s>>>(mA, mB0,
-                                                                                     mB1, kp);
+    kern<<<2 * n_pairs, GATHER ? GATHER_BLOCK : THREADS, SMEM2_BYTES, s>>>(mA, mB0, mB1, kp);
     return MOE_OK;
 }
 
@@ -403,7 +436,7 @@ int max_pairs() {
     int pairs = num_sms() / 2;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(2 * pairs);
-    cfg.blockDim = dim3(THREADS + GATHER_THREADS);
+    cfg.blockDim = dim3(GATHER_BLOCK);
     cfg.dynamicSmemBytes = SMEM2_BYTES;
     cudaLaunchAttribute attr;
     attr.id = cudaLaunchAttributeClusterDimension;

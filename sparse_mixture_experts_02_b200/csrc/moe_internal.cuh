@@ -64,9 +64,9 @@ struct GemmArgs {
 int launch_grouped_gemm(const GemmArgs &a, cudaStream_t s);
 // Same operation on CTA pairs (tcgen05 cta_group::2, 256-row tiles).
 int launch_grouped_gemm_2sm(const GemmArgs &a, cudaStream_t s);
-// Picks the two-CTA kernel for contiguous A when experts hold >= 384 rows on average (256-row
+// Picks the two-CTA kernel when experts hold >= 384 rows on average (256-row
 // pair tiles waste little there); the environment variable MOE_GEMM_2SM=0/1 forces either kernel.
-bool prefer_2sm(int64_t R, int32_t E, bool gather);
+bool prefer_2sm(int64_t R, int32_t E);
 int launch_debug_wait(int64_t limit_ns, unsigned *status, cudaStream_t s);
 // Router on the tensor cores (bf16, E % 8 == 0): logits of 128-token tiles in TMEM, top-k and
 // softmax in the epilogue.
@@ -191,11 +191,6 @@ __device__ __forceinline__ void cp_async_wait_all() {
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
-// The same ordering for shared memory of any CTA of the cluster (the pair MMA reads operands
-// that the other CTA's threads wrote).
-__device__ __forceinline__ void fence_proxy_async_cluster() {
-    asm volatile("fence.proxy.async.shared::cluster;" ::: "memory");
-}
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -310,6 +305,14 @@ __device__ __forceinline__ void cluster_sync() {
 // Arrive on an mbarrier given by its shared::cluster address (possibly in the peer CTA).
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+                 : "memory");
+}
+// Arrive on a barrier of any CTA of the cluster without release ordering. Used only to say
+// "this CTA's A rows of a stage are in its own shared memory and fenced for the async proxy":
+// in a CTA-pair MMA each SM's tensor core reads its own CTA's A rows, so the signal carries no
+// data that another SM must observe. (A release at cluster scope cost ~0.5 us per arrive.)
+__device__ __forceinline__ void mbar_arrive_relaxed_cluster(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
                  : "memory");
 }
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
