@@ -248,13 +248,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                 ent[i] = __ldg(p.sorted_rows + ti.row_begin + min(r, ti.rows - 1));
             }
         };
-        // x row pointers of tile t from its entries; returns whether it is an M=64 tile (the
-        // MMA then reads rows 0-63 only)
+        // x row pointers of tile t from its entries; returns the tile's rows
         auto row_ptrs = [&](int t, const int *ent, const uint8_t **src) {
             const TileInfo ti = decode_tile<BM>(t, st.off, st.tstart, E_sched);
 #pragma unroll
             for (int i = 0; i < 8; ++i) src[i] = xa + (int64_t)(ent[i] / p.k) * row_bytes;
-            return ti.rows <= 64;
+            return ti.rows;
         };
         // Shared memory is saturated by the tensor core, so a tile's schedule lookups, index
         // loads and divisions take ~2 us: the next tile's pointers are formed after the current
@@ -265,10 +264,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         const uint8_t *src[8], *nsrc[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) src[i] = nsrc[i] = xa;
-        bool half = false, nhalf = false;
+        int rows = 0, nrows = 0;
         if (t0 < total) {
             fetch_rows(t0, ent);
-            half = row_ptrs(t0, ent, src);
+            rows = row_ptrs(t0, ent, src);
             if (t0 + tstep < total) fetch_rows(t0 + tstep, ent);
         }
         const int prep_kb = min(1, p.num_kb - 1);
@@ -288,15 +287,17 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                 const uint32_t sA = dev::smem_u32(smem + (size_t)s * sbytes);
                 const int64_t cb = (int64_t)kb * KBYTES + chunk * 16;
                 const uint32_t nbytes = cb < row_bytes ? 16u : 0u;  // zero-fill past K
+                // rows past the tile's end are not copied: an A row only feeds its own output
+                // row, which the epilogue discards (an M=64 tile's MMA reads rows 0-63 only)
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     const int r = gw * 32 + i * 4 + rsub;
                     const uint32_t dst = sA + r * KBYTES + ((chunk ^ (r & 7)) << 4);
-                    if (r < 64 || !half) dev::cp_async16(dst, nbytes ? src[i] + cb : src[i], nbytes);
+                    if (r < rows) dev::cp_async16(dst, nbytes ? src[i] + cb : src[i], nbytes);
                 }
                 dev::cp_async_arrive_noinc(&st.full[s]);
                 if (kb == prep_kb && t + tstep < total) {
-                    nhalf = row_ptrs(t + tstep, ent, nsrc);
+                    nrows = row_ptrs(t + tstep, ent, nsrc);
                     if (t + 2 * tstep < total) fetch_rows(t + 2 * tstep, ent);
                 }
                 if (++s == (uint32_t)nst) {
@@ -306,7 +307,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             }
 #pragma unroll
             for (int i = 0; i < 8; ++i) src[i] = nsrc[i];
-            half = nhalf;
+            rows = nrows;
         }
         dev::cp_async_wait_all();
     } else {

@@ -299,12 +299,14 @@ grouped_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
                 }
                 const uint32_t sA = dev::smem_u32(smem + (size_t)s * STAGE2_BYTES);
                 const int64_t cb = (int64_t)kb * KBYTES + chunk * 16;
-                const uint32_t nbytes = (rows > 0 && cb < row_bytes) ? 16u : 0u;
+                const uint32_t nbytes = cb < row_bytes ? 16u : 0u;  // zero-fill past K
+                // rows past this CTA's share are not copied: an A row only feeds its own output
+                // row, which the epilogue discards
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     const int r = gw * 32 + i * 4 + rsub;
                     const uint32_t dst = sA + r * KBYTES + ((chunk ^ (r & 7)) << 4);
-                    dev::cp_async16(dst, nbytes ? src[i] + cb : xa, nbytes);
+                    if (r < rows) dev::cp_async16(dst, nbytes ? src[i] + cb : src[i], nbytes);
                 }
                 dev::cp_async_arrive_noinc(&st.afull[s]);
                 if (kb == prep_kb && t + npairs < total) {

@@ -99,3 +99,35 @@ def test_scatter_linear_all_routes_one_expert(oracle_lib, moe, gemm_kernel):
                            torch.from_numpy(offsets).cuda())
     torch.cuda.synchronize()
     assert rel_frob(Y.cpu().numpy(), ref) < 2e-5
+
+
+EDGE_COUNTS = [1, 64, 65, 128, 129, 256, 257, 384, 385]
+
+
+@pytest.mark.parametrize("gather_in,scatter_out", [(True, True), (False, True), (True, False),
+                                                   (False, False)])
+def test_scatter_linear_tile_edges(oracle_lib, moe, gemm_kernel, gather_in, scatter_out):
+    # experts whose row counts sit on every tile edge: 64 (an M=64 / half pair-tile share),
+    # 128 (a one-CTA tile, a half pair tile), 256 (a pair tile) and one past each
+    k, Din, Dout = 1, 96, 264
+    E = len(EDGE_COUNTS)
+    owners = np.repeat(np.arange(E, dtype=np.int32), EDGE_COUNTS)
+    perm = np.random.default_rng(7).permutation(len(owners))
+    te = torch.from_numpy(owners[perm].reshape(-1, k).copy())
+    S = te.shape[0]
+    counts, offsets, _, sorted_rows = oracle_lib.sparse_map(te.numpy(), E)
+    assert list(counts) == EDGE_COUNTS
+    gen = torch.Generator().manual_seed(11)
+    X = torch.randn(S, Din, generator=gen).to(torch.bfloat16)
+    Wt = (torch.randn(E, Din, Dout, generator=gen) * 0.05).to(torch.bfloat16)
+    g = torch.rand(S * k, generator=gen)
+    ref = oracle_lib.scatter_linear(X, Wt, k, sorted_rows, offsets, g, gather_in=gather_in,
+                                    scatter_out=scatter_out, S=S)
+    Y = moe.scatter_linear(X.cuda(), Wt.cuda(), k, torch.from_numpy(sorted_rows).cuda(),
+                           torch.from_numpy(offsets).cuda(), g.cuda(), gather_in=gather_in,
+                           scatter_out=scatter_out, S=S)
+    torch.cuda.synchronize()
+    got = Y.float().cpu().numpy()
+    assert rel_frob(got, ref) < _tol("bf16", scatter_out)
+    scale = np.abs(ref).max()
+    assert np.abs(got - ref).max() / scale < 10 * _tol("bf16", scatter_out)
