@@ -261,9 +261,9 @@ def bench_ours(args, w, ws, rank, local):
         t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         ms_total = float(t.item())
-    stage = {"zero+route": [], "sparse_map": [], "gemm1": [], "gemm2": []}
+    stage = {"route": [], "sparse_map": [], "gemm1": [], "gemm2": []}
     for row in evs:
-        stage["zero+route"].append(row[0].elapsed_time(row[1]))
+        stage["route"].append(row[0].elapsed_time(row[1]))
         stage["sparse_map"].append(row[1].elapsed_time(row[2]))
         stage["gemm1"].append(row[2].elapsed_time(row[3]))
         stage["gemm2"].append(row[3].elapsed_time(row[4]))
