@@ -355,6 +355,51 @@ def bench_ours(args, w, ws, rank, local):
     return line
 
 
+def map_sweep(args):
+    """Sparse-map bandwidth over route counts 2^20..2^26 and E in {8, 64, 128, 256} (k = 8,
+    distinct experts per token, uniform marginals). Each point is the median of CUDA-event-timed
+    moe_sparse_map calls on the launch stream, L2 flushed (a 256 MiB write) before every call.
+    Algorithmic bytes: top_experts read (4R), sparse_rows and sorted_rows written (8R), counts and
+    offsets ((2E+1)*4)."""
+    import sparse_mixture_experts_02_b200 as moe
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    pk, pk_kind = peaks()
+    points = []
+    for log_r in range(20, 27):
+        R = 1 << log_r
+        for E in (8, 64, 128, 256):
+            k = 8
+            te = W.make_top_experts(R // k, k, E, seed=log_r * 1000 + E, mode="stride", device=dev)
+            need = moe.workspace_size("sparse_map", R // k, 0, 0, E, k, moe.MOE_BF16)
+            wsp = moe.alloc_workspace(need, dev)
+            reps = max(5, min(args.steps, (1 << 27) // R))
+            times = []
+            for i in range(args.warmup + reps):
+                flush.zero_()
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record()
+                moe.sparse_map(te, E, ws=wsp)
+                e1.record()
+                torch.cuda.synchronize(dev)
+                if i >= args.warmup:
+                    times.append(e0.elapsed_time(e1))
+            moe.check_device_status(wsp)
+            t_ms = sorted(times)[len(times) // 2]
+            nbytes = 4 * R + 8 * R + (2 * E + 1) * 4
+            gbs = nbytes / (t_ms * 1e-3) / 1e9
+            points.append({"R": R, "E": E, "us": round(t_ms * 1e3, 2), "GB/s": round(gbs, 1),
+                           "frac_of_hbm_peak": round(gbs / pk["hbm_gbs"], 3)})
+            del te, wsp
+    return {"metric": "sparse-map GB/s sweep", "unit": "GB/s", "n_gpus": 1,
+            "data": "synthetic (seeded stride routing: k = 8 distinct experts per token)",
+            "l2": "flushed before every call", "launches_per_call": 3,
+            "peak_hbm_gbs": pk["hbm_gbs"], "peak_kind": pk_kind, "points": points}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -366,9 +411,14 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     ap.add_argument("--ref-step-s", type=float, default=None)
+    ap.add_argument("--map-sweep", action="store_true",
+                    help="instead of the forward: sparse-map GB/s over R = 2^20..2^26 routes")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.map_sweep:
+        print(json.dumps(map_sweep(args)), flush=True)
+        return
     w = {**W.WORKLOADS, **W.PROFILE_WORKLOADS}[args.workload]
     if args.impl == "reference":
         # the oracle runs on rank 0's host cores only; other ranks have nothing to do

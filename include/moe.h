@@ -104,8 +104,8 @@ int moe_sparse_map(const int32_t *top_experts, int64_t S, int32_t k, int32_t E,
  * fail or stall the device. The pages have no counterpart of this entry point.
  * The scratch is a fixed array inside the library: 1 MiB of counters plus a 256-byte status area,
  * held on every device that loads the library until the process exits. Sizes must satisfy
- * ceil(S*k / 512) * E * 4 <= 1 MiB (for example S*k <= 524288 routes at E = 256); larger sizes
- * are rejected with MOE_ERR_INVALID_ARG before any launch. The call allocates nothing.
+ * (ceil(S*k / 4096) + 1) * E * 4 <= 1 MiB (for example S*k <= 4190208 routes at E = 256); larger
+ * sizes are rejected with MOE_ERR_INVALID_ARG before any launch. The call allocates nothing.
  * The first call on a device looks up the array's device address (with that device current);
  * make that first call before any stream capture. All calls share the array, which keeps the
  * last call's contents; calls whose kernels overlap on the GPU (e.g. on two streams) race on it

@@ -125,7 +125,19 @@ def make_top_experts(S: int, k: int, E: int, seed: int = 0, mode: str = "uniform
     mode "zipf":    distinct experts drawn by Zipf(1.2) popularity (Gumbel top-k of log-masses).
     mode "one":     every route of every row is expert 0 (rows are then not distinct: a stress case).
     mode "any":     k independent uniform draws (repeats allowed inside a row).
+    mode "stride":  row s holds (b_s + j*c_s) mod E for j < k, with b_s uniform and c_s uniform among
+                    the residues coprime to E: k distinct experts, uniform marginals, drawn on
+                    `device` without an S x E key matrix (for route counts up to 2^26).
     """
+    if mode == "stride":
+        g2 = torch.Generator(device=device)
+        g2.manual_seed(seed)
+        units = torch.tensor([c for c in range(1, E) if math.gcd(c, E) == 1] or [1],
+                             dtype=torch.int64, device=device)
+        b = torch.randint(0, E, (S, 1), generator=g2, device=device)
+        c = units[torch.randint(0, units.numel(), (S, 1), generator=g2, device=device)]
+        j = torch.arange(k, dtype=torch.int64, device=device)[None, :]
+        return ((b + j * c) % E).to(torch.int32).contiguous()
     gen = torch.Generator(device="cpu")
     gen.manual_seed(seed)
     if mode == "one":

@@ -69,7 +69,7 @@ extern "C" int moe_sparse_map_noalloc(const int32_t *top_experts, int64_t S, int
     if (need > kNoallocScratchBytes)
         return set_error(MOE_ERR_INVALID_ARG,
                          "sparse_map_noalloc: S*k=%lld routes over E=%d experts need %zu bytes of "
-                         "scratch, above its fixed %zu bytes (ceil(S*k/512)*E*4 must be <= %zu); "
+                         "scratch, above its fixed %zu bytes ((ceil(S*k/4096)+1)*E*4 must be <= %zu); "
                          "use moe_sparse_map with a workspace",
                          (long long)R, E, need, kNoallocScratchBytes, kNoallocScratchBytes);
     const struct { const char *name; const void *p; bool nullable; } ptrs[] = {

@@ -75,6 +75,25 @@ def test_map_large_route_count(oracle_lib, moe):
     _compare(oracle_lib, moe, te, 256)
 
 
+# Grid-parallel path: routes per count/assign block = 8 warps x 512; sizes one past and one short
+# of block multiples, and the first size past the one-block path.
+@pytest.mark.parametrize("R", [16385, 4096 * 5 - 1, 4096 * 5 + 1, 4096 * 64, 4096 * 1024 + 7])
+def test_map_block_edges(oracle_lib, moe, R):
+    te = W.make_top_experts(R, 1, 64, seed=R, mode="any")
+    _compare(oracle_lib, moe, te, 64)
+
+
+@pytest.mark.parametrize("E,mode", [(8, "stride"), (64, "zipf"), (128, "stride"), (256, "zipf")])
+def test_map_2pow20_routes(oracle_lib, moe, E, mode):
+    te = W.make_top_experts(1 << 17, 8, E, seed=E, mode=mode)
+    _compare(oracle_lib, moe, te, E)
+
+
+def test_map_2pow23_routes_256_experts(oracle_lib, moe):
+    te = W.make_top_experts(1 << 20, 8, 256, seed=23, mode="stride")
+    _compare(oracle_lib, moe, te, 256)
+
+
 def test_map_bad_expert_id_is_reported(moe):
     te = W.make_top_experts(100, 2, 8, seed=2).clone()
     te[17, 1] = 8

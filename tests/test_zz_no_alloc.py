@@ -66,11 +66,11 @@ def test_noalloc_matches_workspace_map_twice(moe):
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch(moe):
-    # ceil(S*k/512) * E * 4 bytes must fit in 1 MiB: 2^21 routes at E = 256 need 4 MiB
-    te = torch.zeros((1 << 18, 8), dtype=torch.int32, device="cuda")
-    outs = _outputs(1 << 18, 8, 256)
+    # (ceil(S*k/4096) + 1) * E * 4 bytes must fit in 1 MiB: 2^23 routes at E = 256 need 2 MiB
+    te = torch.zeros((1 << 20, 8), dtype=torch.int32, device="cuda")
+    outs = _outputs(1 << 20, 8, 256)
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
-    rc = moe.lib.moe_sparse_map_noalloc(_p(te), 1 << 18, 8, 256, *[_p(o) for o in outs], stream)
+    rc = moe.lib.moe_sparse_map_noalloc(_p(te), 1 << 20, 8, 256, *[_p(o) for o in outs], stream)
     assert rc == -1
     assert b"scratch" in moe.lib.moe_last_error()
     # nothing was launched: the outputs keep their fill value
