@@ -368,32 +368,34 @@ def map_sweep(args):
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     pk, pk_kind = peaks()
     points = []
-    for log_r in range(20, 27):
+    grid = [(log_r, E) for log_r in range(20, 27) for E in (8, 64, 128, 256)]
+    if args.map_points:
+        grid = [tuple(int(v) for v in pt.split(":")) for pt in args.map_points.split(",")]
+    for log_r, E in grid:
         R = 1 << log_r
-        for E in (8, 64, 128, 256):
-            k = 8
-            te = W.make_top_experts(R // k, k, E, seed=log_r * 1000 + E, mode="stride", device=dev)
-            need = moe.workspace_size("sparse_map", R // k, 0, 0, E, k, moe.MOE_BF16)
-            wsp = moe.alloc_workspace(need, dev)
-            reps = max(5, min(args.steps, (1 << 27) // R))
-            times = []
-            for i in range(args.warmup + reps):
-                flush.zero_()
-                e0 = torch.cuda.Event(enable_timing=True)
-                e1 = torch.cuda.Event(enable_timing=True)
-                e0.record()
-                moe.sparse_map(te, E, ws=wsp)
-                e1.record()
-                torch.cuda.synchronize(dev)
-                if i >= args.warmup:
-                    times.append(e0.elapsed_time(e1))
-            moe.check_device_status(wsp)
-            t_ms = sorted(times)[len(times) // 2]
-            nbytes = 4 * R + 8 * R + (2 * E + 1) * 4
-            gbs = nbytes / (t_ms * 1e-3) / 1e9
-            points.append({"R": R, "E": E, "us": round(t_ms * 1e3, 2), "GB/s": round(gbs, 1),
-                           "frac_of_hbm_peak": round(gbs / pk["hbm_gbs"], 3)})
-            del te, wsp
+        k = 8
+        te = W.make_top_experts(R // k, k, E, seed=log_r * 1000 + E, mode="stride", device=dev)
+        need = moe.workspace_size("sparse_map", R // k, 0, 0, E, k, moe.MOE_BF16)
+        wsp = moe.alloc_workspace(need, dev)
+        reps = args.steps if args.map_points else max(5, min(args.steps, (1 << 27) // R))
+        times = []
+        for i in range(args.warmup + reps):
+            flush.zero_()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            moe.sparse_map(te, E, ws=wsp)
+            e1.record()
+            torch.cuda.synchronize(dev)
+            if i >= args.warmup:
+                times.append(e0.elapsed_time(e1))
+        moe.check_device_status(wsp)
+        t_ms = sorted(times)[len(times) // 2]
+        nbytes = 4 * R + 8 * R + (2 * E + 1) * 4
+        gbs = nbytes / (t_ms * 1e-3) / 1e9
+        points.append({"R": R, "E": E, "us": round(t_ms * 1e3, 2), "GB/s": round(gbs, 1),
+                       "frac_of_hbm_peak": round(gbs / pk["hbm_gbs"], 3)})
+        del te, wsp
     return {"metric": "sparse-map GB/s sweep", "unit": "GB/s", "n_gpus": 1,
             "data": "synthetic (seeded stride routing: k = 8 distinct experts per token)",
             "l2": "flushed before every call", "launches_per_call": 3,
@@ -413,6 +415,8 @@ def main():
     ap.add_argument("--ref-step-s", type=float, default=None)
     ap.add_argument("--map-sweep", action="store_true",
                     help="instead of the forward: sparse-map GB/s over R = 2^20..2^26 routes")
+    ap.add_argument("--map-points", default="",
+                    help="with --map-sweep: only these points, 'log2R:E,...' (e.g. 26:256)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
