@@ -47,6 +47,8 @@ def lib():
         L.oracle_mlp_forward.argtypes = [P, P, P, P, P, P, i64, i64, i32, i32, P, i64, P, P, P, P]
         L.oracle_scatter_linear.argtypes = [P, P, i64, i64, i64, i32, i32, P, P, P, ctypes.c_int,
                                             ctypes.c_int, P]
+        L.oracle_scatter_linear_backward.argtypes = [P, P, P, i64, i64, i64, i32, i32, P, P, P,
+                                                     ctypes.c_int, ctypes.c_int, P, P, P]
     return _lib
 
 
@@ -172,3 +174,26 @@ def scatter_linear(X, W, k, sorted_rows, offsets, gates=None, gather_in=True, sc
                                 _p(gates.reshape(-1) if gates is not None else None),
                                 int(bool(gather_in)), int(bool(scatter_out)), _p(Y))
     return Y
+
+
+def scatter_linear_backward(X, W, dY, k, sorted_rows, offsets, gates=None, gather_in=True,
+                            scatter_out=True, S=None):
+    """Backward of ParallelLinear in fp64: {"dX", "dW", "dgates"} (dgates only with gates).
+    dY has Y's shape: [S, Dout] when scatter_out, else [R, Dout]; dX has X's shape."""
+    X, W, dY, gates = _f32(X), _f32(W), _f32(dY), _f32(gates)
+    sorted_rows, offsets = _i32(sorted_rows), _i32(offsets)
+    E, Din, Dout = W.shape
+    if S is None:
+        S = X.shape[0] if gather_in else (sorted_rows.shape[0] // k)
+    P = int(offsets[E])
+    dX = np.zeros((S if gather_in else max(P, 0), Din), dtype=np.float64)
+    dW = np.zeros((E, Din, Dout), dtype=np.float64)
+    dg = np.zeros(S * k, dtype=np.float64) if gates is not None else None
+    lib().oracle_scatter_linear_backward(
+        _p(X), _p(W), _p(dY), S, Din, Dout, E, k, _p(sorted_rows), _p(offsets),
+        _p(gates.reshape(-1) if gates is not None else None), int(bool(gather_in)),
+        int(bool(scatter_out)), _p(dX), _p(dW), _p(dg))
+    out = {"dX": dX, "dW": dW}
+    if dg is not None:
+        out["dgates"] = dg
+    return out

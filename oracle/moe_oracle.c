@@ -276,3 +276,87 @@ void oracle_scatter_linear(const float *X, const float *W, int64_t S, int64_t Di
     }
     free(grouped);
 }
+
+/* Backward of ParallelLinear, the ScatterMoE guide's "3. Fused Backward Pass Dynamics": the input
+ * gradient gathers the output gradient of each slot, multiplies by the transposed expert weight and
+ * the gate, and sums back into the token (the guide's grad-X sum over TopK); the weight gradient of
+ * expert e sums the outer products of its slots' inputs and gated output gradients (the guide's
+ * grad-W_e sum over Tokens(e)); the gate gradient is the derivative of Y in g. With dY shaped like
+ * Y ([S, Dout] if scatter_out, else [R, Dout]), for every slot p of expert e, route i, token s:
+ *   dc_p = dY[s] if scatter_out else dY[p];   dv_p = g_i * dc_p  (g_i = 1 without gates)
+ *   dsrc_p = dv_p . W[e]^T          -> dX[s] += dsrc_p (gather_in, dX [S, Din]) or dX[p] = dsrc_p
+ *   dW[e] += src_p^T dv_p           -> dW [E, Din, Dout]
+ *   dgates[i] = dc_p . (src_p . W[e])  (only with gates)
+ * fp64 throughout; dX, dW and dgates may each be null (not computed); outputs are overwritten. */
+void oracle_scatter_linear_backward(const float *X, const float *W, const float *dY, int64_t S,
+                                    int64_t Din, int64_t Dout, int32_t E, int32_t k,
+                                    const int32_t *sorted_rows, const int32_t *offsets,
+                                    const float *gates, int gather_in, int scatter_out, double *dX,
+                                    double *dW, double *dgates) {
+    const int64_t P = offsets[E];
+    int32_t *slot_e = (int32_t *)malloc(sizeof(int32_t) * (size_t)(P > 0 ? P : 1));
+    for (int32_t e = 0; e < E; ++e)
+        for (int64_t p = offsets[e]; p < offsets[e + 1]; ++p) slot_e[p] = e;
+    if (dX) {
+        const int64_t rows = gather_in ? S : P;
+        double *dsrc = (double *)calloc((size_t)(P > 0 ? P : 1) * (size_t)Din, sizeof(double));
+        #pragma omp parallel for schedule(dynamic, 4)
+        for (int64_t p = 0; p < P; ++p) {
+            const int32_t e = slot_e[p];
+            const int64_t i = sorted_rows[p];
+            const int64_t s = i / k;
+            const float *dc = dY + (scatter_out ? s : p) * Dout;
+            const double g = gates ? (double)gates[i] : 1.0;
+            const float *We = W + (int64_t)e * Din * Dout;
+            for (int64_t d = 0; d < Din; ++d) {
+                double acc = 0.0;
+                for (int64_t n = 0; n < Dout; ++n) acc += (double)dc[n] * (double)We[d * Dout + n];
+                dsrc[p * Din + d] = g * acc;
+            }
+        }
+        memset(dX, 0, sizeof(double) * (size_t)rows * (size_t)Din);
+        for (int64_t p = 0; p < P; ++p) {
+            const int64_t r = gather_in ? (int64_t)sorted_rows[p] / k : p;
+            for (int64_t d = 0; d < Din; ++d) dX[r * Din + d] += dsrc[p * Din + d];
+        }
+        free(dsrc);
+    }
+    if (dW) {
+        #pragma omp parallel for schedule(dynamic, 1) collapse(2)
+        for (int32_t e = 0; e < E; ++e) {
+            for (int64_t d = 0; d < Din; ++d) {
+                double *row = dW + ((int64_t)e * Din + d) * Dout;
+                for (int64_t n = 0; n < Dout; ++n) row[n] = 0.0;
+                for (int64_t p = offsets[e]; p < offsets[e + 1]; ++p) {
+                    const int64_t i = sorted_rows[p];
+                    const int64_t s = i / k;
+                    const double xv = (double)X[(gather_in ? s : p) * Din + d];
+                    const double g = gates ? (double)gates[i] : 1.0;
+                    const float *dc = dY + (scatter_out ? s : p) * Dout;
+                    for (int64_t n = 0; n < Dout; ++n) row[n] += xv * g * (double)dc[n];
+                }
+            }
+        }
+    }
+    if (dgates && gates) {
+        const int64_t R = (int64_t)S * k;
+        for (int64_t i = 0; i < R; ++i) dgates[i] = 0.0;
+        #pragma omp parallel for schedule(dynamic, 4)
+        for (int64_t p = 0; p < P; ++p) {
+            const int32_t e = slot_e[p];
+            const int64_t i = sorted_rows[p];
+            const int64_t s = i / k;
+            const float *src = X + (gather_in ? s : p) * Din;
+            const float *dc = dY + (scatter_out ? s : p) * Dout;
+            const float *We = W + (int64_t)e * Din * Dout;
+            double acc = 0.0;
+            for (int64_t n = 0; n < Dout; ++n) {
+                double v = 0.0;
+                for (int64_t d = 0; d < Din; ++d) v += (double)src[d] * (double)We[d * Dout + n];
+                acc += (double)dc[n] * v;
+            }
+            dgates[i] = acc;
+        }
+    }
+    free(slot_e);
+}
