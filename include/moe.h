@@ -138,6 +138,31 @@ int moe_scatter_linear(const void *X, const void *W, int64_t S, int64_t Din, int
                        moe_stream_t stream);
 
 /*
+ * Backward of moe_scatter_linear (ScatterMoE guide, "3. Fused Backward Pass Dynamics"): with the
+ * forward's X, W, sorted_rows, expert_offsets, top_weights, gather_in and scatter_out, and dY
+ * shaped like the forward's Y, for every slot p of expert e (route i, token s):
+ *   dc_p = dY[s] (scatter_out) or dY[p];  dv_p = top_weights[i] * dc_p (1 without top_weights)
+ *   dX[s] += dv_p . W[e]^T  (gather_in: dX [S, Din] float32, overwritten)
+ *   dX[p]  = dv_p . W[e]^T  (else:      dX [S*k, Din] bf16)
+ *   dW[e]  = sum over e's slots of src_p^T (x) dv_p, src_p = X[s] or X[p]  ([E, Din, Dout] f32)
+ *   dgates[i] = dc_p . (src_p . W[e])   ([S*k] float32; needs top_weights)
+ * dY: float32 [S, Dout] when scatter_out, else bf16 [S*k, Dout]. dX, dW and dgates are each
+ * nullable (not computed) and 16-byte aligned; every output is overwritten (dW is zero for an
+ * expert without slots; dgates is zero for a route whose expert id was out of range).
+ * bf16 only (dt = MOE_BF16; MOE_ERR_UNSUPPORTED otherwise). The input gradient runs the forward's
+ * grouped GEMM with the gather and scatter roles exchanged and W read transposed (K-major, no
+ * copy); the weight gradient is a grouped GEMM whose reduction runs over each expert's slots
+ * (fp32 accumulation in TMEM, bf16 operands: dY is rounded to bf16 once).
+ * ws: moe_workspace_size("scatter_linear_backward", S, Din, Dout, E, k, dt) bytes.
+ */
+int moe_scatter_linear_backward(const void *X, const void *W, const void *dY, int64_t S,
+                                int64_t Din, int64_t Dout, int32_t E, int32_t k,
+                                const int32_t *sorted_rows, const int32_t *expert_offsets,
+                                const float *top_weights, int gather_in, int scatter_out,
+                                moe_dtype dt, void *dX, float *dW, float *dgates, void *ws,
+                                size_t ws_bytes, moe_stream_t stream);
+
+/*
  * Whole MoE expert-MLP forward:
  *   out[s] = sum_j w_j * ( silu(x[s] W_gate_e[e_j]) * (x[s] W_up[e_j]) ) W_down[e_j]
  * with (e_j, w_j) from moe_route_topk. Steps on `stream`: zero out, route, sparse map, GEMM1
@@ -156,8 +181,9 @@ int moe_mlp_forward(const void *x, const void *w_gate, const float *logit_bias,
                     size_t ws_bytes, moe_stream_t stream);
 
 /*
- * Workspace bytes for op = "sparse_map", "scatter_linear" or "mlp_forward" (unused sizes may be
- * 0). Returns 0 for an unknown op or sizes outside the limits.
+ * Workspace bytes for op = "sparse_map", "scatter_linear", "scatter_linear_backward" (D = Din,
+ * F = Dout) or "mlp_forward" (unused sizes may be 0). Returns 0 for an unknown op or sizes
+ * outside the limits.
  */
 size_t moe_workspace_size(const char *op, int64_t S, int64_t D, int64_t F, int32_t E, int32_t k,
                           moe_dtype dt);

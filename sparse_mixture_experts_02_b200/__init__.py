@@ -24,7 +24,7 @@ STATUS_NAMES = {0: "MOE_OK", -1: "MOE_ERR_INVALID_ARG", -2: "MOE_ERR_UNSUPPORTED
                 -6: "MOE_ERR_DEVICE_TIMEOUT"}
 
 EXPORTS = ["moe_route_topk", "moe_sparse_map", "moe_sparse_map_noalloc", "moe_scatter_linear",
-           "moe_mlp_forward",
+           "moe_scatter_linear_backward", "moe_mlp_forward",
            "moe_workspace_size", "moe_workspace_view", "moe_last_error",
            "moe_check_device_status", "moe_profile_events", "moe_debug_wait_timeout",
            "moe_last_launch_count"]
@@ -48,6 +48,8 @@ def _load():
     lib.moe_sparse_map_noalloc.argtypes = [P, i64, i32, i32, P, P, P, P, P]
     lib.moe_scatter_linear.argtypes = [P, P, i64, i64, i64, i32, i32, P, P, P, c_int, c_int,
                                        c_int, P, P, ctypes.c_size_t, P]
+    lib.moe_scatter_linear_backward.argtypes = [P, P, P, i64, i64, i64, i32, i32, P, P, P, c_int,
+                                                c_int, c_int, P, P, P, P, ctypes.c_size_t, P]
     lib.moe_mlp_forward.argtypes = [P, P, P, P, P, P, i64, i64, i64, i32, i32, c_int, P, P,
                                     ctypes.c_size_t, P]
     lib.moe_workspace_size.argtypes = [ctypes.c_char_p, i64, i64, i64, i32, i32, c_int]
@@ -59,7 +61,7 @@ def _load():
     lib.moe_profile_events.argtypes = [P, c_int]
     lib.moe_debug_wait_timeout.argtypes = [i64, P, ctypes.c_size_t, P]
     for name in ("moe_route_topk", "moe_sparse_map", "moe_sparse_map_noalloc",
-                 "moe_scatter_linear", "moe_mlp_forward",
+                 "moe_scatter_linear", "moe_scatter_linear_backward", "moe_mlp_forward",
                  "moe_check_device_status", "moe_profile_events", "moe_debug_wait_timeout",
                  "moe_last_launch_count"):
         getattr(lib, name).restype = c_int
@@ -210,6 +212,54 @@ def scatter_linear(X: torch.Tensor, W: torch.Tensor, k: int, sorted_rows: torch.
                                   int(bool(scatter_out)), _dtype_code(X), _ptr(Y), _ptr(ws),
                                   ws.numel(), _stream(dev)))
     return Y
+
+
+def scatter_linear_backward(X: torch.Tensor, W: torch.Tensor, dY: torch.Tensor, k: int,
+                            sorted_rows: torch.Tensor, expert_offsets: torch.Tensor,
+                            gates: Optional[torch.Tensor] = None, gather_in: bool = True,
+                            scatter_out: bool = True, S: Optional[int] = None,
+                            need=("dX", "dW", "dgates"), ws: Optional[torch.Tensor] = None):
+    """Backward of scatter_linear (moe_scatter_linear_backward), bf16 inputs. dY has the forward
+    output's shape and dtype (float32 [S, Dout] when scatter_out, else X's dtype [S*k, Dout]).
+    Returns {"dX", "dW", "dgates"} for the names in `need` (dgates only with gates): dX float32
+    [S, Din] when gather_in, else [S*k, Din] in X's dtype; dW float32 [E, Din, Dout]; dgates
+    float32 [S*k]."""
+    _req(X, "X", dim=2)
+    _req(W, "W", dtype=X.dtype, dim=3, device=X.device)
+    _req(sorted_rows, "sorted_rows", dtype=torch.int32, dim=1, device=X.device)
+    _req(expert_offsets, "expert_offsets", dtype=torch.int32, dim=1, device=X.device)
+    E, Din, Dout = W.shape
+    R = sorted_rows.shape[0]
+    if S is None:
+        S = X.shape[0] if gather_in else R // k
+    if S * k != R or X.shape[1] != Din:
+        raise ValueError("shapes of X, W and sorted_rows disagree")
+    _req(dY, "dY", dtype=torch.float32 if scatter_out else X.dtype, dim=2, device=X.device)
+    if dY.shape != ((S if scatter_out else R), Dout):
+        raise ValueError("dY must have the forward output's shape")
+    if gates is not None:
+        _req(gates, "gates", dtype=torch.float32, device=X.device)
+    dev = X.device
+    out = {}
+    dX = dW = dg = None
+    if "dX" in need:
+        dX = torch.empty((S, Din), dtype=torch.float32, device=dev) if gather_in else \
+            torch.empty((R, Din), dtype=X.dtype, device=dev)
+        out["dX"] = dX
+    if "dW" in need:
+        dW = torch.empty((E, Din, Dout), dtype=torch.float32, device=dev)
+        out["dW"] = dW
+    if "dgates" in need and gates is not None:
+        dg = torch.empty(R, dtype=torch.float32, device=dev)
+        out["dgates"] = dg
+    if ws is None:
+        ws = alloc_workspace(workspace_size("scatter_linear_backward", S, Din, Dout, E, k, X.dtype),
+                             dev)
+    _check(_lib().moe_scatter_linear_backward(
+        _ptr(X), _ptr(W), _ptr(dY), S, Din, Dout, E, k, _ptr(sorted_rows), _ptr(expert_offsets),
+        _ptr(gates), int(bool(gather_in)), int(bool(scatter_out)), _dtype_code(X), _ptr(dX),
+        _ptr(dW), _ptr(dg), _ptr(ws), ws.numel(), _stream(dev)))
+    return out
 
 
 class ForwardWorkspace:

@@ -129,6 +129,24 @@ MlpLayout mlp_layout(int64_t S, int64_t F, int32_t E, int32_t k, moe_dtype dt) {
     return L;
 }
 
+// ParallelLinear backward scratch: status, bf16 copy of an fp32 dY [S, Dout], gated rows dv
+// [R, Dout] bf16 (weight gradient), ungated forward rows v [R, Dout] bf16 (gate gradient).
+struct BwdLayout {
+    size_t status, dyb, dv, v, total;
+};
+
+BwdLayout bwd_layout(int64_t S, int64_t Dout, int32_t k) {
+    const int64_t R = S * k;
+    BwdLayout L;
+    size_t o = 0;
+    L.status = o; o += kStatusBytes;
+    L.dyb = o; o = align_up(o + 2 * (size_t)S * (size_t)Dout);
+    L.dv = o; o = align_up(o + 2 * (size_t)R * (size_t)Dout);
+    L.v = o; o = align_up(o + 2 * (size_t)R * (size_t)Dout);
+    L.total = o;
+    return L;
+}
+
 size_t map_ws_bytes(int64_t S, int32_t E, int32_t k) {
     return kStatusBytes + align_up(map_scratch_bytes(S * k, E));
 }
@@ -177,6 +195,10 @@ size_t moe_workspace_size(const char *op, int64_t S, int64_t D, int64_t F, int32
     if (S * (int64_t)k >= (int64_t(1) << 31)) return 0;
     if (strcmp(op, "sparse_map") == 0) return map_ws_bytes(S, E, k);
     if (strcmp(op, "scatter_linear") == 0) return kStatusBytes;
+    if (strcmp(op, "scatter_linear_backward") == 0) {
+        if (F <= 0) return 0;
+        return bwd_layout(S, F, k).total;  // D = Din, F = Dout
+    }
     if (strcmp(op, "mlp_forward") == 0) {
         if (F <= 0 || (dt != MOE_F32 && dt != MOE_BF16)) return 0;
         return mlp_layout(S, F, E, k, dt).total;
@@ -297,6 +319,128 @@ int moe_scatter_linear(const void *X, const void *W, int64_t S, int64_t Din, int
         return rc;
     g_launches = 1;
     return check_launch("scatter_linear");
+}
+
+int moe_scatter_linear_backward(const void *X, const void *W, const void *dY, int64_t S,
+                                int64_t Din, int64_t Dout, int32_t E, int32_t k,
+                                const int32_t *sorted_rows, const int32_t *expert_offsets,
+                                const float *top_weights, int gather_in, int scatter_out,
+                                moe_dtype dt, void *dX, float *dW, float *dgates, void *ws,
+                                size_t ws_bytes, moe_stream_t stream) {
+    g_launches = 0;
+    int rc;
+    if ((rc = check_dtype(dt)) || (rc = check_dims(S, E, k)) || (rc = check_feat("Din", Din)) ||
+        (rc = check_feat("Dout", Dout)))
+        return rc;
+    if (dt != MOE_BF16)
+        return set_error(MOE_ERR_UNSUPPORTED, "scatter_linear_backward: bf16 inputs only");
+    if (dgates != nullptr && top_weights == nullptr)
+        return set_error(MOE_ERR_INVALID_ARG, "dgates needs top_weights (the forward's gates)");
+    const int64_t R = S * k;
+    if ((rc = check_ptr("X", X, 16, R == 0)) || (rc = check_ptr("W", W, 16)) ||
+        (rc = check_ptr("dY", dY, 16, R == 0)) ||
+        (rc = check_ptr("sorted_rows", sorted_rows, 4, R == 0)) ||
+        (rc = check_ptr("expert_offsets", expert_offsets, 4)) ||
+        (rc = check_ptr("top_weights", top_weights, 4, true)) ||
+        (rc = check_ptr("dX", dX, 16, true)) || (rc = check_ptr("dW", dW, 16, true)) ||
+        (rc = check_ptr("dgates", dgates, 16, true)))
+        return rc;
+    const BwdLayout L = bwd_layout(S, Dout, k);
+    if ((rc = check_ws(ws, ws_bytes, L.total))) return rc;
+    if ((rc = check_device())) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    unsigned *status = at<unsigned>(ws, L.status);
+    if (cudaMemsetAsync(status, 0, sizeof(unsigned), s) != cudaSuccess)
+        return set_error(MOE_ERR_CUDA, "cudaMemsetAsync of the status word failed");
+    int n = 0;
+    // input gradient accumulates into token rows: start from zero
+    if (dX != nullptr && gather_in) {
+        launch_zero_f32(static_cast<float *>(dX), S * Din, nullptr, s);
+        ++n;
+    }
+    if (R == 0) {
+        if (dW != nullptr) {
+            launch_zero_f32(dW, (int64_t)E * Din * Dout, nullptr, s);
+            ++n;
+        }
+        g_launches = n;
+        return check_launch("scatter_linear_backward");
+    }
+    // the output gradient as a bf16 operand: dY is fp32 [S, Dout] when the forward scattered
+    const void *dyb = dY;
+    if (scatter_out) {
+        launch_cast_bf16(static_cast<const float *>(dY), at<void>(ws, L.dyb), S * Dout, s);
+        dyb = at<void>(ws, L.dyb);
+        ++n;
+    }
+    GemmArgs a{};
+    a.offsets = expert_offsets;
+    a.sorted_rows = sorted_rows;
+    a.S = S;
+    a.R = R;
+    a.E = E;
+    a.k = k;
+    a.bf16 = true;
+    a.glu = false;
+    a.status = status;
+    a.wait_limit_ns = kWaitLimitNs;
+    if (dX != nullptr) {
+        // dX = ParallelLinear(dY, W^T, I, G) with the gather and scatter roles exchanged
+        GemmArgs b = a;
+        b.A = dyb;
+        b.a_rows = scatter_out ? S : R;
+        b.B0 = W;  // [E, Din, Dout] read K-major as W^T: N = Din, K = Dout
+        b.b_kmajor = true;
+        b.gates = top_weights;
+        b.out = dX;
+        b.K = Dout;
+        b.N = Din;
+        b.gather = scatter_out != 0;
+        b.scatter = gather_in != 0;
+        if ((rc = launch_grouped_gemm(b, s))) return rc;
+        ++n;
+    }
+    if (dW != nullptr) {
+        launch_gate_rows(dY, !scatter_out, sorted_rows, top_weights, k, R, Dout, scatter_out != 0,
+                         at<void>(ws, L.dv), s);
+        WgradArgs w{};
+        w.X = X;
+        w.dv = at<void>(ws, L.dv);
+        w.offsets = expert_offsets;
+        w.sorted_rows = sorted_rows;
+        w.Din = Din;
+        w.Dout = Dout;
+        w.R = R;
+        w.E = E;
+        w.k = k;
+        w.gather = gather_in != 0;
+        w.dW = dW;
+        w.status = status;
+        w.wait_limit_ns = kWaitLimitNs;
+        if ((rc = launch_grouped_wgrad(w, s))) return rc;
+        n += 2;
+    }
+    if (dgates != nullptr) {
+        // v = the ungated forward rows in slot order; dgates[i] = dY[row] . v[p]
+        GemmArgs f = a;
+        f.A = X;
+        f.a_rows = gather_in ? S : R;
+        f.B0 = W;
+        f.gates = nullptr;
+        f.out = at<void>(ws, L.v);
+        f.K = Din;
+        f.N = Dout;
+        f.gather = gather_in != 0;
+        f.scatter = false;
+        if ((rc = prefer_2sm(R, E) ? launch_grouped_gemm_2sm(f, s) : launch_grouped_gemm(f, s)))
+            return rc;
+        launch_zero_f32(dgates, R, nullptr, s);
+        launch_rowdot(dY, !scatter_out, at<void>(ws, L.v), sorted_rows, k, R, Dout,
+                      scatter_out != 0, dgates, s);
+        n += 3;
+    }
+    g_launches = n;
+    return check_launch("scatter_linear_backward");
 }
 
 int moe_mlp_forward(const void *x, const void *w_gate, const float *logit_bias,

@@ -1,0 +1,135 @@
+// Elementwise and row-reduction kernels of the ParallelLinear backward (ScatterMoE guide,
+// "3. Fused Backward Pass Dynamics"); the GEMMs are the tensor-core kernels of grouped_gemm.cu
+// (input gradient: the forward's form with W read transposed) and grouped_gemm_wgrad.cu (weight
+// gradient).
+//   cast:      an fp32 output gradient [rows, Dout] -> bf16 (the tensor cores' operand type);
+//   gate_rows: dv[p] = bf16(g_i * dY[row(p)]) in slot order, the weight gradient's B operand
+//              (row(p) = sorted_rows[p] / k when the forward scattered into tokens, else p);
+//   rowdot:    dgates[i] = sum_n dY[row(p)][n] * v[p][n], v = the ungated forward rows.
+// One warp per slot; rows move in 16-byte pieces (Dout is a multiple of 8).
+#include "moe_internal.cuh"
+
+#include <cuda_bf16.h>
+
+namespace moe {
+namespace {
+
+constexpr int kWarps = 8;
+
+__device__ __forceinline__ void load8(const void *row, bool bf16, int64_t c, float (&v)[8]) {
+    if (bf16) {
+        const uint4 u = *reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(row) + c);
+        const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float2 f = __bfloat1622float2(h[j]);
+            v[2 * j] = f.x;
+            v[2 * j + 1] = f.y;
+        }
+    } else {
+        const float4 a = *reinterpret_cast<const float4 *>(static_cast<const float *>(row) + c);
+        const float4 b = *reinterpret_cast<const float4 *>(static_cast<const float *>(row) + c + 4);
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+        v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    }
+}
+
+__device__ __forceinline__ uint4 pack8(const float (&v)[8]) {
+    uint4 u;
+    uint32_t *w = reinterpret_cast<uint32_t *>(&u);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        __nv_bfloat162 t = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
+        w[j] = *reinterpret_cast<uint32_t *>(&t);
+    }
+    return u;
+}
+
+__global__ void cast_bf16_kernel(const float *__restrict__ src, __nv_bfloat16 *__restrict__ dst,
+                                 int64_t n8) {
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += stride) {
+        float v[8];
+        load8(src, false, i * 8, v);
+        *reinterpret_cast<uint4 *>(dst + i * 8) = pack8(v);
+    }
+}
+
+__global__ void __launch_bounds__(kWarps * 32)
+gate_rows_kernel(const void *__restrict__ dY, bool dy_bf16, const int32_t *__restrict__ sorted_rows,
+                 const float *__restrict__ gates, int32_t k, int64_t R, int64_t Dout,
+                 bool by_token, __nv_bfloat16 *__restrict__ dv) {
+    const int lane = threadIdx.x & 31;
+    const int64_t wstride = (int64_t)gridDim.x * kWarps;
+    for (int64_t p = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5); p < R; p += wstride) {
+        const int32_t i = __ldg(sorted_rows + p);
+        const float g = gates != nullptr ? __ldg(gates + i) : 1.0f;
+        const int64_t row = by_token ? (int64_t)(i / k) : p;
+        const uint8_t *src = static_cast<const uint8_t *>(dY) + row * Dout * (dy_bf16 ? 2 : 4);
+        for (int64_t c = (int64_t)lane * 8; c < Dout; c += 32 * 8) {
+            float v[8];
+            load8(src, dy_bf16, c, v);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) v[j] *= g;
+            *reinterpret_cast<uint4 *>(dv + p * Dout + c) = pack8(v);
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kWarps * 32)
+rowdot_kernel(const void *__restrict__ dY, bool dy_bf16, const __nv_bfloat16 *__restrict__ v,
+              const int32_t *__restrict__ sorted_rows, int32_t k, int64_t R, int64_t Dout,
+              bool by_token, float *__restrict__ dg) {
+    const int lane = threadIdx.x & 31;
+    const int64_t wstride = (int64_t)gridDim.x * kWarps;
+    for (int64_t p = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5); p < R; p += wstride) {
+        const int32_t i = __ldg(sorted_rows + p);
+        const int64_t row = by_token ? (int64_t)(i / k) : p;
+        const uint8_t *src = static_cast<const uint8_t *>(dY) + row * Dout * (dy_bf16 ? 2 : 4);
+        float acc = 0.f;
+        for (int64_t c = (int64_t)lane * 8; c < Dout; c += 32 * 8) {
+            float a[8], b[8];
+            load8(src, dy_bf16, c, a);
+            load8(v + p * Dout, true, c, b);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc = fmaf(a[j], b[j], acc);
+        }
+#pragma unroll
+        for (int d = 16; d > 0; d >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, d);
+        if (lane == 0) dg[i] = acc;
+    }
+}
+
+unsigned warp_grid(int64_t rows) {
+    int64_t blocks = (rows + kWarps - 1) / kWarps;
+    const int64_t cap = (int64_t)num_sms() * 16;
+    if (blocks > cap) blocks = cap;
+    return (unsigned)(blocks < 1 ? 1 : blocks);
+}
+
+}  // namespace
+
+void launch_cast_bf16(const float *src, void *dst, int64_t n, cudaStream_t s) {
+    const int64_t n8 = n / 8;
+    int64_t blocks = (n8 + 255) / 256;
+    const int64_t cap = (int64_t)num_sms() * 8;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    cast_bf16_kernel<<<(unsigned)blocks, 256, 0, s>>>(src, static_cast<__nv_bfloat16 *>(dst), n8);
+}
+
+void launch_gate_rows(const void *dY, bool dy_bf16, const int32_t *sorted_rows, const float *gates,
+                      int32_t k, int64_t R, int64_t Dout, bool by_token, void *dv, cudaStream_t s) {
+    gate_rows_kernel<<<warp_grid(R), kWarps * 32, 0, s>>>(dY, dy_bf16, sorted_rows, gates, k, R,
+                                                          Dout, by_token,
+                                                          static_cast<__nv_bfloat16 *>(dv));
+}
+
+void launch_rowdot(const void *dY, bool dy_bf16, const void *v, const int32_t *sorted_rows,
+                   int32_t k, int64_t R, int64_t Dout, bool by_token, float *dg, cudaStream_t s) {
+    rowdot_kernel<<<warp_grid(R), kWarps * 32, 0, s>>>(dY, dy_bf16,
+                                                       static_cast<const __nv_bfloat16 *>(v),
+                                                       sorted_rows, k, R, Dout, by_token, dg);
+}
+
+}  // namespace moe

@@ -29,7 +29,9 @@
 //   warps 2-5   epilogue: tcgen05.ld of the accumulator (thread = tile row), then SwiGLU + bf16
 //               store, or gate * acc and red.global.add.v4.f32 into out[token].
 // Stages: 4 x (A 16 KB + B 32 KB), 128-byte swizzle; A is K-major, B (weights, N contiguous)
-// is MN-major. Two accumulators let the epilogue of tile i overlap the mainloop of tile i+1.
+// is MN-major, or K-major for the transposed weights of the backward pass (BKM: a weight
+// [E, Din, Dout] read as W^T, one 64 x 256 box per stage). Two accumulators let the epilogue of
+// tile i overlap the mainloop of tile i+1.
 // Tile schedule: every CTA derives it from expert_offsets on the device (no host sync):
 // tiles are ordered expert-major, then N tile, then M tile, so the CTAs running at one time
 // share expert weight tiles and gathered rows through L2. Waits are bounded (see mbar_wait).
@@ -43,7 +45,7 @@ namespace {
 
 using namespace gemm;
 
-template <bool BF16, bool GATHER, bool GLU, bool SCATTER, bool ROUTER>
+template <bool BF16, bool GATHER, bool GLU, bool SCATTER, bool ROUTER, bool BKM>
 __global__ void __launch_bounds__(GATHER ? THREADS + GATHER_THREADS : THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     const __grid_constant__ CUtensorMap tmB0,
@@ -55,10 +57,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     constexpr int CHUNK = BK * KBYTES;        // bytes of one B chunk
     constexpr int B_KSTEP = (32 / EB) * KBYTES;  // bytes of B per MMA K step (32 bytes of K)
     constexpr int OUT_COLS = GLU ? BN / 2 : BN;  // output columns per tile
-    constexpr uint32_t IDESC = dev::idesc_f32acc(BF16, BM, BN, true);
+    static_assert(!(BKM && (GLU || ROUTER)), "K-major B is for the plain grouped GEMM");
+    constexpr uint32_t IDESC = dev::idesc_f32acc(BF16, BM, BN, !BKM);
     // A tile with at most 64 rows (an expert's short last tile) runs an M=64 MMA: half the tensor
     // work; its accumulator rows 16j + i (i < 16) sit in TMEM lanes 32j + i.
-    constexpr uint32_t IDESC64 = dev::idesc_f32acc(BF16, 64, BN, true);
+    constexpr uint32_t IDESC64 = dev::idesc_f32acc(BF16, 64, BN, !BKM);
     // B (weights, N contiguous) is MN-major: 128-byte swizzle for bf16 (8-row atoms of 1024 B);
     // tf32 needs the 32-byte-unit variant (4-row atoms of 512 B).
     constexpr uint32_t B_LAYOUT = BF16 ? dev::kLayoutSw128 : dev::kLayoutSw128Base32;
@@ -95,7 +98,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     if (warp == 0 && lane == 0) {
         dev::prefetch_tmap(&tmA);
         dev::prefetch_tmap(&tmB0);
-        if (GLU) dev::prefetch_tmap(&tmB1);
+        if (GLU || BKM) dev::prefetch_tmap(&tmB1);
     }
     if (warp == 1) {
         dev::tmem_alloc(&st.tmem_base, TMEM_COLS);
@@ -150,7 +153,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                 __syncwarp();
                 const int kc = kb * BK;
                 if (!GATHER && lane == 0) dev::tma_load_2d(sA, &tmA, &st.full[s], kc, ti.row_begin);
-                if (lane == 0) {
+                if (BKM && lane == 0) {
+                    const bool hi = kc >= p.k_split;
+                    dev::tma_load_3d(sB, hi ? &tmB1 : &tmB0, &st.full[s], hi ? kc - p.k_split : kc,
+                                     n0, ti.e);
+                } else if (lane == 0) {
 #pragma unroll
                     for (int c = 0; c < NCH; ++c) {
                         if (c >= nch) break;
@@ -211,7 +218,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     for (int kk = 0; kk < KBYTES / 32; ++kk) {
                         const uint64_t ad =
                             dev::sdesc(sA + kk * 32, 16, 1024, dev::kLayoutSw128);
-                        const uint64_t bd = dev::sdesc(sB + kk * B_KSTEP, CHUNK, B_SBO, B_LAYOUT);
+                        const uint64_t bd =
+                            BKM ? dev::sdesc(sB + kk * 32, 16, 1024, dev::kLayoutSw128)
+                                : dev::sdesc(sB + kk * B_KSTEP, CHUNK, B_SBO, B_LAYOUT);
                         if (BF16) dev::mma_bf16(d_tmem, ad, bd, tile_idesc, (kb | kk) != 0);
                         else dev::mma_tf32(d_tmem, ad, bd, tile_idesc, (kb | kk) != 0);
                     }
@@ -462,12 +471,12 @@ int encode_tmap(CUtensorMap *m, bool bf16, int rank, const void *base, const uin
 
 namespace {
 
-template <bool BF16, bool GATHER, bool GLU, bool SCATTER, bool ROUTER = false>
+template <bool BF16, bool GATHER, bool GLU, bool SCATTER, bool ROUTER = false, bool BKM = false>
 int launch_t(const GemmArgs &a, cudaStream_t s) {
     constexpr int EB = BF16 ? 2 : 4;
     constexpr int BK = KBYTES / EB;
     constexpr int CW = KBYTES / EB;
-    auto kern = grouped_gemm_kernel<BF16, GATHER, GLU, SCATTER, ROUTER>;
+    auto kern = grouped_gemm_kernel<BF16, GATHER, GLU, SCATTER, ROUTER, BKM>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [&] {
@@ -485,7 +494,26 @@ int launch_t(const GemmArgs &a, cudaStream_t s) {
         int rc = encode_tmap(&mA, BF16, 2, a.A, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
         if (rc) return rc;
     }
-    {
+    if (BKM) {
+        // [E, N, K0] and [E, N, K - K0] with K contiguous, one (BK x BN) box per stage
+        const int64_t k0 = a.B1 != nullptr ? a.k_split : a.K;
+        if (a.B1 != nullptr && (k0 <= 0 || k0 >= a.K || k0 % BK != 0))
+            return set_error(MOE_ERR_UNSUPPORTED, "K split %lld is not a positive multiple of %d "
+                             "below K=%lld", (long long)k0, BK, (long long)a.K);
+        const uint32_t box[3] = {(uint32_t)BK, (uint32_t)BN, 1u};
+        const uint64_t dims0[3] = {(uint64_t)k0, (uint64_t)a.N, (uint64_t)a.E};
+        const uint64_t str0[2] = {(uint64_t)k0 * EB, (uint64_t)a.N * k0 * EB};
+        int rc = encode_tmap(&mB0, BF16, 3, a.B0, dims0, str0, box, CU_TENSOR_MAP_SWIZZLE_128B);
+        if (rc) return rc;
+        if (a.B1 != nullptr) {
+            const uint64_t dims1[3] = {(uint64_t)(a.K - k0), (uint64_t)a.N, (uint64_t)a.E};
+            const uint64_t str1[2] = {(uint64_t)(a.K - k0) * EB, (uint64_t)a.N * (a.K - k0) * EB};
+            rc = encode_tmap(&mB1, BF16, 3, a.B1, dims1, str1, box, CU_TENSOR_MAP_SWIZZLE_128B);
+            if (rc) return rc;
+        } else {
+            mB1 = mB0;
+        }
+    } else {
         const uint64_t dims[3] = {(uint64_t)a.N, (uint64_t)a.K, ROUTER ? 1u : (uint64_t)a.E};
         const uint64_t str[2] = {(uint64_t)a.N * EB, (uint64_t)a.N * a.K * EB};
         const uint32_t box[3] = {(uint32_t)CW, (uint32_t)BK, 1u};
@@ -527,6 +555,7 @@ int launch_t(const GemmArgs &a, cudaStream_t s) {
         kp.stage_bytes = STAGE_BYTES;
         kp.stages = STAGES;
     }
+    kp.k_split = (int32_t)(BKM && a.B1 != nullptr ? a.k_split : a.K + BK);
     kp.zero_ptr = reinterpret_cast<float4 *>(a.zero_ptr);
     kp.zero_n4 = a.zero_n / 4;
     kp.status = a.status;
@@ -542,8 +571,17 @@ int launch_grouped_gemm(const GemmArgs &a, cudaStream_t s) {
     // instantiated forms: (gather, glu, scatter) in {(1,1,0), (0,0,1), (1,0,0), (1,0,1),
     // (0,0,0)} x {bf16, f32}
 #define MOE_DISPATCH(BF, G, L, SC)                                                          \
-    if (a.bf16 == BF && a.gather == G && a.glu == L && a.scatter == SC)                     \
+    if (!a.b_kmajor && a.bf16 == BF && a.gather == G && a.glu == L && a.scatter == SC)      \
         return launch_t<BF, G, L, SC>(a, s);
+#define MOE_DISPATCH_KM(G, SC)                                                              \
+    if (a.b_kmajor && a.bf16 && a.gather == G && !a.glu && a.scatter == SC)                 \
+        return launch_t<true, G, false, SC, false, true>(a, s);
+    // B K-major (bf16): the input-gradient GEMMs of the backward pass
+    MOE_DISPATCH_KM(true, true)
+    MOE_DISPATCH_KM(true, false)
+    MOE_DISPATCH_KM(false, true)
+    MOE_DISPATCH_KM(false, false)
+#undef MOE_DISPATCH_KM
     MOE_DISPATCH(true, true, true, false)
     MOE_DISPATCH(true, false, false, true)
     MOE_DISPATCH(true, true, false, false)

@@ -1,0 +1,336 @@
+// Weight gradient of ParallelLinear on the sm_100a tensor cores: for every expert e,
+//   dW[e] = sum over the slots p of e of  src_p^T (x) dv_p        ([Din, Dout], fp32)
+// with src_p = X[sorted_rows[p] / k] (gathered token rows) or X[p] (slot-ordered rows) and dv_p
+// the gated output-gradient rows in slot order. The reduction runs over an expert's slots, so the
+// K extent of a tile is that expert's row count: any value, zero included.
+//
+// Source: ScatterMoE guide, "3. Fused Backward Pass Dynamics" (the weight gradient of expert e
+// accumulates the outer products of its tokens' inputs and gated output gradients). The guide
+// reduces inside shared memory to avoid global atomics; here each output tile is owned by one CTA
+// and reduced in TMEM over the expert's slots, so no atomics are needed either.
+//
+// Design (one CTA per SM, persistent, the forward kernel's warp roles):
+//   warp 0     TMA producer of B: the stage's 64 dv rows x 256 columns (4 boxes of 64 x 64,
+//              128-byte swizzle: MN-major, the K index is the row).
+//   warps 6-9  cp.async gatherers of A: the stage's 64 source rows x 128 columns of Din, written
+//              MN-major in the same swizzle (row r of the stage at 128-byte line r of each
+//              64-column chunk); slots past the expert's end and columns past Din are zero-filled.
+//              The row indices of the next stage are loaded one stage ahead.
+//   warp 1     TMEM owner (two 128 x 256 fp32 accumulators) and MMA issuer: 4 MMAs of M=128
+//              (Din), N=256 (Dout), K=16 rows per stage, both operands MN-major.
+//   warps 2-5  epilogue: accumulator lane m -> dW[e][m0 + m][n0 .. n0 + 255]; a tile of an
+//              expert without slots stores zeros.
+// Tiles are (expert, N tile, M tile), expert-major, so the CTAs running at once share an
+// expert's rows through L2. Every wait is bounded (mbar_wait).
+#include "gemm_common.cuh"
+
+#include <mutex>
+
+namespace moe {
+namespace {
+
+using namespace gemm;
+
+constexpr int WK = 64;                     // slots (K rows) per stage
+constexpr int WCH = 64 * KBYTES;           // one 64-column chunk of a stage: 64 rows x 128 B
+constexpr int WA_BYTES = 2 * WCH;          // A: 128 columns of Din
+constexpr int WB_BYTES = 4 * WCH;          // B: 256 columns of Dout
+static_assert(WA_BYTES == A_BYTES && WB_BYTES == B_BYTES, "stage layout of the forward kernel");
+
+struct WParams {
+    const uint8_t *X;
+    int64_t Din, Dout;
+    const int32_t *offsets;
+    const int32_t *sorted_rows;
+    int32_t E, k, gather;
+    float *dW;
+    int32_t m_tiles, n_tiles;
+    unsigned *status;
+    int64_t wait_limit_ns;
+};
+
+__device__ __forceinline__ void wtile(int t, int per_e, int m_tiles, int &e, int &n, int &m) {
+    e = t / per_e;
+    const int local = t - e * per_e;
+    n = local / m_tiles;
+    m = local - n * m_tiles;
+}
+
+__global__ void __launch_bounds__(THREADS + GATHER_THREADS, 1)
+grouped_wgrad_kernel(const __grid_constant__ CUtensorMap tmB, const WParams p) {
+    constexpr uint32_t IDESC = dev::idesc_f32acc(true, BM, BN, true, true);
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    SmemTail &st = *reinterpret_cast<SmemTail *>(smem + STAGE_AREA);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int E = p.E;
+    const int per_e = p.m_tiles * p.n_tiles;
+    const int total = E * per_e;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            dev::mbar_init(&st.full[s], 1 + GATHER_THREADS);
+            dev::mbar_init(&st.empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            dev::mbar_init(&st.tfull[b], 1);
+            dev::mbar_init(&st.tempty[b], 4);
+        }
+        dev::mbar_init(&st.drain, 1);
+        st.abort = 0;
+        dev::fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) dev::prefetch_tmap(&tmB);
+    if (warp == 1) {
+        dev::tmem_alloc(&st.tmem_base, TMEM_COLS);
+        dev::tmem_relinquish();
+        dev::tc_fence_before();
+    }
+    for (int e = threadIdx.x; e <= E; e += blockDim.x) st.off[e] = __ldg(p.offsets + e);
+    __syncthreads();
+    dev::tc_fence_after();
+    const uint32_t tmem_base = st.tmem_base;
+    volatile int *abort = &st.abort;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------------ TMA producer (B)
+        uint32_t s = 0, ph = 0, issued = 0, last_par = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+            int e, n, m;
+            wtile(t, per_e, p.m_tiles, e, n, m);
+            const int r0 = st.off[e], nkb = (st.off[e + 1] - r0 + WK - 1) / WK;
+            for (int kb = 0; kb < nkb; ++kb) {
+                bool w = true;
+                if (lane == 0)
+                    w = dev::mbar_wait(&st.empty[s], ph ^ 1u, abort, p.status, p.wait_limit_ns,
+                                       kKernelGemm);
+                w = __shfl_sync(0xffffffffu, w, 0);
+                if (!w) {
+                    ok = false;
+                    break;
+                }
+                if (lane == 0) {
+                    uint8_t *sB = smem + (size_t)s * STAGE_BYTES + WA_BYTES;
+                    dev::mbar_arrive_expect_tx(&st.full[s], (uint32_t)WB_BYTES);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+                        dev::tma_load_2d(sB + c * WCH, &tmB, &st.full[s], n * BN + c * 64,
+                                         r0 + kb * WK);
+                }
+                issued |= 1u << s;
+                last_par = (last_par & ~(1u << s)) | (ph << s);
+                if (++s == STAGES) {
+                    s = 0;
+                    ph ^= 1u;
+                }
+            }
+        }
+        if (lane == 0) {
+            for (int s2 = 0; s2 < STAGES; ++s2)
+                if (issued & (1u << s2))
+                    dev::mbar_wait(&st.full[s2], (last_par >> s2) & 1u, nullptr, p.status,
+                                   kDrainLimitNs, kKernelGemm);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            uint32_t s = 0, ph = 0;
+            int it = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++it) {
+                int e, n, m;
+                wtile(t, per_e, p.m_tiles, e, n, m);
+                const int nkb = (st.off[e + 1] - st.off[e] + WK - 1) / WK;
+                const uint32_t b = it & 1, aph = (it >> 1) & 1;
+                if (!dev::mbar_wait(&st.tempty[b], aph ^ 1u, abort, p.status, p.wait_limit_ns,
+                                    kKernelGemm))
+                    break;
+                dev::tc_fence_after();
+                const uint32_t d_tmem = tmem_base + b * BN;
+                for (int kb = 0; kb < nkb; ++kb) {
+                    if (!dev::mbar_wait(&st.full[s], ph, abort, p.status, p.wait_limit_ns,
+                                        kKernelGemm)) {
+                        ok = false;
+                        break;
+                    }
+                    dev::tc_fence_after();
+                    dev::fence_proxy_async_smem();  // cp.async rows -> tensor core
+                    const uint32_t sA = dev::smem_u32(smem + (size_t)s * STAGE_BYTES);
+                    const uint32_t sB = sA + WA_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < WK / 16; ++kk) {
+                        // 16 K rows per MMA: 16 lines of 128 B into every 64-column chunk
+                        const uint64_t ad =
+                            dev::sdesc(sA + kk * 16 * KBYTES, WCH, 1024, dev::kLayoutSw128);
+                        const uint64_t bd =
+                            dev::sdesc(sB + kk * 16 * KBYTES, WCH, 1024, dev::kLayoutSw128);
+                        dev::mma_bf16(d_tmem, ad, bd, IDESC, (kb | kk) != 0);
+                    }
+                    dev::mma_commit(&st.empty[s]);
+                    if (++s == STAGES) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                dev::mma_commit(&st.tfull[b]);  // also for a tile without slots (nothing pending)
+            }
+            dev::mma_commit(&st.drain);
+            dev::mbar_wait(&st.drain, 0, nullptr, p.status, kDrainLimitNs, kKernelGemm);
+            dev::tc_fence_before();
+        }
+        __syncwarp();
+    } else if (warp >= THREADS / 32) {
+        // ------------------------------------------------------------------ A gatherers
+        // thread -> stage row r = gt / 2 (a slot), half h = gt % 2 (64 columns = 128 B)
+        const int gt = threadIdx.x - THREADS;
+        const int r = gt >> 1, h = gt & 1;
+        const int64_t row_bytes = p.Din * 2;
+        uint32_t s = 0, ph = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+            int e, n, m;
+            wtile(t, per_e, p.m_tiles, e, n, m);
+            const int r0 = st.off[e], r1 = st.off[e + 1];
+            const int nkb = (r1 - r0 + WK - 1) / WK;
+            const int64_t col0 = ((int64_t)m * BM + h * 64) * 2;  // byte offset in a row
+            // source row of this thread's slot, one stage ahead
+            auto src_row = [&](int kb) -> int64_t {
+                const int slot = r0 + kb * WK + r;
+                if (slot >= r1) return -1;
+                return p.gather ? (int64_t)(__ldg(p.sorted_rows + slot) / p.k) : (int64_t)slot;
+            };
+            int64_t row = nkb > 0 ? src_row(0) : -1;
+            for (int kb = 0; kb < nkb; ++kb) {
+                const int64_t next = kb + 1 < nkb ? src_row(kb + 1) : -1;
+                bool w = true;
+                if (lane == 0)
+                    w = dev::mbar_wait(&st.empty[s], ph ^ 1u, abort, p.status, p.wait_limit_ns,
+                                       kKernelGemm);
+                w = __shfl_sync(0xffffffffu, w, 0);
+                if (!w) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t dst0 = dev::smem_u32(smem + (size_t)s * STAGE_BYTES) + h * WCH +
+                                      r * KBYTES;
+                const uint8_t *src = row >= 0 ? p.X + row * row_bytes + col0 : p.X;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const bool in = row >= 0 && col0 + j * 16 < row_bytes;
+                    dev::cp_async16(dst0 + ((j ^ (r & 7)) << 4), in ? src + j * 16 : p.X,
+                                    in ? 16u : 0u);
+                }
+                dev::cp_async_arrive_noinc(&st.full[s]);
+                row = next;
+                if (++s == STAGES) {
+                    s = 0;
+                    ph ^= 1u;
+                }
+            }
+        }
+        dev::cp_async_wait_all();
+    } else {
+        // ------------------------------------------------------------------ epilogue
+        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        const int mr = q * 32 + lane;
+        int it = 0;
+        for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
+            int e, n, m;
+            wtile(t, per_e, p.m_tiles, e, n, m);
+            const bool empty_e = st.off[e + 1] == st.off[e];
+            const uint32_t b = it & 1, aph = (it >> 1) & 1;
+            bool w = true;
+            if (lane == 0)
+                w = dev::mbar_wait(&st.tfull[b], aph, abort, p.status, p.wait_limit_ns,
+                                   kKernelGemm);
+            w = __shfl_sync(0xffffffffu, w, 0);
+            if (!w) break;
+            dev::tc_fence_after();
+            const int64_t grow = (int64_t)m * BM + mr;  // row of dW[e]
+            const bool row_ok = grow < p.Din;
+            float *dst = p.dW + ((int64_t)e * p.Din + (row_ok ? grow : 0)) * p.Dout;
+            const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + b * BN;
+#pragma unroll 1
+            for (int c = 0; c < BN / 32; ++c) {
+                uint32_t v[32];
+                if (!empty_e) {
+                    dev::tmem_ld32(tbase + c * 32, v);
+                    dev::tmem_ld_wait();
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] = 0u;
+                }
+                const int64_t col0 = (int64_t)n * BN + c * 32;
+                if (row_ok) {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        if (col0 + j * 4 < p.Dout)
+                            *reinterpret_cast<float4 *>(dst + col0 + j * 4) = make_float4(
+                                __uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+                }
+            }
+            dev::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) dev::mbar_arrive(&st.tempty[b]);
+        }
+    }
+
+    __syncthreads();
+    if (warp == 1) {
+        dev::tc_fence_after();
+        dev::tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+}  // namespace
+
+int launch_grouped_wgrad(const WgradArgs &a, cudaStream_t s) {
+    const int64_t m_tiles = (a.Din + BM - 1) / BM, n_tiles = (a.Dout + BN - 1) / BN;
+    if (a.R <= 0 || a.E <= 0) {
+        // no slot at all: every expert's gradient is zero
+        launch_zero_f32(a.dW, (int64_t)a.E * a.Din * a.Dout, nullptr, s);
+        return MOE_OK;
+    }
+    if ((int64_t)a.E * m_tiles * n_tiles >= (int64_t(1) << 31))
+        return set_error(MOE_ERR_UNSUPPORTED, "weight-gradient tile count too large");
+    auto kern = grouped_wgrad_kernel;
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [&] {
+        attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)SMEM_BYTES);
+    });
+    if (attr_err != cudaSuccess)
+        return set_error(MOE_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(attr_err));
+    CUtensorMap mB;
+    {
+        const uint64_t dims[2] = {(uint64_t)a.Dout, (uint64_t)a.R};
+        const uint64_t str[1] = {(uint64_t)a.Dout * 2};
+        const uint32_t box[2] = {64u, (uint32_t)WK};
+        int rc = encode_tmap(&mB, true, 2, a.dv, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
+        if (rc) return rc;
+    }
+    WParams wp;
+    wp.X = reinterpret_cast<const uint8_t *>(a.X);
+    wp.Din = a.Din;
+    wp.Dout = a.Dout;
+    wp.offsets = a.offsets;
+    wp.sorted_rows = a.sorted_rows;
+    wp.E = a.E;
+    wp.k = a.k;
+    wp.gather = a.gather ? 1 : 0;
+    wp.dW = a.dW;
+    wp.m_tiles = (int32_t)m_tiles;
+    wp.n_tiles = (int32_t)n_tiles;
+    wp.status = a.status;
+    wp.wait_limit_ns = a.wait_limit_ns;
+    kern<<<num_sms(), THREADS + GATHER_THREADS, SMEM_BYTES, s>>>(mB, wp);
+    return MOE_OK;
+}
+
+}  // namespace moe

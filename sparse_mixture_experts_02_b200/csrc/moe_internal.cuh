@@ -53,6 +53,11 @@ struct GemmArgs {
     int32_t E, k;
     int64_t K, N;
     bool bf16, gather, glu, scatter;
+    // B K-major (one-CTA kernel, non-GLU): B0 is [E, N, K] with K contiguous (a weight [E, N, K]
+    // read as its transpose); with B1 set, B0 covers K indices < k_split ([E, N, k_split]) and
+    // B1 the rest ([E, N, K - k_split]); k_split is a multiple of 64 bf16 elements.
+    bool b_kmajor;
+    int64_t k_split;
     const float *bias;      // router mode only
     int32_t *top_e;
     float *top_w;
@@ -68,6 +73,28 @@ int launch_grouped_gemm_2sm(const GemmArgs &a, cudaStream_t s);
 // pair tiles waste little there); the environment variable MOE_GEMM_2SM=0/1 forces either kernel.
 bool prefer_2sm(int64_t R, int32_t E);
 int launch_debug_wait(int64_t limit_ns, unsigned *status, cudaStream_t s);
+// Weight gradient of ParallelLinear: dW[e] = sum over the slots p of expert e of
+// src_p^T (x) dv_p, src_p = X[sorted_rows[p] / k] (gather) or X[p], dv [R, Dout] bf16 in slot
+// order; dW [E, Din, Dout] fp32 is overwritten (zeros for experts without slots). bf16 only.
+struct WgradArgs {
+    const void *X;          // [S, Din] (gather) or [R, Din]
+    const void *dv;         // [R, Dout]
+    const int32_t *offsets; // [E+1]
+    const int32_t *sorted_rows;
+    int64_t Din, Dout, R;
+    int32_t E, k;
+    bool gather;
+    float *dW;
+    unsigned *status;
+    int64_t wait_limit_ns;
+};
+int launch_grouped_wgrad(const WgradArgs &a, cudaStream_t s);
+// Backward helpers (backward.cu), one warp per slot; Dout a multiple of 8, rows 16-byte aligned.
+void launch_cast_bf16(const float *src, void *dst, int64_t n, cudaStream_t s);
+void launch_gate_rows(const void *dY, bool dy_bf16, const int32_t *sorted_rows, const float *gates,
+                      int32_t k, int64_t R, int64_t Dout, bool by_token, void *dv, cudaStream_t s);
+void launch_rowdot(const void *dY, bool dy_bf16, const void *v, const int32_t *sorted_rows,
+                   int32_t k, int64_t R, int64_t Dout, bool by_token, float *dg, cudaStream_t s);
 // Router on the tensor cores (bf16, E % 8 == 0): logits of 128-token tiles in TMEM, top-k and
 // softmax in the epilogue.
 int launch_route_tc(const void *x, const void *w_gate, const float *bias, int64_t S, int64_t D,
@@ -281,9 +308,10 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t
 // [4,6) D format = 1 (f32); [7,10) A format, [10,13) B format (1 = bf16, 2 = tf32);
 // [15] A major (0 = K-major); [16] B major (1 = MN-major); [17,23) N>>3; [24,29) M>>4.
 __host__ __device__ constexpr uint32_t idesc_f32acc(bool bf16, uint32_t M, uint32_t N,
-                                                     bool b_mn_major) {
+                                                     bool b_mn_major, bool a_mn_major = false) {
     return (1u << 4) | ((bf16 ? 1u : 2u) << 7) | ((bf16 ? 1u : 2u) << 10) |
-           ((b_mn_major ? 1u : 0u) << 16) | ((N >> 3) << 17) | ((M >> 4) << 24);
+           ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) | ((N >> 3) << 17) |
+           ((M >> 4) << 24);
 }
 
 // ---- clusters of two CTAs (tcgen05 cta_group::2) ---------------------------------------------------
