@@ -360,3 +360,94 @@ void oracle_scatter_linear_backward(const float *X, const float *W, const float 
     }
     free(slot_e);
 }
+
+/* Backward of the expert MLP forward (oracle_mlp_forward) for all S tokens, given the gradient of
+ * the output dout [S, D]. The routing is the oracle's own top-k, or given_top_experts ([S, k]) if
+ * non-null; the selection itself has no derivative. Per token s and selected expert e = J_j,
+ * with a = x W_gate_e[e], b = x W_up[e], h = silu(a) * b, v = h W_down[e], w = softmax(l_J):
+ *   dw_j = dout . v;  dv = w_j dout;  dh = dv W_down[e]^T;  dW_down[e] += h^T dv
+ *   da = dh * b * silu'(a), silu'(z) = sig(z) (1 + z (1 - sig(z)));  db = dh * silu(a)
+ *   dW_gate_e[e] += x^T da;  dW_up[e] += x^T db;  dx += da W_gate_e[e]^T + db W_up[e]^T
+ *   softmax over the selected logits: dl_j = w_j (dw_j - sum_j' w_j' dw_j')
+ *   dW_gate[:, e] += x dl_j;  dx += dl_j W_gate[:, e]
+ * (the ScatterMoE guide's backward of each ParallelLinear, "3. Fused Backward Pass Dynamics",
+ * chained through SwiGLU and the router softmax). fp64; every output is overwritten:
+ * dx [S, D], dw_gate [D, E], dw_gate_e and dw_up [E, D, F], dw_down [E, F, D]. */
+void oracle_mlp_backward(const float *x, const float *w_gate, const float *bias,
+                         const float *w_gate_e, const float *w_up, const float *w_down,
+                         const float *dout, int64_t S, int64_t D, int64_t F, int32_t E, int32_t k,
+                         const int32_t *given_top_experts, double *dx, double *dw_gate,
+                         double *dw_gate_e, double *dw_up, double *dw_down) {
+    memset(dx, 0, sizeof(double) * (size_t)S * (size_t)D);
+    memset(dw_gate, 0, sizeof(double) * (size_t)D * (size_t)E);
+    memset(dw_gate_e, 0, sizeof(double) * (size_t)E * (size_t)D * (size_t)F);
+    memset(dw_up, 0, sizeof(double) * (size_t)E * (size_t)D * (size_t)F);
+    memset(dw_down, 0, sizeof(double) * (size_t)E * (size_t)F * (size_t)D);
+    double *l = (double *)malloc(sizeof(double) * (size_t)E);
+    double *a = (double *)malloc(sizeof(double) * (size_t)F);
+    double *b = (double *)malloc(sizeof(double) * (size_t)F);
+    double *h = (double *)malloc(sizeof(double) * (size_t)F);
+    double *dh = (double *)malloc(sizeof(double) * (size_t)F);
+    double *da = (double *)malloc(sizeof(double) * (size_t)F);
+    double *db = (double *)malloc(sizeof(double) * (size_t)F);
+    double *dv = (double *)malloc(sizeof(double) * (size_t)D);
+    int32_t J[64];
+    double w[64], dwj[64];
+    for (int64_t s = 0; s < S; ++s) {
+        const float *xs = x + s * D;
+        const float *ds = dout + s * D;
+        double *dxs = dx + s * D;
+        logits_one(xs, w_gate, bias, D, E, l, NULL);
+        if (given_top_experts) {
+            for (int32_t j = 0; j < k; ++j) J[j] = given_top_experts[s * k + j];
+            oracle_weights_for(l, J, 1, E, k, w);
+        } else {
+            topk_one(l, E, k, J, w);
+        }
+        for (int32_t j = 0; j < k; ++j) {
+            const int64_t e = J[j];
+            const float *wge = w_gate_e + e * D * F, *wu = w_up + e * D * F;
+            const float *wd = w_down + e * F * D;
+            expert_hidden(xs, wge, wu, D, F, a, b, h);
+            double dwv = 0.0;
+            for (int64_t f = 0; f < F; ++f) {
+                double vd_dot = 0.0;  /* (W_down[e] row f) . dout */
+                for (int64_t d = 0; d < D; ++d) vd_dot += (double)wd[f * D + d] * (double)ds[d];
+                dwv += h[f] * vd_dot;
+                dh[f] = w[j] * vd_dot;
+            }
+            dwj[j] = dwv;
+            for (int64_t d = 0; d < D; ++d) dv[d] = w[j] * (double)ds[d];
+            double *dwd = dw_down + e * F * D;
+            for (int64_t f = 0; f < F; ++f)
+                for (int64_t d = 0; d < D; ++d) dwd[f * D + d] += h[f] * dv[d];
+            for (int64_t f = 0; f < F; ++f) {
+                const double sg = 1.0 / (1.0 + exp(-a[f]));
+                da[f] = dh[f] * b[f] * sg * (1.0 + a[f] * (1.0 - sg));
+                db[f] = dh[f] * a[f] * sg;
+            }
+            double *dge = dw_gate_e + e * D * F, *dup = dw_up + e * D * F;
+            for (int64_t d = 0; d < D; ++d) {
+                const double xd = (double)xs[d];
+                double acc = 0.0;
+                for (int64_t f = 0; f < F; ++f) {
+                    dge[d * F + f] += xd * da[f];
+                    dup[d * F + f] += xd * db[f];
+                    acc += da[f] * (double)wge[d * F + f] + db[f] * (double)wu[d * F + f];
+                }
+                dxs[d] += acc;
+            }
+        }
+        double mean = 0.0;
+        for (int32_t j = 0; j < k; ++j) mean += w[j] * dwj[j];
+        for (int32_t j = 0; j < k; ++j) {
+            const double dl = w[j] * (dwj[j] - mean);
+            const int64_t e = J[j];
+            for (int64_t d = 0; d < D; ++d) {
+                dw_gate[d * E + e] += (double)xs[d] * dl;
+                dxs[d] += dl * (double)w_gate[d * E + e];
+            }
+        }
+    }
+    free(l); free(a); free(b); free(h); free(dh); free(da); free(db); free(dv);
+}
