@@ -181,8 +181,33 @@ int moe_mlp_forward(const void *x, const void *w_gate, const float *logit_bias,
                     size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * Backward of moe_mlp_forward (bf16): given dout [S, D] float32 (the gradient of out) and the
+ * workspace of the forward call on the same inputs (fwd_ws: its routing, sparse map and h), the
+ * float32 gradients (all overwritten, all required):
+ *   dx [S, D], dw_gate [D, E], dw_gate_e [E, D, F], dw_up [E, D, F], dw_down [E, F, D].
+ * The selection of the top-k experts has no derivative; the weights are the softmax over the
+ * selected logits, differentiated through it. Steps on `stream`:
+ *   1. dout -> bf16.
+ *   2. dh = dout[s] . W_down[e]^T per slot (the forward's grouped GEMM, W_down read K-major).
+ *   3. a = x W_gate_e[e] and b = x W_up[e] recomputed.
+ *   4. SwiGLU backward: the route-weight gradient dh . h, then da and db.
+ *   5. dW_down (weight-gradient GEMM over each expert's slots).
+ *   6. dx += [da | db] . [W_gate_e ; W_up]^T (scatter-added into tokens).
+ *   7. dW_gate_e and dW_up.
+ *   8. Router backward: the softmax Jacobian, then dx += dl W_gate^T and dW_gate = x^T dl.
+ * ScatterMoE guide, "3. Fused Backward Pass Dynamics" (each ParallelLinear's input and weight
+ * gradients). Constraints beyond the forward's: bf16 only, E a multiple of 8, F a multiple of 64.
+ * ws: moe_workspace_size("mlp_backward", S, D, F, E, k, dt) bytes.
+ */
+int moe_mlp_backward(const void *x, const void *w_gate, const void *w_gate_e, const void *w_up,
+                     const void *w_down, const float *dout, int64_t S, int64_t D, int64_t F,
+                     int32_t E, int32_t k, moe_dtype dt, const void *fwd_ws, size_t fwd_ws_bytes,
+                     float *dx, float *dw_gate, float *dw_gate_e, float *dw_up, float *dw_down,
+                     void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
  * Workspace bytes for op = "sparse_map", "scatter_linear", "scatter_linear_backward" (D = Din,
- * F = Dout) or "mlp_forward" (unused sizes may be 0). Returns 0 for an unknown op or sizes
+ * F = Dout), "mlp_forward" or "mlp_backward" (unused sizes may be 0). Returns 0 for an unknown op or sizes
  * outside the limits.
  */
 size_t moe_workspace_size(const char *op, int64_t S, int64_t D, int64_t F, int32_t E, int32_t k,

@@ -24,7 +24,7 @@ STATUS_NAMES = {0: "MOE_OK", -1: "MOE_ERR_INVALID_ARG", -2: "MOE_ERR_UNSUPPORTED
                 -6: "MOE_ERR_DEVICE_TIMEOUT"}
 
 EXPORTS = ["moe_route_topk", "moe_sparse_map", "moe_sparse_map_noalloc", "moe_scatter_linear",
-           "moe_scatter_linear_backward", "moe_mlp_forward",
+           "moe_scatter_linear_backward", "moe_mlp_forward", "moe_mlp_backward",
            "moe_workspace_size", "moe_workspace_view", "moe_last_error",
            "moe_check_device_status", "moe_profile_events", "moe_debug_wait_timeout",
            "moe_last_launch_count"]
@@ -52,6 +52,8 @@ def _load():
                                                 c_int, c_int, P, P, P, P, ctypes.c_size_t, P]
     lib.moe_mlp_forward.argtypes = [P, P, P, P, P, P, i64, i64, i64, i32, i32, c_int, P, P,
                                     ctypes.c_size_t, P]
+    lib.moe_mlp_backward.argtypes = [P, P, P, P, P, P, i64, i64, i64, i32, i32, c_int, P,
+                                     ctypes.c_size_t, P, P, P, P, P, P, ctypes.c_size_t, P]
     lib.moe_workspace_size.argtypes = [ctypes.c_char_p, i64, i64, i64, i32, i32, c_int]
     lib.moe_workspace_size.restype = ctypes.c_size_t
     lib.moe_workspace_view.argtypes = [ctypes.c_char_p, i64, i64, i64, i32, i32, c_int]
@@ -62,6 +64,7 @@ def _load():
     lib.moe_debug_wait_timeout.argtypes = [i64, P, ctypes.c_size_t, P]
     for name in ("moe_route_topk", "moe_sparse_map", "moe_sparse_map_noalloc",
                  "moe_scatter_linear", "moe_scatter_linear_backward", "moe_mlp_forward",
+                 "moe_mlp_backward",
                  "moe_check_device_status", "moe_profile_events", "moe_debug_wait_timeout",
                  "moe_last_launch_count"):
         getattr(lib, name).restype = c_int
@@ -320,6 +323,35 @@ def mlp_forward(x: torch.Tensor, w_gate: torch.Tensor, w_gate_e: torch.Tensor,
     _check(_lib().moe_mlp_forward(_ptr(x), _ptr(w_gate), _ptr(logit_bias), _ptr(w_gate_e),
                                _ptr(w_up), _ptr(w_down), S, D, F, E, k, _dtype_code(x),
                                _ptr(out), _ptr(ws.buf), ws.buf.numel(), _stream(dev)))
+    return out
+
+
+def mlp_backward(x: torch.Tensor, w_gate: torch.Tensor, w_gate_e: torch.Tensor,
+                 w_up: torch.Tensor, w_down: torch.Tensor, k: int, dout: torch.Tensor,
+                 fwd_ws: ForwardWorkspace, ws: Optional[torch.Tensor] = None) -> dict:
+    """Backward of mlp_forward (moe_mlp_backward), bf16: given dout [S, D] float32 and the
+    workspace of the forward call on the same inputs (its routing, map and h), returns float32
+    {"dx" [S, D], "dw_gate" [D, E], "dw_gate_e" [E, D, F], "dw_up" [E, D, F],
+    "dw_down" [E, F, D]}."""
+    _req(x, "x", dim=2)
+    dev = x.device
+    S, D = x.shape
+    E, F = w_gate.shape[1], w_gate_e.shape[2]
+    if fwd_ws.shape != (S, D, F, E, k):
+        raise ValueError("the forward workspace was made for other sizes")
+    _req(dout, "dout", dtype=torch.float32, dim=2, device=dev)
+    out = {"dx": torch.empty((S, D), dtype=torch.float32, device=dev),
+           "dw_gate": torch.empty((D, E), dtype=torch.float32, device=dev),
+           "dw_gate_e": torch.empty((E, D, F), dtype=torch.float32, device=dev),
+           "dw_up": torch.empty((E, D, F), dtype=torch.float32, device=dev),
+           "dw_down": torch.empty((E, F, D), dtype=torch.float32, device=dev)}
+    if ws is None:
+        ws = alloc_workspace(workspace_size("mlp_backward", S, D, F, E, k, x.dtype), dev)
+    _check(_lib().moe_mlp_backward(
+        _ptr(x), _ptr(w_gate), _ptr(w_gate_e), _ptr(w_up), _ptr(w_down), _ptr(dout), S, D, F, E,
+        k, _dtype_code(x), _ptr(fwd_ws.buf), fwd_ws.buf.numel(), _ptr(out["dx"]),
+        _ptr(out["dw_gate"]), _ptr(out["dw_gate_e"]), _ptr(out["dw_up"]), _ptr(out["dw_down"]),
+        _ptr(ws), ws.numel(), _stream(dev)))
     return out
 
 

@@ -147,6 +147,29 @@ BwdLayout bwd_layout(int64_t S, int64_t Dout, int32_t k) {
     return L;
 }
 
+// MLP backward scratch (the forward's workspace supplies routing, map and h).
+struct MlpBwdLayout {
+    size_t status, dyb, dhp, a, b, dpre, dw, dv, dl, off1, total;
+};
+
+MlpBwdLayout mlp_bwd_layout(int64_t S, int64_t D, int64_t F, int32_t E, int32_t k) {
+    const int64_t R = S * k;
+    MlpBwdLayout L;
+    size_t o = 0;
+    L.status = o; o += kStatusBytes;
+    L.dyb = o; o = align_up(o + 2 * (size_t)S * (size_t)D);
+    L.dhp = o; o = align_up(o + 2 * (size_t)R * (size_t)F);
+    L.a = o; o = align_up(o + 2 * (size_t)R * (size_t)F);
+    L.b = o; o = align_up(o + 2 * (size_t)R * (size_t)F);
+    L.dpre = o; o = align_up(o + 4 * (size_t)R * (size_t)F);
+    L.dw = o; o = align_up(o + 4 * (size_t)R);
+    L.dv = o; o = align_up(o + 2 * (size_t)R * (size_t)D);
+    L.dl = o; o = align_up(o + 2 * (size_t)S * (size_t)E);
+    L.off1 = o; o = align_up(o + 2 * sizeof(int32_t));
+    L.total = o;
+    return L;
+}
+
 size_t map_ws_bytes(int64_t S, int32_t E, int32_t k) {
     return kStatusBytes + align_up(map_scratch_bytes(S * k, E));
 }
@@ -198,6 +221,10 @@ size_t moe_workspace_size(const char *op, int64_t S, int64_t D, int64_t F, int32
     if (strcmp(op, "scatter_linear_backward") == 0) {
         if (F <= 0) return 0;
         return bwd_layout(S, F, k).total;  // D = Din, F = Dout
+    }
+    if (strcmp(op, "mlp_backward") == 0) {
+        if (F <= 0 || D <= 0) return 0;
+        return mlp_bwd_layout(S, D, F, E, k).total;
     }
     if (strcmp(op, "mlp_forward") == 0) {
         if (F <= 0 || (dt != MOE_F32 && dt != MOE_BF16)) return 0;
@@ -581,3 +608,186 @@ int moe_debug_wait_timeout(int64_t limit_ns, void *ws, size_t ws_bytes, moe_stre
 }
 
 }  // extern "C"
+
+extern "C" int moe_mlp_backward(const void *x, const void *w_gate, const void *w_gate_e,
+                                const void *w_up, const void *w_down, const float *dout, int64_t S,
+                                int64_t D, int64_t F, int32_t E, int32_t k, moe_dtype dt,
+                                const void *fwd_ws, size_t fwd_ws_bytes, float *dx, float *dw_gate,
+                                float *dw_gate_e, float *dw_up, float *dw_down, void *ws,
+                                size_t ws_bytes, moe_stream_t stream) {
+    g_launches = 0;
+    int rc;
+    if ((rc = check_dtype(dt)) || (rc = check_dims(S, E, k)) || (rc = check_feat("D", D)) ||
+        (rc = check_feat("F", F)))
+        return rc;
+    if (dt != MOE_BF16) return set_error(MOE_ERR_UNSUPPORTED, "mlp_backward: bf16 inputs only");
+    if (E % 8 != 0)
+        return set_error(MOE_ERR_UNSUPPORTED, "mlp_backward: E must be a multiple of 8 (got %d)", E);
+    if (F % 64 != 0)
+        return set_error(MOE_ERR_UNSUPPORTED, "mlp_backward: F must be a multiple of 64 (got %lld)",
+                         (long long)F);
+    const int64_t R = S * k;
+    if ((rc = check_ptr("x", x, 16, S == 0)) || (rc = check_ptr("w_gate", w_gate, 16)) ||
+        (rc = check_ptr("w_gate_e", w_gate_e, 16)) || (rc = check_ptr("w_up", w_up, 16)) ||
+        (rc = check_ptr("w_down", w_down, 16)) || (rc = check_ptr("dout", dout, 16, S == 0)) ||
+        (rc = check_ptr("dx", dx, 16, S == 0)) || (rc = check_ptr("dw_gate", dw_gate, 16)) ||
+        (rc = check_ptr("dw_gate_e", dw_gate_e, 16)) || (rc = check_ptr("dw_up", dw_up, 16)) ||
+        (rc = check_ptr("dw_down", dw_down, 16)))
+        return rc;
+    const MlpLayout FL = mlp_layout(S, F, E, k, dt);
+    if (fwd_ws == nullptr || fwd_ws_bytes < FL.total)
+        return set_error(MOE_ERR_WORKSPACE, "the forward's workspace is missing or too small");
+    const MlpBwdLayout L = mlp_bwd_layout(S, D, F, E, k);
+    if ((rc = check_ws(ws, ws_bytes, L.total))) return rc;
+    if ((rc = check_device())) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    void *fws = const_cast<void *>(fwd_ws);
+    const int32_t *top_e = at<int32_t>(fws, FL.top_e);
+    const float *top_w = at<float>(fws, FL.top_w);
+    const int32_t *offsets = at<int32_t>(fws, FL.offsets);
+    const int32_t *sorted_rows = at<int32_t>(fws, FL.sorted_rows);
+    const void *h = at<void>(fws, FL.h);
+    unsigned *status = at<unsigned>(ws, L.status);
+    if (cudaMemsetAsync(status, 0, sizeof(unsigned), s) != cudaSuccess)
+        return set_error(MOE_ERR_CUDA, "cudaMemsetAsync of the status word failed");
+    int n = 0;
+    launch_zero_f32(dx, S * D, nullptr, s);
+    ++n;
+    if (R == 0) {
+        launch_zero_f32(dw_gate, D * E, nullptr, s);
+        launch_zero_f32(dw_gate_e, (int64_t)E * D * F, nullptr, s);
+        launch_zero_f32(dw_up, (int64_t)E * D * F, nullptr, s);
+        launch_zero_f32(dw_down, (int64_t)E * F * D, nullptr, s);
+        g_launches = n + 4;
+        return check_launch("mlp_backward");
+    }
+    void *dyb = at<void>(ws, L.dyb), *dhp = at<void>(ws, L.dhp), *av = at<void>(ws, L.a);
+    void *bv = at<void>(ws, L.b), *dpre = at<void>(ws, L.dpre), *dv = at<void>(ws, L.dv);
+    void *dl = at<void>(ws, L.dl);
+    float *dwr = at<float>(ws, L.dw);
+    int32_t *off1 = at<int32_t>(ws, L.off1);
+    launch_cast_bf16(dout, dyb, S * D, s);
+    ++n;
+    GemmArgs g{};
+    g.offsets = offsets;
+    g.sorted_rows = sorted_rows;
+    g.S = S;
+    g.R = R;
+    g.E = E;
+    g.k = k;
+    g.bf16 = true;
+    g.status = status;
+    g.wait_limit_ns = kWaitLimitNs;
+    // GEMM2 backward, ungated: dhp[p] = dout[s] . W_down[e]^T (W_down [E, F, D] read K-major)
+    {
+        GemmArgs a = g;
+        a.A = dyb;
+        a.a_rows = S;
+        a.B0 = w_down;
+        a.b_kmajor = true;
+        a.out = dhp;
+        a.K = D;
+        a.N = F;
+        a.gather = true;
+        if ((rc = launch_grouped_gemm(a, s))) return rc;
+        ++n;
+    }
+    // GEMM1 pre-activations recomputed: a = x W_gate_e[e], b = x W_up[e] (slot order)
+    for (int half = 0; half < 2; ++half) {
+        GemmArgs a = g;
+        a.A = x;
+        a.a_rows = S;
+        a.B0 = half == 0 ? w_gate_e : w_up;
+        a.out = half == 0 ? av : bv;
+        a.K = D;
+        a.N = F;
+        a.gather = true;
+        if ((rc = prefer_2sm(R, E) ? launch_grouped_gemm_2sm(a, s) : launch_grouped_gemm(a, s)))
+            return rc;
+        ++n;
+    }
+    // route-weight gradient and [da | db]
+    launch_zero_f32(dwr, R, nullptr, s);
+    launch_swiglu_bwd(dhp, h, av, bv, sorted_rows, top_w, R, F, dpre, dwr, s);
+    n += 2;
+    // dW_down[e] = sum over e's slots of h_p^T (w_i dout[s])
+    launch_gate_rows(dout, false, sorted_rows, top_w, k, R, D, true, dv, s);
+    {
+        WgradArgs w{};
+        w.X = h;
+        w.dv = dv;
+        w.offsets = offsets;
+        w.sorted_rows = sorted_rows;
+        w.Din = F;
+        w.Dout = D;
+        w.R = R;
+        w.E = E;
+        w.k = k;
+        w.gather = false;
+        w.dW = dw_down;
+        w.status = status;
+        w.wait_limit_ns = kWaitLimitNs;
+        if ((rc = launch_grouped_wgrad(w, s))) return rc;
+        n += 2;
+    }
+    // dx (experts) += [da | db] . [W_gate_e ; W_up]^T, scatter-added into tokens
+    {
+        GemmArgs a = g;
+        a.A = dpre;
+        a.a_rows = R;
+        a.B0 = w_gate_e;
+        a.B1 = w_up;
+        a.k_split = F;
+        a.b_kmajor = true;
+        a.out = dx;
+        a.K = 2 * F;
+        a.N = D;
+        a.gather = false;
+        a.scatter = true;
+        if ((rc = launch_grouped_gemm(a, s))) return rc;
+        ++n;
+    }
+    // dW_gate_e, dW_up from the gathered x rows and the two halves of [da | db]
+    for (int half = 0; half < 2; ++half) {
+        WgradArgs w{};
+        w.X = x;
+        w.dv = static_cast<const uint8_t *>(dpre) + (size_t)half * F * 2;
+        w.dv_ld = 2 * F;
+        w.offsets = offsets;
+        w.sorted_rows = sorted_rows;
+        w.Din = D;
+        w.Dout = F;
+        w.R = R;
+        w.E = E;
+        w.k = k;
+        w.gather = true;
+        w.dW = half == 0 ? dw_gate_e : dw_up;
+        w.status = status;
+        w.wait_limit_ns = kWaitLimitNs;
+        if ((rc = launch_grouped_wgrad(w, s))) return rc;
+        ++n;
+    }
+    // router: dl (softmax over the selection), dx += dl W_gate^T, dW_gate = x^T dl
+    launch_router_bwd(top_e, top_w, dwr, w_gate, S, D, E, k, dl, dx, off1, s);
+    ++n;
+    {
+        WgradArgs w{};
+        w.X = x;
+        w.dv = dl;
+        w.offsets = off1;
+        w.sorted_rows = nullptr;
+        w.Din = D;
+        w.Dout = E;
+        w.R = S;
+        w.E = 1;
+        w.k = 1;
+        w.gather = false;
+        w.dW = dw_gate;
+        w.status = status;
+        w.wait_limit_ns = kWaitLimitNs;
+        if ((rc = launch_grouped_wgrad(w, s))) return rc;
+        ++n;
+    }
+    g_launches = n;
+    return check_launch("mlp_backward");
+}

@@ -100,6 +100,84 @@ rowdot_kernel(const void *__restrict__ dY, bool dy_bf16, const __nv_bfloat16 *__
     }
 }
 
+// SwiGLU backward of one slot p (route i, gate g = top_w[i]) from the ungated gradient of h,
+// dhp = dout[s] . W_down[e]^T, the forward's h and the recomputed pre-activations a, b:
+//   dw[i] = dhp . h;  dh = g * dhp;  da = dh * b * silu'(a);  db = dh * silu(a)
+// with silu'(z) = sig(z) (1 + z (1 - sig(z))); writes dpre[p] = [da | db] (bf16, 2F wide).
+__global__ void __launch_bounds__(kWarps * 32)
+swiglu_bwd_kernel(const __nv_bfloat16 *__restrict__ dhp, const __nv_bfloat16 *__restrict__ h,
+                  const __nv_bfloat16 *__restrict__ a, const __nv_bfloat16 *__restrict__ b,
+                  const int32_t *__restrict__ sorted_rows, const float *__restrict__ top_w,
+                  int64_t R, int64_t F, __nv_bfloat16 *__restrict__ dpre, float *__restrict__ dw) {
+    const int lane = threadIdx.x & 31;
+    const int64_t wstride = (int64_t)gridDim.x * kWarps;
+    for (int64_t p = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5); p < R; p += wstride) {
+        const int32_t i = __ldg(sorted_rows + p);
+        const float g = __ldg(top_w + i);
+        float acc = 0.f;
+        for (int64_t c = (int64_t)lane * 8; c < F; c += 32 * 8) {
+            float vd[8], vh[8], va[8], vb[8], da[8], db[8];
+            load8(dhp + p * F, true, c, vd);
+            load8(h + p * F, true, c, vh);
+            load8(a + p * F, true, c, va);
+            load8(b + p * F, true, c, vb);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                acc = fmaf(vd[j], vh[j], acc);
+                const float dh = g * vd[j];
+                const float sg = 1.0f / (1.0f + __expf(-va[j]));
+                da[j] = dh * vb[j] * sg * (1.0f + va[j] * (1.0f - sg));
+                db[j] = dh * va[j] * sg;
+            }
+            *reinterpret_cast<uint4 *>(dpre + p * 2 * F + c) = pack8(da);
+            *reinterpret_cast<uint4 *>(dpre + p * 2 * F + F + c) = pack8(db);
+        }
+#pragma unroll
+        for (int d = 16; d > 0; d >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, d);
+        if (lane == 0) dw[i] = acc;
+    }
+}
+
+// Router backward of one token s: the softmax over its k selected logits gives
+//   dl_j = w_j (dw_j - sum_j' w_j' dw_j');
+// dl is written as a dense bf16 row [E] (zero outside the selection, the weight gradient's
+// operand) and dx[s] += sum_j dl_j W_gate[:, e_j] (after the expert part of dx is complete).
+// Block 0 also writes the one-"expert" offsets {0, S} of the W_gate gradient.
+__global__ void __launch_bounds__(kWarps * 32)
+router_bwd_kernel(const int32_t *__restrict__ top_e, const float *__restrict__ top_w,
+                  const float *__restrict__ dw, const __nv_bfloat16 *__restrict__ w_gate,
+                  int64_t S, int64_t D, int32_t E, int32_t k, __nv_bfloat16 *__restrict__ dl,
+                  float *__restrict__ dx, int32_t *__restrict__ offsets1) {
+    const int lane = threadIdx.x & 31;
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        offsets1[0] = 0;
+        offsets1[1] = (int32_t)S;
+    }
+    const int64_t wstride = (int64_t)gridDim.x * kWarps;
+    for (int64_t s = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5); s < S; s += wstride) {
+        float mean = 0.f;
+        for (int j = 0; j < k; ++j) mean += top_w[s * k + j] * dw[s * k + j];
+        float dlj[8];
+        int32_t ej[8];
+        for (int j = 0; j < k; ++j) {
+            dlj[j] = top_w[s * k + j] * (dw[s * k + j] - mean);
+            ej[j] = top_e[s * k + j];
+        }
+        for (int e = lane; e < E; e += 32) {
+            float v = 0.f;
+            for (int j = 0; j < k; ++j)
+                if (ej[j] == e) v = dlj[j];
+            dl[s * E + e] = __float2bfloat16_rn(v);
+        }
+        for (int64_t d = lane; d < D; d += 32) {
+            float acc = 0.f;
+            for (int j = 0; j < k; ++j)
+                acc = fmaf(dlj[j], __bfloat162float(w_gate[d * E + ej[j]]), acc);
+            dx[s * D + d] += acc;
+        }
+    }
+}
+
 unsigned warp_grid(int64_t rows) {
     int64_t blocks = (rows + kWarps - 1) / kWarps;
     const int64_t cap = (int64_t)num_sms() * 16;
@@ -130,6 +208,23 @@ void launch_rowdot(const void *dY, bool dy_bf16, const void *v, const int32_t *s
     rowdot_kernel<<<warp_grid(R), kWarps * 32, 0, s>>>(dY, dy_bf16,
                                                        static_cast<const __nv_bfloat16 *>(v),
                                                        sorted_rows, k, R, Dout, by_token, dg);
+}
+
+void launch_swiglu_bwd(const void *dhp, const void *h, const void *a, const void *b,
+                       const int32_t *sorted_rows, const float *top_w, int64_t R, int64_t F,
+                       void *dpre, float *dw, cudaStream_t s) {
+    swiglu_bwd_kernel<<<warp_grid(R), kWarps * 32, 0, s>>>(
+        static_cast<const __nv_bfloat16 *>(dhp), static_cast<const __nv_bfloat16 *>(h),
+        static_cast<const __nv_bfloat16 *>(a), static_cast<const __nv_bfloat16 *>(b), sorted_rows,
+        top_w, R, F, static_cast<__nv_bfloat16 *>(dpre), dw);
+}
+
+void launch_router_bwd(const int32_t *top_e, const float *top_w, const float *dw,
+                       const void *w_gate, int64_t S, int64_t D, int32_t E, int32_t k, void *dl,
+                       float *dx, int32_t *offsets1, cudaStream_t s) {
+    router_bwd_kernel<<<warp_grid(S), kWarps * 32, 0, s>>>(
+        top_e, top_w, dw, static_cast<const __nv_bfloat16 *>(w_gate), S, D, E, k,
+        static_cast<__nv_bfloat16 *>(dl), dx, offsets1);
 }
 
 }  // namespace moe

@@ -310,7 +310,7 @@ int launch_grouped_wgrad(const WgradArgs &a, cudaStream_t s) {
     CUtensorMap mB;
     {
         const uint64_t dims[2] = {(uint64_t)a.Dout, (uint64_t)a.R};
-        const uint64_t str[1] = {(uint64_t)a.Dout * 2};
+        const uint64_t str[1] = {(uint64_t)(a.dv_ld > 0 ? a.dv_ld : a.Dout) * 2};
         const uint32_t box[2] = {64u, (uint32_t)WK};
         int rc = encode_tmap(&mB, true, 2, a.dv, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
         if (rc) return rc;

@@ -78,7 +78,8 @@ int launch_debug_wait(int64_t limit_ns, unsigned *status, cudaStream_t s);
 // order; dW [E, Din, Dout] fp32 is overwritten (zeros for experts without slots). bf16 only.
 struct WgradArgs {
     const void *X;          // [S, Din] (gather) or [R, Din]
-    const void *dv;         // [R, Dout]
+    const void *dv;         // [R, Dout] with row stride dv_ld elements (0: Dout)
+    int64_t dv_ld;
     const int32_t *offsets; // [E+1]
     const int32_t *sorted_rows;
     int64_t Din, Dout, R;
@@ -95,6 +96,12 @@ void launch_gate_rows(const void *dY, bool dy_bf16, const int32_t *sorted_rows, 
                       int32_t k, int64_t R, int64_t Dout, bool by_token, void *dv, cudaStream_t s);
 void launch_rowdot(const void *dY, bool dy_bf16, const void *v, const int32_t *sorted_rows,
                    int32_t k, int64_t R, int64_t Dout, bool by_token, float *dg, cudaStream_t s);
+void launch_swiglu_bwd(const void *dhp, const void *h, const void *a, const void *b,
+                       const int32_t *sorted_rows, const float *top_w, int64_t R, int64_t F,
+                       void *dpre, float *dw, cudaStream_t s);
+void launch_router_bwd(const int32_t *top_e, const float *top_w, const float *dw,
+                       const void *w_gate, int64_t S, int64_t D, int32_t E, int32_t k, void *dl,
+                       float *dx, int32_t *offsets1, cudaStream_t s);
 // Router on the tensor cores (bf16, E % 8 == 0): logits of 128-token tiles in TMEM, top-k and
 // softmax in the epilogue.
 int launch_route_tc(const void *x, const void *w_gate, const float *bias, int64_t S, int64_t D,
