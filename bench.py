@@ -402,6 +402,70 @@ def map_sweep(args):
             "peak_hbm_gbs": pk["hbm_gbs"], "peak_kind": pk_kind, "points": points}
 
 
+def backward_bench(args, w):
+    """Time moe_mlp_backward on workload w (bf16): one forward fills the workspace with routing,
+    map and h, then W warm-up and K timed backward steps (CUDA events on the launch stream). A
+    step's algorithmic work: 12*R*D*F expert FLOPs (dh, dW_down, dx, dW_gate_e, dW_up) plus the
+    router's 2*S*D*E (dW_gate) and 2*S*k*D (dx); the kernels also recompute a and b (4*R*D*F)."""
+    import sparse_mixture_experts_02_b200 as moe
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    inp = W.make_inputs(w, device=dev, seed=0)
+    fws = moe.ForwardWorkspace(w.S, w.D, w.F, w.E, w.k, inp["x"].dtype, dev)
+    out = torch.empty((w.S, w.D), dtype=torch.float32, device=dev)
+    moe.mlp_forward(inp["x"], inp["w_gate"], inp["w_gate_e"], inp["w_up"], inp["w_down"], w.k,
+                    logit_bias=inp["logit_bias"], out=out, ws=fws)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1)
+    dout = torch.randn((w.S, w.D), generator=gen, device=dev)
+    bws = moe.alloc_workspace(moe.workspace_size("mlp_backward", w.S, w.D, w.F, w.E, w.k,
+                                                 inp["x"].dtype), dev)
+
+    def step(evs=None):
+        if evs is not None:
+            moe.profile_events(evs)
+        return moe.mlp_backward(inp["x"], inp["w_gate"], inp["w_gate_e"], inp["w_up"],
+                                inp["w_down"], w.k, dout, fws, ws=bws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    moe.check_device_status(bws)
+    launches = moe.last_launch_count()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+    for row in evs:
+        for e in row:
+            e.record()
+    torch.cuda.synchronize(dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        t0.record()
+        for i in range(args.steps):
+            step(evs[i])
+        t1.record()
+        torch.cuda.synchronize(dev)
+    ms = t0.elapsed_time(t1) / args.steps
+    names = ["dh", "recompute_a_b", "swiglu_bwd_and_dW_down", "dx", "dW_gate_e_and_dW_up",
+             "router"]
+    stage = {n: sum(r[q].elapsed_time(r[q + 1]) for r in evs) / args.steps
+             for q, n in enumerate(names)}
+    R = w.S * w.k
+    flop = 12.0 * R * w.D * w.F + 2.0 * w.S * w.D * w.E + 2.0 * w.S * w.k * w.D
+    pk, pk_kind = peaks()
+    tflops = flop / (ms * 1e-3) / 1e12
+    return {"metric": "MoE-layer backward tokens/s and TFLOP/s (bf16)", "value": w.S / (ms * 1e-3),
+            "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "dtype": w.dtype, "data": "synthetic",
+            "config": {"workload": w.name, "S": w.S, "D": w.D, "F": w.F, "E": w.E, "k": w.k,
+                       "l2": "inputs larger than L2 (all expert weights streamed every step)"},
+            "tflops": tflops, "flop_per_step": flop,
+            "tflops_frac": {"of_measured_sustained": tflops / pk["bf16_tflops_sustained"],
+                            "of_nominal": tflops / 2250.0, "peaks": pk_kind},
+            "extra_flop_recompute": 4.0 * R * w.D * w.F, "stage_ms": stage,
+            "gpu_launches": launches * args.steps, "clocks": clk.summary()}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -415,6 +479,8 @@ def main():
     ap.add_argument("--ref-step-s", type=float, default=None)
     ap.add_argument("--map-sweep", action="store_true",
                     help="instead of the forward: sparse-map GB/s over R = 2^20..2^26 routes")
+    ap.add_argument("--backward", action="store_true",
+                    help="instead of the forward: time moe_mlp_backward on --workload")
     ap.add_argument("--map-points", default="",
                     help="with --map-sweep: only these points, 'log2R:E,...' (e.g. 26:256)")
     args = ap.parse_args()
@@ -422,6 +488,10 @@ def main():
         ap.error("--warmup must be >= 3")
     if args.map_sweep:
         print(json.dumps(map_sweep(args)), flush=True)
+        return
+    if args.backward:
+        wl = {**W.WORKLOADS, **W.PROFILE_WORKLOADS}[args.workload]
+        print(json.dumps(backward_bench(args, wl)), flush=True)
         return
     w = {**W.WORKLOADS, **W.PROFILE_WORKLOADS}[args.workload]
     if args.impl == "reference":

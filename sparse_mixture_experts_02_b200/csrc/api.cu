@@ -661,6 +661,9 @@ extern "C" int moe_mlp_backward(const void *x, const void *w_gate, const void *w
         g_launches = n + 4;
         return check_launch("mlp_backward");
     }
+    // profile events (moe_profile_events): 0 start, 1 after dh, 2 after the a/b recompute,
+    // 3 after the SwiGLU backward and dW_down, 4 after dx, 5 after dW_gate_e/dW_up, 6 end
+    record_prof(0, s);
     void *dyb = at<void>(ws, L.dyb), *dhp = at<void>(ws, L.dhp), *av = at<void>(ws, L.a);
     void *bv = at<void>(ws, L.b), *dpre = at<void>(ws, L.dpre), *dv = at<void>(ws, L.dv);
     void *dl = at<void>(ws, L.dl);
@@ -692,6 +695,7 @@ extern "C" int moe_mlp_backward(const void *x, const void *w_gate, const void *w
         if ((rc = launch_grouped_gemm(a, s))) return rc;
         ++n;
     }
+    record_prof(1, s);
     // GEMM1 pre-activations recomputed: a = x W_gate_e[e], b = x W_up[e] (slot order)
     for (int half = 0; half < 2; ++half) {
         GemmArgs a = g;
@@ -706,6 +710,7 @@ extern "C" int moe_mlp_backward(const void *x, const void *w_gate, const void *w
             return rc;
         ++n;
     }
+    record_prof(2, s);
     // route-weight gradient and [da | db]
     launch_zero_f32(dwr, R, nullptr, s);
     launch_swiglu_bwd(dhp, h, av, bv, sorted_rows, top_w, R, F, dpre, dwr, s);
@@ -730,6 +735,7 @@ extern "C" int moe_mlp_backward(const void *x, const void *w_gate, const void *w
         if ((rc = launch_grouped_wgrad(w, s))) return rc;
         n += 2;
     }
+    record_prof(3, s);
     // dx (experts) += [da | db] . [W_gate_e ; W_up]^T, scatter-added into tokens
     {
         GemmArgs a = g;
@@ -747,6 +753,7 @@ extern "C" int moe_mlp_backward(const void *x, const void *w_gate, const void *w
         if ((rc = launch_grouped_gemm(a, s))) return rc;
         ++n;
     }
+    record_prof(4, s);
     // dW_gate_e, dW_up from the gathered x rows and the two halves of [da | db]
     for (int half = 0; half < 2; ++half) {
         WgradArgs w{};
@@ -767,6 +774,7 @@ extern "C" int moe_mlp_backward(const void *x, const void *w_gate, const void *w
         if ((rc = launch_grouped_wgrad(w, s))) return rc;
         ++n;
     }
+    record_prof(5, s);
     // router: dl (softmax over the selection), dx += dl W_gate^T, dW_gate = x^T dl
     launch_router_bwd(top_e, top_w, dwr, w_gate, S, D, E, k, dl, dx, off1, s);
     ++n;
@@ -788,6 +796,7 @@ extern "C" int moe_mlp_backward(const void *x, const void *w_gate, const void *w
         if ((rc = launch_grouped_wgrad(w, s))) return rc;
         ++n;
     }
+    record_prof(6, s);
     g_launches = n;
     return check_launch("mlp_backward");
 }

@@ -15,11 +15,14 @@
 //   warps 6-9  cp.async gatherers of A: the stage's 64 source rows x 128 columns of Din, written
 //              MN-major in the same swizzle (row r of the stage at 128-byte line r of each
 //              64-column chunk); slots past the expert's end and columns past Din are zero-filled.
-//              The row indices of the next stage are loaded one stage ahead.
+//              Each copy instruction covers 4 whole 128-byte segments (one per 8 lanes); the row
+//              indices of the next stage are loaded one stage ahead. (One thread per half-row,
+//              16 bytes per instruction, touched 32 segments per instruction and cost ~40%.)
 //   warp 1     TMEM owner (two 128 x 256 fp32 accumulators) and MMA issuer: 4 MMAs of M=128
 //              (Din), N=256 (Dout), K=16 rows per stage, both operands MN-major.
-//   warps 2-5  epilogue: accumulator lane m -> dW[e][m0 + m][n0 .. n0 + 255]; a tile of an
-//              expert without slots stores zeros.
+//   warps 2-5  epilogue: accumulator lane m -> dW[e][m0 + m][n0 .. n0 + 255], staged through
+//              shared memory in 32 x 32 chunks so each store covers 4 rows x 128 bytes; a tile of
+//              an expert without slots stores zeros.
 // Tiles are (expert, N tile, M tile), expert-major, so the CTAs running at once share an
 // expert's rows through L2. Every wait is bounded (mbar_wait).
 #include "gemm_common.cuh"
@@ -185,9 +188,13 @@ grouped_wgrad_kernel(const __grid_constant__ CUtensorMap tmB, const WParams p) {
         __syncwarp();
     } else if (warp >= THREADS / 32) {
         // ------------------------------------------------------------------ A gatherers
-        // thread -> stage row r = gt / 2 (a slot), half h = gt % 2 (64 columns = 128 B)
-        const int gt = threadIdx.x - THREADS;
-        const int r = gt >> 1, h = gt & 1;
+        // Warp gw fills stage rows gw*16 .. gw*16+15, both 128-byte halves of each. Per copy
+        // instruction i, lanes 8u..8u+7 (u = lane / 8) copy the 16-byte pieces 0..7 of row
+        // 2i + u/2, half u%2: a warp instruction covers 4 whole 128-byte segments. Lane l < 16
+        // holds the source row of the warp's row l (loaded one stage ahead; lanes 16-31 repeat
+        // it), and the copies take it by shuffle.
+        const int gw = (threadIdx.x - THREADS) >> 5;
+        const int j = lane & 7, sub = lane >> 3;
         const int64_t row_bytes = p.Din * 2;
         uint32_t s = 0, ph = 0;
         bool ok = true;
@@ -196,16 +203,14 @@ grouped_wgrad_kernel(const __grid_constant__ CUtensorMap tmB, const WParams p) {
             wtile(t, per_e, p.m_tiles, e, n, m);
             const int r0 = st.off[e], r1 = st.off[e + 1];
             const int nkb = (r1 - r0 + WK - 1) / WK;
-            const int64_t col0 = ((int64_t)m * BM + h * 64) * 2;  // byte offset in a row
-            // source row of this thread's slot, one stage ahead
-            auto src_row = [&](int kb) -> int64_t {
-                const int slot = r0 + kb * WK + r;
+            auto row_index = [&](int kb) -> long long {
+                const int slot = r0 + kb * WK + gw * 16 + (lane & 15);
                 if (slot >= r1) return -1;
-                return p.gather ? (int64_t)(__ldg(p.sorted_rows + slot) / p.k) : (int64_t)slot;
+                return p.gather ? (long long)(__ldg(p.sorted_rows + slot) / p.k) : (long long)slot;
             };
-            int64_t row = nkb > 0 ? src_row(0) : -1;
+            long long myrow = nkb > 0 ? row_index(0) : -1;
             for (int kb = 0; kb < nkb; ++kb) {
-                const int64_t next = kb + 1 < nkb ? src_row(kb + 1) : -1;
+                const long long next = kb + 1 < nkb ? row_index(kb + 1) : -1;
                 bool w = true;
                 if (lane == 0)
                     w = dev::mbar_wait(&st.empty[s], ph ^ 1u, abort, p.status, p.wait_limit_ns,
@@ -215,17 +220,19 @@ grouped_wgrad_kernel(const __grid_constant__ CUtensorMap tmB, const WParams p) {
                     ok = false;
                     break;
                 }
-                const uint32_t dst0 = dev::smem_u32(smem + (size_t)s * STAGE_BYTES) + h * WCH +
-                                      r * KBYTES;
-                const uint8_t *src = row >= 0 ? p.X + row * row_bytes + col0 : p.X;
+                const uint32_t sA = dev::smem_u32(smem + (size_t)s * STAGE_BYTES);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const bool in = row >= 0 && col0 + j * 16 < row_bytes;
-                    dev::cp_async16(dst0 + ((j ^ (r & 7)) << 4), in ? src + j * 16 : p.X,
-                                    in ? 16u : 0u);
+                for (int i = 0; i < 8; ++i) {
+                    const int rl = 2 * i + (sub >> 1), h = sub & 1;
+                    const int r = gw * 16 + rl;
+                    const long long row = __shfl_sync(0xffffffffu, myrow, rl);
+                    const int64_t cb = ((int64_t)m * BM + h * 64) * 2 + j * 16;
+                    const bool in = row >= 0 && cb < row_bytes;
+                    const uint32_t dst = sA + h * WCH + r * KBYTES + ((j ^ (r & 7)) << 4);
+                    dev::cp_async16(dst, in ? p.X + row * row_bytes + cb : p.X, in ? 16u : 0u);
                 }
                 dev::cp_async_arrive_noinc(&st.full[s]);
-                row = next;
+                myrow = next;
                 if (++s == STAGES) {
                     s = 0;
                     ph ^= 1u;
@@ -236,7 +243,6 @@ grouped_wgrad_kernel(const __grid_constant__ CUtensorMap tmB, const WParams p) {
     } else {
         // ------------------------------------------------------------------ epilogue
         const int q = warp & 3;  // TMEM lane quarter this warp may access
-        const int mr = q * 32 + lane;
         int it = 0;
         for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
             int e, n, m;
@@ -250,12 +256,19 @@ grouped_wgrad_kernel(const __grid_constant__ CUtensorMap tmB, const WParams p) {
             w = __shfl_sync(0xffffffffu, w, 0);
             if (!w) break;
             dev::tc_fence_after();
-            const int64_t grow = (int64_t)m * BM + mr;  // row of dW[e]
-            const bool row_ok = grow < p.Din;
-            float *dst = p.dW + ((int64_t)e * p.Din + (row_ok ? grow : 0)) * p.Dout;
+            // Each 32 x 32 chunk of the warp's rows goes through shared memory (row stride 33
+            // floats), so a store instruction covers 4 rows x 128 contiguous bytes of dW instead
+            // of 16 bytes in each of 32 rows: the weight gradient writes 16x more bytes per FLOP
+            // than the forward GEMMs.
+            float *stg = st.stage[q];
+            const int rsub = lane >> 3, cc = (lane & 7) * 4;
+            const int64_t row0 = (int64_t)m * BM + q * 32;  // first dW[e] row of this warp
+            float *dWe = p.dW + (int64_t)e * p.Din * p.Dout;
             const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + b * BN;
 #pragma unroll 1
             for (int c = 0; c < BN / 32; ++c) {
+                const int64_t col0 = (int64_t)n * BN + c * 32;
+                if (col0 >= p.Dout) break;  // warp-uniform
                 uint32_t v[32];
                 if (!empty_e) {
                     dev::tmem_ld32(tbase + c * 32, v);
@@ -264,15 +277,20 @@ grouped_wgrad_kernel(const __grid_constant__ CUtensorMap tmB, const WParams p) {
 #pragma unroll
                     for (int j = 0; j < 32; ++j) v[j] = 0u;
                 }
-                const int64_t col0 = (int64_t)n * BN + c * 32;
-                if (row_ok) {
 #pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        if (col0 + j * 4 < p.Dout)
-                            *reinterpret_cast<float4 *>(dst + col0 + j * 4) = make_float4(
-                                __uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
-                                __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+                for (int j = 0; j < 32; ++j) stg[lane * 33 + j] = __uint_as_float(v[j]);
+                __syncwarp();
+#pragma unroll
+                for (int pass = 0; pass < 8; ++pass) {
+                    const int rr = pass * 4 + rsub;
+                    const int64_t grow = row0 + rr;
+                    if (grow < p.Din && col0 + cc < p.Dout) {
+                        const float *sv = stg + rr * 33 + cc;
+                        *reinterpret_cast<float4 *>(dWe + grow * p.Dout + col0 + cc) =
+                            make_float4(sv[0], sv[1], sv[2], sv[3]);
+                    }
                 }
+                __syncwarp();
             }
             dev::tc_fence_before();
             __syncwarp();
