@@ -129,19 +129,21 @@ MlpLayout mlp_layout(int64_t S, int64_t F, int32_t E, int32_t k, moe_dtype dt) {
     return L;
 }
 
-// ParallelLinear backward scratch: status, bf16 copy of an fp32 dY [S, Dout], gated rows dv
-// [R, Dout] bf16 (weight gradient), ungated forward rows v [R, Dout] bf16 (gate gradient).
+// ParallelLinear backward scratch: status, bf16 copy of an fp32 dY [S, Dout], gated rows dv in
+// the weight gradient's padded layout [R + 64 E, Dout] bf16, x rows in slot order [R, Din] (for
+// gathered inputs), ungated forward rows v [R, Dout] bf16 (gate gradient).
 struct BwdLayout {
-    size_t status, dyb, dv, v, total;
+    size_t status, dyb, dv, xs, v, total;
 };
 
-BwdLayout bwd_layout(int64_t S, int64_t Dout, int32_t k) {
+BwdLayout bwd_layout(int64_t S, int64_t Din, int64_t Dout, int32_t E, int32_t k) {
     const int64_t R = S * k;
     BwdLayout L;
     size_t o = 0;
     L.status = o; o += kStatusBytes;
     L.dyb = o; o = align_up(o + 2 * (size_t)S * (size_t)Dout);
-    L.dv = o; o = align_up(o + 2 * (size_t)R * (size_t)Dout);
+    L.dv = o; o = align_up(o + 2 * (size_t)(R + (int64_t)kWgradPad * E) * (size_t)Dout);
+    L.xs = o; o = align_up(o + 2 * (size_t)R * (size_t)Din);
     L.v = o; o = align_up(o + 2 * (size_t)R * (size_t)Dout);
     L.total = o;
     return L;
@@ -149,7 +151,7 @@ BwdLayout bwd_layout(int64_t S, int64_t Dout, int32_t k) {
 
 // MLP backward scratch (the forward's workspace supplies routing, map and h).
 struct MlpBwdLayout {
-    size_t status, dyb, dhp, a, b, dpre, dw, dv, dl, off1, total;
+    size_t status, dyb, dhp, a, b, dpre, dw, dv, dl, xs, off1, total;
 };
 
 MlpBwdLayout mlp_bwd_layout(int64_t S, int64_t D, int64_t F, int32_t E, int32_t k) {
@@ -161,10 +163,13 @@ MlpBwdLayout mlp_bwd_layout(int64_t S, int64_t D, int64_t F, int32_t E, int32_t 
     L.dhp = o; o = align_up(o + 2 * (size_t)R * (size_t)F);
     L.a = o; o = align_up(o + 2 * (size_t)R * (size_t)F);
     L.b = o; o = align_up(o + 2 * (size_t)R * (size_t)F);
-    L.dpre = o; o = align_up(o + 4 * (size_t)R * (size_t)F);
+    // [da | db], the gated dout rows and the router's dl in the weight gradient's padded layout
+    const int64_t Rp = R + (int64_t)kWgradPad * E;
+    L.dpre = o; o = align_up(o + 4 * (size_t)Rp * (size_t)F);
     L.dw = o; o = align_up(o + 4 * (size_t)R);
-    L.dv = o; o = align_up(o + 2 * (size_t)R * (size_t)D);
-    L.dl = o; o = align_up(o + 2 * (size_t)S * (size_t)E);
+    L.dv = o; o = align_up(o + 2 * (size_t)Rp * (size_t)D);
+    L.dl = o; o = align_up(o + 2 * (size_t)(S + kWgradPad) * (size_t)E);
+    L.xs = o; o = align_up(o + 2 * (size_t)R * (size_t)D);
     L.off1 = o; o = align_up(o + 2 * sizeof(int32_t));
     L.total = o;
     return L;
@@ -220,7 +225,8 @@ size_t moe_workspace_size(const char *op, int64_t S, int64_t D, int64_t F, int32
     if (strcmp(op, "scatter_linear") == 0) return kStatusBytes;
     if (strcmp(op, "scatter_linear_backward") == 0) {
         if (F <= 0) return 0;
-        return bwd_layout(S, F, k).total;  // D = Din, F = Dout
+        if (D <= 0) return 0;
+        return bwd_layout(S, D, F, E, k).total;  // D = Din, F = Dout
     }
     if (strcmp(op, "mlp_backward") == 0) {
         if (F <= 0 || D <= 0) return 0;
@@ -372,7 +378,7 @@ int moe_scatter_linear_backward(const void *X, const void *W, const void *dY, in
         (rc = check_ptr("dX", dX, 16, true)) || (rc = check_ptr("dW", dW, 16, true)) ||
         (rc = check_ptr("dgates", dgates, 16, true)))
         return rc;
-    const BwdLayout L = bwd_layout(S, Dout, k);
+    const BwdLayout L = bwd_layout(S, Din, Dout, E, k);
     if ((rc = check_ws(ws, ws_bytes, L.total))) return rc;
     if ((rc = check_device())) return rc;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -428,24 +434,30 @@ int moe_scatter_linear_backward(const void *X, const void *W, const void *dY, in
         ++n;
     }
     if (dW != nullptr) {
+        // B: the gated dY rows in the padded layout; A: the input rows in slot order
         launch_gate_rows(dY, !scatter_out, sorted_rows, top_weights, k, R, Dout, scatter_out != 0,
-                         at<void>(ws, L.dv), s);
+                         at<void>(ws, L.dv), expert_offsets, E, s);
+        launch_zero_pad_rows(at<void>(ws, L.dv), Dout, Dout, expert_offsets, E, s);
+        const void *As = X;
+        if (gather_in) {
+            launch_gather_rows(X, sorted_rows, k, R, Din, at<void>(ws, L.xs), s);
+            As = at<void>(ws, L.xs);
+            ++n;
+        }
         WgradArgs w{};
-        w.X = X;
+        w.A = As;
+        w.a_rows = R;
         w.dv = at<void>(ws, L.dv);
+        w.dv_rows = R + (int64_t)kWgradPad * E;
         w.offsets = expert_offsets;
-        w.sorted_rows = sorted_rows;
         w.Din = Din;
         w.Dout = Dout;
-        w.R = R;
         w.E = E;
-        w.k = k;
-        w.gather = gather_in != 0;
         w.dW = dW;
         w.status = status;
         w.wait_limit_ns = kWaitLimitNs;
         if ((rc = launch_grouped_wgrad(w, s))) return rc;
-        n += 2;
+        n += 3;
     }
     if (dgates != nullptr) {
         // v = the ungated forward rows in slot order; dgates[i] = dY[row] . v[p]
@@ -713,34 +725,36 @@ extern "C" int moe_mlp_backward(const void *x, const void *w_gate, const void *w
     record_prof(2, s);
     // route-weight gradient and [da | db]
     launch_zero_f32(dwr, R, nullptr, s);
-    launch_swiglu_bwd(dhp, h, av, bv, sorted_rows, top_w, R, F, dpre, dwr, s);
-    n += 2;
+    const int64_t Rp = R + (int64_t)kWgradPad * E;
+    launch_swiglu_bwd(dhp, h, av, bv, sorted_rows, top_w, offsets, E, R, F, dpre, dwr, s);
+    launch_zero_pad_rows(dpre, 2 * F, 2 * F, offsets, E, s);
+    n += 3;
     // dW_down[e] = sum over e's slots of h_p^T (w_i dout[s])
-    launch_gate_rows(dout, false, sorted_rows, top_w, k, R, D, true, dv, s);
+    launch_gate_rows(dout, false, sorted_rows, top_w, k, R, D, true, dv, offsets, E, s);
+    launch_zero_pad_rows(dv, D, D, offsets, E, s);
     {
         WgradArgs w{};
-        w.X = h;
+        w.A = h;
+        w.a_rows = R;
         w.dv = dv;
+        w.dv_rows = Rp;
         w.offsets = offsets;
-        w.sorted_rows = sorted_rows;
         w.Din = F;
         w.Dout = D;
-        w.R = R;
         w.E = E;
-        w.k = k;
-        w.gather = false;
         w.dW = dw_down;
         w.status = status;
         w.wait_limit_ns = kWaitLimitNs;
         if ((rc = launch_grouped_wgrad(w, s))) return rc;
-        n += 2;
+        n += 3;
     }
     record_prof(3, s);
     // dx (experts) += [da | db] . [W_gate_e ; W_up]^T, scatter-added into tokens
     {
         GemmArgs a = g;
         a.A = dpre;
-        a.a_rows = R;
+        a.a_rows = Rp;
+        a.a_row_pad = kWgradPad;
         a.B0 = w_gate_e;
         a.B1 = w_up;
         a.k_split = F;
@@ -754,20 +768,21 @@ extern "C" int moe_mlp_backward(const void *x, const void *w_gate, const void *w
         ++n;
     }
     record_prof(4, s);
-    // dW_gate_e, dW_up from the gathered x rows and the two halves of [da | db]
+    // dW_gate_e, dW_up from the x rows in slot order and the two halves of [da | db]
+    void *xs = at<void>(ws, L.xs);
+    launch_gather_rows(x, sorted_rows, k, R, D, xs, s);
+    ++n;
     for (int half = 0; half < 2; ++half) {
         WgradArgs w{};
-        w.X = x;
+        w.A = xs;
+        w.a_rows = R;
         w.dv = static_cast<const uint8_t *>(dpre) + (size_t)half * F * 2;
+        w.dv_rows = Rp;
         w.dv_ld = 2 * F;
         w.offsets = offsets;
-        w.sorted_rows = sorted_rows;
         w.Din = D;
         w.Dout = F;
-        w.R = R;
         w.E = E;
-        w.k = k;
-        w.gather = true;
         w.dW = half == 0 ? dw_gate_e : dw_up;
         w.status = status;
         w.wait_limit_ns = kWaitLimitNs;
@@ -777,19 +792,18 @@ extern "C" int moe_mlp_backward(const void *x, const void *w_gate, const void *w
     record_prof(5, s);
     // router: dl (softmax over the selection), dx += dl W_gate^T, dW_gate = x^T dl
     launch_router_bwd(top_e, top_w, dwr, w_gate, S, D, E, k, dl, dx, off1, s);
-    ++n;
+    launch_zero_pad_rows(dl, E, E, off1, 1, s);
+    n += 2;
     {
         WgradArgs w{};
-        w.X = x;
+        w.A = x;
+        w.a_rows = S;
         w.dv = dl;
+        w.dv_rows = S + kWgradPad;
         w.offsets = off1;
-        w.sorted_rows = nullptr;
         w.Din = D;
         w.Dout = E;
-        w.R = S;
         w.E = 1;
-        w.k = 1;
-        w.gather = false;
         w.dW = dw_gate;
         w.status = status;
         w.wait_limit_ns = kWaitLimitNs;

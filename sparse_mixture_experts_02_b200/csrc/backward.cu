@@ -3,8 +3,10 @@
 // (input gradient: the forward's form with W read transposed) and grouped_gemm_wgrad.cu (weight
 // gradient).
 //   cast:      an fp32 output gradient [rows, Dout] -> bf16 (the tensor cores' operand type);
-//   gate_rows: dv[p] = bf16(g_i * dY[row(p)]) in slot order, the weight gradient's B operand
-//              (row(p) = sorted_rows[p] / k when the forward scattered into tokens, else p);
+//   gate_rows: dv[p] = bf16(g_i * dY[row(p)]), the weight gradient's B operand, in slot order or
+//              in its padded layout (row p + 64 e(p); row(p) = sorted_rows[p] / k when the forward
+//              scattered into tokens, else p); zero_pad_rows zeroes that layout's padding rows;
+//   gather_rows: x rows in slot order (the weight gradient's A operand for gathered inputs);
 //   rowdot:    dgates[i] = sum_n dY[row(p)][n] * v[p][n], v = the ungated forward rows.
 // One warp per slot; rows move in 16-byte pieces (Dout is a multiple of 8).
 #include "moe_internal.cuh"
@@ -45,6 +47,18 @@ __device__ __forceinline__ uint4 pack8(const float (&v)[8]) {
     return u;
 }
 
+// Expert of slot p: the largest e with offsets[e] <= p (empty experts share their start with the
+// next one, which is the one that holds p).
+__device__ __forceinline__ int expert_of(const int32_t *__restrict__ offsets, int32_t E, int64_t p) {
+    int lo = 0, hi = E;
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (__ldg(offsets + mid) <= p) lo = mid;
+        else hi = mid;
+    }
+    return lo;
+}
+
 __global__ void cast_bf16_kernel(const float *__restrict__ src, __nv_bfloat16 *__restrict__ dst,
                                  int64_t n8) {
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
@@ -58,7 +72,8 @@ __global__ void cast_bf16_kernel(const float *__restrict__ src, __nv_bfloat16 *_
 __global__ void __launch_bounds__(kWarps * 32)
 gate_rows_kernel(const void *__restrict__ dY, bool dy_bf16, const int32_t *__restrict__ sorted_rows,
                  const float *__restrict__ gates, int32_t k, int64_t R, int64_t Dout,
-                 bool by_token, __nv_bfloat16 *__restrict__ dv) {
+                 bool by_token, __nv_bfloat16 *__restrict__ dv,
+                 const int32_t *__restrict__ pad_offsets, int32_t E) {
     const int lane = threadIdx.x & 31;
     const int64_t wstride = (int64_t)gridDim.x * kWarps;
     for (int64_t p = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5); p < R; p += wstride) {
@@ -66,12 +81,14 @@ gate_rows_kernel(const void *__restrict__ dY, bool dy_bf16, const int32_t *__res
         const float g = gates != nullptr ? __ldg(gates + i) : 1.0f;
         const int64_t row = by_token ? (int64_t)(i / k) : p;
         const uint8_t *src = static_cast<const uint8_t *>(dY) + row * Dout * (dy_bf16 ? 2 : 4);
+        const int64_t out = pad_offsets != nullptr ? p + (int64_t)kWgradPad * expert_of(pad_offsets, E, p)
+                                                   : p;
         for (int64_t c = (int64_t)lane * 8; c < Dout; c += 32 * 8) {
             float v[8];
             load8(src, dy_bf16, c, v);
 #pragma unroll
             for (int j = 0; j < 8; ++j) v[j] *= g;
-            *reinterpret_cast<uint4 *>(dv + p * Dout + c) = pack8(v);
+            *reinterpret_cast<uint4 *>(dv + out * Dout + c) = pack8(v);
         }
     }
 }
@@ -108,12 +125,14 @@ __global__ void __launch_bounds__(kWarps * 32)
 swiglu_bwd_kernel(const __nv_bfloat16 *__restrict__ dhp, const __nv_bfloat16 *__restrict__ h,
                   const __nv_bfloat16 *__restrict__ a, const __nv_bfloat16 *__restrict__ b,
                   const int32_t *__restrict__ sorted_rows, const float *__restrict__ top_w,
-                  int64_t R, int64_t F, __nv_bfloat16 *__restrict__ dpre, float *__restrict__ dw) {
+                  const int32_t *__restrict__ offsets, int32_t E, int64_t R, int64_t F,
+                  __nv_bfloat16 *__restrict__ dpre, float *__restrict__ dw) {
     const int lane = threadIdx.x & 31;
     const int64_t wstride = (int64_t)gridDim.x * kWarps;
     for (int64_t p = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5); p < R; p += wstride) {
         const int32_t i = __ldg(sorted_rows + p);
         const float g = __ldg(top_w + i);
+        const int64_t out = p + (int64_t)kWgradPad * expert_of(offsets, E, p);
         float acc = 0.f;
         for (int64_t c = (int64_t)lane * 8; c < F; c += 32 * 8) {
             float vd[8], vh[8], va[8], vb[8], da[8], db[8];
@@ -129,8 +148,8 @@ swiglu_bwd_kernel(const __nv_bfloat16 *__restrict__ dhp, const __nv_bfloat16 *__
                 da[j] = dh * vb[j] * sg * (1.0f + va[j] * (1.0f - sg));
                 db[j] = dh * va[j] * sg;
             }
-            *reinterpret_cast<uint4 *>(dpre + p * 2 * F + c) = pack8(da);
-            *reinterpret_cast<uint4 *>(dpre + p * 2 * F + F + c) = pack8(db);
+            *reinterpret_cast<uint4 *>(dpre + out * 2 * F + c) = pack8(da);
+            *reinterpret_cast<uint4 *>(dpre + out * 2 * F + F + c) = pack8(db);
         }
 #pragma unroll
         for (int d = 16; d > 0; d >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, d);
@@ -178,6 +197,31 @@ router_bwd_kernel(const int32_t *__restrict__ top_e, const float *__restrict__ t
     }
 }
 
+// Padding rows of expert e (blockIdx.x) in the padded layout: rows offsets[e] + 64 e + n_e up to
+// offsets[e] + 64 e + roundup(n_e, 64) are zeroed.
+__global__ void zero_pad_rows_kernel(uint4 *__restrict__ rows, int64_t ld16, int64_t cols16,
+                                     const int32_t *__restrict__ offsets) {
+    const int e = blockIdx.x;
+    const int64_t n = __ldg(offsets + e + 1) - __ldg(offsets + e);
+    const int64_t first = __ldg(offsets + e) + (int64_t)kWgradPad * e + n;
+    const int64_t count = (n + kWgradPad - 1) / kWgradPad * kWgradPad - n;
+    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+    for (int64_t q = threadIdx.x; q < count * cols16; q += blockDim.x)
+        rows[(first + q / cols16) * ld16 + q % cols16] = z;
+}
+
+// xs[p] = x[sorted_rows[p] / k], bf16 rows of D elements, one warp per slot.
+__global__ void __launch_bounds__(kWarps * 32)
+gather_rows_kernel(const uint4 *__restrict__ x, const int32_t *__restrict__ sorted_rows, int32_t k,
+                   int64_t R, int64_t d16, uint4 *__restrict__ xs) {
+    const int lane = threadIdx.x & 31;
+    const int64_t wstride = (int64_t)gridDim.x * kWarps;
+    for (int64_t p = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5); p < R; p += wstride) {
+        const int64_t s = __ldg(sorted_rows + p) / k;
+        for (int64_t c = lane; c < d16; c += 32) xs[p * d16 + c] = __ldg(x + s * d16 + c);
+    }
+}
+
 unsigned warp_grid(int64_t rows) {
     int64_t blocks = (rows + kWarps - 1) / kWarps;
     const int64_t cap = (int64_t)num_sms() * 16;
@@ -197,10 +241,25 @@ void launch_cast_bf16(const float *src, void *dst, int64_t n, cudaStream_t s) {
 }
 
 void launch_gate_rows(const void *dY, bool dy_bf16, const int32_t *sorted_rows, const float *gates,
-                      int32_t k, int64_t R, int64_t Dout, bool by_token, void *dv, cudaStream_t s) {
+                      int32_t k, int64_t R, int64_t Dout, bool by_token, void *dv,
+                      const int32_t *pad_offsets, int32_t E, cudaStream_t s) {
     gate_rows_kernel<<<warp_grid(R), kWarps * 32, 0, s>>>(dY, dy_bf16, sorted_rows, gates, k, R,
                                                           Dout, by_token,
-                                                          static_cast<__nv_bfloat16 *>(dv));
+                                                          static_cast<__nv_bfloat16 *>(dv),
+                                                          pad_offsets, E);
+}
+
+void launch_zero_pad_rows(void *rows, int64_t ld, int64_t cols, const int32_t *offsets, int32_t E,
+                          cudaStream_t s) {
+    zero_pad_rows_kernel<<<(unsigned)E, 256, 0, s>>>(static_cast<uint4 *>(rows), ld / 8, cols / 8,
+                                                     offsets);
+}
+
+void launch_gather_rows(const void *x, const int32_t *sorted_rows, int32_t k, int64_t R, int64_t D,
+                        void *xs, cudaStream_t s) {
+    gather_rows_kernel<<<warp_grid(R), kWarps * 32, 0, s>>>(static_cast<const uint4 *>(x),
+                                                            sorted_rows, k, R, D / 8,
+                                                            static_cast<uint4 *>(xs));
 }
 
 void launch_rowdot(const void *dY, bool dy_bf16, const void *v, const int32_t *sorted_rows,
@@ -211,12 +270,12 @@ void launch_rowdot(const void *dY, bool dy_bf16, const void *v, const int32_t *s
 }
 
 void launch_swiglu_bwd(const void *dhp, const void *h, const void *a, const void *b,
-                       const int32_t *sorted_rows, const float *top_w, int64_t R, int64_t F,
-                       void *dpre, float *dw, cudaStream_t s) {
+                       const int32_t *sorted_rows, const float *top_w, const int32_t *offsets,
+                       int32_t E, int64_t R, int64_t F, void *dpre, float *dw, cudaStream_t s) {
     swiglu_bwd_kernel<<<warp_grid(R), kWarps * 32, 0, s>>>(
         static_cast<const __nv_bfloat16 *>(dhp), static_cast<const __nv_bfloat16 *>(h),
         static_cast<const __nv_bfloat16 *>(a), static_cast<const __nv_bfloat16 *>(b), sorted_rows,
-        top_w, R, F, static_cast<__nv_bfloat16 *>(dpre), dw);
+        top_w, offsets, E, R, F, static_cast<__nv_bfloat16 *>(dpre), dw);
 }
 
 void launch_router_bwd(const int32_t *top_e, const float *top_w, const float *dw,

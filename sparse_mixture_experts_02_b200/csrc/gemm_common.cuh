@@ -56,6 +56,7 @@ struct KParams {
     int32_t stages;   // router mode: pipeline depth and stage size (bytes, multiple of 1024)
     int32_t stage_bytes;
     int32_t k_split;  // K-major B: first K index read from the second B tensor map
+    int32_t a_row_pad;  // contiguous A: slot row p of expert e is read at row p + a_row_pad * e
     // optional side job of the epilogue warps before their first tile: zero zero_n4 float4s
     float4 *zero_ptr;
     int64_t zero_n4;

@@ -152,7 +152,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                 if (lane == 0) dev::mbar_arrive_expect_tx(&st.full[s], stage_tx);
                 __syncwarp();
                 const int kc = kb * BK;
-                if (!GATHER && lane == 0) dev::tma_load_2d(sA, &tmA, &st.full[s], kc, ti.row_begin);
+                if (!GATHER && lane == 0)
+                    dev::tma_load_2d(sA, &tmA, &st.full[s], kc,
+                                     ti.row_begin + p.a_row_pad * ti.e);
                 if (BKM && lane == 0) {
                     const bool hi = kc >= p.k_split;
                     dev::tma_load_3d(sB, hi ? &tmB1 : &tmB0, &st.full[s], hi ? kc - p.k_split : kc,
@@ -556,6 +558,7 @@ int launch_t(const GemmArgs &a, cudaStream_t s) {
         kp.stages = STAGES;
     }
     kp.k_split = (int32_t)(BKM && a.B1 != nullptr ? a.k_split : a.K + BK);
+    kp.a_row_pad = GATHER ? 0 : a.a_row_pad;
     kp.zero_ptr = reinterpret_cast<float4 *>(a.zero_ptr);
     kp.zero_n4 = a.zero_n / 4;
     kp.status = a.status;

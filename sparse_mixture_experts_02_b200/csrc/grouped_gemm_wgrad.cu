@@ -1,30 +1,29 @@
 // Weight gradient of ParallelLinear on the sm_100a tensor cores: for every expert e,
-//   dW[e] = sum over the slots p of e of  src_p^T (x) dv_p        ([Din, Dout], fp32)
-// with src_p = X[sorted_rows[p] / k] (gathered token rows) or X[p] (slot-ordered rows) and dv_p
-// the gated output-gradient rows in slot order. The reduction runs over an expert's slots, so the
-// K extent of a tile is that expert's row count: any value, zero included.
+//   dW[e] = sum over the slots p of e of  A_p^T (x) dv_p        ([Din, Dout], fp32)
+// with A_p the input row of slot p and dv_p its gated output-gradient row. The reduction runs
+// over an expert's slots, so the K extent of a tile is that expert's row count: any value, zero
+// included.
 //
 // Source: ScatterMoE guide, "3. Fused Backward Pass Dynamics" (the weight gradient of expert e
 // accumulates the outer products of its tokens' inputs and gated output gradients). The guide
 // reduces inside shared memory to avoid global atomics; here each output tile is owned by one CTA
 // and reduced in TMEM over the expert's slots, so no atomics are needed either.
 //
-// Design (one CTA per SM, persistent, the forward kernel's warp roles):
-//   warp 0     TMA producer of B: the stage's 64 dv rows x 256 columns (4 boxes of 64 x 64,
-//              128-byte swizzle: MN-major, the K index is the row).
-//   warps 6-9  cp.async gatherers of A: the stage's 64 source rows x 128 columns of Din, written
-//              MN-major in the same swizzle (row r of the stage at 128-byte line r of each
-//              64-column chunk); slots past the expert's end and columns past Din are zero-filled.
-//              Each copy instruction covers 4 whole 128-byte segments (one per 8 lanes); the row
-//              indices of the next stage are loaded one stage ahead. (One thread per half-row,
-//              16 bytes per instruction, touched 32 segments per instruction and cost ~40%.)
+// Operands (both MN-major: the K index, a slot, is the row): A in slot order, dv in a padded
+// slot order where expert e's rows start at offsets[e] + 64 e and are followed by zero rows up
+// to the next multiple of 64. A stage of 64 slots may run past the expert's last slot; those A
+// rows belong to the next expert, but their dv rows are zero, so they add nothing. Both come by
+// TMA (cp.async gathers of A cost ~40% here: the epilogue already loads the LSU path).
+//
+// Design (one CTA per SM, persistent):
+//   warp 0     TMA producer: per stage 64 A rows x 128 columns (2 boxes of 64 x 64) and 64 dv
+//              rows x 256 columns (4 boxes), 128-byte swizzle.
 //   warp 1     TMEM owner (two 128 x 256 fp32 accumulators) and MMA issuer: 4 MMAs of M=128
-//              (Din), N=256 (Dout), K=16 rows per stage, both operands MN-major.
+//              (Din), N=256 (Dout), K=16 rows per stage.
 //   warps 2-5  epilogue: accumulator lane m -> dW[e][m0 + m][n0 .. n0 + 255], staged through
 //              shared memory in 32 x 32 chunks so each store covers 4 rows x 128 bytes; a tile of
 //              an expert without slots stores zeros.
-// Tiles are (expert, N tile, M tile), expert-major, so the CTAs running at once share an
-// expert's rows through L2. Every wait is bounded (mbar_wait).
+// Tiles are (expert, N tile, M tile), expert-major. Every wait is bounded (mbar_wait).
 #include "gemm_common.cuh"
 
 #include <mutex>
@@ -41,11 +40,9 @@ constexpr int WB_BYTES = 4 * WCH;          // B: 256 columns of Dout
 static_assert(WA_BYTES == A_BYTES && WB_BYTES == B_BYTES, "stage layout of the forward kernel");
 
 struct WParams {
-    const uint8_t *X;
-    int64_t Din, Dout;
     const int32_t *offsets;
-    const int32_t *sorted_rows;
-    int32_t E, k, gather;
+    int64_t Din, Dout;
+    int32_t E;
     float *dW;
     int32_t m_tiles, n_tiles;
     unsigned *status;
@@ -59,8 +56,9 @@ __device__ __forceinline__ void wtile(int t, int per_e, int m_tiles, int &e, int
     m = local - n * m_tiles;
 }
 
-__global__ void __launch_bounds__(THREADS + GATHER_THREADS, 1)
-grouped_wgrad_kernel(const __grid_constant__ CUtensorMap tmB, const WParams p) {
+__global__ void __launch_bounds__(THREADS, 1)
+grouped_wgrad_kernel(const __grid_constant__ CUtensorMap tmA,
+                     const __grid_constant__ CUtensorMap tmB, const WParams p) {
     constexpr uint32_t IDESC = dev::idesc_f32acc(true, BM, BN, true, true);
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -73,7 +71,7 @@ grouped_wgrad_kernel(const __grid_constant__ CUtensorMap tmB, const WParams p) {
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            dev::mbar_init(&st.full[s], 1 + GATHER_THREADS);
+            dev::mbar_init(&st.full[s], 1);
             dev::mbar_init(&st.empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -84,7 +82,10 @@ grouped_wgrad_kernel(const __grid_constant__ CUtensorMap tmB, const WParams p) {
         st.abort = 0;
         dev::fence_mbar_init();
     }
-    if (warp == 0 && lane == 0) dev::prefetch_tmap(&tmB);
+    if (warp == 0 && lane == 0) {
+        dev::prefetch_tmap(&tmA);
+        dev::prefetch_tmap(&tmB);
+    }
     if (warp == 1) {
         dev::tmem_alloc(&st.tmem_base, TMEM_COLS);
         dev::tmem_relinquish();
@@ -115,12 +116,17 @@ grouped_wgrad_kernel(const __grid_constant__ CUtensorMap tmB, const WParams p) {
                     break;
                 }
                 if (lane == 0) {
-                    uint8_t *sB = smem + (size_t)s * STAGE_BYTES + WA_BYTES;
-                    dev::mbar_arrive_expect_tx(&st.full[s], (uint32_t)WB_BYTES);
+                    uint8_t *sA = smem + (size_t)s * STAGE_BYTES;
+                    uint8_t *sB = sA + WA_BYTES;
+                    dev::mbar_arrive_expect_tx(&st.full[s], (uint32_t)(WA_BYTES + WB_BYTES));
+#pragma unroll
+                    for (int c = 0; c < 2; ++c)
+                        dev::tma_load_2d(sA + c * WCH, &tmA, &st.full[s], m * BM + c * 64,
+                                         r0 + kb * WK);
 #pragma unroll
                     for (int c = 0; c < 4; ++c)
                         dev::tma_load_2d(sB + c * WCH, &tmB, &st.full[s], n * BN + c * 64,
-                                         r0 + kb * WK);
+                                         r0 + kWgradPad * e + kb * WK);
                 }
                 issued |= 1u << s;
                 last_par = (last_par & ~(1u << s)) | (ph << s);
@@ -160,7 +166,6 @@ grouped_wgrad_kernel(const __grid_constant__ CUtensorMap tmB, const WParams p) {
                         break;
                     }
                     dev::tc_fence_after();
-                    dev::fence_proxy_async_smem();  // cp.async rows -> tensor core
                     const uint32_t sA = dev::smem_u32(smem + (size_t)s * STAGE_BYTES);
                     const uint32_t sB = sA + WA_BYTES;
 #pragma unroll
@@ -186,60 +191,6 @@ grouped_wgrad_kernel(const __grid_constant__ CUtensorMap tmB, const WParams p) {
             dev::tc_fence_before();
         }
         __syncwarp();
-    } else if (warp >= THREADS / 32) {
-        // ------------------------------------------------------------------ A gatherers
-        // Warp gw fills stage rows gw*16 .. gw*16+15, both 128-byte halves of each. Per copy
-        // instruction i, lanes 8u..8u+7 (u = lane / 8) copy the 16-byte pieces 0..7 of row
-        // 2i + u/2, half u%2: a warp instruction covers 4 whole 128-byte segments. Lane l < 16
-        // holds the source row of the warp's row l (loaded one stage ahead; lanes 16-31 repeat
-        // it), and the copies take it by shuffle.
-        const int gw = (threadIdx.x - THREADS) >> 5;
-        const int j = lane & 7, sub = lane >> 3;
-        const int64_t row_bytes = p.Din * 2;
-        uint32_t s = 0, ph = 0;
-        bool ok = true;
-        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-            int e, n, m;
-            wtile(t, per_e, p.m_tiles, e, n, m);
-            const int r0 = st.off[e], r1 = st.off[e + 1];
-            const int nkb = (r1 - r0 + WK - 1) / WK;
-            auto row_index = [&](int kb) -> long long {
-                const int slot = r0 + kb * WK + gw * 16 + (lane & 15);
-                if (slot >= r1) return -1;
-                return p.gather ? (long long)(__ldg(p.sorted_rows + slot) / p.k) : (long long)slot;
-            };
-            long long myrow = nkb > 0 ? row_index(0) : -1;
-            for (int kb = 0; kb < nkb; ++kb) {
-                const long long next = kb + 1 < nkb ? row_index(kb + 1) : -1;
-                bool w = true;
-                if (lane == 0)
-                    w = dev::mbar_wait(&st.empty[s], ph ^ 1u, abort, p.status, p.wait_limit_ns,
-                                       kKernelGemm);
-                w = __shfl_sync(0xffffffffu, w, 0);
-                if (!w) {
-                    ok = false;
-                    break;
-                }
-                const uint32_t sA = dev::smem_u32(smem + (size_t)s * STAGE_BYTES);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int rl = 2 * i + (sub >> 1), h = sub & 1;
-                    const int r = gw * 16 + rl;
-                    const long long row = __shfl_sync(0xffffffffu, myrow, rl);
-                    const int64_t cb = ((int64_t)m * BM + h * 64) * 2 + j * 16;
-                    const bool in = row >= 0 && cb < row_bytes;
-                    const uint32_t dst = sA + h * WCH + r * KBYTES + ((j ^ (r & 7)) << 4);
-                    dev::cp_async16(dst, in ? p.X + row * row_bytes + cb : p.X, in ? 16u : 0u);
-                }
-                dev::cp_async_arrive_noinc(&st.full[s]);
-                myrow = next;
-                if (++s == STAGES) {
-                    s = 0;
-                    ph ^= 1u;
-                }
-            }
-        }
-        dev::cp_async_wait_all();
     } else {
         // ------------------------------------------------------------------ epilogue
         const int q = warp & 3;  // TMEM lane quarter this warp may access
@@ -309,7 +260,7 @@ grouped_wgrad_kernel(const __grid_constant__ CUtensorMap tmB, const WParams p) {
 
 int launch_grouped_wgrad(const WgradArgs &a, cudaStream_t s) {
     const int64_t m_tiles = (a.Din + BM - 1) / BM, n_tiles = (a.Dout + BN - 1) / BN;
-    if (a.R <= 0 || a.E <= 0) {
+    if (a.a_rows <= 0 || a.E <= 0) {
         // no slot at all: every expert's gradient is zero
         launch_zero_f32(a.dW, (int64_t)a.E * a.Din * a.Dout, nullptr, s);
         return MOE_OK;
@@ -325,29 +276,32 @@ int launch_grouped_wgrad(const WgradArgs &a, cudaStream_t s) {
     });
     if (attr_err != cudaSuccess)
         return set_error(MOE_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(attr_err));
-    CUtensorMap mB;
+    CUtensorMap mA, mB;
     {
-        const uint64_t dims[2] = {(uint64_t)a.Dout, (uint64_t)a.R};
+        const uint64_t dims[2] = {(uint64_t)a.Din, (uint64_t)a.a_rows};
+        const uint64_t str[1] = {(uint64_t)(a.a_ld > 0 ? a.a_ld : a.Din) * 2};
+        const uint32_t box[2] = {64u, (uint32_t)WK};
+        int rc = encode_tmap(&mA, true, 2, a.A, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
+        if (rc) return rc;
+    }
+    {
+        const uint64_t dims[2] = {(uint64_t)a.Dout, (uint64_t)a.dv_rows};
         const uint64_t str[1] = {(uint64_t)(a.dv_ld > 0 ? a.dv_ld : a.Dout) * 2};
         const uint32_t box[2] = {64u, (uint32_t)WK};
         int rc = encode_tmap(&mB, true, 2, a.dv, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
         if (rc) return rc;
     }
     WParams wp;
-    wp.X = reinterpret_cast<const uint8_t *>(a.X);
+    wp.offsets = a.offsets;
     wp.Din = a.Din;
     wp.Dout = a.Dout;
-    wp.offsets = a.offsets;
-    wp.sorted_rows = a.sorted_rows;
     wp.E = a.E;
-    wp.k = a.k;
-    wp.gather = a.gather ? 1 : 0;
     wp.dW = a.dW;
     wp.m_tiles = (int32_t)m_tiles;
     wp.n_tiles = (int32_t)n_tiles;
     wp.status = a.status;
     wp.wait_limit_ns = a.wait_limit_ns;
-    kern<<<num_sms(), THREADS + GATHER_THREADS, SMEM_BYTES, s>>>(mB, wp);
+    kern<<<num_sms(), THREADS, SMEM_BYTES, s>>>(mA, mB, wp);
     return MOE_OK;
 }
 

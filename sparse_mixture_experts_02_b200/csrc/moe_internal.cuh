@@ -58,6 +58,8 @@ struct GemmArgs {
     // B1 the rest ([E, N, K - k_split]); k_split is a multiple of 64 bf16 elements.
     bool b_kmajor;
     int64_t k_split;
+    // contiguous A only: slot row p of expert e is read at row p + a_row_pad * e (a padded layout)
+    int32_t a_row_pad;
     const float *bias;      // router mode only
     int32_t *top_e;
     float *top_w;
@@ -73,32 +75,46 @@ int launch_grouped_gemm_2sm(const GemmArgs &a, cudaStream_t s);
 // pair tiles waste little there); the environment variable MOE_GEMM_2SM=0/1 forces either kernel.
 bool prefer_2sm(int64_t R, int32_t E);
 int launch_debug_wait(int64_t limit_ns, unsigned *status, cudaStream_t s);
-// Weight gradient of ParallelLinear: dW[e] = sum over the slots p of expert e of
-// src_p^T (x) dv_p, src_p = X[sorted_rows[p] / k] (gather) or X[p], dv [R, Dout] bf16 in slot
-// order; dW [E, Din, Dout] fp32 is overwritten (zeros for experts without slots). bf16 only.
+// Weight gradient of ParallelLinear: dW[e] = sum over the slots p of expert e of A_p^T (x) dv_p,
+// A [a_rows, Din] the source rows in slot order (row stride a_ld elements, 0: Din), dv the
+// output-gradient rows in the padded slot layout: expert e's rows start at row offsets[e] + 64 e
+// and are followed by zero rows up to the next multiple of 64 (dv_rows >= R + 64 E). dW
+// [E, Din, Dout] fp32 is overwritten (zeros for experts without slots). bf16 operands.
 struct WgradArgs {
-    const void *X;          // [S, Din] (gather) or [R, Din]
-    const void *dv;         // [R, Dout] with row stride dv_ld elements (0: Dout)
-    int64_t dv_ld;
+    const void *A;
+    int64_t a_rows, a_ld;
+    const void *dv;
+    int64_t dv_rows, dv_ld;
     const int32_t *offsets; // [E+1]
-    const int32_t *sorted_rows;
-    int64_t Din, Dout, R;
-    int32_t E, k;
-    bool gather;
+    int64_t Din, Dout;
+    int32_t E;
     float *dW;
     unsigned *status;
     int64_t wait_limit_ns;
 };
+constexpr int kWgradPad = 64;  // rows of zero padding per expert in the dv layout
 int launch_grouped_wgrad(const WgradArgs &a, cudaStream_t s);
 // Backward helpers (backward.cu), one warp per slot; Dout a multiple of 8, rows 16-byte aligned.
 void launch_cast_bf16(const float *src, void *dst, int64_t n, cudaStream_t s);
+// dv[p'] = bf16(gate * dY[row(p)]) with p' = p + 64 e(p) when pad_offsets (the expert offsets)
+// is given (the weight gradient's padded layout), else p' = p.
 void launch_gate_rows(const void *dY, bool dy_bf16, const int32_t *sorted_rows, const float *gates,
-                      int32_t k, int64_t R, int64_t Dout, bool by_token, void *dv, cudaStream_t s);
+                      int32_t k, int64_t R, int64_t Dout, bool by_token, void *dv,
+                      const int32_t *pad_offsets, int32_t E, cudaStream_t s);
+// Zeroes, for every expert, the padding rows after its rows in the padded layout (bf16 rows of
+// `cols` elements, row stride ld).
+void launch_zero_pad_rows(void *rows, int64_t ld, int64_t cols, const int32_t *offsets, int32_t E,
+                          cudaStream_t s);
+// xs[p] = x[sorted_rows[p] / k] (bf16 rows of D elements): the slot-ordered rows the weight
+// gradient reads by TMA.
+void launch_gather_rows(const void *x, const int32_t *sorted_rows, int32_t k, int64_t R, int64_t D,
+                        void *xs, cudaStream_t s);
 void launch_rowdot(const void *dY, bool dy_bf16, const void *v, const int32_t *sorted_rows,
                    int32_t k, int64_t R, int64_t Dout, bool by_token, float *dg, cudaStream_t s);
+// [da | db] rows are written in the padded layout (slot p at row p + 64 e(p)).
 void launch_swiglu_bwd(const void *dhp, const void *h, const void *a, const void *b,
-                       const int32_t *sorted_rows, const float *top_w, int64_t R, int64_t F,
-                       void *dpre, float *dw, cudaStream_t s);
+                       const int32_t *sorted_rows, const float *top_w, const int32_t *offsets,
+                       int32_t E, int64_t R, int64_t F, void *dpre, float *dw, cudaStream_t s);
 void launch_router_bwd(const int32_t *top_e, const float *top_w, const float *dw,
                        const void *w_gate, int64_t S, int64_t D, int32_t E, int32_t k, void *dl,
                        float *dx, int32_t *offsets1, cudaStream_t s);
