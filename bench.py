@@ -446,7 +446,7 @@ def backward_bench(args, w):
         t1.record()
         torch.cuda.synchronize(dev)
     ms = t0.elapsed_time(t1) / args.steps
-    names = ["dh", "recompute_a_b", "swiglu_bwd_and_dW_down", "dx", "dW_gate_e_and_dW_up",
+    names = ["dh", "gemm1_recompute_with_swiglu_bwd", "dW_down", "dx", "dW_gate_e_and_dW_up",
              "router"]
     stage = {n: sum(r[q].elapsed_time(r[q + 1]) for r in evs) / args.steps
              for q, n in enumerate(names)}

@@ -189,12 +189,12 @@ int moe_mlp_forward(const void *x, const void *w_gate, const float *logit_bias,
  * selected logits, differentiated through it. Steps on `stream`:
  *   1. dout -> bf16.
  *   2. dh = dout[s] . W_down[e]^T per slot (the forward's grouped GEMM, W_down read K-major).
- *   3. a = x W_gate_e[e] and b = x W_up[e] recomputed.
- *   4. SwiGLU backward: the route-weight gradient dh . h, then da and db.
- *   5. dW_down (weight-gradient GEMM over each expert's slots).
- *   6. dx += [da | db] . [W_gate_e ; W_up]^T (scatter-added into tokens).
- *   7. dW_gate_e and dW_up.
- *   8. Router backward: the softmax Jacobian, then dx += dl W_gate^T and dW_gate = x^T dl.
+ *   3. The fused gate+up GEMM recomputed, with the SwiGLU backward in its epilogue: the
+ *      route-weight gradient dh . h, then da and db.
+ *   4. dW_down (weight-gradient GEMM over each expert's slots).
+ *   5. dx += [da | db] . [W_gate_e ; W_up]^T (scatter-added into tokens).
+ *   6. dW_gate_e and dW_up.
+ *   7. Router backward: the softmax Jacobian, then dx += dl W_gate^T and dW_gate = x^T dl.
  * ScatterMoE guide, "3. Fused Backward Pass Dynamics" (each ParallelLinear's input and weight
  * gradients). Constraints beyond the forward's: bf16 only, E a multiple of 8, F a multiple of 64.
  * ws: moe_workspace_size("mlp_backward", S, D, F, E, k, dt) bytes.

@@ -151,7 +151,7 @@ BwdLayout bwd_layout(int64_t S, int64_t Din, int64_t Dout, int32_t E, int32_t k)
 
 // MLP backward scratch (the forward's workspace supplies routing, map and h).
 struct MlpBwdLayout {
-    size_t status, dyb, dhp, a, b, dpre, dw, dv, dl, xs, off1, total;
+    size_t status, dyb, dhp, dpre, dw, dv, dl, xs, off1, total;
 };
 
 MlpBwdLayout mlp_bwd_layout(int64_t S, int64_t D, int64_t F, int32_t E, int32_t k) {
@@ -161,8 +161,6 @@ MlpBwdLayout mlp_bwd_layout(int64_t S, int64_t D, int64_t F, int32_t E, int32_t 
     L.status = o; o += kStatusBytes;
     L.dyb = o; o = align_up(o + 2 * (size_t)S * (size_t)D);
     L.dhp = o; o = align_up(o + 2 * (size_t)R * (size_t)F);
-    L.a = o; o = align_up(o + 2 * (size_t)R * (size_t)F);
-    L.b = o; o = align_up(o + 2 * (size_t)R * (size_t)F);
     // [da | db], the gated dout rows and the router's dl in the weight gradient's padded layout
     const int64_t Rp = R + (int64_t)kWgradPad * E;
     L.dpre = o; o = align_up(o + 4 * (size_t)Rp * (size_t)F);
@@ -673,11 +671,11 @@ extern "C" int moe_mlp_backward(const void *x, const void *w_gate, const void *w
         g_launches = n + 4;
         return check_launch("mlp_backward");
     }
-    // profile events (moe_profile_events): 0 start, 1 after dh, 2 after the a/b recompute,
-    // 3 after the SwiGLU backward and dW_down, 4 after dx, 5 after dW_gate_e/dW_up, 6 end
+    // profile events (moe_profile_events): 0 start, 1 after dh, 2 after the GEMM1 recompute with
+    // the SwiGLU backward, 3 after dW_down, 4 after dx, 5 after dW_gate_e/dW_up, 6 end
     record_prof(0, s);
-    void *dyb = at<void>(ws, L.dyb), *dhp = at<void>(ws, L.dhp), *av = at<void>(ws, L.a);
-    void *bv = at<void>(ws, L.b), *dpre = at<void>(ws, L.dpre), *dv = at<void>(ws, L.dv);
+    void *dyb = at<void>(ws, L.dyb), *dhp = at<void>(ws, L.dhp);
+    void *dpre = at<void>(ws, L.dpre), *dv = at<void>(ws, L.dv);
     void *dl = at<void>(ws, L.dl);
     float *dwr = at<float>(ws, L.dw);
     int32_t *off1 = at<int32_t>(ws, L.off1);
@@ -708,27 +706,31 @@ extern "C" int moe_mlp_backward(const void *x, const void *w_gate, const void *w
         ++n;
     }
     record_prof(1, s);
-    // GEMM1 pre-activations recomputed: a = x W_gate_e[e], b = x W_up[e] (slot order)
-    for (int half = 0; half < 2; ++half) {
+    // GEMM1 recomputed (fused gate+up, gathered x) with the SwiGLU backward in its epilogue: the
+    // route-weight gradient dh_u . h (atomically per N tile) and [da | db] in the padded layout
+    const int64_t Rp = R + (int64_t)kWgradPad * E;
+    launch_zero_f32(dwr, R, nullptr, s);
+    {
         GemmArgs a = g;
         a.A = x;
         a.a_rows = S;
-        a.B0 = half == 0 ? w_gate_e : w_up;
-        a.out = half == 0 ? av : bv;
+        a.B0 = w_gate_e;
+        a.B1 = w_up;
+        a.gates = top_w;
+        a.out = dpre;
         a.K = D;
         a.N = F;
         a.gather = true;
-        if ((rc = prefer_2sm(R, E) ? launch_grouped_gemm_2sm(a, s) : launch_grouped_gemm(a, s)))
-            return rc;
-        ++n;
+        a.glu = true;
+        a.glu_bwd = true;
+        a.bwd_dh = dhp;
+        a.bwd_dw = dwr;
+        a.out_row_pad = kWgradPad;
+        if ((rc = launch_grouped_gemm(a, s))) return rc;
     }
-    record_prof(2, s);
-    // route-weight gradient and [da | db]
-    launch_zero_f32(dwr, R, nullptr, s);
-    const int64_t Rp = R + (int64_t)kWgradPad * E;
-    launch_swiglu_bwd(dhp, h, av, bv, sorted_rows, top_w, offsets, E, R, F, dpre, dwr, s);
     launch_zero_pad_rows(dpre, 2 * F, 2 * F, offsets, E, s);
     n += 3;
+    record_prof(2, s);
     // dW_down[e] = sum over e's slots of h_p^T (w_i dout[s])
     launch_gate_rows(dout, false, sorted_rows, top_w, k, R, D, true, dv, offsets, E, s);
     launch_zero_pad_rows(dv, D, D, offsets, E, s);

@@ -117,46 +117,6 @@ rowdot_kernel(const void *__restrict__ dY, bool dy_bf16, const __nv_bfloat16 *__
     }
 }
 
-// SwiGLU backward of one slot p (route i, gate g = top_w[i]) from the ungated gradient of h,
-// dhp = dout[s] . W_down[e]^T, the forward's h and the recomputed pre-activations a, b:
-//   dw[i] = dhp . h;  dh = g * dhp;  da = dh * b * silu'(a);  db = dh * silu(a)
-// with silu'(z) = sig(z) (1 + z (1 - sig(z))); writes dpre[p] = [da | db] (bf16, 2F wide).
-__global__ void __launch_bounds__(kWarps * 32)
-swiglu_bwd_kernel(const __nv_bfloat16 *__restrict__ dhp, const __nv_bfloat16 *__restrict__ h,
-                  const __nv_bfloat16 *__restrict__ a, const __nv_bfloat16 *__restrict__ b,
-                  const int32_t *__restrict__ sorted_rows, const float *__restrict__ top_w,
-                  const int32_t *__restrict__ offsets, int32_t E, int64_t R, int64_t F,
-                  __nv_bfloat16 *__restrict__ dpre, float *__restrict__ dw) {
-    const int lane = threadIdx.x & 31;
-    const int64_t wstride = (int64_t)gridDim.x * kWarps;
-    for (int64_t p = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5); p < R; p += wstride) {
-        const int32_t i = __ldg(sorted_rows + p);
-        const float g = __ldg(top_w + i);
-        const int64_t out = p + (int64_t)kWgradPad * expert_of(offsets, E, p);
-        float acc = 0.f;
-        for (int64_t c = (int64_t)lane * 8; c < F; c += 32 * 8) {
-            float vd[8], vh[8], va[8], vb[8], da[8], db[8];
-            load8(dhp + p * F, true, c, vd);
-            load8(h + p * F, true, c, vh);
-            load8(a + p * F, true, c, va);
-            load8(b + p * F, true, c, vb);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                acc = fmaf(vd[j], vh[j], acc);
-                const float dh = g * vd[j];
-                const float sg = 1.0f / (1.0f + __expf(-va[j]));
-                da[j] = dh * vb[j] * sg * (1.0f + va[j] * (1.0f - sg));
-                db[j] = dh * va[j] * sg;
-            }
-            *reinterpret_cast<uint4 *>(dpre + out * 2 * F + c) = pack8(da);
-            *reinterpret_cast<uint4 *>(dpre + out * 2 * F + F + c) = pack8(db);
-        }
-#pragma unroll
-        for (int d = 16; d > 0; d >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, d);
-        if (lane == 0) dw[i] = acc;
-    }
-}
-
 // Router backward of one token s: the softmax over its k selected logits gives
 //   dl_j = w_j (dw_j - sum_j' w_j' dw_j');
 // dl is written as a dense bf16 row [E] (zero outside the selection, the weight gradient's
@@ -267,15 +227,6 @@ void launch_rowdot(const void *dY, bool dy_bf16, const void *v, const int32_t *s
     rowdot_kernel<<<warp_grid(R), kWarps * 32, 0, s>>>(dY, dy_bf16,
                                                        static_cast<const __nv_bfloat16 *>(v),
                                                        sorted_rows, k, R, Dout, by_token, dg);
-}
-
-void launch_swiglu_bwd(const void *dhp, const void *h, const void *a, const void *b,
-                       const int32_t *sorted_rows, const float *top_w, const int32_t *offsets,
-                       int32_t E, int64_t R, int64_t F, void *dpre, float *dw, cudaStream_t s) {
-    swiglu_bwd_kernel<<<warp_grid(R), kWarps * 32, 0, s>>>(
-        static_cast<const __nv_bfloat16 *>(dhp), static_cast<const __nv_bfloat16 *>(h),
-        static_cast<const __nv_bfloat16 *>(a), static_cast<const __nv_bfloat16 *>(b), sorted_rows,
-        top_w, offsets, E, R, F, static_cast<__nv_bfloat16 *>(dpre), dw);
 }
 
 void launch_router_bwd(const int32_t *top_e, const float *top_w, const float *dw,

@@ -57,6 +57,11 @@ struct KParams {
     int32_t stage_bytes;
     int32_t k_split;  // K-major B: first K index read from the second B tensor map
     int32_t a_row_pad;  // contiguous A: slot row p of expert e is read at row p + a_row_pad * e
+    // GLU backward epilogue (the MLP backward's recompute of GEMM1): the ungated gradient of h
+    // [R, N] bf16 in slot order, the route-weight gradient [R] (accumulated), the output row pad
+    const void *bwd_dh;
+    float *bwd_dw;
+    int32_t out_row_pad;
     // optional side job of the epilogue warps before their first tile: zero zero_n4 float4s
     float4 *zero_ptr;
     int64_t zero_n4;
@@ -239,6 +244,63 @@ __device__ __forceinline__ void epilogue_row(const KParams &p, uint32_t tbase, b
             }
         }
     }
+}
+
+// SwiGLU backward in the epilogue of the fused gate+up GEMM (MLP backward): the accumulator holds
+// a = x W_gate_e[e] in columns 0..127 and b = x W_up[e] in 128..255 for output columns n0.. of
+// slot `slot` (route `route`, router weight g). With dh = g * dh_u (dh_u = the ungated gradient
+// of h, read from bwd_dh) and h = silu(a) * b recomputed in fp32:
+//   dw[route] += dh_u . h  (atomically: one partial per N tile)
+//   da = dh * b * silu'(a), silu'(z) = sig(z) (1 + z (1 - sig(z)));  db = dh * silu(a)
+// written as bf16 to out[out_row][n0 + c] and out[out_row][N + n0 + c] (row stride 2N).
+__device__ __forceinline__ void glu_bwd_row(const KParams &p, uint32_t tbase, bool valid,
+                                            int64_t slot, int64_t route, float g, int64_t out_row,
+                                            int n0) {
+    constexpr int HALF = BN / 2;
+    float dw_acc = 0.f;
+    const __nv_bfloat16 *dh_row = static_cast<const __nv_bfloat16 *>(p.bwd_dh) + slot * p.N;
+    __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(p.out) + out_row * (2 * (int64_t)p.N);
+#pragma unroll 1
+    for (int c = 0; c < HALF / 32; ++c) {
+        uint32_t av[32], bv[32];
+        dev::tmem_ld32(tbase + c * 32, av);
+        dev::tmem_ld32(tbase + HALF + c * 32, bv);
+        dev::tmem_ld_wait();
+        const int col0 = n0 + c * 32;
+        if (!valid || col0 >= p.N) continue;
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+            if (col0 + v * 8 >= p.N) break;
+            const uint4 u = *reinterpret_cast<const uint4 *>(dh_row + col0 + v * 8);
+            const __nv_bfloat162 *hp = reinterpret_cast<const __nv_bfloat162 *>(&u);
+            float da[8], db[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const float2 d2 = __bfloat1622float2(hp[j >> 1]);
+                const float du = (j & 1) ? d2.y : d2.x;
+                const float a = __uint_as_float(av[v * 8 + j]);
+                const float b = __uint_as_float(bv[v * 8 + j]);
+                const float sg = 1.0f / (1.0f + __expf(-a));
+                const float sl = a * sg;
+                dw_acc = fmaf(du, sl * b, dw_acc);
+                const float dh = g * du;
+                da[j] = dh * b * sg * (1.0f + a * (1.0f - sg));
+                db[j] = dh * sl;
+            }
+            uint4 pa, pb;
+            uint32_t *wa = reinterpret_cast<uint32_t *>(&pa), *wb = reinterpret_cast<uint32_t *>(&pb);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                __nv_bfloat162 ta = __floats2bfloat162_rn(da[2 * j], da[2 * j + 1]);
+                __nv_bfloat162 tb = __floats2bfloat162_rn(db[2 * j], db[2 * j + 1]);
+                wa[j] = *reinterpret_cast<uint32_t *>(&ta);
+                wb[j] = *reinterpret_cast<uint32_t *>(&tb);
+            }
+            *reinterpret_cast<uint4 *>(o + col0 + v * 8) = pa;
+            *reinterpret_cast<uint4 *>(o + p.N + col0 + v * 8) = pb;
+        }
+    }
+    if (valid) atomicAdd(p.bwd_dw + route, dw_acc);
 }
 
 }  // namespace gemm

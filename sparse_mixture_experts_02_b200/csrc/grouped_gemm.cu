@@ -45,7 +45,7 @@ namespace {
 
 using namespace gemm;
 
-template <bool BF16, bool GATHER, bool GLU, bool SCATTER, bool ROUTER, bool BKM>
+template <bool BF16, bool GATHER, bool GLU, bool SCATTER, bool ROUTER, bool BKM, bool GBWD>
 __global__ void __launch_bounds__(GATHER ? THREADS + GATHER_THREADS : THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     const __grid_constant__ CUtensorMap tmB0,
@@ -58,6 +58,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     constexpr int B_KSTEP = (32 / EB) * KBYTES;  // bytes of B per MMA K step (32 bytes of K)
     constexpr int OUT_COLS = GLU ? BN / 2 : BN;  // output columns per tile
     static_assert(!(BKM && (GLU || ROUTER)), "K-major B is for the plain grouped GEMM");
+    static_assert(!GBWD || (BF16 && GLU && !SCATTER && !ROUTER), "GLU backward epilogue form");
     constexpr uint32_t IDESC = dev::idesc_f32acc(BF16, BM, BN, !BKM);
     // A tile with at most 64 rows (an expert's short last tile) runs an M=64 MMA: half the tensor
     // work; its accumulator rows 16j + i (i < 16) sit in TMEM lanes 32j + i.
@@ -401,6 +402,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         }
                     }
                 }
+            } else if constexpr (GBWD) {
+                const int64_t route = valid ? (int64_t)__ldg(p.sorted_rows + prow) : 0;
+                glu_bwd_row(p, tbase, valid, prow, route, g,
+                            prow + (int64_t)p.out_row_pad * ti.e, n0);
             } else {
                 epilogue_row<BF16, GLU, SCATTER>(p, tbase, valid, orow, g, n0, st.stage[q]);
             }
@@ -473,12 +478,13 @@ int encode_tmap(CUtensorMap *m, bool bf16, int rank, const void *base, const uin
 
 namespace {
 
-template <bool BF16, bool GATHER, bool GLU, bool SCATTER, bool ROUTER = false, bool BKM = false>
+template <bool BF16, bool GATHER, bool GLU, bool SCATTER, bool ROUTER = false, bool BKM = false,
+          bool GBWD = false>
 int launch_t(const GemmArgs &a, cudaStream_t s) {
     constexpr int EB = BF16 ? 2 : 4;
     constexpr int BK = KBYTES / EB;
     constexpr int CW = KBYTES / EB;
-    auto kern = grouped_gemm_kernel<BF16, GATHER, GLU, SCATTER, ROUTER, BKM>;
+    auto kern = grouped_gemm_kernel<BF16, GATHER, GLU, SCATTER, ROUTER, BKM, GBWD>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [&] {
@@ -559,6 +565,9 @@ int launch_t(const GemmArgs &a, cudaStream_t s) {
     }
     kp.k_split = (int32_t)(BKM && a.B1 != nullptr ? a.k_split : a.K + BK);
     kp.a_row_pad = GATHER ? 0 : a.a_row_pad;
+    kp.bwd_dh = a.bwd_dh;
+    kp.bwd_dw = a.bwd_dw;
+    kp.out_row_pad = a.out_row_pad;
     kp.zero_ptr = reinterpret_cast<float4 *>(a.zero_ptr);
     kp.zero_n4 = a.zero_n / 4;
     kp.status = a.status;
@@ -573,6 +582,12 @@ int launch_t(const GemmArgs &a, cudaStream_t s) {
 int launch_grouped_gemm(const GemmArgs &a, cudaStream_t s) {
     // instantiated forms: (gather, glu, scatter) in {(1,1,0), (0,0,1), (1,0,0), (1,0,1),
     // (0,0,0)} x {bf16, f32}
+    // GLU backward epilogue (bf16, gathered x, fused gate+up): the MLP backward's recompute
+    if (a.glu_bwd) {
+        if (a.bf16 && a.gather && a.glu && !a.scatter && !a.b_kmajor)
+            return launch_t<true, true, true, false, false, false, true>(a, s);
+        return set_error(MOE_ERR_UNSUPPORTED, "GLU backward epilogue form not built");
+    }
 #define MOE_DISPATCH(BF, G, L, SC)                                                          \
     if (!a.b_kmajor && a.bf16 == BF && a.gather == G && a.glu == L && a.scatter == SC)      \
         return launch_t<BF, G, L, SC>(a, s);

@@ -461,8 +461,9 @@ int max_pairs() {
 }  // namespace
 
 int launch_grouped_gemm_2sm(const GemmArgs &a, cudaStream_t s) {
-    if (a.b_kmajor || a.a_row_pad != 0)
-        return set_error(MOE_ERR_UNSUPPORTED, "two-CTA grouped GEMM: K-major B / padded A not built");
+    if (a.b_kmajor || a.a_row_pad != 0 || a.glu_bwd)
+        return set_error(MOE_ERR_UNSUPPORTED,
+                         "two-CTA grouped GEMM: K-major B / padded A / GLU backward not built");
     const int pairs = max_pairs();
 #define MOE_DISPATCH2(BF, G, L, SC)                                                         \
     if (a.bf16 == BF && a.gather == G && a.glu == L && a.scatter == SC)                     \

@@ -60,6 +60,13 @@ struct GemmArgs {
     int64_t k_split;
     // contiguous A only: slot row p of expert e is read at row p + a_row_pad * e (a padded layout)
     int32_t a_row_pad;
+    // GLU backward epilogue (one-CTA kernel, bf16, gathered A, GLU): out is [da | db] bf16 rows
+    // of 2N at row p + out_row_pad * e; bwd_dh [R, N] the ungated gradient of h; bwd_dw [R] the
+    // route-weight gradient (accumulated atomically, zeroed by the caller); gates = router weights
+    bool glu_bwd;
+    const void *bwd_dh;
+    float *bwd_dw;
+    int32_t out_row_pad;
     const float *bias;      // router mode only
     int32_t *top_e;
     float *top_w;
@@ -111,10 +118,6 @@ void launch_gather_rows(const void *x, const int32_t *sorted_rows, int32_t k, in
                         void *xs, cudaStream_t s);
 void launch_rowdot(const void *dY, bool dy_bf16, const void *v, const int32_t *sorted_rows,
                    int32_t k, int64_t R, int64_t Dout, bool by_token, float *dg, cudaStream_t s);
-// [da | db] rows are written in the padded layout (slot p at row p + 64 e(p)).
-void launch_swiglu_bwd(const void *dhp, const void *h, const void *a, const void *b,
-                       const int32_t *sorted_rows, const float *top_w, const int32_t *offsets,
-                       int32_t E, int64_t R, int64_t F, void *dpre, float *dw, cudaStream_t s);
 void launch_router_bwd(const int32_t *top_e, const float *top_w, const float *dw,
                        const void *w_gate, int64_t S, int64_t D, int32_t E, int32_t k, void *dl,
                        float *dx, int32_t *offsets1, cudaStream_t s);
