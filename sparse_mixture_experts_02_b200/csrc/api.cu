@@ -149,9 +149,20 @@ BwdLayout bwd_layout(int64_t S, int64_t Din, int64_t Dout, int32_t E, int32_t k)
     return L;
 }
 
+// The W_gate gradient reduces over all S tokens in one "expert": split into P chunks of
+// consecutive tokens (at least 256 each) so that about 296 tiles (two per SM) run, then summed.
+int32_t router_chunks(int64_t S, int64_t D) {
+    const int64_t m_tiles = (D + 127) / 128;
+    int64_t P = (296 + m_tiles - 1) / m_tiles;
+    const int64_t by_rows = (S + 255) / 256;
+    if (P > by_rows) P = by_rows;
+    if (P > 256) P = 256;  // the weight-gradient kernel holds at most 256 "experts"
+    return (int32_t)(P < 1 ? 1 : P);
+}
+
 // MLP backward scratch (the forward's workspace supplies routing, map and h).
 struct MlpBwdLayout {
-    size_t status, dyb, dhp, dpre, dw, dv, dl, xs, off1, total;
+    size_t status, dyb, dhp, dpre, dw, dv, dl, xs, off1, partial, wgt, total;
 };
 
 MlpBwdLayout mlp_bwd_layout(int64_t S, int64_t D, int64_t F, int32_t E, int32_t k) {
@@ -166,9 +177,12 @@ MlpBwdLayout mlp_bwd_layout(int64_t S, int64_t D, int64_t F, int32_t E, int32_t 
     L.dpre = o; o = align_up(o + 4 * (size_t)Rp * (size_t)F);
     L.dw = o; o = align_up(o + 4 * (size_t)R);
     L.dv = o; o = align_up(o + 2 * (size_t)Rp * (size_t)D);
-    L.dl = o; o = align_up(o + 2 * (size_t)(S + kWgradPad) * (size_t)E);
+    const int32_t P = router_chunks(S, D);
+    L.dl = o; o = align_up(o + 2 * (size_t)(S + (int64_t)kWgradPad * P) * (size_t)E);
     L.xs = o; o = align_up(o + 2 * (size_t)R * (size_t)D);
-    L.off1 = o; o = align_up(o + 2 * sizeof(int32_t));
+    L.off1 = o; o = align_up(o + sizeof(int32_t) * (size_t)(P + 1));
+    L.partial = o; o = align_up(o + sizeof(float) * (size_t)P * (size_t)D * (size_t)E);
+    L.wgt = o; o = align_up(o + 2 * (size_t)E * (size_t)D);
     L.total = o;
     return L;
 }
@@ -793,24 +807,30 @@ extern "C" int moe_mlp_backward(const void *x, const void *w_gate, const void *w
     }
     record_prof(5, s);
     // router: dl (softmax over the selection), dx += dl W_gate^T, dW_gate = x^T dl
-    launch_router_bwd(top_e, top_w, dwr, w_gate, S, D, E, k, dl, dx, off1, s);
-    launch_zero_pad_rows(dl, E, E, off1, 1, s);
-    n += 2;
+    // the W_gate gradient in P token chunks (partial gradients), then summed
+    const int32_t P = router_chunks(S, D);
+    const int32_t chunk = (int32_t)((S + P - 1) / P);
+    float *partial = at<float>(ws, L.partial);
+    launch_router_bwd(top_e, top_w, dwr, w_gate, at<void>(ws, L.wgt), S, D, E, k, dl, dx, off1,
+                      chunk, P, s);
+    launch_zero_pad_rows(dl, E, E, off1, P, s);
+    n += 3;
     {
         WgradArgs w{};
         w.A = x;
         w.a_rows = S;
         w.dv = dl;
-        w.dv_rows = S + kWgradPad;
+        w.dv_rows = S + (int64_t)kWgradPad * P;
         w.offsets = off1;
         w.Din = D;
         w.Dout = E;
-        w.E = 1;
-        w.dW = dw_gate;
+        w.E = P;
+        w.dW = partial;
         w.status = status;
         w.wait_limit_ns = kWaitLimitNs;
         if ((rc = launch_grouped_wgrad(w, s))) return rc;
-        ++n;
+        launch_sum_partials(partial, D * E, P, dw_gate, s);
+        n += 2;
     }
     record_prof(6, s);
     g_launches = n;

@@ -120,18 +120,21 @@ rowdot_kernel(const void *__restrict__ dY, bool dy_bf16, const __nv_bfloat16 *__
 // Router backward of one token s: the softmax over its k selected logits gives
 //   dl_j = w_j (dw_j - sum_j' w_j' dw_j');
 // dl is written as a dense bf16 row [E] (zero outside the selection, the weight gradient's
-// operand) and dx[s] += sum_j dl_j W_gate[:, e_j] (after the expert part of dx is complete).
-// Block 0 also writes the one-"expert" offsets {0, S} of the W_gate gradient.
+// operand) and dx[s] += sum_j dl_j W_gate[:, e_j] (after the expert part of dx is complete),
+// read from W_gate^T [E, D] so that the lanes' loads are consecutive.
+// The W_gate gradient splits the tokens into P chunks of `chunk` consecutive tokens (partial
+// gradients, summed afterwards): dl rows go to the padded layout of those chunks (token s at
+// row s + 64 (s / chunk)), and block 0 writes the chunk offsets min(j chunk, S), j = 0..P.
 __global__ void __launch_bounds__(kWarps * 32)
 router_bwd_kernel(const int32_t *__restrict__ top_e, const float *__restrict__ top_w,
-                  const float *__restrict__ dw, const __nv_bfloat16 *__restrict__ w_gate,
+                  const float *__restrict__ dw, const __nv_bfloat16 *__restrict__ w_gate_t,
                   int64_t S, int64_t D, int32_t E, int32_t k, __nv_bfloat16 *__restrict__ dl,
-                  float *__restrict__ dx, int32_t *__restrict__ offsets1) {
+                  float *__restrict__ dx, int32_t *__restrict__ chunk_offsets, int32_t chunk,
+                  int32_t P) {
     const int lane = threadIdx.x & 31;
-    if (blockIdx.x == 0 && threadIdx.x == 0) {
-        offsets1[0] = 0;
-        offsets1[1] = (int32_t)S;
-    }
+    if (blockIdx.x == 0)
+        for (int j = threadIdx.x; j <= P; j += blockDim.x)
+            chunk_offsets[j] = (int32_t)((int64_t)j * chunk < S ? (int64_t)j * chunk : S);
     const int64_t wstride = (int64_t)gridDim.x * kWarps;
     for (int64_t s = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5); s < S; s += wstride) {
         float mean = 0.f;
@@ -142,16 +145,17 @@ router_bwd_kernel(const int32_t *__restrict__ top_e, const float *__restrict__ t
             dlj[j] = top_w[s * k + j] * (dw[s * k + j] - mean);
             ej[j] = top_e[s * k + j];
         }
+        const int64_t drow = s + (int64_t)kWgradPad * (s / chunk);
         for (int e = lane; e < E; e += 32) {
             float v = 0.f;
             for (int j = 0; j < k; ++j)
                 if (ej[j] == e) v = dlj[j];
-            dl[s * E + e] = __float2bfloat16_rn(v);
+            dl[drow * E + e] = __float2bfloat16_rn(v);
         }
         for (int64_t d = lane; d < D; d += 32) {
             float acc = 0.f;
             for (int j = 0; j < k; ++j)
-                acc = fmaf(dlj[j], __bfloat162float(w_gate[d * E + ej[j]]), acc);
+                acc = fmaf(dlj[j], __bfloat162float(w_gate_t[(int64_t)ej[j] * D + d]), acc);
             dx[s * D + d] += acc;
         }
     }
@@ -179,6 +183,33 @@ gather_rows_kernel(const uint4 *__restrict__ x, const int32_t *__restrict__ sort
     for (int64_t p = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5); p < R; p += wstride) {
         const int64_t s = __ldg(sorted_rows + p) / k;
         for (int64_t c = lane; c < d16; c += 32) xs[p * d16 + c] = __ldg(x + s * d16 + c);
+    }
+}
+
+// dst [cols, rows] = src [rows, cols]^T (bf16), through 32 x 33 shared tiles.
+__global__ void transpose_bf16_kernel(const __nv_bfloat16 *__restrict__ src, int64_t rows,
+                                      int64_t cols, __nv_bfloat16 *__restrict__ dst) {
+    __shared__ __nv_bfloat16 tile[32][33];
+    const int64_t r0 = (int64_t)blockIdx.y * 32, c0 = (int64_t)blockIdx.x * 32;
+    for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+        const int64_t r = r0 + i, c = c0 + threadIdx.x;
+        if (r < rows && c < cols) tile[i][threadIdx.x] = src[r * cols + c];
+    }
+    __syncthreads();
+    for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+        const int64_t c = c0 + i, r = r0 + threadIdx.x;
+        if (c < cols && r < rows) dst[c * rows + r] = tile[threadIdx.x][i];
+    }
+}
+
+// out[i] = sum over j < P of partial[j][i], i < n (the chunks' partial W_gate gradients).
+__global__ void sum_partials_kernel(const float *__restrict__ partial, int64_t n, int32_t P,
+                                    float *__restrict__ out) {
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
+        float acc = 0.f;
+        for (int j = 0; j < P; ++j) acc += partial[(int64_t)j * n + i];
+        out[i] = acc;
     }
 }
 
@@ -230,11 +261,24 @@ void launch_rowdot(const void *dY, bool dy_bf16, const void *v, const int32_t *s
 }
 
 void launch_router_bwd(const int32_t *top_e, const float *top_w, const float *dw,
-                       const void *w_gate, int64_t S, int64_t D, int32_t E, int32_t k, void *dl,
-                       float *dx, int32_t *offsets1, cudaStream_t s) {
+                       const void *w_gate, void *w_gate_t, int64_t S, int64_t D, int32_t E,
+                       int32_t k, void *dl, float *dx, int32_t *chunk_offsets, int32_t chunk,
+                       int32_t P, cudaStream_t s) {
+    const dim3 grid((unsigned)((E + 31) / 32), (unsigned)((D + 31) / 32));
+    transpose_bf16_kernel<<<grid, dim3(32, 8), 0, s>>>(static_cast<const __nv_bfloat16 *>(w_gate),
+                                                       D, E,
+                                                       static_cast<__nv_bfloat16 *>(w_gate_t));
     router_bwd_kernel<<<warp_grid(S), kWarps * 32, 0, s>>>(
-        top_e, top_w, dw, static_cast<const __nv_bfloat16 *>(w_gate), S, D, E, k,
-        static_cast<__nv_bfloat16 *>(dl), dx, offsets1);
+        top_e, top_w, dw, static_cast<const __nv_bfloat16 *>(w_gate_t), S, D, E, k,
+        static_cast<__nv_bfloat16 *>(dl), dx, chunk_offsets, chunk, P);
+}
+
+void launch_sum_partials(const float *partial, int64_t n, int32_t P, float *out, cudaStream_t s) {
+    int64_t blocks = (n + 255) / 256;
+    const int64_t cap = (int64_t)num_sms() * 8;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    sum_partials_kernel<<<(unsigned)blocks, 256, 0, s>>>(partial, n, P, out);
 }
 
 }  // namespace moe

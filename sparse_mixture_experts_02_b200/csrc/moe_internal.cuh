@@ -118,9 +118,12 @@ void launch_gather_rows(const void *x, const int32_t *sorted_rows, int32_t k, in
                         void *xs, cudaStream_t s);
 void launch_rowdot(const void *dY, bool dy_bf16, const void *v, const int32_t *sorted_rows,
                    int32_t k, int64_t R, int64_t Dout, bool by_token, float *dg, cudaStream_t s);
+// (two launches: W_gate^T into w_gate_t [E, D], then the per-token router backward)
 void launch_router_bwd(const int32_t *top_e, const float *top_w, const float *dw,
-                       const void *w_gate, int64_t S, int64_t D, int32_t E, int32_t k, void *dl,
-                       float *dx, int32_t *offsets1, cudaStream_t s);
+                       const void *w_gate, void *w_gate_t, int64_t S, int64_t D, int32_t E,
+                       int32_t k, void *dl, float *dx, int32_t *chunk_offsets, int32_t chunk,
+                       int32_t P, cudaStream_t s);
+void launch_sum_partials(const float *partial, int64_t n, int32_t P, float *out, cudaStream_t s);
 // Router on the tensor cores (bf16, E % 8 == 0): logits of 128-token tiles in TMEM, top-k and
 // softmax in the epilogue.
 int launch_route_tc(const void *x, const void *w_gate, const float *bias, int64_t S, int64_t D,
