@@ -162,7 +162,7 @@ router_bwd_kernel(const int32_t *__restrict__ top_e, const float *__restrict__ t
 }
 
 // Padding rows of expert e (blockIdx.x) in the padded layout: rows offsets[e] + 64 e + n_e up to
-// offsets[e] + 64 e + roundup(n_e, 64) are zeroed.
+// offsets[e] + 64 e + roundup(n_e, 64) are zeroed, by gridDim.y blocks per expert.
 __global__ void zero_pad_rows_kernel(uint4 *__restrict__ rows, int64_t ld16, int64_t cols16,
                                      const int32_t *__restrict__ offsets) {
     const int e = blockIdx.x;
@@ -170,7 +170,8 @@ __global__ void zero_pad_rows_kernel(uint4 *__restrict__ rows, int64_t ld16, int
     const int64_t first = __ldg(offsets + e) + (int64_t)kWgradPad * e + n;
     const int64_t count = (n + kWgradPad - 1) / kWgradPad * kWgradPad - n;
     const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-    for (int64_t q = threadIdx.x; q < count * cols16; q += blockDim.x)
+    for (int64_t q = (int64_t)blockIdx.y * blockDim.x + threadIdx.x; q < count * cols16;
+         q += (int64_t)gridDim.y * blockDim.x)
         rows[(first + q / cols16) * ld16 + q % cols16] = z;
 }
 
@@ -242,8 +243,13 @@ void launch_gate_rows(const void *dY, bool dy_bf16, const int32_t *sorted_rows, 
 
 void launch_zero_pad_rows(void *rows, int64_t ld, int64_t cols, const int32_t *offsets, int32_t E,
                           cudaStream_t s) {
-    zero_pad_rows_kernel<<<(unsigned)E, 256, 0, s>>>(static_cast<uint4 *>(rows), ld / 8, cols / 8,
-                                                     offsets);
+    // up to 63 rows per expert: spread each expert's rows over several blocks
+    const int64_t per_expert = 63 * (cols / 8);
+    int64_t ys = (per_expert + 4095) / 4096;
+    if (ys > 32) ys = 32;
+    const dim3 grid((unsigned)E, (unsigned)(ys < 1 ? 1 : ys));
+    zero_pad_rows_kernel<<<grid, 256, 0, s>>>(static_cast<uint4 *>(rows), ld / 8, cols / 8,
+                                              offsets);
 }
 
 void launch_gather_rows(const void *x, const int32_t *sorted_rows, int32_t k, int64_t R, int64_t D,
