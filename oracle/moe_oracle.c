@@ -451,3 +451,96 @@ void oracle_mlp_backward(const float *x, const float *w_gate, const float *bias,
     }
     free(l); free(a); free(b); free(h); free(dh); free(da); free(db); free(dv);
 }
+
+/* Mixture of Attention through ParallelLinear (ScatterMoE guide, "2. Generalization to Mixture of
+ * Attention (MoA)"; the ScatterMoE abstract's MoA demonstration): the router and top-k softmax
+ * of the expert MLP select k of E attention experts per token; expert e owns a query projection
+ * W_q[e] [D, H*dh] and an output projection W_o[e] [H*dh, D]; keys and values are shared,
+ * K = x W_k, V = x W_v ([S, H*dh]). For token s and selected expert e = J_j, per head h:
+ *   q = x_s W_q[e];  o_h = sum_{t <= s} softmax_t(q_h . K[t,h] / sqrt(dh)) V[t,h]  (causal)
+ *   y_s += w_j * (o W_o[e]).
+ * fp64; routing given ([S, k]) or the oracle's own. Outputs out [S, D] and, nullable, the
+ * routing top_experts_out [S, k] / top_weights_out [S, k]. */
+void oracle_moa_forward(const float *x, const float *w_gate, const float *bias, const float *w_q,
+                        const float *w_k, const float *w_v, const float *w_o, int64_t S, int64_t D,
+                        int32_t H, int32_t dh, int32_t E, int32_t k,
+                        const int32_t *given_top_experts, double *out, int32_t *top_experts_out,
+                        double *top_weights_out) {
+    const int64_t HD = (int64_t)H * dh;
+    double *K = (double *)calloc((size_t)S * (size_t)HD, sizeof(double));
+    double *V = (double *)calloc((size_t)S * (size_t)HD, sizeof(double));
+    #pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < S; ++t) {
+        for (int64_t d = 0; d < D; ++d) {
+            const double xv = (double)x[t * D + d];
+            for (int64_t c = 0; c < HD; ++c) {
+                K[t * HD + c] += xv * (double)w_k[d * HD + c];
+                V[t * HD + c] += xv * (double)w_v[d * HD + c];
+            }
+        }
+    }
+    const double scale = 1.0 / sqrt((double)dh);
+    #pragma omp parallel
+    {
+        double *l = (double *)malloc(sizeof(double) * (size_t)E);
+        double *q = (double *)malloc(sizeof(double) * (size_t)HD);
+        double *o = (double *)malloc(sizeof(double) * (size_t)HD);
+        double *sc = (double *)malloc(sizeof(double) * (size_t)(S > 0 ? S : 1));
+        int32_t J[64];
+        double w[64];
+        #pragma omp for schedule(dynamic, 1)
+        for (int64_t s = 0; s < S; ++s) {
+            const float *xs = x + s * D;
+            logits_one(xs, w_gate, bias, D, E, l, NULL);
+            if (given_top_experts) {
+                for (int32_t j = 0; j < k; ++j) J[j] = given_top_experts[s * k + j];
+                oracle_weights_for(l, J, 1, E, k, w);
+            } else {
+                topk_one(l, E, k, J, w);
+            }
+            double *y = out + s * D;
+            for (int64_t d = 0; d < D; ++d) y[d] = 0.0;
+            for (int32_t j = 0; j < k; ++j) {
+                const int64_t e = J[j];
+                const float *wq = w_q + e * D * HD, *wo = w_o + e * HD * D;
+                for (int64_t c = 0; c < HD; ++c) q[c] = 0.0;
+                for (int64_t d = 0; d < D; ++d) {
+                    const double xv = (double)xs[d];
+                    for (int64_t c = 0; c < HD; ++c) q[c] += xv * (double)wq[d * HD + c];
+                }
+                for (int32_t h = 0; h < H; ++h) {
+                    const double *qh = q + (int64_t)h * dh;
+                    double mx = -INFINITY;
+                    for (int64_t t = 0; t <= s; ++t) {
+                        double acc = 0.0;
+                        for (int32_t c = 0; c < dh; ++c) acc += qh[c] * K[t * HD + (int64_t)h * dh + c];
+                        sc[t] = acc * scale;
+                        if (sc[t] > mx) mx = sc[t];
+                    }
+                    double den = 0.0;
+                    for (int64_t t = 0; t <= s; ++t) {
+                        sc[t] = exp(sc[t] - mx);
+                        den += sc[t];
+                    }
+                    double *oh = o + (int64_t)h * dh;
+                    for (int32_t c = 0; c < dh; ++c) oh[c] = 0.0;
+                    for (int64_t t = 0; t <= s; ++t) {
+                        const double pt = sc[t] / den;
+                        for (int32_t c = 0; c < dh; ++c) oh[c] += pt * V[t * HD + (int64_t)h * dh + c];
+                    }
+                }
+                for (int64_t c = 0; c < HD; ++c) {
+                    const double cw = w[j] * o[c];
+                    for (int64_t d = 0; d < D; ++d) y[d] += cw * (double)wo[c * D + d];
+                }
+            }
+            if (top_experts_out)
+                for (int32_t j = 0; j < k; ++j) top_experts_out[s * k + j] = J[j];
+            if (top_weights_out)
+                for (int32_t j = 0; j < k; ++j) top_weights_out[s * k + j] = w[j];
+        }
+        free(l); free(q); free(o); free(sc);
+    }
+    free(K);
+    free(V);
+}
