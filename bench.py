@@ -466,6 +466,76 @@ def backward_bench(args, w):
             "gpu_launches": launches * args.steps, "clocks": clk.summary()}
 
 
+def moa_flops(w: W.MoaWorkload) -> dict:
+    """Algorithmic FLOPs of one Mixture-of-Attention forward: router, shared key/value projection,
+    routed query projection, causal attention (route at token s: 4*dh*(s+1) per head, summed over
+    the k routes of every token) and routed output projection."""
+    return {
+        "router": 2.0 * w.S * w.D * w.E,
+        "kv_projection": 2.0 * w.S * w.D * 2 * w.HD,
+        "q_projection": 2.0 * w.R * w.D * w.HD,
+        "attention": 2.0 * w.HD * w.k * w.S * (w.S + 1),
+        "o_projection": 2.0 * w.R * w.HD * w.D,
+    }
+
+
+def moa_bench(args, w):
+    """Time moe_moa_forward on workload w (bf16): W warm-up and K timed steps, CUDA events on the
+    launch stream, per-stage events from the library."""
+    import sparse_mixture_experts_02_b200 as moe
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    inp = W.make_moa_inputs(w, device=dev, seed=0)
+    ws = moe.MoaWorkspace(w.S, w.D, w.HD, w.E, w.k, dev)
+    out = torch.empty((w.S, w.D), dtype=torch.float32, device=dev)
+
+    def step(evs=None):
+        if evs is not None:
+            moe.profile_events(evs)
+        return moe.moa_forward(inp["x"], inp["w_gate"], inp["w_q"], inp["w_kv"], inp["w_o"], w.k,
+                               w.H, logit_bias=inp["logit_bias"], out=out, ws=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    moe.check_device_status(ws)
+    launches = moe.last_launch_count()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+    for row in evs:
+        for e in row:
+            e.record()
+    torch.cuda.synchronize(dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        t0.record()
+        for i in range(args.steps):
+            step(evs[i])
+        t1.record()
+        torch.cuda.synchronize(dev)
+    ms = t0.elapsed_time(t1) / args.steps
+    names = ["route", "sparse_map", "kv_projection", "q_projection", "attention", "o_projection"]
+    stage = {n: sum(r[q].elapsed_time(r[q + 1]) for r in evs) / args.steps
+             for q, n in enumerate(names)}
+    fl = moa_flops(w)
+    flop = sum(fl.values())
+    pk, pk_kind = peaks()
+    tflops = flop / (ms * 1e-3) / 1e12
+    att = fl["attention"] / (stage["attention"] * 1e-3) / 1e12
+    return {"metric": "MoA-layer fwd tokens/s and TFLOP/s (bf16)", "value": w.S / (ms * 1e-3),
+            "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "S": w.S, "D": w.D, "H": w.H, "dh": w.dh, "E": w.E,
+                       "k": w.k, "l2": "inputs larger than L2 (expert weights streamed)"},
+            "tflops": tflops, "flop_per_step": flop, "flop_by_stage": fl,
+            "tflops_frac": {"of_measured_sustained": tflops / pk["bf16_tflops_sustained"],
+                            "of_nominal": tflops / 2250.0, "peaks": pk_kind},
+            "roofline": {"kernel": "attention core", "bound": "tensor", "achieved": att,
+                         "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": att / pk["bf16_tflops"], "traffic": None},
+            "stage_ms": stage, "gpu_launches": launches * args.steps, "clocks": clk.summary()}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -481,6 +551,8 @@ def main():
                     help="instead of the forward: sparse-map GB/s over R = 2^20..2^26 routes")
     ap.add_argument("--backward", action="store_true",
                     help="instead of the forward: time moe_mlp_backward on --workload")
+    ap.add_argument("--moa", action="store_true",
+                    help="instead of the MLP forward: time moe_moa_forward (Mixture of Attention)")
     ap.add_argument("--map-points", default="",
                     help="with --map-sweep: only these points, 'log2R:E,...' (e.g. 26:256)")
     args = ap.parse_args()
@@ -488,6 +560,9 @@ def main():
         ap.error("--warmup must be >= 3")
     if args.map_sweep:
         print(json.dumps(map_sweep(args)), flush=True)
+        return
+    if args.moa:
+        print(json.dumps(moa_bench(args, W.MOA_WORKLOADS["moa_prefill"])), flush=True)
         return
     if args.backward:
         wl = {**W.WORKLOADS, **W.PROFILE_WORKLOADS}[args.workload]

@@ -206,8 +206,34 @@ int moe_mlp_backward(const void *x, const void *w_gate, const void *w_gate_e, co
                      void *ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * Mixture of Attention forward (ScatterMoE guide, "2. Generalization to Mixture of Attention
+ * (MoA)"; the ScatterMoE abstract's MoA demonstration), bf16. The router of moe_route_topk picks
+ * k of E attention experts per token; expert e owns a query projection W_q[e] and an output
+ * projection W_o[e]; keys and values are shared by all experts. For token s, selected expert
+ * e_j with router weight w_j, and head h (H heads of dh columns, HD = H * dh):
+ *   q = x[s] W_q[e_j];  K = x W_kv[:, :HD];  V = x W_kv[:, HD:]
+ *   o_h = sum_{t <= s} softmax_t(q_h . K[t, h] / sqrt(dh)) V[t, h]   (causal, one sequence)
+ *   out[s] = sum_j w_j * (o W_o[e_j])
+ * Steps on `stream`: route, sparse map, the shared key/value projection (one group of all S
+ * tokens, [S, D] x [D, 2 HD]; its epilogue warps zero `out`), the routed query projection
+ * (ParallelLinear with gathered x rows, q in slot order), the attention core over the slot-ordered
+ * query rows (tensor cores, running-max softmax, each row masked at its own token position), and
+ * the routed output projection (ParallelLinear from slot order, router weight, scatter-add into
+ * tokens). No host synchronisation.
+ *   x [S, D], w_gate [D, E], w_q [E, D, HD], w_kv [D, 2 HD], w_o [E, HD, D]: bf16;
+ *   logit_bias [E] float32 nullable; out [S, D] float32 (overwritten). dh is 64 or 128.
+ *   ws: moe_workspace_size("moa_forward", S, D, HD, E, k, MOE_BF16) bytes; the routing views of
+ *   moe_workspace_view (top_experts ... sorted_rows, any F) apply to it.
+ * MOE_ERR_UNSUPPORTED for another dtype or head size.
+ */
+int moe_moa_forward(const void *x, const void *w_gate, const float *logit_bias, const void *w_q,
+                    const void *w_kv, const void *w_o, int64_t S, int64_t D, int32_t H, int32_t dh,
+                    int32_t E, int32_t k, moe_dtype dt, float *out, void *ws, size_t ws_bytes,
+                    moe_stream_t stream);
+
+/*
  * Workspace bytes for op = "sparse_map", "scatter_linear", "scatter_linear_backward" (D = Din,
- * F = Dout), "mlp_forward" or "mlp_backward" (unused sizes may be 0). Returns 0 for an unknown op or sizes
+ * F = Dout), "mlp_forward", "mlp_backward" or "moa_forward" (F = H * dh) (unused sizes may be 0). Returns 0 for an unknown op or sizes
  * outside the limits.
  */
 size_t moe_workspace_size(const char *op, int64_t S, int64_t D, int64_t F, int32_t E, int32_t k,
@@ -232,9 +258,15 @@ const char *moe_last_error(void);
 int moe_check_device_status(void *ws, moe_stream_t stream);
 
 /*
- * Optional per-stage timing of moe_mlp_forward on the calling host thread: when `events` holds
- * n >= 5 cudaEvent_t handles, the next moe_mlp_forward records them on its stream at: start,
- * after route, after the sparse map, after GEMM1, after GEMM2; then the registration clears.
+ * Optional per-stage timing on the calling host thread: when `events` holds n cudaEvent_t
+ * handles (n <= 8), the next moe_mlp_forward, moe_mlp_backward or moe_moa_forward records the
+ * first n of its stage events on its stream; then the registration clears.
+ *   moe_mlp_forward (5): start, after route, after the sparse map, after GEMM1, after GEMM2.
+ *   moe_mlp_backward (7): start, after dh, after the recomputed GEMM1 with the SwiGLU backward,
+ *     after dW_down, after dx, after dW_gate_e and dW_up, after the router backward.
+ *   moe_moa_forward (7): start, after route, after the sparse map, after the key/value
+ *     projection, after the query projection, after the attention core, after the output
+ *     projection.
  * Pass n = 0 to clear. Returns MOE_OK or MOE_ERR_INVALID_ARG.
  */
 int moe_profile_events(void *const *events, int n);

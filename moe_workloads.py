@@ -117,6 +117,65 @@ def make_inputs(w: Workload, device="cpu", seed: int = 0) -> dict:
     return dict(x=x, w_gate=w_gate, w_gate_e=w_gate_e, w_up=w_up, w_down=w_down, logit_bias=bias)
 
 
+@dataclasses.dataclass(frozen=True)
+class MoaWorkload:
+    """A Mixture-of-Attention layer: E attention experts with H heads of dh columns each (own
+    query and output projections), keys and values shared, one causal sequence of S tokens."""
+    name: str
+    S: int
+    D: int
+    H: int
+    dh: int
+    E: int
+    k: int
+    router_std: str = "0.02"
+    zipf_s: float = 0.0
+    weight_std: float = 0.02
+
+    @property
+    def R(self) -> int:
+        return self.S * self.k
+
+    @property
+    def HD(self) -> int:
+        return self.H * self.dh
+
+    def describe(self) -> dict:
+        return dataclasses.asdict(self)
+
+
+# The MoA layer at the Mixtral-8x7B prefill shape: 8 attention experts of 8 heads x 128 (each
+# token's k = 2 experts give 16 query heads, half of a 32-head dense layer), one 4096-token sequence.
+MOA_WORKLOADS = {
+    "moa_prefill": MoaWorkload("moa_prefill", S=4096, D=4096, H=8, dh=128, E=8, k=2),
+}
+
+
+def make_moa_inputs(w: MoaWorkload, device="cpu", seed: int = 0) -> dict:
+    """bf16 x [S,D] ~ N(0,1), w_gate [D,E], w_q [E,D,HD], w_kv [D,2HD] (key columns first),
+    w_o [E,HD,D] ~ N(0, weight_std^2); router std as for the MLP workloads; logit_bias [E] float32
+    (Zipf popularity, as for the MLP workloads) or None. Draw order x, w_gate, w_q, w_kv, w_o,
+    then the popularity permutation."""
+    device = torch.device(device)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    dt = torch.bfloat16
+    rstd = 0.02 if w.router_std == "0.02" else 1.0 / math.sqrt(w.D)
+    x = _draw(gen, (w.S, w.D), 1.0, dt, device)
+    w_gate = _draw(gen, (w.D, w.E), rstd, dt, device)
+    w_q = _draw(gen, (w.E, w.D, w.HD), w.weight_std, dt, device)
+    w_kv = _draw(gen, (w.D, 2 * w.HD), w.weight_std, dt, device)
+    w_o = _draw(gen, (w.E, w.HD, w.D), w.weight_std, dt, device)
+    bias: Optional[torch.Tensor] = None
+    if w.zipf_s > 0:
+        perm = torch.randperm(w.E, generator=gen, device=device)
+        ranks = torch.arange(w.E, dtype=torch.float64)
+        vals = (-w.zipf_s * torch.log(ranks + 1.0)).to(torch.float32).to(device)
+        bias = torch.empty(w.E, dtype=torch.float32, device=device)
+        bias[perm] = vals
+    return dict(x=x, w_gate=w_gate, w_q=w_q, w_kv=w_kv, w_o=w_o, logit_bias=bias)
+
+
 def make_top_experts(S: int, k: int, E: int, seed: int = 0, mode: str = "uniform",
                      device="cpu") -> torch.Tensor:
     """Seeded routing tables [S,k] int32 for the sparse-map tests, without any router.

@@ -25,7 +25,7 @@ STATUS_NAMES = {0: "MOE_OK", -1: "MOE_ERR_INVALID_ARG", -2: "MOE_ERR_UNSUPPORTED
 
 EXPORTS = ["moe_route_topk", "moe_sparse_map", "moe_sparse_map_noalloc", "moe_scatter_linear",
            "moe_scatter_linear_backward", "moe_mlp_forward", "moe_mlp_backward",
-           "moe_workspace_size", "moe_workspace_view", "moe_last_error",
+           "moe_moa_forward", "moe_workspace_size", "moe_workspace_view", "moe_last_error",
            "moe_check_device_status", "moe_profile_events", "moe_debug_wait_timeout",
            "moe_last_launch_count"]
 
@@ -52,6 +52,8 @@ def _load():
                                                 c_int, c_int, P, P, P, P, ctypes.c_size_t, P]
     lib.moe_mlp_forward.argtypes = [P, P, P, P, P, P, i64, i64, i64, i32, i32, c_int, P, P,
                                     ctypes.c_size_t, P]
+    lib.moe_moa_forward.argtypes = [P, P, P, P, P, P, i64, i64, i32, i32, i32, i32, c_int, P, P,
+                                    ctypes.c_size_t, P]
     lib.moe_mlp_backward.argtypes = [P, P, P, P, P, P, i64, i64, i64, i32, i32, c_int, P,
                                      ctypes.c_size_t, P, P, P, P, P, P, ctypes.c_size_t, P]
     lib.moe_workspace_size.argtypes = [ctypes.c_char_p, i64, i64, i64, i32, i32, c_int]
@@ -64,7 +66,7 @@ def _load():
     lib.moe_debug_wait_timeout.argtypes = [i64, P, ctypes.c_size_t, P]
     for name in ("moe_route_topk", "moe_sparse_map", "moe_sparse_map_noalloc",
                  "moe_scatter_linear", "moe_scatter_linear_backward", "moe_mlp_forward",
-                 "moe_mlp_backward",
+                 "moe_mlp_backward", "moe_moa_forward",
                  "moe_check_device_status", "moe_profile_events", "moe_debug_wait_timeout",
                  "moe_last_launch_count"):
         getattr(lib, name).restype = c_int
@@ -326,6 +328,70 @@ def mlp_forward(x: torch.Tensor, w_gate: torch.Tensor, w_gate_e: torch.Tensor,
     return out
 
 
+class MoaWorkspace:
+    """A workspace for moa_forward plus views of the routing it leaves there."""
+
+    def __init__(self, S, D, HD, E, k, device):
+        self.shape = (S, D, HD, E, k)
+        code = _dtype_code(torch.empty(0, dtype=torch.bfloat16))
+        self.code = code
+        n = workspace_size("moa_forward", S, D, HD, E, k, code)
+        if n == 0:
+            raise ValueError("sizes outside the library's limits")
+        self.buf = alloc_workspace(n, device)
+
+    def view(self, which: str) -> torch.Tensor:
+        S, D, HD, E, k = self.shape
+        R = S * k
+        shapes = {
+            "top_experts": (R, torch.int32, (S, k)),
+            "top_weights": (R, torch.float32, (S, k)),
+            "expert_counts": (E, torch.int32, (E,)),
+            "expert_offsets": (E + 1, torch.int32, (E + 1,)),
+            "sparse_rows": (R, torch.int32, (R,)),
+            "sorted_rows": (R, torch.int32, (R,)),
+        }
+        if which not in shapes:
+            raise KeyError(which)
+        # the routing sits at the same offsets as in an mlp_forward workspace (F is irrelevant)
+        off = workspace_view(which, S, D, 0, E, k, self.code)
+        n, dt, shape = shapes[which]
+        nbytes = n * torch.empty(0, dtype=dt).element_size()
+        return self.buf[off:off + nbytes].view(dt).view(shape)
+
+
+def moa_forward(x: torch.Tensor, w_gate: torch.Tensor, w_q: torch.Tensor, w_kv: torch.Tensor,
+                w_o: torch.Tensor, k: int, heads: int, logit_bias: Optional[torch.Tensor] = None,
+                out: Optional[torch.Tensor] = None,
+                ws: Optional[MoaWorkspace] = None) -> torch.Tensor:
+    """Mixture of Attention forward (moe_moa_forward), bf16; returns out [S, D] float32.
+    w_gate [D,E], w_q [E,D,H*dh], w_kv [D,2*H*dh] (key columns first), w_o [E,H*dh,D]."""
+    _req(x, "x", dim=2)
+    dev = x.device
+    for t, n, d in ((w_gate, "w_gate", 2), (w_q, "w_q", 3), (w_kv, "w_kv", 2), (w_o, "w_o", 3)):
+        _req(t, n, dtype=x.dtype, dim=d, device=dev)
+    S, D = x.shape
+    E = w_gate.shape[1]
+    HD = w_q.shape[2]
+    if heads < 1 or HD % heads != 0:
+        raise ValueError("w_q's last dimension must be heads * dh")
+    if w_gate.shape[0] != D or tuple(w_q.shape) != (E, D, HD) or \
+            tuple(w_kv.shape) != (D, 2 * HD) or tuple(w_o.shape) != (E, HD, D):
+        raise ValueError("expected w_gate [D,E], w_q [E,D,HD], w_kv [D,2HD], w_o [E,HD,D]")
+    if logit_bias is not None:
+        _req(logit_bias, "logit_bias", dtype=torch.float32, dim=1, device=dev)
+    if out is None:
+        out = torch.empty((S, D), dtype=torch.float32, device=dev)
+    _req(out, "out", dtype=torch.float32, dim=2, device=dev)
+    if ws is None:
+        ws = MoaWorkspace(S, D, HD, E, k, dev)
+    _check(_lib().moe_moa_forward(_ptr(x), _ptr(w_gate), _ptr(logit_bias), _ptr(w_q),
+                               _ptr(w_kv), _ptr(w_o), S, D, heads, HD // heads, E, k,
+                               _dtype_code(x), _ptr(out), _ptr(ws.buf), ws.buf.numel(),
+                               _stream(dev)))
+    return out
+
+
 def mlp_backward(x: torch.Tensor, w_gate: torch.Tensor, w_gate_e: torch.Tensor,
                  w_up: torch.Tensor, w_down: torch.Tensor, k: int, dout: torch.Tensor,
                  fwd_ws: ForwardWorkspace, ws: Optional[torch.Tensor] = None) -> dict:
@@ -357,12 +423,13 @@ def mlp_backward(x: torch.Tensor, w_gate: torch.Tensor, w_gate_e: torch.Tensor,
 
 def check_device_status(ws: torch.Tensor):
     """Synchronises and raises MoeError if the device flagged a bad expert id or a timeout."""
-    buf = ws.buf if isinstance(ws, ForwardWorkspace) else ws
+    buf = ws.buf if isinstance(ws, (ForwardWorkspace, MoaWorkspace)) else ws
     _check(_lib().moe_check_device_status(_ptr(buf), _stream(buf.device)))
 
 
 def profile_events(events):
-    """Registers torch.cuda.Event objects (>= 5) for the next mlp_forward on this thread."""
+    """Registers torch.cuda.Event objects (>= 5) for the next mlp_forward, mlp_backward or
+    moa_forward on this thread."""
     if not events:
         _check(_lib().moe_profile_events(None, 0))
         return

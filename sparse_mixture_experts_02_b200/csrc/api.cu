@@ -129,6 +129,28 @@ MlpLayout mlp_layout(int64_t S, int64_t F, int32_t E, int32_t k, moe_dtype dt) {
     return L;
 }
 
+// Mixture of Attention forward: the routing prefix of the MLP layout (identical offsets, so the
+// routing views of an "mlp_forward" workspace apply), then the one-group offsets of the shared
+// key/value projection, kv [S, 2 HD], q and the attention output o ([R, HD] each, slot order),
+// all bf16.
+struct MoaLayout {
+    MlpLayout base;
+    size_t kv_off, kv, q, o, total;
+};
+
+MoaLayout moa_layout(int64_t S, int64_t HD, int32_t E, int32_t k) {
+    const int64_t R = S * k;
+    MoaLayout L;
+    L.base = mlp_layout(S, 0, E, k, MOE_BF16);
+    size_t o = L.base.total;
+    L.kv_off = o; o = align_up(o + 2 * sizeof(int32_t));
+    L.kv = o; o = align_up(o + 2 * (size_t)S * 2 * (size_t)HD);
+    L.q = o; o = align_up(o + 2 * (size_t)R * (size_t)HD);
+    L.o = o; o = align_up(o + 2 * (size_t)R * (size_t)HD);
+    L.total = o;
+    return L;
+}
+
 // ParallelLinear backward scratch: status, bf16 copy of an fp32 dY [S, Dout], gated rows dv in
 // the weight gradient's padded layout [R + 64 E, Dout] bf16, x rows in slot order [R, Din] (for
 // gathered inputs), ungated forward rows v [R, Dout] bf16 (gate gradient).
@@ -243,6 +265,10 @@ size_t moe_workspace_size(const char *op, int64_t S, int64_t D, int64_t F, int32
     if (strcmp(op, "mlp_backward") == 0) {
         if (F <= 0 || D <= 0) return 0;
         return mlp_bwd_layout(S, D, F, E, k).total;
+    }
+    if (strcmp(op, "moa_forward") == 0) {  // F = H * dh
+        if (F <= 0 || dt != MOE_BF16) return 0;
+        return moa_layout(S, F, E, k).total;
     }
     if (strcmp(op, "mlp_forward") == 0) {
         if (F <= 0 || (dt != MOE_F32 && dt != MOE_BF16)) return 0;
@@ -833,6 +859,136 @@ extern "C" int moe_mlp_backward(const void *x, const void *w_gate, const void *w
         n += 2;
     }
     record_prof(6, s);
+    g_prof_n = 0;
     g_launches = n;
     return check_launch("mlp_backward");
+}
+
+int moe_moa_forward(const void *x, const void *w_gate, const float *logit_bias, const void *w_q,
+                    const void *w_kv, const void *w_o, int64_t S, int64_t D, int32_t H, int32_t dh,
+                    int32_t E, int32_t k, moe_dtype dt, float *out, void *ws, size_t ws_bytes,
+                    moe_stream_t stream) {
+    g_launches = 0;
+    int rc;
+    if ((rc = check_dtype(dt)) || (rc = check_dims(S, E, k)) || (rc = check_feat("D", D)))
+        return rc;
+    if (dt != MOE_BF16) return set_error(MOE_ERR_UNSUPPORTED, "moa_forward: bf16 inputs only");
+    if (dh != 64 && dh != 128)
+        return set_error(MOE_ERR_UNSUPPORTED, "moa_forward: head size %d (64 or 128 are built)", dh);
+    if (H < 1 || (int64_t)H * dh * 2 >= (int64_t(1) << 31))
+        return set_error(MOE_ERR_INVALID_ARG, "moa_forward: H must be positive with 2*H*dh < 2^31");
+    const int64_t HD = (int64_t)H * dh;
+    if ((rc = check_ptr("x", x, 16, S == 0)) || (rc = check_ptr("w_gate", w_gate, 16)) ||
+        (rc = check_ptr("logit_bias", logit_bias, 4, true)) || (rc = check_ptr("w_q", w_q, 16)) ||
+        (rc = check_ptr("w_kv", w_kv, 16)) || (rc = check_ptr("w_o", w_o, 16)) ||
+        (rc = check_ptr("out", out, 16, S == 0)))
+        return rc;
+    const MoaLayout L = moa_layout(S, HD, E, k);
+    if ((rc = check_ws(ws, ws_bytes, L.total))) return rc;
+    if ((rc = check_device())) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int64_t R = S * k;
+    unsigned *status = at<unsigned>(ws, L.base.status);
+    int32_t *top_e = at<int32_t>(ws, L.base.top_e);
+    float *top_w = at<float>(ws, L.base.top_w);
+    int32_t *offsets = at<int32_t>(ws, L.base.offsets);
+    int32_t *sorted_rows = at<int32_t>(ws, L.base.sorted_rows);
+    int32_t *kv_off = at<int32_t>(ws, L.kv_off);
+    void *kv = at<void>(ws, L.kv), *q = at<void>(ws, L.q), *o = at<void>(ws, L.o);
+    int n = 0;
+
+    record_prof(0, s);
+    if (R == 0) {
+        n += launch_zero_f32(out, S * D, status, s);
+        if ((rc = check_launch("zero"))) return rc;
+    }
+    {
+        const int nr = launch_route(x, w_gate, logit_bias, S, D, E, k, true, top_e, top_w, status, s);
+        if (nr < 0) return MOE_ERR_CUDA;
+        n += nr;
+    }
+    if ((rc = check_launch("route"))) return rc;
+    record_prof(1, s);
+    launch_sparse_map(top_e, R, E, at<int32_t>(ws, L.base.counts), offsets,
+                      at<int32_t>(ws, L.base.sparse_rows), sorted_rows,
+                      at<int32_t>(ws, L.base.scratch), status, s, &n);
+    if ((rc = check_launch("sparse_map"))) return rc;
+    record_prof(2, s);
+    if (R > 0) {
+        // shared keys and values: one group of all S tokens, [S, D] . [D, 2 HD]; its epilogue
+        // warps also zero `out` for the final scatter-add
+        launch_kv_offsets(kv_off, S, s);
+        GemmArgs a{};
+        a.A = x;
+        a.a_rows = S;
+        a.B0 = w_kv;
+        a.offsets = kv_off;
+        a.sorted_rows = sorted_rows;
+        a.out = kv;
+        a.S = S;
+        a.R = S;
+        a.E = 1;
+        a.k = 1;
+        a.K = D;
+        a.N = 2 * HD;
+        a.bf16 = true;
+        a.zero_ptr = out;
+        a.zero_n = S * D;
+        a.status = status;
+        a.wait_limit_ns = kWaitLimitNs;
+        if ((rc = prefer_2sm(S, 1) ? launch_grouped_gemm_2sm(a, s) : launch_grouped_gemm(a, s)))
+            return rc;
+        if ((rc = check_launch("kv projection"))) return rc;
+        n += 2;
+        record_prof(3, s);
+        // routed query projection: gathered x rows, W_q[e], q in slot order
+        GemmArgs b{};
+        b.A = x;
+        b.a_rows = S;
+        b.B0 = w_q;
+        b.offsets = offsets;
+        b.sorted_rows = sorted_rows;
+        b.out = q;
+        b.S = S;
+        b.R = R;
+        b.E = E;
+        b.k = k;
+        b.K = D;
+        b.N = HD;
+        b.bf16 = true;
+        b.gather = true;
+        b.status = status;
+        b.wait_limit_ns = kWaitLimitNs;
+        if ((rc = prefer_2sm(R, E) ? launch_grouped_gemm_2sm(b, s) : launch_grouped_gemm(b, s)))
+            return rc;
+        if ((rc = check_launch("q projection"))) return rc;
+        ++n;
+        record_prof(4, s);
+        if ((rc = launch_moa_attention(q, kv, sorted_rows, offsets, o, R, S, H, dh, k, E, s)))
+            return rc;
+        if ((rc = check_launch("attention"))) return rc;
+        ++n;
+        record_prof(5, s);
+        // routed output projection: o rows in slot order, W_o[e], router weight, scatter-add
+        GemmArgs c = b;
+        c.A = o;
+        c.a_rows = R;
+        c.B0 = w_o;
+        c.gates = top_w;
+        c.out = out;
+        c.K = HD;
+        c.N = D;
+        c.gather = false;
+        c.scatter = true;
+        if ((rc = prefer_2sm(R, E) ? launch_grouped_gemm_2sm(c, s) : launch_grouped_gemm(c, s)))
+            return rc;
+        if ((rc = check_launch("o projection"))) return rc;
+        ++n;
+        record_prof(6, s);
+    } else {
+        for (int q = 3; q <= 6; ++q) record_prof(q, s);
+    }
+    g_prof_n = 0;
+    g_launches = n;
+    return MOE_OK;
 }

@@ -126,6 +126,15 @@ void launch_router_bwd(const int32_t *top_e, const float *top_w, const float *dw
 void launch_sum_partials(const float *partial, int64_t n, int32_t P, float *out, cudaStream_t s);
 // Router on the tensor cores (bf16, E % 8 == 0): logits of 128-token tiles in TMEM, top-k and
 // softmax in the epilogue.
+// Attention core of Mixture of Attention: o[p] = causal attention of query row q[p] (slot order,
+// [R, H*dh] bf16) over the shared keys/values kv [S, 2*H*dh] bf16 (K columns first), the query's
+// token position being sorted_rows[p] / k; slots at or past offsets[E] are skipped. dh is 64 or
+// 128.
+int launch_moa_attention(const void *q, const void *kv, const int32_t *sorted_rows,
+                         const int32_t *offsets, void *o, int64_t R, int64_t S, int32_t H,
+                         int32_t dh, int32_t k, int32_t E, cudaStream_t s);
+// Writes {0, S}: the offsets of one group holding every token.
+void launch_kv_offsets(int32_t *off, int64_t S, cudaStream_t s);
 int launch_route_tc(const void *x, const void *w_gate, const float *bias, int64_t S, int64_t D,
                     int32_t E, int32_t k, int32_t *top_e, float *top_w, unsigned *status,
                     cudaStream_t s);
