@@ -19,7 +19,7 @@ enum : unsigned {
     kStatusBadExpert = 1u << 0,
     kStatusTimeout = 1u << 1,
     // bits 8..15: id of the first kernel whose wait ran out
-    kKernelGemm = 1u, kKernelDebugWait = 2u,
+    kKernelGemm = 1u, kKernelDebugWait = 2u, kKernelAttention = 3u,
 };
 constexpr size_t kStatusBytes = 256;
 
@@ -126,13 +126,14 @@ void launch_router_bwd(const int32_t *top_e, const float *top_w, const float *dw
 void launch_sum_partials(const float *partial, int64_t n, int32_t P, float *out, cudaStream_t s);
 // Router on the tensor cores (bf16, E % 8 == 0): logits of 128-token tiles in TMEM, top-k and
 // softmax in the epilogue.
-// Attention core of Mixture of Attention: o[p] = causal attention of query row q[p] (slot order,
-// [R, H*dh] bf16) over the shared keys/values kv [S, 2*H*dh] bf16 (K columns first), the query's
-// token position being sorted_rows[p] / k; slots at or past offsets[E] are skipped. dh is 64 or
-// 128.
+// Attention core of Mixture of Attention: for every route i (token i / k) with slot
+// p = sparse_rows[i], o[p] = causal attention of query row q[p] ([R, H*dh] bf16, slot order)
+// over the shared keys/values kv [S, 2*H*dh] bf16 (K columns first) up to token i / k. dh is 64
+// or 128. Waits are bounded (status word, kernel id kKernelAttention).
 int launch_moa_attention(const void *q, const void *kv, const int32_t *sorted_rows,
-                         const int32_t *offsets, void *o, int64_t R, int64_t S, int32_t H,
-                         int32_t dh, int32_t k, int32_t E, cudaStream_t s);
+                         const int32_t *sparse_rows, const int32_t *offsets, void *o, int64_t R,
+                         int64_t S, int32_t H, int32_t dh, int32_t k, int32_t E, unsigned *status,
+                         cudaStream_t s);
 // Writes {0, S}: the offsets of one group holding every token.
 void launch_kv_offsets(int32_t *off, int64_t S, cudaStream_t s);
 int launch_route_tc(const void *x, const void *w_gate, const float *bias, int64_t S, int64_t D,
@@ -321,6 +322,23 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 }
 __device__ __forceinline__ void tmem_ld_wait() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+// 32 lanes x 32 consecutive 32-bit columns from registers: thread t of the warp writes lane
+// (base lane + t).
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+        "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+        "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 // ---- shared-memory matrix descriptors (tcgen05 format) -----------------------------------------
