@@ -533,7 +533,31 @@ def moa_bench(args, w):
             "roofline": {"kernel": "attention core", "bound": "tensor", "achieved": att,
                          "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
                          "frac": att / pk["bf16_tflops"], "traffic": None},
-            "stage_ms": stage, "gpu_launches": launches * args.steps, "clocks": clk.summary()}
+            "stage_ms": stage, "gpu_launches": launches * args.steps, "clocks": clk.summary(),
+            "cpu_baseline": None if args.no_cpu_baseline else moa_oracle_baseline(w, inp,
+                                                                                  args.cpu_budget_s)}
+
+
+def moa_oracle_baseline(w, inp, budget_s):
+    """The oracle's MoA forward on a causal prefix of the sequence (tokens 0..n-1 depend on
+    nothing later), n sized from a 16-token probe to take about budget_s seconds."""
+    import oracle
+    cpu = host_inputs(inp)
+    HD = w.HD
+
+    def run(n):
+        t0 = time.perf_counter()
+        oracle.moa_forward(cpu["x"][:n], cpu["w_gate"], cpu["w_q"], cpu["w_kv"][:, :HD],
+                           cpu["w_kv"][:, HD:], cpu["w_o"], w.k, w.H, bias=cpu["logit_bias"])
+        return time.perf_counter() - t0
+
+    n0 = min(w.S, 16)
+    t = run(n0)
+    n = max(n0, min(w.S, int(n0 * budget_s / max(t, 1e-6))))
+    t = run(n)
+    return {"value": n / t, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"the first {n} tokens of the sequence (a causal prefix: shorter attention "
+                      f"spans than the full sequence's average)"}
 
 
 def main():

@@ -964,8 +964,8 @@ int moe_moa_forward(const void *x, const void *w_gate, const float *logit_bias, 
         if ((rc = check_launch("q projection"))) return rc;
         ++n;
         record_prof(4, s);
-        if ((rc = launch_moa_attention(q, kv, sorted_rows, at<int32_t>(ws, L.base.sparse_rows),
-                                       offsets, o, R, S, H, dh, k, E, status, s)))
+        if ((rc = launch_moa_attention(q, kv, at<int32_t>(ws, L.base.sparse_rows), o, R, S, H, dh,
+                                       k, status, s)))
             return rc;
         if ((rc = check_launch("attention"))) return rc;
         ++n;

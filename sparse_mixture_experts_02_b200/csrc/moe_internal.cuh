@@ -130,9 +130,8 @@ void launch_sum_partials(const float *partial, int64_t n, int32_t P, float *out,
 // p = sparse_rows[i], o[p] = causal attention of query row q[p] ([R, H*dh] bf16, slot order)
 // over the shared keys/values kv [S, 2*H*dh] bf16 (K columns first) up to token i / k. dh is 64
 // or 128. Waits are bounded (status word, kernel id kKernelAttention).
-int launch_moa_attention(const void *q, const void *kv, const int32_t *sorted_rows,
-                         const int32_t *sparse_rows, const int32_t *offsets, void *o, int64_t R,
-                         int64_t S, int32_t H, int32_t dh, int32_t k, int32_t E, unsigned *status,
+int launch_moa_attention(const void *q, const void *kv, const int32_t *sparse_rows, void *o,
+                         int64_t R, int64_t S, int32_t H, int32_t dh, int32_t k, unsigned *status,
                          cudaStream_t s);
 // Writes {0, S}: the offsets of one group holding every token.
 void launch_kv_offsets(int32_t *off, int64_t S, cudaStream_t s);
