@@ -232,8 +232,55 @@ int moe_moa_forward(const void *x, const void *w_gate, const float *logit_bias, 
                     moe_stream_t stream);
 
 /*
+ * Expert parallelism (ScatterMoE guide, "Combine with Tensor and Pipeline Parallelism": expert
+ * weights spread over expert-parallel ranks, ParallelLinear running each rank's local experts).
+ * The E experts are split into contiguous ranges, one per rank. A forward is:
+ *   route (moe_route_topk) -> moe_ep_dispatch -> all-to-all of the rows (caller, e.g. NCCL)
+ *   -> moe_expert_mlp_forward on the received rows -> all-to-all back -> moe_ep_combine.
+ * The library does no communication; these calls prepare and consume the exchanged buffers.
+ *
+ * moe_ep_dispatch: the sparse map of top_experts (outputs as moe_sparse_map) plus the send
+ * buffer in slot order: send_x[p] = x[sorted_rows[p] / k] ([S*k, D], dt) and
+ * send_e[p] = top_experts[sorted_rows[p]] (the global expert id of row p). Slots are grouped by
+ * expert, so rank r's rows are the contiguous range [expert_offsets[r*E/n], expert_offsets[(r+1)*E/n])
+ * for n ranks of E/n experts each. Slots at or past expert_offsets[E] (routes with an id outside
+ * [0,E)) are not written.
+ *   ws: moe_workspace_size("ep_dispatch", S, D, 0, E, k, dt) bytes (status word + map scratch).
+ */
+int moe_ep_dispatch(const void *x, const int32_t *top_experts, int64_t S, int64_t D, int32_t E,
+                    int32_t k, moe_dtype dt, int32_t *expert_counts, int32_t *expert_offsets,
+                    int32_t *sparse_rows, int32_t *sorted_rows, void *send_x, int32_t *send_e,
+                    void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * The expert MLP on rows that arrive with their expert ids (the receiving side of expert
+ * parallelism): for row i with local expert e = expert_ids[i] - expert_base (0 <= e < E),
+ *   y[i] = (silu(x_rows[i] W_gate_e[e]) * (x_rows[i] W_up[e])) W_down[e]   (unweighted, fp32)
+ * Steps: local ids, sparse map over the rows, GEMM1 (rows gathered on load, fused gate+up, SwiGLU),
+ * GEMM2 (scatter-add into row order). A row whose id is out of range is reported through the
+ * status word (MOE_ERR_BAD_EXPERT_ID) and its y row stays zero.
+ *   x_rows [R, D], w_gate_e / w_up [E, D, F], w_down [E, F, D]: dt; expert_ids [R] int32;
+ *   y [R, D] float32 (overwritten).
+ *   ws: moe_workspace_size("expert_mlp_forward", R, D, F, E, 1, dt) bytes.
+ */
+int moe_expert_mlp_forward(const void *x_rows, const int32_t *expert_ids, int32_t expert_base,
+                           int64_t R, int64_t D, int64_t F, int32_t E, const void *w_gate_e,
+                           const void *w_up, const void *w_down, moe_dtype dt, float *y, void *ws,
+                           size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Expert-parallel combine: out[s] = sum_j top_weights[s*k + j] * y_ret[sparse_rows[s*k + j]],
+ * with y_ret [S*k, D] float32 the expert outputs returned into the send buffer's slot order and
+ * sparse_rows the dispatch's map. Routes with sparse_rows outside [0, S*k) add nothing. out
+ * [S, D] float32 is overwritten; every token sums its k rows in order (deterministic, no atomics).
+ */
+int moe_ep_combine(const float *y_ret, const int32_t *sparse_rows, const float *top_weights,
+                   int64_t S, int64_t D, int32_t k, float *out, moe_stream_t stream);
+
+/*
  * Workspace bytes for op = "sparse_map", "scatter_linear", "scatter_linear_backward" (D = Din,
- * F = Dout), "mlp_forward", "mlp_backward" or "moa_forward" (F = H * dh) (unused sizes may be 0). Returns 0 for an unknown op or sizes
+ * F = Dout), "mlp_forward", "mlp_backward", "moa_forward" (F = H * dh), "ep_dispatch" or
+ * "expert_mlp_forward" (S = rows, k = 1) (unused sizes may be 0). Returns 0 for an unknown op or sizes
  * outside the limits.
  */
 size_t moe_workspace_size(const char *op, int64_t S, int64_t D, int64_t F, int32_t E, int32_t k,

@@ -25,7 +25,8 @@ STATUS_NAMES = {0: "MOE_OK", -1: "MOE_ERR_INVALID_ARG", -2: "MOE_ERR_UNSUPPORTED
 
 EXPORTS = ["moe_route_topk", "moe_sparse_map", "moe_sparse_map_noalloc", "moe_scatter_linear",
            "moe_scatter_linear_backward", "moe_mlp_forward", "moe_mlp_backward",
-           "moe_moa_forward", "moe_workspace_size", "moe_workspace_view", "moe_last_error",
+           "moe_moa_forward", "moe_ep_dispatch", "moe_expert_mlp_forward", "moe_ep_combine",
+           "moe_workspace_size", "moe_workspace_view", "moe_last_error",
            "moe_check_device_status", "moe_profile_events", "moe_debug_wait_timeout",
            "moe_last_launch_count"]
 
@@ -54,6 +55,11 @@ def _load():
                                     ctypes.c_size_t, P]
     lib.moe_moa_forward.argtypes = [P, P, P, P, P, P, i64, i64, i32, i32, i32, i32, c_int, P, P,
                                     ctypes.c_size_t, P]
+    lib.moe_ep_dispatch.argtypes = [P, P, i64, i64, i32, i32, c_int, P, P, P, P, P, P, P,
+                                    ctypes.c_size_t, P]
+    lib.moe_expert_mlp_forward.argtypes = [P, P, i32, i64, i64, i64, i32, P, P, P, c_int, P, P,
+                                           ctypes.c_size_t, P]
+    lib.moe_ep_combine.argtypes = [P, P, P, i64, i64, i32, P, P]
     lib.moe_mlp_backward.argtypes = [P, P, P, P, P, P, i64, i64, i64, i32, i32, c_int, P,
                                      ctypes.c_size_t, P, P, P, P, P, P, ctypes.c_size_t, P]
     lib.moe_workspace_size.argtypes = [ctypes.c_char_p, i64, i64, i64, i32, i32, c_int]
@@ -66,7 +72,8 @@ def _load():
     lib.moe_debug_wait_timeout.argtypes = [i64, P, ctypes.c_size_t, P]
     for name in ("moe_route_topk", "moe_sparse_map", "moe_sparse_map_noalloc",
                  "moe_scatter_linear", "moe_scatter_linear_backward", "moe_mlp_forward",
-                 "moe_mlp_backward", "moe_moa_forward",
+                 "moe_mlp_backward", "moe_moa_forward", "moe_ep_dispatch",
+                 "moe_expert_mlp_forward", "moe_ep_combine",
                  "moe_check_device_status", "moe_profile_events", "moe_debug_wait_timeout",
                  "moe_last_launch_count"):
         getattr(lib, name).restype = c_int
@@ -389,6 +396,85 @@ def moa_forward(x: torch.Tensor, w_gate: torch.Tensor, w_q: torch.Tensor, w_kv: 
                                _ptr(w_kv), _ptr(w_o), S, D, heads, HD // heads, E, k,
                                _dtype_code(x), _ptr(out), _ptr(ws.buf), ws.buf.numel(),
                                _stream(dev)))
+    return out
+
+
+def ep_dispatch(x: torch.Tensor, top_experts: torch.Tensor, E: int,
+                ws: Optional[torch.Tensor] = None) -> dict:
+    """Sending side of expert parallelism (moe_ep_dispatch): the sparse map of top_experts
+    [S, k] and the routed rows in slot order. Returns a dict with send_x [S*k, D] (x's dtype),
+    send_e [S*k] int32, expert_counts [E], expert_offsets [E+1], sparse_rows and sorted_rows
+    [S*k]."""
+    _req(x, "x", dim=2)
+    dev = x.device
+    _req(top_experts, "top_experts", dtype=torch.int32, dim=2, device=dev)
+    S, D = x.shape
+    k = top_experts.shape[1]
+    if top_experts.shape[0] != S:
+        raise ValueError("top_experts must be [S, k]")
+    R = S * k
+    out = {
+        "send_x": torch.empty((R, D), dtype=x.dtype, device=dev),
+        "send_e": torch.empty(R, dtype=torch.int32, device=dev),
+        "expert_counts": torch.empty(E, dtype=torch.int32, device=dev),
+        "expert_offsets": torch.empty(E + 1, dtype=torch.int32, device=dev),
+        "sparse_rows": torch.empty(R, dtype=torch.int32, device=dev),
+        "sorted_rows": torch.empty(R, dtype=torch.int32, device=dev),
+    }
+    if ws is None:
+        ws = alloc_workspace(workspace_size("ep_dispatch", S, D, 0, E, k, _dtype_code(x)), dev)
+    _check(_lib().moe_ep_dispatch(
+        _ptr(x), _ptr(top_experts), S, D, E, k, _dtype_code(x), _ptr(out["expert_counts"]),
+        _ptr(out["expert_offsets"]), _ptr(out["sparse_rows"]), _ptr(out["sorted_rows"]),
+        _ptr(out["send_x"]), _ptr(out["send_e"]), _ptr(ws), ws.numel(), _stream(dev)))
+    return out
+
+
+def expert_mlp_forward(x_rows: torch.Tensor, expert_ids: torch.Tensor, expert_base: int,
+                       w_gate_e: torch.Tensor, w_up: torch.Tensor, w_down: torch.Tensor,
+                       y: Optional[torch.Tensor] = None,
+                       ws: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Expert MLP on rows with given expert ids (moe_expert_mlp_forward): row i goes through
+    expert expert_ids[i] - expert_base of the given weights, unweighted; returns y [R, D] float32."""
+    _req(x_rows, "x_rows", dim=2)
+    dev = x_rows.device
+    _req(expert_ids, "expert_ids", dtype=torch.int32, dim=1, device=dev)
+    for t, n in ((w_gate_e, "w_gate_e"), (w_up, "w_up"), (w_down, "w_down")):
+        _req(t, n, dtype=x_rows.dtype, dim=3, device=dev)
+    R, D = x_rows.shape
+    E, _, F = w_gate_e.shape
+    if expert_ids.shape[0] != R or tuple(w_gate_e.shape) != (E, D, F) or \
+            tuple(w_up.shape) != (E, D, F) or tuple(w_down.shape) != (E, F, D):
+        raise ValueError("expected expert_ids [R], w_gate_e/w_up [E,D,F], w_down [E,F,D]")
+    if y is None:
+        y = torch.empty((R, D), dtype=torch.float32, device=dev)
+    _req(y, "y", dtype=torch.float32, dim=2, device=dev)
+    if ws is None:
+        ws = alloc_workspace(workspace_size("expert_mlp_forward", R, D, F, E, 1,
+                                            _dtype_code(x_rows)), dev)
+    _check(_lib().moe_expert_mlp_forward(
+        _ptr(x_rows), _ptr(expert_ids), int(expert_base), R, D, F, E, _ptr(w_gate_e), _ptr(w_up),
+        _ptr(w_down), _dtype_code(x_rows), _ptr(y), _ptr(ws), ws.numel(), _stream(dev)))
+    return y
+
+
+def ep_combine(y_ret: torch.Tensor, sparse_rows: torch.Tensor, top_weights: torch.Tensor,
+               out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Expert-parallel combine (moe_ep_combine): out[s] = sum_j w[s, j] * y_ret[sparse_rows[s k + j]];
+    returns out [S, D] float32."""
+    _req(y_ret, "y_ret", dtype=torch.float32, dim=2)
+    dev = y_ret.device
+    _req(top_weights, "top_weights", dtype=torch.float32, dim=2, device=dev)
+    _req(sparse_rows, "sparse_rows", dtype=torch.int32, dim=1, device=dev)
+    S, k = top_weights.shape
+    D = y_ret.shape[1]
+    if sparse_rows.shape[0] != S * k or y_ret.shape[0] != S * k:
+        raise ValueError("expected y_ret [S*k, D] and sparse_rows [S*k] for top_weights [S, k]")
+    if out is None:
+        out = torch.empty((S, D), dtype=torch.float32, device=dev)
+    _req(out, "out", dtype=torch.float32, dim=2, device=dev)
+    _check(_lib().moe_ep_combine(_ptr(y_ret), _ptr(sparse_rows), _ptr(top_weights), S, D, k,
+                                 _ptr(out), _stream(dev)))
     return out
 
 

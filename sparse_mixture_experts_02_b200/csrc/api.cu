@@ -270,6 +270,11 @@ size_t moe_workspace_size(const char *op, int64_t S, int64_t D, int64_t F, int32
         if (F <= 0 || dt != MOE_BF16) return 0;
         return moa_layout(S, F, E, k).total;
     }
+    if (strcmp(op, "ep_dispatch") == 0) return map_ws_bytes(S, E, k);
+    if (strcmp(op, "expert_mlp_forward") == 0) {  // S = rows, k = 1
+        if (F <= 0 || k != 1 || (dt != MOE_F32 && dt != MOE_BF16)) return 0;
+        return mlp_layout(S, F, E, 1, dt).total;
+    }
     if (strcmp(op, "mlp_forward") == 0) {
         if (F <= 0 || (dt != MOE_F32 && dt != MOE_BF16)) return 0;
         return mlp_layout(S, F, E, k, dt).total;
@@ -992,4 +997,140 @@ int moe_moa_forward(const void *x, const void *w_gate, const float *logit_bias, 
     g_prof_n = 0;
     g_launches = n;
     return MOE_OK;
+}
+
+int moe_ep_dispatch(const void *x, const int32_t *top_experts, int64_t S, int64_t D, int32_t E,
+                    int32_t k, moe_dtype dt, int32_t *expert_counts, int32_t *expert_offsets,
+                    int32_t *sparse_rows, int32_t *sorted_rows, void *send_x, int32_t *send_e,
+                    void *ws, size_t ws_bytes, moe_stream_t stream) {
+    g_launches = 0;
+    int rc;
+    if ((rc = check_dtype(dt)) || (rc = check_dims(S, E, k)) || (rc = check_feat("D", D)))
+        return rc;
+    const int64_t R = S * k;
+    if ((rc = check_ptr("x", x, 16, R == 0)) ||
+        (rc = check_ptr("top_experts", top_experts, 4, R == 0)) ||
+        (rc = check_ptr("expert_counts", expert_counts, 4)) ||
+        (rc = check_ptr("expert_offsets", expert_offsets, 4)) ||
+        (rc = check_ptr("sparse_rows", sparse_rows, 4, R == 0)) ||
+        (rc = check_ptr("sorted_rows", sorted_rows, 4, R == 0)) ||
+        (rc = check_ptr("send_x", send_x, 16, R == 0)) ||
+        (rc = check_ptr("send_e", send_e, 4, R == 0)))
+        return rc;
+    if ((rc = check_ws(ws, ws_bytes, map_ws_bytes(S, E, k)))) return rc;
+    if ((rc = check_device())) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    unsigned *status = at<unsigned>(ws, 0);
+    if (cudaMemsetAsync(status, 0, sizeof(unsigned), s) != cudaSuccess)
+        return set_error(MOE_ERR_CUDA, "cudaMemsetAsync of the status word failed");
+    int n = 0;
+    launch_sparse_map(top_experts, R, E, expert_counts, expert_offsets, sparse_rows, sorted_rows,
+                      at<int32_t>(ws, kStatusBytes), status, s, &n);
+    if ((rc = check_launch("sparse_map"))) return rc;
+    if (R > 0) {
+        launch_ep_pack(x, (size_t)D * esize(dt), top_experts, sorted_rows, expert_offsets, E, k,
+                       R, send_x, send_e, s);
+        ++n;
+    }
+    g_launches = n;
+    return check_launch("ep_pack");
+}
+
+int moe_expert_mlp_forward(const void *x_rows, const int32_t *expert_ids, int32_t expert_base,
+                           int64_t R, int64_t D, int64_t F, int32_t E, const void *w_gate_e,
+                           const void *w_up, const void *w_down, moe_dtype dt, float *y, void *ws,
+                           size_t ws_bytes, moe_stream_t stream) {
+    g_launches = 0;
+    int rc;
+    if ((rc = check_dtype(dt)) || (rc = check_dims(R, E, 1)) || (rc = check_feat("D", D)) ||
+        (rc = check_feat("F", F)))
+        return rc;
+    if ((rc = check_ptr("x_rows", x_rows, 16, R == 0)) ||
+        (rc = check_ptr("expert_ids", expert_ids, 4, R == 0)) ||
+        (rc = check_ptr("w_gate_e", w_gate_e, 16)) || (rc = check_ptr("w_up", w_up, 16)) ||
+        (rc = check_ptr("w_down", w_down, 16)) || (rc = check_ptr("y", y, 16, R == 0)))
+        return rc;
+    // the forward's layout with one route per row: top_e holds the local ids
+    const MlpLayout L = mlp_layout(R, F, E, 1, dt);
+    if ((rc = check_ws(ws, ws_bytes, L.total))) return rc;
+    if ((rc = check_device())) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    unsigned *status = at<unsigned>(ws, L.status);
+    int32_t *local = at<int32_t>(ws, L.top_e);
+    int32_t *offsets = at<int32_t>(ws, L.offsets);
+    int32_t *sorted_rows = at<int32_t>(ws, L.sorted_rows);
+    int n = 0;
+    launch_local_ids(expert_ids, expert_base, R, local, status, s);
+    ++n;
+    if ((rc = check_launch("local_ids"))) return rc;
+    if (R == 0) {
+        g_launches = n;
+        return MOE_OK;
+    }
+    launch_sparse_map(local, R, E, at<int32_t>(ws, L.counts), offsets,
+                      at<int32_t>(ws, L.sparse_rows), sorted_rows, at<int32_t>(ws, L.scratch),
+                      status, s, &n);
+    if ((rc = check_launch("sparse_map"))) return rc;
+    GemmArgs a{};
+    a.A = x_rows;
+    a.a_rows = R;
+    a.B0 = w_gate_e;
+    a.B1 = w_up;
+    a.offsets = offsets;
+    a.sorted_rows = sorted_rows;
+    a.out = at<void>(ws, L.h);
+    a.S = R;
+    a.R = R;
+    a.E = E;
+    a.k = 1;
+    a.K = D;
+    a.N = F;
+    a.bf16 = dt == MOE_BF16;
+    a.gather = true;
+    a.glu = true;
+    a.zero_ptr = y;  // zeroed by GEMM1's epilogue warps before GEMM2 adds into it
+    a.zero_n = R * D;
+    a.status = status;
+    a.wait_limit_ns = kWaitLimitNs;
+    if ((rc = prefer_2sm(R, E) ? launch_grouped_gemm_2sm(a, s) : launch_grouped_gemm(a, s)))
+        return rc;
+    if ((rc = check_launch("gemm1"))) return rc;
+    GemmArgs b = a;
+    b.zero_ptr = nullptr;
+    b.zero_n = 0;
+    b.A = at<void>(ws, L.h);
+    b.B0 = w_down;
+    b.B1 = nullptr;
+    b.out = y;
+    b.K = F;
+    b.N = D;
+    b.gather = false;
+    b.glu = false;
+    b.scatter = true;
+    if ((rc = prefer_2sm(R, E) ? launch_grouped_gemm_2sm(b, s) : launch_grouped_gemm(b, s)))
+        return rc;
+    n += 2;
+    g_launches = n;
+    return check_launch("gemm2");
+}
+
+int moe_ep_combine(const float *y_ret, const int32_t *sparse_rows, const float *top_weights,
+                   int64_t S, int64_t D, int32_t k, float *out, moe_stream_t stream) {
+    g_launches = 0;
+    int rc;
+    if (S < 0 || k < 1 || k > 8 || S * (int64_t)k >= (int64_t(1) << 31))
+        return set_error(MOE_ERR_INVALID_ARG, "ep_combine: need S >= 0, 1 <= k <= 8, S*k < 2^31");
+    if ((rc = check_feat("D", D))) return rc;
+    const int64_t R = S * k;
+    if ((rc = check_ptr("y_ret", y_ret, 16, R == 0)) ||
+        (rc = check_ptr("sparse_rows", sparse_rows, 4, R == 0)) ||
+        (rc = check_ptr("top_weights", top_weights, 4, R == 0)) ||
+        (rc = check_ptr("out", out, 16, S == 0)))
+        return rc;
+    if ((rc = check_device())) return rc;
+    if (S == 0) return MOE_OK;
+    launch_ep_combine(y_ret, sparse_rows, top_weights, S, k, R, D, out,
+                      reinterpret_cast<cudaStream_t>(stream));
+    g_launches = 1;
+    return check_launch("ep_combine");
 }

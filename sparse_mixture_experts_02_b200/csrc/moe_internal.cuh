@@ -133,6 +133,16 @@ void launch_sum_partials(const float *partial, int64_t n, int32_t P, float *out,
 int launch_moa_attention(const void *q, const void *kv, const int32_t *sparse_rows, void *o,
                          int64_t R, int64_t S, int32_t H, int32_t dh, int32_t k, unsigned *status,
                          cudaStream_t s);
+// Expert parallelism (expert_parallel.cu): pack the routed rows in slot order (row_bytes a
+// multiple of 16) with their expert ids; local expert ids of received rows (also clears the
+// status word); combine returned fp32 rows per token with the router weights (D % 4 == 0).
+void launch_ep_pack(const void *x, size_t row_bytes, const int32_t *top_e,
+                    const int32_t *sorted_rows, const int32_t *offsets, int32_t E, int32_t k,
+                    int64_t R, void *send, int32_t *send_e, cudaStream_t s);
+void launch_local_ids(const int32_t *ids, int32_t base, int64_t R, int32_t *local,
+                      unsigned *status, cudaStream_t s);
+void launch_ep_combine(const float *ret, const int32_t *sparse_rows, const float *w, int64_t S,
+                       int32_t k, int64_t R, int64_t D, float *out, cudaStream_t s);
 // Writes {0, S}: the offsets of one group holding every token.
 void launch_kv_offsets(int32_t *off, int64_t S, cudaStream_t s);
 int launch_route_tc(const void *x, const void *w_gate, const float *bias, int64_t S, int64_t D,
