@@ -466,6 +466,84 @@ def backward_bench(args, w):
             "gpu_launches": launches * args.steps, "clocks": clk.summary()}
 
 
+def ep_bench(args, w):
+    """Expert-parallel forward (expert_parallel.ep_mlp_forward) on N ranks, one GPU each: the E
+    experts split into N contiguous ranges, every rank routing its own S tokens (weak scaling).
+    The timed region includes the count exchange's host synchronisation and the three
+    all-to-alls (NCCL); time is the max over ranks of CUDA-event time."""
+    import datetime
+    import socket
+
+    import sparse_mixture_experts_02_b200 as moe  # noqa: F401 (loads the library)
+    from sparse_mixture_experts_02_b200.expert_parallel import STAGES, ep_mlp_forward
+
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if "MASTER_ADDR" not in os.environ:
+        with socket.socket() as sk:
+            sk.bind(("127.0.0.1", 0))
+            os.environ["MASTER_PORT"] = str(sk.getsockname()[1])
+        os.environ["MASTER_ADDR"] = "127.0.0.1"
+    torch.distributed.init_process_group("nccl", rank=rank, world_size=ws,
+                                         timeout=datetime.timedelta(seconds=120), device_id=dev)
+    try:
+        if w.E % ws != 0:
+            raise SystemExit(f"E={w.E} does not split over {ws} ranks")
+        el = w.E // ws
+        inp = W.make_inputs(w, device=dev, seed=0)  # the same weights on every rank
+        sl = slice(rank * el, (rank + 1) * el)
+        wge, wup, wd = (inp[n][sl].contiguous() for n in ("w_gate_e", "w_up", "w_down"))
+        del inp["w_gate_e"], inp["w_up"], inp["w_down"]
+        g = torch.Generator(device=dev)
+        g.manual_seed(1000 + rank)  # every rank its own tokens
+        x = torch.randn((w.S, w.D), generator=g, device=dev).to(inp["x"].dtype)
+
+        def step(evs=None):
+            return ep_mlp_forward(x, inp["w_gate"], wge, wup, wd, w.E, w.k,
+                                  logit_bias=inp["logit_bias"], events=evs)
+
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize(dev)
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)]
+               for _ in range(args.steps)]
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.distributed.barrier()
+        torch.cuda.synchronize(dev)
+        with ClockSampler(torch.cuda.current_device()) as clk:
+            t0.record()
+            for i in range(args.steps):
+                step(evs[i])
+            t1.record()
+            torch.cuda.synchronize(dev)
+        torch.distributed.barrier()
+        ms = t0.elapsed_time(t1) / args.steps
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_max = float(t.item())
+        stage = {n: sum(r[q].elapsed_time(r[q + 1]) for r in evs) / args.steps
+                 for q, n in enumerate(STAGES)}
+        if rank != 0:
+            return None
+        fl = flops_of(w)
+        flop = ws * (fl["router"] + fl["gemm1"] + fl["gemm2"])
+        return {"metric": "expert-parallel MoE-layer fwd tokens/s (bf16)",
+                "value": ws * w.S / (ms_max * 1e-3), "unit": "tokens/s", "n_gpus": ws,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+                "higher_is_better": True, "scaling": "weak", "dtype": w.dtype,
+                "data": "synthetic",
+                "config": {"workload": w.name, "S_per_rank": w.S, "D": w.D, "F": w.F, "E": w.E,
+                           "k": w.k, "experts_per_rank": el, "parallelism": f"ep{ws}",
+                           "l2": "inputs larger than L2 (expert weights streamed)"},
+                "tflops": flop / (ms_max * 1e-3) / 1e12, "stage_ms_rank0": stage,
+                "clocks": clk.summary()}
+    finally:
+        torch.distributed.destroy_process_group()
+
+
 def moa_flops(w: W.MoaWorkload) -> dict:
     """Algorithmic FLOPs of one Mixture-of-Attention forward: router, shared key/value projection,
     routed query projection, causal attention (route at token s: 4*dh*(s+1) per head, summed over
@@ -577,6 +655,9 @@ def main():
                     help="instead of the forward: time moe_mlp_backward on --workload")
     ap.add_argument("--moa", action="store_true",
                     help="instead of the MLP forward: time moe_moa_forward (Mixture of Attention)")
+    ap.add_argument("--ep", action="store_true",
+                    help="instead of the replicated forward: the expert-parallel forward, experts "
+                         "split over the ranks (all-to-all dispatch and combine over NCCL)")
     ap.add_argument("--map-points", default="",
                     help="with --map-sweep: only these points, 'log2R:E,...' (e.g. 26:256)")
     args = ap.parse_args()
@@ -584,6 +665,12 @@ def main():
         ap.error("--warmup must be >= 3")
     if args.map_sweep:
         print(json.dumps(map_sweep(args)), flush=True)
+        return
+    if args.ep:
+        wl = {**W.WORKLOADS, **W.PROFILE_WORKLOADS}[args.workload]
+        line = ep_bench(args, wl)
+        if line is not None:
+            print(json.dumps(line), flush=True)
         return
     if args.moa:
         print(json.dumps(moa_bench(args, W.MOA_WORKLOADS["moa_prefill"])), flush=True)

@@ -38,14 +38,25 @@ def split_sizes(expert_offsets, E: int, n_ranks: int):
     return [off[(r + 1) * el] - off[r * el] for r in range(n_ranks)]
 
 
+STAGES = ("route", "dispatch", "exchange", "experts", "return", "combine")
+
+
 def ep_mlp_forward(x: torch.Tensor, w_gate: torch.Tensor, w_gate_e: torch.Tensor,
                    w_up: torch.Tensor, w_down: torch.Tensor, E: int, k: int,
-                   group=None, logit_bias: Optional[torch.Tensor] = None, ops=None):
+                   group=None, logit_bias: Optional[torch.Tensor] = None, ops=None,
+                   events=None):
     """Expert-parallel forward of this rank's tokens x [S, D]; w_gate [D, E] replicated;
     w_gate_e / w_up [E/n, D, F] and w_down [E/n, F, D] this rank's experts. Returns
     (out [S, D] float32, top_experts [S, k], top_weights [S, k]). Every rank of `group` must call
-    it (the exchanges are collective). `ops` replaces the row kernels (tests only)."""
+    it (the exchanges are collective). `ops` replaces the row kernels (tests only); `events`, 7
+    torch.cuda.Event objects, are recorded on the current stream around the STAGES."""
     ops = CUDA_OPS if ops is None else ops
+
+    def mark(i):
+        if events is not None:
+            events[i].record()
+
+    mark(0)
     n = dist.get_world_size(group)
     rank = dist.get_rank(group)
     if E % n != 0:
@@ -56,7 +67,9 @@ def ep_mlp_forward(x: torch.Tensor, w_gate: torch.Tensor, w_gate_e: torch.Tensor
     S, D = x.shape
     dev = x.device
     top_e, top_w = ops.route(x, w_gate, k, logit_bias)
+    mark(1)
     d = ops.dispatch(x, top_e, E)
+    mark(2)
     off = d["expert_offsets"].to("cpu")
     send = split_sizes(off.tolist(), E, n)
     n_send = int(off[E])
@@ -70,10 +83,14 @@ def ep_mlp_forward(x: torch.Tensor, w_gate: torch.Tensor, w_gate_e: torch.Tensor
     recv_e = torch.empty(n_recv, dtype=torch.int32, device=dev)
     dist.all_to_all_single(recv_x, d["send_x"][:n_send], recv, send, group=group)
     dist.all_to_all_single(recv_e, d["send_e"][:n_send], recv, send, group=group)
+    mark(3)
     y = ops.experts(recv_x, recv_e, rank * el, w_gate_e, w_up, w_down)
+    mark(4)
     # expert outputs back into the slots they were sent from (slots past n_send carry routes
     # with an out-of-range id, which the combine skips)
     ret = torch.empty((S * k, D), dtype=torch.float32, device=dev)
     dist.all_to_all_single(ret[:n_send], y, send, recv, group=group)
+    mark(5)
     out = ops.combine(ret, d["sparse_rows"], top_w)
+    mark(6)
     return out, top_e, top_w
