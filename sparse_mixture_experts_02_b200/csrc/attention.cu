@@ -30,51 +30,53 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 // consecutive tokens, so a tile's rows share nearly one causal limit and the cost of a tile grows
 // with t. Row i reads q from slot sparse_rows[i] and writes o there. A work item is a pair of
 // adjacent tiles (2u, 2u + 1) and one head; both tiles walk the key blocks the later tile needs
-// (the earlier one's extra blocks are masked). Items run in order of decreasing cost, dealt to
+// (the earlier one's extra keys are masked). Items run in order of decreasing cost, dealt to
 // persistent CTAs forwards in even rounds and backwards in odd rounds.
 //
-// Roles (320 threads): warp 0 loads blocks of 64 keys of K and V by TMA (two stages each; K runs
-// one block ahead of V, since a K block is released by its score MMAs and a V block only by its
-// P V MMAs). Warp 1 issues the MMAs: for every block, S = Q K^T of both tiles into their TMEM
-// score buffers (two per tile), then O += P V of both tiles for the previous block into their TMEM
-// outputs. Warps 2-5 and 6-9 are one softmax group per tile: a thread owns one query row (= its
-// TMEM lane). It reads its score row, masks keys past the row's token, and keeps a reference
-// maximum that moves only when the row maximum exceeds it by more than 2^8 (the exponentials
-// stay below 256). It writes the bf16 probabilities P into shared memory as the A operand of the
-// next MMA (128-byte swizzle), and rescales its O row in TMEM when its reference moved. The two
-// groups work on different tiles, so one group's loads, reductions and waits overlap the other's
-// exponentials. After the last block the group normalises O by the row sum and stores bf16 rows
-// to the slots; Q of the group's next tile is gathered by cp.async as soon as the tile's last
-// score MMA has completed.
+// Roles (320 threads):
+//   warp 0     loads blocks of 128 keys of K and V by TMA (two stages each; K runs one block ahead
+//              of V, since a K block is released by its score MMAs and a V block by its P V MMAs);
+//   warp 1     issues the MMAs, alternating the tiles: for block j and tile x, O_x += P_x V (block
+//              j - 1), then S_x = Q_x K^T (block j). Each tile has one TMEM score buffer; P is
+//              written over it and read from TMEM as the A operand of P V, so the score MMA of
+//              block j, issued after that P V, may overwrite it (tcgen05 MMAs of one thread run in
+//              issue order). While one tile's softmax runs, the tensor cores work on the other's;
+//   warps 2-5  the softmax group of tile 0, warps 6-9 that of tile 1: a thread owns one query row
+//              (= its TMEM lane). It reads its 128 scores (two halves of 64 columns), masks keys past
+//              its token, keeps a reference maximum that moves only when the row maximum exceeds
+//              it by more than 2^8 (the exponentials stay below 256), writes the bf16
+//              probabilities over the score buffer and rescales its O row when the reference
+//              moved. After the last block it normalises O by the row sum and stores bf16 rows to
+//              the slots; Q of its next tile is gathered by cp.async as soon as the tile's last
+//              score MMA has completed.
 namespace tc {
 
 constexpr int BM = 128;                   // query rows per tile (two tiles per item)
-constexpr int BN = 64;                    // keys per block
+constexpr int BN = 128;                   // keys per block
 constexpr int THREADS = 320;              // producer warp, MMA warp, two softmax groups
 constexpr int GROUP_WARPS = 4;
-constexpr uint32_t QCHUNK = 128u * 128u;  // 128 rows x 128 bytes: Q columns, a P block
-constexpr uint32_t KCHUNK = 64u * 128u;   // 64 rows x 128 bytes: K or V columns of a block
-constexpr uint32_t TMEM_COLS = 512;       // tile x: S[x][b] at 128 x + 64 b, O[x] at 256 + 128 x
+constexpr uint32_t CHUNK = 128u * 128u;   // 128 rows x 128 bytes, swizzled
+constexpr uint32_t TMEM_COLS = 512;       // tile x: S / P at 128 x, O at 256 + 128 x
 constexpr float kRescaleLog2 = 8.0f;
+constexpr uint32_t NST = 2;               // stages of the K ring and of the V ring
 
 template <int DH>
 struct Layout {
     static constexpr int NCH = DH / 64;
-    static constexpr uint32_t Q = NCH * QCHUNK;   // one Q tile
-    static constexpr uint32_t KV = NCH * KCHUNK;  // one K (or V) block
-    static constexpr uint32_t P = QCHUNK;         // one P block
+    static constexpr uint32_t Q = NCH * CHUNK;   // one Q tile
+    static constexpr uint32_t KV = NCH * CHUNK;  // one K (or V) block
     static constexpr uint32_t OFF_K = 2 * Q;
-    static constexpr uint32_t OFF_V = OFF_K + 2 * KV;
-    static constexpr uint32_t OFF_P = OFF_V + 2 * KV;  // [tile][buffer]
-    static constexpr uint32_t OFF_BAR = OFF_P + 4 * P;
+    static constexpr uint32_t OFF_V = OFF_K + NST * KV;
+    static constexpr uint32_t OFF_BAR = OFF_V + NST * KV;
     static constexpr uint32_t SMEM = OFF_BAR + 256 + 1024;  // + barriers + alignment slack
     static constexpr uint32_t TX = KV;
 };
 
 struct Bars {
-    uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
-    uint64_t s_full[2][2], s_free[2][2], p_full[2][2], p_empty[2][2];  // [tile][buffer]
-    uint64_t q_full[2], o_free[2];                                     // [tile]
+    uint64_t k_full[NST], k_empty[NST], v_full[NST], v_empty[NST];
+    uint64_t s_full[2], p_full[2];  // [tile]: score block ready; P written (and O rescaled)
+    uint64_t o_done[2];             // [tile]: the item's last P V completed
+    uint64_t q_full[2], o_free[2];  // [tile]
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
@@ -93,9 +95,9 @@ struct Params {
 };
 
 // Byte offset of 16-byte unit u (8 bf16) of row r in a K-major tile of 128 rows with 128-byte
-// swizzle: 64-column chunks of QCHUNK bytes, 8-row atoms of 1024 bytes.
+// swizzle: 64-column chunks of CHUNK bytes, 8-row atoms of 1024 bytes.
 __device__ __forceinline__ uint32_t sw_off(int r, int u) {
-    return (uint32_t)(u >> 3) * QCHUNK + (uint32_t)(r >> 3) * 1024u + (uint32_t)(r & 7) * 128u +
+    return (uint32_t)(u >> 3) * CHUNK + (uint32_t)(r >> 3) * 1024u + (uint32_t)(r & 7) * 128u +
            ((uint32_t)((u & 7) ^ (r & 7)) << 4);
 }
 
@@ -120,19 +122,16 @@ moa_attention_tc_kernel(const __grid_constant__ CUtensorMap tmKV, const Params p
     const int64_t HD = (int64_t)p.H * DH;
 
     if (threadIdx.x == 0) {
-        for (int b = 0; b < 2; ++b) {
-            dev::mbar_init(&bar.k_full[b], 1);
-            dev::mbar_init(&bar.k_empty[b], 1);
-            dev::mbar_init(&bar.v_full[b], 1);
-            dev::mbar_init(&bar.v_empty[b], 1);
-            for (int x = 0; x < 2; ++x) {
-                dev::mbar_init(&bar.s_full[x][b], 1);
-                dev::mbar_init(&bar.s_free[x][b], GROUP_WARPS);
-                dev::mbar_init(&bar.p_full[x][b], GROUP_WARPS);
-                dev::mbar_init(&bar.p_empty[x][b], 1);
-            }
+        for (uint32_t st = 0; st < NST; ++st) {
+            dev::mbar_init(&bar.k_full[st], 1);
+            dev::mbar_init(&bar.k_empty[st], 1);
+            dev::mbar_init(&bar.v_full[st], 1);
+            dev::mbar_init(&bar.v_empty[st], 1);
         }
         for (int x = 0; x < 2; ++x) {
+            dev::mbar_init(&bar.s_full[x], 1);
+            dev::mbar_init(&bar.p_full[x], GROUP_WARPS);
+            dev::mbar_init(&bar.o_done[x], 1);
             dev::mbar_init(&bar.q_full[x], GROUP_WARPS);
             dev::mbar_init(&bar.o_free[x], GROUP_WARPS);
         }
@@ -156,7 +155,7 @@ moa_attention_tc_kernel(const __grid_constant__ CUtensorMap tmKV, const Params p
         const int64_t G = gridDim.x;
         return (int64_t)r * G + ((r & 1) ? G - 1 - blockIdx.x : blockIdx.x);
     };
-    // item -> (tile pair, head); blocks of 64 keys the pair needs (up to its last token)
+    // item -> (tile pair, head); blocks of 128 keys the pair needs (up to its last token)
     auto pair_of = [&](int64_t it) { return (int64_t)p.npairs - 1 - it / p.H; };
     auto head_of = [&](int64_t it) { return (int)(it % p.H); };
     auto nblocks = [&](int64_t pair) {
@@ -167,25 +166,26 @@ moa_attention_tc_kernel(const __grid_constant__ CUtensorMap tmKV, const Params p
     if (warp == 0) {
         // ---------------------------------------------------------------- K/V producer
         if (lane == 0) {
-            uint32_t issued = 0, last_par = 0;  // bit b: K stage b (0, 1) / V stage b (2, 3)
+            // bit st: K stage st; bit NST + st: V stage st
+            uint32_t issued = 0, last_par = 0;
             bool ok = true;
             auto load = [&](bool is_v, uint32_t gb, int h, int jb) {
-                const uint32_t b = gb & 1u;
-                uint64_t *empty = is_v ? &bar.v_empty[b] : &bar.k_empty[b];
-                uint64_t *full = is_v ? &bar.v_full[b] : &bar.k_full[b];
-                if (gb >= 2 && !dev::mbar_wait(empty, ((gb - 2) >> 1) & 1u, abort, p.status,
-                                               p.wait_limit_ns, kKernelAttention))
+                const uint32_t st = gb % NST;
+                uint64_t *empty = is_v ? &bar.v_empty[st] : &bar.k_empty[st];
+                uint64_t *full = is_v ? &bar.v_full[st] : &bar.k_full[st];
+                if (gb >= NST && !dev::mbar_wait(empty, ((gb - NST) / NST) & 1u, abort, p.status,
+                                                 p.wait_limit_ns, kKernelAttention))
                     return false;
                 dev::mbar_arrive_expect_tx(full, L::TX);
-                uint8_t *dst = smem + (is_v ? L::OFF_V : L::OFF_K) + b * L::KV;
+                uint8_t *dst = smem + (is_v ? L::OFF_V : L::OFF_K) + st * L::KV;
 #pragma unroll
                 for (int c = 0; c < L::NCH; ++c)
-                    dev::tma_load_2d(dst + c * KCHUNK, &tmKV, full,
+                    dev::tma_load_2d(dst + c * CHUNK, &tmKV, full,
                                      (int32_t)((is_v ? HD : 0) + h * DH + c * 64),
                                      (int32_t)(jb * BN));
-                const uint32_t bit = (is_v ? 2u : 0u) + b;
+                const uint32_t bit = (is_v ? NST : 0u) + st;
                 issued |= 1u << bit;
-                last_par = (last_par & ~(1u << bit)) | (((gb >> 1) & 1u) << bit);
+                last_par = (last_par & ~(1u << bit)) | (((gb / NST) & 1u) << bit);
                 return true;
             };
             uint32_t g = 0, vg = 0;
@@ -206,9 +206,9 @@ moa_attention_tc_kernel(const __grid_constant__ CUtensorMap tmKV, const Params p
             }
             if (ok && vh >= 0) load(true, vg, vh, vj);
             // teardown: every load issued must land before the CTA may exit
-            for (int bit = 0; bit < 4; ++bit)
+            for (uint32_t bit = 0; bit < 2 * NST; ++bit)
                 if (issued & (1u << bit))
-                    dev::mbar_wait(bit < 2 ? &bar.k_full[bit] : &bar.v_full[bit - 2],
+                    dev::mbar_wait(bit < NST ? &bar.k_full[bit] : &bar.v_full[bit - NST],
                                    (last_par >> bit) & 1u, nullptr, p.status, kDrainLimitNs,
                                    kKernelAttention);
         }
@@ -219,66 +219,73 @@ moa_attention_tc_kernel(const __grid_constant__ CUtensorMap tmKV, const Params p
             auto wait = [&](uint64_t *b, uint32_t par) {
                 return dev::mbar_wait(b, par, abort, p.status, p.wait_limit_ns, kKernelAttention);
             };
-            // O += P V of both tiles for global block gp (the first block of an item overwrites
-            // O, after the softmax group has read the previous item's O)
-            auto pv = [&](uint32_t gp, bool first, uint32_t icnt) {
-                const uint32_t b = gp & 1u;
-                if (!wait(&bar.v_full[b], (gp >> 1) & 1u)) return false;
-                const uint32_t sV = sbase + L::OFF_V + b * L::KV;
-                for (int x = 0; x < 2; ++x) {
-                    if (!wait(&bar.p_full[x][b], (gp >> 1) & 1u)) return false;
-                    if (first && icnt > 0 && !wait(&bar.o_free[x], (icnt - 1) & 1u)) return false;
-                    dev::tc_fence_after();
-                    const uint32_t sP = sbase + L::OFF_P + (uint32_t)(2 * x + b) * L::P;
+            // O_x += P_x V for global block gp (the first block of an item overwrites O_x, after
+            // the softmax group has read the previous item's O_x)
+            auto pv = [&](int x, uint32_t gp, bool first, uint32_t icnt) {
+                const uint32_t vs = gp % NST;
+                if ((x == 0 && !wait(&bar.v_full[vs], (gp / NST) & 1u)) ||
+                    !wait(&bar.p_full[x], gp & 1u) ||
+                    (first && icnt > 0 && !wait(&bar.o_free[x], (icnt - 1) & 1u)))
+                    return false;
+                dev::tc_fence_after();
+                const uint32_t sV = sbase + L::OFF_V + vs * L::KV;
 #pragma unroll
-                    for (int kk = 0; kk < BN / 16; ++kk)
-                        dev::mma_bf16(tmem + 256 + 128 * x,
-                                      dev::sdesc(sP + kk * 32, 16, 1024, dev::kLayoutSw128),
-                                      dev::sdesc(sV + kk * 2048, KCHUNK, 1024, dev::kLayoutSw128),
-                                      IDESC_O, (!first || kk > 0) ? 1u : 0u);
-                    dev::mma_commit(&bar.p_empty[x][b]);
-                }
-                dev::mma_commit(&bar.v_empty[b]);
+                for (int kk = 0; kk < BN / 16; ++kk)
+                    dev::mma_bf16_ts(tmem + 256 + 128 * x, tmem + 128 * x + kk * 8,
+                                     dev::sdesc(sV + kk * 2048, CHUNK, 1024, dev::kLayoutSw128),
+                                     IDESC_O, (!first || kk > 0) ? 1u : 0u);
                 return true;
+            };
+            auto score = [&](int x, uint32_t ks) {
+                const uint32_t sQ = sbase + (uint32_t)x * L::Q;
+                const uint32_t sK = sbase + L::OFF_K + ks * L::KV;
+#pragma unroll
+                for (int kk = 0; kk < DH / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * CHUNK + (kk & 3) * 32;
+                    dev::mma_bf16(tmem + 128 * x,
+                                  dev::sdesc(sQ + off, 16, 1024, dev::kLayoutSw128),
+                                  dev::sdesc(sK + off, 16, 1024, dev::kLayoutSw128), IDESC_S,
+                                  kk > 0 ? 1u : 0u);
+                }
+                dev::mma_commit(&bar.s_full[x]);
             };
             uint32_t g = 0, icnt = 0;
             bool ok = true;
             for (int r = 0; item_of(r) < p.nitems && ok; ++r, ++icnt) {
                 const int n = nblocks(pair_of(item_of(r)));
-                if (!wait(&bar.q_full[0], icnt & 1u) || !wait(&bar.q_full[1], icnt & 1u)) break;
-                for (int j = 0; j < n; ++j) {
-                    const uint32_t gj = g + j, b = gj & 1u;
-                    if (!wait(&bar.k_full[b], (gj >> 1) & 1u)) {
+                for (int j = 0; j < n && ok; ++j) {
+                    const uint32_t gj = g + j, ks = gj % NST;
+                    if (!wait(&bar.k_full[ks], (gj / NST) & 1u)) {
                         ok = false;
                         break;
                     }
-                    const uint32_t sK = sbase + L::OFF_K + b * L::KV;
-                    for (int x = 0; x < 2 && ok; ++x) {
-                        if (gj >= 2 && !wait(&bar.s_free[x][b], ((gj - 2) >> 1) & 1u)) {
+                    for (int x = 0; x < 2; ++x) {
+                        if (j >= 1 && !pv(x, gj - 1, j == 1, icnt)) {
+                            ok = false;
+                            break;
+                        }
+                        if (j == 0 && !wait(&bar.q_full[x], icnt & 1u)) {
                             ok = false;
                             break;
                         }
                         dev::tc_fence_after();
-                        const uint32_t sQ = sbase + (uint32_t)x * L::Q;
-#pragma unroll
-                        for (int kk = 0; kk < DH / 16; ++kk)
-                            dev::mma_bf16(
-                                tmem + 128 * x + 64 * b,
-                                dev::sdesc(sQ + (kk >> 2) * QCHUNK + (kk & 3) * 32, 16, 1024,
-                                           dev::kLayoutSw128),
-                                dev::sdesc(sK + (kk >> 2) * KCHUNK + (kk & 3) * 32, 16, 1024,
-                                           dev::kLayoutSw128),
-                                IDESC_S, kk > 0 ? 1u : 0u);
-                        dev::mma_commit(&bar.s_full[x][b]);
+                        score(x, ks);
                     }
                     if (!ok) break;
-                    dev::mma_commit(&bar.k_empty[b]);
-                    if (j >= 1 && !pv(gj - 1, j == 1, icnt)) {
+                    dev::mma_commit(&bar.k_empty[ks]);
+                    if (j >= 1) dev::mma_commit(&bar.v_empty[(gj - 1) % NST]);
+                }
+                if (!ok) break;
+                const uint32_t gl = g + n - 1;
+                for (int x = 0; x < 2 && ok; ++x) {
+                    if (!pv(x, gl, n == 1, icnt)) {
                         ok = false;
                         break;
                     }
+                    dev::mma_commit(&bar.o_done[x]);
                 }
-                if (!ok || !pv(g + n - 1, n == 1, icnt)) break;
+                if (!ok) break;
+                dev::mma_commit(&bar.v_empty[gl % NST]);
                 g += n;
             }
             // teardown: all issued MMAs complete before TMEM is released
@@ -293,8 +300,8 @@ moa_attention_tc_kernel(const __grid_constant__ CUtensorMap tmKV, const Params p
         const int qw = warp & 3;                 // TMEM lane quarter this warp may access
         const int row = qw * 32 + lane;          // query row of the tile = TMEM lane
         const uint32_t tl = tmem + ((uint32_t)(qw * 32) << 16);
+        const uint32_t s_col = 128 * x, o_col = 256 + 128 * x;
         const uint32_t sQ = sbase + (uint32_t)x * L::Q;
-        const uint32_t o_col = 256 + 128 * x;
         auto wait = [&](uint64_t *b, uint32_t par) {  // warp-uniform bounded wait
             bool w = true;
             if (lane == 0)
@@ -320,7 +327,19 @@ moa_attention_tc_kernel(const __grid_constant__ CUtensorMap tmKV, const Params p
                 dev::cp_async16(sQ + sw_off(row, u), sl >= 0 ? src + u * 8 : p.q,
                                 sl >= 0 ? 16u : 0u);
         };
-        uint32_t g = 0;
+        // 64 scores (half hh of the block) -> registers, keys past `pos` set to -inf
+        auto load_half = [&](int hh, int key0, int pos, uint32_t (&sr)[2][32]) {
+            dev::tmem_ld32(tl + s_col + 64 * hh, sr[0]);
+            dev::tmem_ld32(tl + s_col + 64 * hh + 32, sr[1]);
+            dev::tmem_ld_wait();
+            const int kh = key0 + 64 * hh;
+            if (kh + 63 > pos) {
+#pragma unroll
+                for (int c = 0; c < 64; ++c)
+                    if (kh + c > pos) sr[c / 32][c % 32] = __float_as_uint(-CUDART_INF_F);
+            }
+        };
+        uint32_t g = 0, icnt = 0;
         bool ok = true;
         int64_t it = item_of(0);
         if (it < p.nitems) {
@@ -329,7 +348,7 @@ moa_attention_tc_kernel(const __grid_constant__ CUtensorMap tmKV, const Params p
             dev::fence_proxy_async_smem();
             arrive(&bar.q_full[x]);
         }
-        for (int r = 0; it < p.nitems && ok; it = item_of(++r)) {
+        for (int r = 0; it < p.nitems && ok; it = item_of(++r), ++icnt) {
             const int64_t pair = pair_of(it);
             const int h = head_of(it);
             const int n = nblocks(pair);
@@ -339,33 +358,27 @@ moa_attention_tc_kernel(const __grid_constant__ CUtensorMap tmKV, const Params p
             const bool has_next = nit < p.nitems;
             float m_ref = -CUDART_INF_F, l = 0.f;
             for (int j = 0; j < n && ok; ++j) {
-                const uint32_t gj = g + j, b = gj & 1u;
-                if (!wait(&bar.s_full[x][b], (gj >> 1) & 1u)) {
+                const uint32_t gj = g + j;
+                if (!wait(&bar.s_full[x], gj & 1u)) {
                     ok = false;
                     break;
                 }
                 dev::tc_fence_after();
-                uint32_t sr[BN / 32][32];
-#pragma unroll
-                for (int c = 0; c < BN / 32; ++c)
-                    dev::tmem_ld32(tl + 128 * x + 64 * b + c * 32, sr[c]);
-                dev::tmem_ld_wait();
-                dev::tc_fence_before();
-                arrive(&bar.s_free[x][b]);
-                // the last score MMA of this tile has completed: Q may be replaced
+                // the tile's last score MMA has completed: its Q may be replaced
                 if (j == n - 1 && has_next) load_q(pair_of(nit), head_of(nit));
                 const int key0 = j * BN;
-                if (key0 + BN - 1 > pos) {
-#pragma unroll
-                    for (int c = 0; c < BN; ++c)
-                        if (key0 + c > pos) sr[c / 32][c % 32] = __float_as_uint(-CUDART_INF_F);
-                }
+                // pass 1: the row maximum over the block (8 independent chains per half)
                 float pm[8];
 #pragma unroll
-                for (int t = 0; t < 8; ++t) pm[t] = __uint_as_float(sr[0][t]);
+                for (int t = 0; t < 8; ++t) pm[t] = -CUDART_INF_F;
 #pragma unroll
-                for (int c = 8; c < BN; ++c)
-                    pm[c % 8] = fmaxf(pm[c % 8], __uint_as_float(sr[c / 32][c % 32]));
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t sr[2][32];
+                    load_half(hh, key0, pos, sr);
+#pragma unroll
+                    for (int c = 0; c < 64; ++c)
+                        pm[c % 8] = fmaxf(pm[c % 8], __uint_as_float(sr[c / 32][c % 32]));
+                }
                 const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
                                        fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
                 const float mxs = mx * p.scale_log2;
@@ -376,38 +389,31 @@ moa_attention_tc_kernel(const __grid_constant__ CUtensorMap tmKV, const Params p
                     m_ref = mxs;
                 }
                 const float mneg = m_ref == -CUDART_INF_F ? 0.f : -m_ref;
-                // the P row (bf16) into P buffer b once P V of block gj - 2 has released it
-                if (gj >= 2 && !wait(&bar.p_empty[x][b], ((gj - 2) >> 1) & 1u)) {
-                    ok = false;
-                    break;
-                }
-                const uint32_t sP = sbase + L::OFF_P + (uint32_t)(2 * x + b) * L::P;
+                // pass 2: probabilities, written as bf16 pairs over the first 64 columns of the
+                // score buffer (half hh's P lands on score columns already read)
                 float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int u = 0; u < BN / 8; ++u) {
-                    float e[8];
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t sr[2][32];
+                    load_half(hh, key0, pos, sr);
+                    uint32_t pk[32];
 #pragma unroll
-                    for (int t = 0; t < 8; ++t) {
-                        e[t] = ex2(fmaf(__uint_as_float(sr[(u * 8 + t) / 32][(u * 8 + t) % 32]),
-                                        p.scale_log2, mneg));
-                        ps[t] += e[t];
+                    for (int c = 0; c < 32; ++c) {
+                        const float e0 = ex2(fmaf(__uint_as_float(sr[c / 16][(2 * c) % 32]),
+                                                  p.scale_log2, mneg));
+                        const float e1 = ex2(fmaf(__uint_as_float(sr[c / 16][(2 * c + 1) % 32]),
+                                                  p.scale_log2, mneg));
+                        ps[(2 * c) % 8] += e0;
+                        ps[(2 * c + 1) % 8] += e1;
+                        pk[c] = pack_bf16(e0, e1);
                     }
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sP + sw_off(row, u)),
-                                 "r"(pack_bf16(e[0], e[1])), "r"(pack_bf16(e[2], e[3])),
-                                 "r"(pack_bf16(e[4], e[5])), "r"(pack_bf16(e[6], e[7]))
-                                 : "memory");
+                    dev::tmem_st32(tl + s_col + 32 * hh, pk);
                 }
                 const float sum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
                 l = l * alpha + sum;
-                dev::fence_proxy_async_smem();
-                // O holds P V of blocks < gj: rescale the rows whose reference moved
+                // O holds P V of blocks < gj (complete: this block's score MMA was issued after
+                // the previous P V): rescale the rows whose reference moved
                 if (j >= 1 && __any_sync(0xffffffffu, need)) {
-                    const uint32_t gp = gj - 1;
-                    if (!wait(&bar.p_empty[x][gp & 1u], (gp >> 1) & 1u)) {
-                        ok = false;
-                        break;
-                    }
-                    dev::tc_fence_after();
 #pragma unroll
                     for (int c = 0; c < DH / 32; ++c) {
                         uint32_t o[32];
@@ -417,15 +423,14 @@ moa_attention_tc_kernel(const __grid_constant__ CUtensorMap tmKV, const Params p
                         for (int t = 0; t < 32; ++t) o[t] = __float_as_uint(__uint_as_float(o[t]) * alpha);
                         dev::tmem_st32(tl + o_col + c * 32, o);
                     }
-                    dev::tmem_st_wait();
                 }
+                dev::tmem_st_wait();
                 dev::tc_fence_before();
-                arrive(&bar.p_full[x][b]);
+                arrive(&bar.p_full[x]);
             }
             if (!ok) break;
-            // O complete after P V of the last block: normalise and store the row
-            const uint32_t gl = g + n - 1;
-            if (!wait(&bar.p_empty[x][gl & 1u], (gl >> 1) & 1u)) break;
+            // O complete after the item's last P V: normalise and store the row
+            if (!wait(&bar.o_done[x], icnt & 1u)) break;
             dev::tc_fence_after();
             const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
