@@ -634,8 +634,9 @@ def moa_oracle_baseline(w, inp, budget_s):
     n = max(n0, min(w.S, int(n0 * budget_s / max(t, 1e-6))))
     t = run(n)
     return {"value": n / t, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"the first {n} tokens of the sequence (a causal prefix: shorter attention "
-                      f"spans than the full sequence's average)"}
+            "sample": ("the whole sequence" if n >= w.S else
+                       f"the first {n} tokens of the sequence (a causal prefix: shorter attention "
+                       f"spans than the full sequence's average)")}
 
 
 def main():
