@@ -21,6 +21,9 @@
  *    float32 side arrays must be 4-byte aligned. The library never allocates device memory in
  *    these calls: scratch space comes from the caller's workspace `ws` (size from
  *    moe_workspace_size, alignment 256 bytes).
+ *  - Environment: MOE_GEMM_2SM=1 (or 0) forces the grouped GEMMs onto CTA pairs (or single CTAs)
+ *    instead of the library's choice by rows per expert; results are the same either way (the
+ *    parity tests run both). No other environment variable is read.
  *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy default stream) and
  *    never synchronise the host. Argument errors are detected on the host and returned before any
  *    launch. Errors the device detects (an expert id outside [0,E), a bounded wait that ran out)
