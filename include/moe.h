@@ -281,6 +281,14 @@ int moe_ep_combine(const float *y_ret, const int32_t *sparse_rows, const float *
                    int64_t S, int64_t D, int32_t k, float *out, moe_stream_t stream);
 
 /*
+ * The optional last step of the forward: an fp32 output (e.g. moe_mlp_forward's `out`) rounded to
+ * bf16, round-to-nearest-even, for callers whose activations are bf16 (the ScatterMoE guide's
+ * forward returns the input's dtype). src [n] float32, dst [n] bf16, n a multiple of 8, both
+ * 16-byte aligned; no workspace.
+ */
+int moe_cast_bf16(const float *src, int64_t n, void *dst, moe_stream_t stream);
+
+/*
  * Workspace bytes for op = "sparse_map", "scatter_linear", "scatter_linear_backward" (D = Din,
  * F = Dout), "mlp_forward", "mlp_backward", "moa_forward" (F = H * dh), "ep_dispatch" or
  * "expert_mlp_forward" (S = rows, k = 1) (unused sizes may be 0). Returns 0 for an unknown op or sizes

@@ -234,3 +234,17 @@ def moa_forward(x, w_gate, w_q, w_k, w_v, w_o, k, heads, bias=None, given_top_ex
     lib().oracle_moa_forward(_p(x), _p(wg), _p(bias), _p(wq), _p(wk), _p(wv), _p(wo), S, D, heads,
                              dh, E, k, _p(given), _p(out), _p(te), _p(tw))
     return out, te, tw
+
+
+def to_bf16_bits(x):
+    """The optional last step of the forward: float32 -> bfloat16 with round-to-nearest-even
+    (ScatterMoE guide, "3. Assembling the ScatterMoE FFN Block": the layer returns the input's
+    dtype). Plain definition on the bit pattern: keep the top 16 bits after adding half an ulp of
+    the kept part minus one, plus the kept part's lowest bit (ties go to the even pattern);
+    overflow carries into the exponent and yields infinity. NaN becomes the quiet NaN 0x7FC0 (sign
+    kept). Returns uint16 bit patterns."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    rounded = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16) & 0xFFFF
+    nan = np.isnan(np.ascontiguousarray(x, dtype=np.float32))
+    qnan = ((u >> 16) & 0x8000) | 0x7FC0
+    return np.where(nan, qnan, rounded).astype(np.uint16)

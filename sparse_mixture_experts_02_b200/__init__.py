@@ -26,7 +26,7 @@ STATUS_NAMES = {0: "MOE_OK", -1: "MOE_ERR_INVALID_ARG", -2: "MOE_ERR_UNSUPPORTED
 EXPORTS = ["moe_route_topk", "moe_sparse_map", "moe_sparse_map_noalloc", "moe_scatter_linear",
            "moe_scatter_linear_backward", "moe_mlp_forward", "moe_mlp_backward",
            "moe_moa_forward", "moe_ep_dispatch", "moe_expert_mlp_forward", "moe_ep_combine",
-           "moe_workspace_size", "moe_workspace_view", "moe_last_error",
+           "moe_cast_bf16", "moe_workspace_size", "moe_workspace_view", "moe_last_error",
            "moe_check_device_status", "moe_profile_events", "moe_debug_wait_timeout",
            "moe_last_launch_count"]
 
@@ -60,6 +60,7 @@ def _load():
     lib.moe_expert_mlp_forward.argtypes = [P, P, i32, i64, i64, i64, i32, P, P, P, c_int, P, P,
                                            ctypes.c_size_t, P]
     lib.moe_ep_combine.argtypes = [P, P, P, i64, i64, i32, P, P]
+    lib.moe_cast_bf16.argtypes = [P, i64, P, P]
     lib.moe_mlp_backward.argtypes = [P, P, P, P, P, P, i64, i64, i64, i32, i32, c_int, P,
                                      ctypes.c_size_t, P, P, P, P, P, P, ctypes.c_size_t, P]
     lib.moe_workspace_size.argtypes = [ctypes.c_char_p, i64, i64, i64, i32, i32, c_int]
@@ -73,7 +74,7 @@ def _load():
     for name in ("moe_route_topk", "moe_sparse_map", "moe_sparse_map_noalloc",
                  "moe_scatter_linear", "moe_scatter_linear_backward", "moe_mlp_forward",
                  "moe_mlp_backward", "moe_moa_forward", "moe_ep_dispatch",
-                 "moe_expert_mlp_forward", "moe_ep_combine",
+                 "moe_expert_mlp_forward", "moe_ep_combine", "moe_cast_bf16",
                  "moe_check_device_status", "moe_profile_events", "moe_debug_wait_timeout",
                  "moe_last_launch_count"):
         getattr(lib, name).restype = c_int
@@ -475,6 +476,18 @@ def ep_combine(y_ret: torch.Tensor, sparse_rows: torch.Tensor, top_weights: torc
     _req(out, "out", dtype=torch.float32, dim=2, device=dev)
     _check(_lib().moe_ep_combine(_ptr(y_ret), _ptr(sparse_rows), _ptr(top_weights), S, D, k,
                                  _ptr(out), _stream(dev)))
+    return out
+
+
+def cast_bf16(src: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """fp32 -> bf16, round-to-nearest-even (moe_cast_bf16); src's element count a multiple of 8."""
+    _req(src, "src", dtype=torch.float32)
+    if out is None:
+        out = torch.empty(src.shape, dtype=torch.bfloat16, device=src.device)
+    _req(out, "out", dtype=torch.bfloat16, device=src.device)
+    if out.numel() != src.numel():
+        raise ValueError("out must have src's element count")
+    _check(_lib().moe_cast_bf16(_ptr(src), src.numel(), _ptr(out), _stream(src.device)))
     return out
 
 

@@ -1134,3 +1134,17 @@ int moe_ep_combine(const float *y_ret, const int32_t *sparse_rows, const float *
     g_launches = 1;
     return check_launch("ep_combine");
 }
+
+int moe_cast_bf16(const float *src, int64_t n, void *dst, moe_stream_t stream) {
+    g_launches = 0;
+    int rc;
+    if (n < 0 || n % 8 != 0 || n >= (int64_t(1) << 40))
+        return set_error(MOE_ERR_INVALID_ARG, "cast_bf16: n must be a non-negative multiple of 8");
+    if ((rc = check_ptr("src", src, 16, n == 0)) || (rc = check_ptr("dst", dst, 16, n == 0)))
+        return rc;
+    if ((rc = check_device())) return rc;
+    if (n == 0) return MOE_OK;
+    launch_cast_bf16(src, dst, n, reinterpret_cast<cudaStream_t>(stream));
+    g_launches = 1;
+    return check_launch("cast_bf16");
+}
