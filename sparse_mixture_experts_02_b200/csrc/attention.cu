@@ -327,16 +327,16 @@ moa_attention_tc_kernel(const __grid_constant__ CUtensorMap tmKV, const Params p
                 dev::cp_async16(sQ + sw_off(row, u), sl >= 0 ? src + u * 8 : p.q,
                                 sl >= 0 ? 16u : 0u);
         };
-        // 64 scores (half hh of the block) -> registers, keys past `pos` set to -inf
-        auto load_half = [&](int hh, int key0, int pos, uint32_t (&sr)[2][32]) {
-            dev::tmem_ld32(tl + s_col + 64 * hh, sr[0]);
-            dev::tmem_ld32(tl + s_col + 64 * hh + 32, sr[1]);
-            dev::tmem_ld_wait();
-            const int kh = key0 + 64 * hh;
-            if (kh + 63 > pos) {
+        // the block's 128 scores -> registers (one wait for the four loads), keys past `pos`
+        // set to -inf
+        auto load_scores = [&](int key0, int pos, uint32_t (&sr)[BN / 32][32]) {
 #pragma unroll
-                for (int c = 0; c < 64; ++c)
-                    if (kh + c > pos) sr[c / 32][c % 32] = __float_as_uint(-CUDART_INF_F);
+            for (int c = 0; c < BN / 32; ++c) dev::tmem_ld32(tl + s_col + 32 * c, sr[c]);
+            dev::tmem_ld_wait();
+            if (key0 + BN - 1 > pos) {
+#pragma unroll
+                for (int c = 0; c < BN; ++c)
+                    if (key0 + c > pos) sr[c / 32][c % 32] = __float_as_uint(-CUDART_INF_F);
             }
         };
         uint32_t g = 0, icnt = 0;
@@ -367,18 +367,15 @@ moa_attention_tc_kernel(const __grid_constant__ CUtensorMap tmKV, const Params p
                 // the tile's last score MMA has completed: its Q may be replaced
                 if (j == n - 1 && has_next) load_q(pair_of(nit), head_of(nit));
                 const int key0 = j * BN;
-                // pass 1: the row maximum over the block (8 independent chains per half)
+                uint32_t sr[BN / 32][32];
+                load_scores(key0, pos, sr);
+                // the row maximum over the block (8 independent chains)
                 float pm[8];
 #pragma unroll
-                for (int t = 0; t < 8; ++t) pm[t] = -CUDART_INF_F;
+                for (int t = 0; t < 8; ++t) pm[t] = __uint_as_float(sr[0][t]);
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    uint32_t sr[2][32];
-                    load_half(hh, key0, pos, sr);
-#pragma unroll
-                    for (int c = 0; c < 64; ++c)
-                        pm[c % 8] = fmaxf(pm[c % 8], __uint_as_float(sr[c / 32][c % 32]));
-                }
+                for (int c = 8; c < BN; ++c)
+                    pm[c % 8] = fmaxf(pm[c % 8], __uint_as_float(sr[c / 32][c % 32]));
                 const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
                                        fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
                 const float mxs = mx * p.scale_log2;
@@ -389,19 +386,18 @@ moa_attention_tc_kernel(const __grid_constant__ CUtensorMap tmKV, const Params p
                     m_ref = mxs;
                 }
                 const float mneg = m_ref == -CUDART_INF_F ? 0.f : -m_ref;
-                // pass 2: probabilities, written as bf16 pairs over the first 64 columns of the
-                // score buffer (half hh's P lands on score columns already read)
+                // probabilities, written as bf16 pairs over the first 64 columns of the score
+                // buffer (all scores are in registers by now)
                 float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
-                    uint32_t sr[2][32];
-                    load_half(hh, key0, pos, sr);
                     uint32_t pk[32];
 #pragma unroll
                     for (int c = 0; c < 32; ++c) {
-                        const float e0 = ex2(fmaf(__uint_as_float(sr[c / 16][(2 * c) % 32]),
+                        const int k0 = 64 * hh + 2 * c;
+                        const float e0 = ex2(fmaf(__uint_as_float(sr[k0 / 32][k0 % 32]),
                                                   p.scale_log2, mneg));
-                        const float e1 = ex2(fmaf(__uint_as_float(sr[c / 16][(2 * c + 1) % 32]),
+                        const float e1 = ex2(fmaf(__uint_as_float(sr[(k0 + 1) / 32][(k0 + 1) % 32]),
                                                   p.scale_log2, mneg));
                         ps[(2 * c) % 8] += e0;
                         ps[(2 * c + 1) % 8] += e1;
