@@ -12,12 +12,17 @@
 
 #include <math.h>
 
+#include <algorithm>
+#include <mutex>
+
 namespace moe {
 namespace {
 
 constexpr int kTokPerWarp = 8;
 constexpr int kWarps = 8;
 constexpr int kChunk = 64;
+constexpr int kRouteE8MaxSmem = 96 * 1024;  // W_gate rows of the eight-expert router: D <= 6144
+constexpr int kE8Batch = 16;                // x pieces a lane has in flight in that router
 
 template <bool BF16>
 __device__ __forceinline__ float ld_elem(const void *p, int64_t i) {
@@ -135,6 +140,116 @@ route_kernel(const void *__restrict__ x, const void *__restrict__ w_gate,
             sel_i[r] = bi;
         }
         if (lane == 0) {
+            const float m = sel_v[0];
+            float den = 0.f;
+            for (int r = 0; r < k; ++r) den += expf(sel_v[r] - m);
+            for (int r = 0; r < k; ++r) {
+                top_e[s * k + r] = sel_i[r];
+                top_w[s * k + r] = expf(sel_v[r] - m) / den;
+            }
+        }
+    }
+}
+
+// Router for E = 8 experts (bf16) at large batches. Persistent blocks stage W_gate [D, 8] (bf16
+// rows of 16 bytes) in shared memory once; a warp owns a token at a time, lane l reads the
+// 16-byte pieces c = l + 32 j of the x row (8 consecutive d each, coalesced across the warp;
+// kE8Batch pieces in flight) and accumulates the 8 dot products in fp32, ascending d within the
+// lane. Row d sits at slot d ^ ((d >> 3) & 7): the rows of a piece keep their 128 bytes, permuted
+// so that, for a given row offset, the eight lanes of a quarter-warp read eight different 16-byte
+// bank groups. The lanes' sums are added by a butterfly, after which lane 0 takes the top-k and
+// the softmax.
+__global__ void __launch_bounds__(kWarps * 32)
+route_e8_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ w_gate,
+                const float *__restrict__ bias, int64_t S, int64_t D, int32_t k,
+                int32_t *__restrict__ top_e, float *__restrict__ top_w, unsigned *status) {
+    constexpr int NE = 8;
+    extern __shared__ __align__(16) uint4 wrow[];  // D rows of 8 bf16
+    if (status != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *status = 0u;  // first kernel
+    const uint4 *wg = reinterpret_cast<const uint4 *>(w_gate);
+    for (int64_t d0 = threadIdx.x; d0 < D; d0 += 8 * (int64_t)blockDim.x) {
+        uint4 r[8];
+#pragma unroll
+        for (int b = 0; b < 8; ++b) {
+            const int64_t d = d0 + (int64_t)b * blockDim.x;
+            if (d < D) r[b] = __ldg(wg + d);
+        }
+#pragma unroll
+        for (int b = 0; b < 8; ++b) {
+            const int64_t d = d0 + (int64_t)b * blockDim.x;
+            if (d < D) wrow[d ^ ((d >> 3) & 7)] = r[b];
+        }
+    }
+    __syncthreads();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t pieces = D / 8;
+    for (int64_t s = (int64_t)blockIdx.x * kWarps + warp; s < S; s += (int64_t)gridDim.x * kWarps) {
+        float acc[NE];
+#pragma unroll
+        for (int e = 0; e < NE; ++e) acc[e] = 0.f;
+        const uint4 *xr = reinterpret_cast<const uint4 *>(x + s * D);
+        // kE8Batch pieces per lane are loaded before any is used, so their latencies overlap
+        for (int64_t c0 = lane; c0 < pieces; c0 += 32 * kE8Batch) {
+            uint4 xv[kE8Batch];
+#pragma unroll
+            for (int b = 0; b < kE8Batch; ++b) {
+                const int64_t c = c0 + 32 * b;
+                xv[b] = c < pieces ? __ldg(xr + c) : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int b = 0; b < kE8Batch; ++b) {
+                const int64_t c = c0 + 32 * b;
+                if (c >= pieces) break;
+                const __nv_bfloat162 *xp = reinterpret_cast<const __nv_bfloat162 *>(&xv[b]);
+                const int64_t base = 8 * c;
+                const int sw = (int)(c & 7);
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    const float2 xf = __bfloat1622float2(xp[h]);
+#pragma unroll
+                    for (int q = 0; q < 2; ++q) {
+                        const int u = 2 * h + q;
+                        const float xu = q == 0 ? xf.x : xf.y;
+                        const uint4 wv = wrow[base + (u ^ sw)];
+                        const __nv_bfloat162 *wp = reinterpret_cast<const __nv_bfloat162 *>(&wv);
+#pragma unroll
+                        for (int t = 0; t < 4; ++t) {
+                            const float2 wf = __bfloat1622float2(wp[t]);
+                            acc[2 * t] = fmaf(xu, wf.x, acc[2 * t]);
+                            acc[2 * t + 1] = fmaf(xu, wf.y, acc[2 * t + 1]);
+                        }
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < NE; ++e)
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], off);
+        if (lane == 0) {
+            float v[NE];
+#pragma unroll
+            for (int e = 0; e < NE; ++e) {
+                float l = acc[e];
+                if (bias != nullptr) l += __ldg(bias + e);
+                v[e] = isnan(l) ? -INFINITY : l;
+            }
+            unsigned taken = 0;
+            float sel_v[8];
+            int sel_i[8];
+            for (int r = 0; r < k; ++r) {
+                float bv = -INFINITY;
+                int bi = 0x7fffffff;
+#pragma unroll
+                for (int e = 0; e < NE; ++e)
+                    if (!(taken & (1u << e)) && better(v[e], e, bv, bi)) {
+                        bv = v[e];
+                        bi = e;
+                    }
+                taken |= 1u << bi;
+                sel_v[r] = bv;
+                sel_i[r] = bi;
+            }
             const float m = sel_v[0];
             float den = 0.f;
             for (int r = 0; r < k; ++r) den += expf(sel_v[r] - m);
@@ -311,6 +426,28 @@ int launch_route(const void *x, const void *w_gate, const float *bias, int64_t S
                  int32_t E, int32_t k, bool bf16, int32_t *top_e, float *top_w, unsigned *status,
                  cudaStream_t s) {
     if (S == 0) return 0;
+    // Eight experts (bf16), a batch too large for one block per token: W_gate fits in shared
+    // memory and every SM streams x rows (measured 25 us against the tensor-core router's 29 us
+    // at S = 4096, D = 4096).
+    if (bf16 && E == 8 && S > 2048 && D * 16 <= kRouteE8MaxSmem) {
+        static std::once_flag once;
+        static cudaError_t attr_err = cudaSuccess;
+        std::call_once(once, [] {
+            attr_err = cudaFuncSetAttribute(route_e8_kernel,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            kRouteE8MaxSmem);
+        });
+        if (attr_err != cudaSuccess) {
+            set_error(MOE_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(attr_err));
+            return -1;
+        }
+        const int64_t want = (S + kWarps - 1) / kWarps;
+        const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(want, 2LL * num_sms()));
+        route_e8_kernel<<<(unsigned)blocks, kWarps * 32, (size_t)(D * 16), s>>>(
+            static_cast<const __nv_bfloat16 *>(x), static_cast<const __nv_bfloat16 *>(w_gate),
+            bias, S, D, k, top_e, top_w, status);
+        return 1;
+    }
     // Few experts and a batch too small to fill the SMs with 128-token tensor-core tiles (or fp32
     // inputs): one block per token on the CUDA cores, exact fp32 accumulation.
     if (E <= 64 && (S <= 2048 || !bf16) && S < (int64_t(1) << 31)) {

@@ -67,3 +67,20 @@ def test_route_full_workloads(oracle_lib, moe, name):
            if k in ("x", "w_gate", "logit_bias")}
     toks = np.random.default_rng(0).choice(w.S, size=2048, replace=False).astype(np.int32)
     _route_and_check(oracle_lib, moe, cpu, w.k, tokens=np.sort(toks))
+
+
+@pytest.mark.parametrize("k", [1, 2, 8])
+def test_route_eight_experts_large_batch(oracle_lib, moe, k):
+    """The eight-expert router used above 2048 tokens (W_gate staged in shared memory); D = 264
+    gives 33 pieces per row, a ragged last round across the lanes; k = 2 adds a skewing bias."""
+    w = W.custom("e8", S=2500, D=264, F=8, E=8, k=k, router_std="1/sqrt(D)",
+                 zipf_s=1.2 if k == 2 else 0.0)
+    _route_and_check(oracle_lib, moe, W.make_inputs(w, seed=k), k)
+
+
+def test_route_eight_experts_exact_ties(moe):
+    x = torch.zeros(3000, 64, dtype=torch.bfloat16, device="cuda")
+    wg = torch.randn(64, 8, device="cuda").to(torch.bfloat16)
+    te, tw = moe.route_topk(x, wg, 3)
+    assert torch.equal(te.cpu(), torch.tensor([[0, 1, 2]] * 3000, dtype=torch.int32))
+    assert torch.allclose(tw.cpu(), torch.full((3000, 3), 1 / 3))
