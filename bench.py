@@ -463,6 +463,16 @@ def backward_bench(args, w):
             "tflops_frac": {"of_measured_sustained": tflops / pk["bf16_tflops_sustained"],
                             "of_nominal": tflops / 2250.0, "peaks": pk_kind},
             "extra_flop_recompute": 4.0 * R * w.D * w.F, "stage_ms": stage,
+            # dominant stage: the weight gradients of the gate and up projections (two grouped
+            # weight-gradient GEMMs, 2 R D F FLOPs each)
+            "roofline": {"kernel": "dW_gate_e_and_dW_up (grouped_wgrad_kernel x2)",
+                         "bound": "tensor",
+                         "achieved": 4.0 * R * w.D * w.F / (stage["dW_gate_e_and_dW_up"] * 1e-3) / 1e12,
+                         "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                         "frac": 4.0 * R * w.D * w.F / (stage["dW_gate_e_and_dW_up"] * 1e-3) / 1e12
+                         / pk["bf16_tflops_sustained"],
+                         "peak_kind": "measured sustained bf16" if pk_kind == "measured" else pk_kind,
+                         "traffic": None},
             "gpu_launches": launches * args.steps, "clocks": clk.summary()}
 
 
@@ -539,6 +549,14 @@ def ep_bench(args, w):
                            "k": w.k, "experts_per_rank": el, "parallelism": f"ep{ws}",
                            "l2": "inputs larger than L2 (expert weights streamed)"},
                 "tflops": flop / (ms_max * 1e-3) / 1e12, "stage_ms_rank0": stage,
+                # dominant stage: the local experts on the received rows (GEMM1 + GEMM2)
+                "roofline": {"kernel": "experts (grouped GEMMs on received rows, rank 0)",
+                             "bound": "tensor",
+                             "achieved": (fl["gemm1"] + fl["gemm2"]) / (stage["experts"] * 1e-3) / 1e12,
+                             "peak": peaks()[0]["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                             "frac": (fl["gemm1"] + fl["gemm2"]) / (stage["experts"] * 1e-3) / 1e12
+                             / peaks()[0]["bf16_tflops_sustained"],
+                             "traffic": None},
                 "clocks": clk.summary()}
     finally:
         torch.distributed.destroy_process_group()
