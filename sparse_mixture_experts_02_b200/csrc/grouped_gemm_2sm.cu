@@ -33,7 +33,6 @@ namespace {
 using namespace gemm;
 
 constexpr int TM2 = 256;            // rows per pair tile
-constexpr int ST2 = 6;              // pipeline stages
 constexpr int A2_BYTES = 128 * KBYTES;
 constexpr int B2_BYTES = 128 * KBYTES;  // this CTA's 128 columns of B
 constexpr int STAGE2_BYTES = A2_BYTES + B2_BYTES;
@@ -41,10 +40,12 @@ constexpr uint16_t kPairMask = 0x3;
 constexpr int RELAY_WARP = (THREADS + GATHER_THREADS) / 32;
 constexpr int GATHER_BLOCK = THREADS + GATHER_THREADS + 32;  // threads of a gathered-A CTA
 
-struct Smem2 {
-    uint64_t full[ST2];    // leader: one phase per stage = both CTAs' TMA bytes (+ both relays)
-    uint64_t afull[ST2];   // both CTAs: this CTA's gathered rows of the stage landed
-    uint64_t empty[ST2];   // both CTAs: the pair MMAs of the stage are done
+// Shared-memory tail after NS pipeline stages; STG: the scatter epilogue's staging buffers.
+template <int NS, bool STG>
+struct Smem2T {
+    uint64_t full[NS];     // leader: one phase per stage = both CTAs' TMA bytes (+ both relays)
+    uint64_t afull[NS];    // both CTAs: this CTA's gathered rows of the stage landed
+    uint64_t empty[NS];    // both CTAs: the pair MMAs of the stage are done
     uint64_t tfull[2];     // both CTAs: accumulator b complete
     uint64_t tempty[2];    // leader: both CTAs' epilogues have read accumulator b
     uint64_t drain;
@@ -52,9 +53,20 @@ struct Smem2 {
     int abort;
     int32_t off[MAX_E + 1];
     int32_t tstart[MAX_E + 1];
-    float stage[4][32 * 33];  // scatter epilogue staging, one buffer per epilogue warp
+    float stage[STG ? 4 : 1][STG ? 32 * 33 : 1];  // one 32 x 33 buffer per epilogue warp
 };
-constexpr size_t SMEM2_BYTES = 1024 + (size_t)ST2 * STAGE2_BYTES + sizeof(Smem2);
+// The SwiGLU form stores h rows straight from registers and needs no staging buffers: it runs a
+// seventh stage in their place, with less alignment slack (the kernel checks that the dynamic
+// shared memory base needs no more).
+template <bool GLU> constexpr int stages2() { return GLU ? 7 : 6; }
+template <bool GLU> constexpr size_t slack2() { return GLU ? 768 : 1024; }
+template <bool GLU>
+constexpr size_t smem2_bytes() {
+    return slack2<GLU>() + (size_t)stages2<GLU>() * STAGE2_BYTES +
+           sizeof(Smem2T<stages2<GLU>(), !GLU>);
+}
+static_assert(smem2_bytes<true>() <= 232448 && smem2_bytes<false>() <= 232448,
+              "dynamic shared memory per CTA");
 
 template <bool BF16, bool GATHER, bool GLU, bool SCATTER>
 __global__ void __cluster_dims__(2, 1, 1)
@@ -74,9 +86,16 @@ grouped_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
     constexpr uint32_t B_SBO = BF16 ? 1024 : 512;
     static_assert(NCH * CHUNK == B2_BYTES, "B half size");
 
-    extern __shared__ uint8_t smem_raw[];
+    constexpr int ST2 = stages2<GLU>();
+    using Smem2 = Smem2T<ST2, !GLU>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    if ((size_t)(smem - smem_raw) > slack2<GLU>()) {  // uniform over the pair; nothing started
+        if (threadIdx.x == 0 && p.status != nullptr)
+            atomicOr(p.status, kStatusTimeout | (kKernelGemm << 8));
+        return;
+    }
     Smem2 &st = *reinterpret_cast<Smem2 *>(smem + (size_t)ST2 * STAGE2_BYTES);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -353,7 +372,10 @@ grouped_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
             }
             const int n0 = ti.n_idx * OUT_COLS;
             const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + b * BN;
-            epilogue_row<BF16, GLU, SCATTER>(p, tbase, valid, orow, g, n0, st.stage[q]);
+            if constexpr (GLU)
+                epilogue_row<BF16, GLU, SCATTER>(p, tbase, valid, orow, g, n0, nullptr);
+            else
+                epilogue_row<BF16, GLU, SCATTER>(p, tbase, valid, orow, g, n0, st.stage[q]);
             dev::tc_fence_before();
             __syncwarp();
             if (lane == 0) dev::mbar_arrive_cluster(tempty0_base + b * (uint32_t)sizeof(uint64_t));
@@ -378,7 +400,7 @@ int launch_2sm_t(const GemmArgs &a, cudaStream_t s, int n_pairs) {
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [&] {
         attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        (int)SMEM2_BYTES);
+                                        (int)smem2_bytes<GLU>());
     });
     if (attr_err != cudaSuccess)
         return set_error(MOE_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(attr_err));
@@ -424,7 +446,8 @@ int launch_2sm_t(const GemmArgs &a, cudaStream_t s, int n_pairs) {
     kp.zero_n4 = a.zero_n / 4;
     kp.status = a.status;
     kp.wait_limit_ns = a.wait_limit_ns;
-    kern<<<2 * n_pairs, GATHER ? GATHER_BLOCK : THREADS, SMEM2_BYTES, s>>>(mA, mB0, mB1, kp);
+    kern<<<2 * n_pairs, GATHER ? GATHER_BLOCK : THREADS, smem2_bytes<GLU>(), s>>>(mA, mB0, mB1,
+                                                                              kp);
     return MOE_OK;
 }
 
@@ -439,7 +462,7 @@ int max_pairs() {
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(2 * pairs);
     cfg.blockDim = dim3(GATHER_BLOCK);
-    cfg.dynamicSmemBytes = SMEM2_BYTES;
+    cfg.dynamicSmemBytes = smem2_bytes<true>();
     cudaLaunchAttribute attr;
     attr.id = cudaLaunchAttributeClusterDimension;
     attr.val.clusterDim.x = 2;
@@ -449,7 +472,8 @@ int max_pairs() {
     cfg.numAttrs = 1;
     int clusters = 0;
     auto kern = grouped_gemm_2sm_kernel<true, true, true, false>;
-    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM2_BYTES);
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)smem2_bytes<true>());
     if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) == cudaSuccess && clusters > 0 &&
         clusters < pairs)
         pairs = clusters;
