@@ -203,19 +203,24 @@ def scatter_linear_backward(X, W, dY, k, sorted_rows, offsets, gates=None, gathe
     return out
 
 
-def mlp_backward(x, w_gate, w_gate_e, w_up, w_down, dout, k, bias=None, given_top_experts=None):
-    """Backward of mlp_forward over all tokens in fp64, given dout [S, D]: {"dx", "dw_gate",
-    "dw_gate_e", "dw_up", "dw_down"}. given_top_experts [S, k] fixes the routing."""
+def mlp_backward(x, w_gate, w_gate_e, w_up, w_down, dout, k, bias=None, given_top_experts=None,
+                 want=("dx", "dw_gate", "dw_gate_e", "dw_up", "dw_down")):
+    """Backward of mlp_forward over all tokens in fp64, given dout [S, D]: a dict with the
+    requested ones of "dx", "dw_gate", "dw_gate_e", "dw_up", "dw_down" (dx is always computed).
+    given_top_experts [S, k] fixes the routing. Without weight gradients the tokens run in
+    parallel (dx of a token depends on that token alone)."""
     x, wg, wge, wu, wd = _f32(x), _f32(w_gate), _f32(w_gate_e), _f32(w_up), _f32(w_down)
     dout, bias = _f32(dout), _f32(bias)
     S, D = x.shape
     E, _, F = wge.shape
     given = _i32(given_top_experts) if given_top_experts is not None else None
-    out = {"dx": np.zeros((S, D)), "dw_gate": np.zeros((D, E)), "dw_gate_e": np.zeros((E, D, F)),
-           "dw_up": np.zeros((E, D, F)), "dw_down": np.zeros((E, F, D))}
+    shapes = {"dx": (S, D), "dw_gate": (D, E), "dw_gate_e": (E, D, F), "dw_up": (E, D, F),
+              "dw_down": (E, F, D)}
+    out = {n: np.zeros(sh) for n, sh in shapes.items() if n == "dx" or n in want}
     lib().oracle_mlp_backward(_p(x), _p(wg), _p(bias), _p(wge), _p(wu), _p(wd), _p(dout), S, D,
-                              F, E, k, _p(given), _p(out["dx"]), _p(out["dw_gate"]),
-                              _p(out["dw_gate_e"]), _p(out["dw_up"]), _p(out["dw_down"]))
+                              F, E, k, _p(given), _p(out["dx"]), _p(out.get("dw_gate")),
+                              _p(out.get("dw_gate_e")), _p(out.get("dw_up")),
+                              _p(out.get("dw_down")))
     return out
 
 

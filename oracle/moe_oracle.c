@@ -372,17 +372,23 @@ void oracle_scatter_linear_backward(const float *X, const float *W, const float 
  *   dW_gate[:, e] += x dl_j;  dx += dl_j W_gate[:, e]
  * (the ScatterMoE guide's backward of each ParallelLinear, "3. Fused Backward Pass Dynamics",
  * chained through SwiGLU and the router softmax). fp64; every output is overwritten:
- * dx [S, D], dw_gate [D, E], dw_gate_e and dw_up [E, D, F], dw_down [E, F, D]. */
+ * dx [S, D], dw_gate [D, E], dw_gate_e and dw_up [E, D, F], dw_down [E, F, D]. The weight
+ * gradients are nullable (not computed); dx of a token depends on that token alone. */
 void oracle_mlp_backward(const float *x, const float *w_gate, const float *bias,
                          const float *w_gate_e, const float *w_up, const float *w_down,
                          const float *dout, int64_t S, int64_t D, int64_t F, int32_t E, int32_t k,
                          const int32_t *given_top_experts, double *dx, double *dw_gate,
                          double *dw_gate_e, double *dw_up, double *dw_down) {
     memset(dx, 0, sizeof(double) * (size_t)S * (size_t)D);
-    memset(dw_gate, 0, sizeof(double) * (size_t)D * (size_t)E);
-    memset(dw_gate_e, 0, sizeof(double) * (size_t)E * (size_t)D * (size_t)F);
-    memset(dw_up, 0, sizeof(double) * (size_t)E * (size_t)D * (size_t)F);
-    memset(dw_down, 0, sizeof(double) * (size_t)E * (size_t)F * (size_t)D);
+    if (dw_gate) memset(dw_gate, 0, sizeof(double) * (size_t)D * (size_t)E);
+    if (dw_gate_e) memset(dw_gate_e, 0, sizeof(double) * (size_t)E * (size_t)D * (size_t)F);
+    if (dw_up) memset(dw_up, 0, sizeof(double) * (size_t)E * (size_t)D * (size_t)F);
+    if (dw_down) memset(dw_down, 0, sizeof(double) * (size_t)E * (size_t)F * (size_t)D);
+    /* Tokens run in parallel only when no weight gradient (a sum over tokens) is requested:
+     * dx rows are per token. */
+    const int tokens_independent = !dw_gate && !dw_gate_e && !dw_up && !dw_down;
+    #pragma omp parallel if (tokens_independent)
+    {
     double *l = (double *)malloc(sizeof(double) * (size_t)E);
     double *a = (double *)malloc(sizeof(double) * (size_t)F);
     double *b = (double *)malloc(sizeof(double) * (size_t)F);
@@ -393,6 +399,7 @@ void oracle_mlp_backward(const float *x, const float *w_gate, const float *bias,
     double *dv = (double *)malloc(sizeof(double) * (size_t)D);
     int32_t J[64];
     double w[64], dwj[64];
+    #pragma omp for schedule(dynamic, 1)
     for (int64_t s = 0; s < S; ++s) {
         const float *xs = x + s * D;
         const float *ds = dout + s * D;
@@ -418,23 +425,27 @@ void oracle_mlp_backward(const float *x, const float *w_gate, const float *bias,
             }
             dwj[j] = dwv;
             for (int64_t d = 0; d < D; ++d) dv[d] = w[j] * (double)ds[d];
-            double *dwd = dw_down + e * F * D;
-            for (int64_t f = 0; f < F; ++f)
-                for (int64_t d = 0; d < D; ++d) dwd[f * D + d] += h[f] * dv[d];
+            if (dw_down) {
+                double *dwd = dw_down + e * F * D;
+                for (int64_t f = 0; f < F; ++f)
+                    for (int64_t d = 0; d < D; ++d) dwd[f * D + d] += h[f] * dv[d];
+            }
             for (int64_t f = 0; f < F; ++f) {
                 const double sg = 1.0 / (1.0 + exp(-a[f]));
                 da[f] = dh[f] * b[f] * sg * (1.0 + a[f] * (1.0 - sg));
                 db[f] = dh[f] * a[f] * sg;
             }
-            double *dge = dw_gate_e + e * D * F, *dup = dw_up + e * D * F;
+            double *dge = dw_gate_e ? dw_gate_e + e * D * F : NULL;
+            double *dup = dw_up ? dw_up + e * D * F : NULL;
             for (int64_t d = 0; d < D; ++d) {
                 const double xd = (double)xs[d];
                 double acc = 0.0;
-                for (int64_t f = 0; f < F; ++f) {
-                    dge[d * F + f] += xd * da[f];
-                    dup[d * F + f] += xd * db[f];
+                if (dge)
+                    for (int64_t f = 0; f < F; ++f) dge[d * F + f] += xd * da[f];
+                if (dup)
+                    for (int64_t f = 0; f < F; ++f) dup[d * F + f] += xd * db[f];
+                for (int64_t f = 0; f < F; ++f)
                     acc += da[f] * (double)wge[d * F + f] + db[f] * (double)wu[d * F + f];
-                }
                 dxs[d] += acc;
             }
         }
@@ -444,12 +455,13 @@ void oracle_mlp_backward(const float *x, const float *w_gate, const float *bias,
             const double dl = w[j] * (dwj[j] - mean);
             const int64_t e = J[j];
             for (int64_t d = 0; d < D; ++d) {
-                dw_gate[d * E + e] += (double)xs[d] * dl;
+                if (dw_gate) dw_gate[d * E + e] += (double)xs[d] * dl;
                 dxs[d] += dl * (double)w_gate[d * E + e];
             }
         }
     }
     free(l); free(a); free(b); free(h); free(dh); free(da); free(db); free(dv);
+    }
 }
 
 /* Mixture of Attention through ParallelLinear (ScatterMoE guide, "2. Generalization to Mixture of

@@ -8,6 +8,7 @@ import numpy as np
 import pytest
 import torch
 
+import moe_workloads as W
 from parity import rel_frob
 
 pytestmark = pytest.mark.gpu
@@ -74,3 +75,33 @@ def test_mlp_backward_argument_errors(moe):
     moe.mlp_forward(*cu, k, ws=ws)
     with pytest.raises(moe.MoeError):
         moe.mlp_backward(*cu, k, dout.to(dev), ws)
+
+
+def test_mlp_backward_full_size_sampled_dx(oracle_lib, moe):
+    """The Mixtral-shaped prefill layer in the configuration the bench's backward times: the input
+    gradient of seeded sample tokens against the oracle's backward run on those tokens alone (a
+    token's dx depends on that token only). This covers the dh GEMM, the fused SwiGLU backward,
+    the dx GEMM and the router backward at full size; the weight gradients are sums over all
+    tokens and are checked at the smaller sizes above."""
+    w = W.WORKLOADS["mixtral_prefill"]
+    dev = torch.device("cuda")
+    inp = W.make_inputs(w, device=dev, seed=0)
+    ws = moe.ForwardWorkspace(w.S, w.D, w.F, w.E, w.k, torch.bfloat16, dev)
+    moe.mlp_forward(inp["x"], inp["w_gate"], inp["w_gate_e"], inp["w_up"], inp["w_down"], w.k,
+                    logit_bias=inp["logit_bias"], ws=ws)
+    g = torch.Generator(device=dev)
+    g.manual_seed(1)
+    dout = torch.randn((w.S, w.D), generator=g, device=dev)
+    grads = moe.mlp_backward(inp["x"], inp["w_gate"], inp["w_gate_e"], inp["w_up"],
+                             inp["w_down"], w.k, dout, ws)
+    torch.cuda.synchronize()
+    moe.check_device_status(ws.buf)
+    te = ws.view("top_experts").cpu().numpy()
+    toks = np.sort(np.random.default_rng(3).choice(w.S, size=12, replace=False))
+    cpu = {n: inp[n].float().cpu().numpy() for n in ("x", "w_gate", "w_gate_e", "w_up", "w_down")}
+    ref = oracle_lib.mlp_backward(cpu["x"][toks], cpu["w_gate"], cpu["w_gate_e"], cpu["w_up"],
+                                  cpu["w_down"], dout.cpu().numpy()[toks], w.k,
+                                  given_top_experts=te[toks], want=("dx",))["dx"]
+    got = grads["dx"].cpu().numpy()[toks]
+    assert rel_frob(got, ref) < REL, rel_frob(got, ref)
+    assert np.abs(got - ref).max() / (np.abs(ref).max() + 1e-30) < MAXREL

@@ -98,3 +98,25 @@ def test_mlp_backward_finite_differences(oracle_lib):
             step = float(up[name][idx]) - float(dn[name][idx])
             fd = (loss(up) - loss(dn)) / step
             assert fd == pytest.approx(got[name][idx], rel=2e-4, abs=2e-6), (name, idx)
+
+
+def test_dx_only_and_per_token(oracle_lib):
+    """Asking for dx alone (tokens in parallel) gives the same dx as the full backward, and the dx
+    rows of a token subset equal those of the whole batch (a token's dx depends on it alone)."""
+    g = np.random.default_rng(5)
+    S, D, F, E, k = 40, 24, 32, 6, 2
+    x = g.standard_normal((S, D)).astype(np.float32)
+    wg = (g.standard_normal((D, E)) / D ** 0.5).astype(np.float32)
+    wge = (g.standard_normal((E, D, F)) / D ** 0.5).astype(np.float32)
+    wu = (g.standard_normal((E, D, F)) / D ** 0.5).astype(np.float32)
+    wd = (g.standard_normal((E, F, D)) / F ** 0.5).astype(np.float32)
+    dout = g.standard_normal((S, D)).astype(np.float32)
+    full = oracle_lib.mlp_backward(x, wg, wge, wu, wd, dout, k)
+    only = oracle_lib.mlp_backward(x, wg, wge, wu, wd, dout, k, want=("dx",))
+    assert set(only) == {"dx"}
+    np.testing.assert_allclose(only["dx"], full["dx"], rtol=1e-12, atol=1e-14)
+    _, te, _ = oracle_lib.mlp_forward(x, wg, wge, wu, wd, k)
+    toks = np.array([3, 17, 29, 38])
+    sub = oracle_lib.mlp_backward(x[toks], wg, wge, wu, wd, dout[toks], k,
+                                  given_top_experts=te[toks], want=("dx",))
+    np.testing.assert_allclose(sub["dx"], full["dx"][toks], rtol=1e-12, atol=1e-14)
