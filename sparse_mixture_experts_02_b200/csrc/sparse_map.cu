@@ -160,7 +160,10 @@ map_assign_kernel(const int32_t *__restrict__ te, int64_t R, int32_t E, int64_t 
     static_assert(NT == kMaxE, "one thread per expert");
     __shared__ int32_t cnt[kWarpsPerBlock][kMaxE];
     __shared__ int32_t wsum[NT / 32];
-    __shared__ int32_t total;
+    __shared__ int32_t total, btotal;
+    __shared__ int32_t s_first[kMaxE], s_pre[kMaxE];  // per expert: first slot, staging offset
+    __shared__ int32_t stage_r[kBlockRoutes];          // routes, grouped by expert
+    __shared__ uint8_t stage_e[kBlockRoutes];          // their experts
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int e_t = threadIdx.x;  // this thread's expert in the per-expert steps
     const int64_t b = blockIdx.x;
@@ -184,6 +187,7 @@ map_assign_kernel(const int32_t *__restrict__ te, int64_t R, int32_t E, int64_t 
     count_unit(ev, cnt[warp]);
     __syncthreads();
     // per expert: expert offset + block base, then exclusive prefix over the block's warps
+    int32_t bcount_e = 0;
     if (e_t < E) {
         int32_t run = eoff_e + bb_e;
 #pragma unroll
@@ -192,6 +196,18 @@ map_assign_kernel(const int32_t *__restrict__ te, int64_t R, int32_t E, int64_t 
             cnt[w][e_t] = run;
             run += c;
         }
+        bcount_e = run - (eoff_e + bb_e);
+    }
+    // the block's slots of expert e are the contiguous range [first, first + bcount_e). With more
+    // than 16 experts a warp's 32 routes spread over many experts and a direct sorted_rows store
+    // is one scattered word per route: the routes are then staged in shared memory, expert after
+    // expert, and written out contiguously below (measured 22% faster at 2^26 routes and 64 or
+    // 256 experts, 10% slower at 8, where a warp's stores already form runs of about four).
+    const bool staged = E > 16;
+    const int32_t pre_e = block_exclusive_scan<NT>(bcount_e, wsum, &btotal);
+    if (e_t < E) {
+        s_first[e_t] = eoff_e + bb_e;
+        s_pre[e_t] = pre_e;
     }
     __syncthreads();
     // stable slots
@@ -210,8 +226,23 @@ map_assign_kernel(const int32_t *__restrict__ te, int64_t R, int32_t E, int64_t 
         __syncwarp();
         if (i < R) {
             sparse_rows[i] = slot;
-            if (slot >= 0) sorted_rows[slot] = (int32_t)i;
+            if (slot >= 0) {
+                if (staged) {
+                    const int32_t local = s_pre[e] + (slot - s_first[e]);
+                    stage_r[local] = (int32_t)i;
+                    stage_e[local] = (uint8_t)e;
+                } else {
+                    sorted_rows[slot] = (int32_t)i;
+                }
+            }
         }
+    }
+    if (!staged) return;  // uniform over the block
+    __syncthreads();
+    // sorted_rows: consecutive threads write consecutive slots of one expert's range
+    for (int j = threadIdx.x; j < btotal; j += NT) {
+        const int e = stage_e[j];
+        sorted_rows[s_first[e] + (j - s_pre[e])] = stage_r[j];
     }
 }
 
