@@ -7,8 +7,10 @@
 // results ("4. Correctness Validation"). Here slots inside an expert follow the flat route index
 // (a stable counting sort), which is unique, so the map is bit-exact run to run.
 //
-// Work split: the route list is cut into units of kUnit consecutive routes, one warp per unit,
-// kBlockWarps units per block (kBlockRoutes routes).
+// Work split: the route list is cut into units of consecutive routes, one warp per unit, eight
+// units per block. A unit is 512 routes (16 steps of 32) when that still gives at least one block
+// per SM; below that (the 10^4-10^5 routes of a forward) it shrinks to 256, 128, 64 or 32 routes
+// so that the grid keeps about one to two blocks per SM instead of leaving most SMs idle.
 //  1. count:  each warp counts its unit into its own shared-memory counters (shared atomics);
 //             the block sums its warps and writes its per-expert counts to scratch,
 //             expert-major: bcount[e][block].
@@ -31,7 +33,6 @@ namespace {
 constexpr int kWarpsPerBlock = 8;
 constexpr int kIters = 16;                // 32-route steps per unit
 constexpr int kUnit = 32 * kIters;        // 512 routes per warp
-constexpr int kBlockRoutes = kUnit * kWarpsPerBlock;
 constexpr int kMaxE = 256;
 constexpr int kScanThreads = 1024;
 
@@ -50,12 +51,13 @@ __device__ __forceinline__ unsigned same_value_lanes(unsigned v, int nbits) {
 // Bits that hold expert ids 0..E (E itself stands for "no expert").
 __device__ __forceinline__ int id_bits(int32_t E) { return 32 - __clz(E); }
 
-// Loads the kIters x 32 routes of a warp's unit (-1 past R or for an id outside [0, E)).
+// Loads the IT x 32 routes of a warp's unit (-1 past R or for an id outside [0, E)).
+template <int IT>
 __device__ __forceinline__ bool load_unit(const int32_t *__restrict__ te, int64_t R, int32_t E,
-                                          int64_t base, int lane, int (&ev)[kIters]) {
+                                          int64_t base, int lane, int (&ev)[IT]) {
     bool bad = false;
 #pragma unroll
-    for (int it = 0; it < kIters; ++it) {
+    for (int it = 0; it < IT; ++it) {
         const int64_t i = base + it * 32 + lane;
         int e = -1;
         if (i < R) {
@@ -72,24 +74,27 @@ __device__ __forceinline__ bool load_unit(const int32_t *__restrict__ te, int64_
 
 // Adds the unit's routes to the warp's per-expert counters. Counting needs no order, so plain
 // shared-memory atomics do it (measured 1.3-1.5x faster than warp-aggregating with ballots).
-__device__ __forceinline__ void count_unit(const int (&ev)[kIters], int32_t *cnt) {
+template <int IT>
+__device__ __forceinline__ void count_unit(const int (&ev)[IT], int32_t *cnt) {
 #pragma unroll
-    for (int it = 0; it < kIters; ++it)
+    for (int it = 0; it < IT; ++it)
         if (ev[it] >= 0) atomicAdd(&cnt[ev[it]], 1);
     __syncwarp();
 }
 
+template <int IT>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
 map_count_kernel(const int32_t *__restrict__ te, int64_t R, int32_t E, int64_t nblk,
                  int32_t *__restrict__ bcount, unsigned *status) {
+    constexpr int UNIT = 32 * IT, BLOCK_ROUTES = UNIT * kWarpsPerBlock;
     __shared__ int32_t cnt[kWarpsPerBlock][kMaxE];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t b = blockIdx.x;
     for (int e = lane; e < E; e += 32) cnt[warp][e] = 0;
     __syncwarp();
-    int ev[kIters];
-    const bool bad = load_unit(te, R, E, b * kBlockRoutes + (int64_t)warp * kUnit, lane, ev);
-    count_unit(ev, cnt[warp]);
+    int ev[IT];
+    const bool bad = load_unit<IT>(te, R, E, b * BLOCK_ROUTES + (int64_t)warp * UNIT, lane, ev);
+    count_unit<IT>(ev, cnt[warp]);
     if (bad) atomicOr(status, kStatusBadExpert);
     __syncthreads();
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
@@ -151,27 +156,29 @@ map_scan_kernel(int32_t *__restrict__ bcount, int64_t nblk, int32_t *__restrict_
 // All of a block's global loads (the expert totals, its block bases, the warps' routes) are
 // issued before any of them is used: with few blocks per SM, three dependent load phases left
 // the kernel waiting on memory latency (ncu: long-scoreboard stalls first, 24% warps active).
+template <int IT>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32, 4)
 map_assign_kernel(const int32_t *__restrict__ te, int64_t R, int32_t E, int64_t nblk,
                   const int32_t *__restrict__ bbase, const int32_t *__restrict__ totals,
                   int32_t *__restrict__ counts, int32_t *__restrict__ offsets,
                   int32_t *__restrict__ sparse_rows, int32_t *__restrict__ sorted_rows) {
     constexpr int NT = kWarpsPerBlock * 32;
+    constexpr int UNIT = 32 * IT, BLOCK_ROUTES = UNIT * kWarpsPerBlock;
     static_assert(NT == kMaxE, "one thread per expert");
     __shared__ int32_t cnt[kWarpsPerBlock][kMaxE];
     __shared__ int32_t wsum[NT / 32];
     __shared__ int32_t total, btotal;
     __shared__ int32_t s_first[kMaxE], s_pre[kMaxE];  // per expert: first slot, staging offset
-    __shared__ int32_t stage_r[kBlockRoutes];          // routes, grouped by expert
-    __shared__ uint8_t stage_e[kBlockRoutes];          // their experts
+    __shared__ int32_t stage_r[BLOCK_ROUTES];          // routes, grouped by expert
+    __shared__ uint8_t stage_e[BLOCK_ROUTES];          // their experts
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int e_t = threadIdx.x;  // this thread's expert in the per-expert steps
     const int64_t b = blockIdx.x;
     const int32_t tot_e = e_t < E ? __ldg(totals + e_t) : 0;
     const int32_t bb_e = e_t < E ? __ldg(bbase + (int64_t)e_t * nblk + b) : 0;
-    int ev[kIters];
-    const int64_t base = b * kBlockRoutes + (int64_t)warp * kUnit;
-    load_unit(te, R, E, base, lane, ev);
+    int ev[IT];
+    const int64_t base = b * BLOCK_ROUTES + (int64_t)warp * UNIT;
+    load_unit<IT>(te, R, E, base, lane, ev);
     // expert offsets: exclusive prefix of the totals
     const int32_t eoff_e = block_exclusive_scan<NT>(tot_e, wsum, &total);
     if (b == 0) {
@@ -184,7 +191,7 @@ map_assign_kernel(const int32_t *__restrict__ te, int64_t R, int32_t E, int64_t 
     // recount this block's units per warp
     for (int e = lane; e < E; e += 32) cnt[warp][e] = 0;
     __syncwarp();
-    count_unit(ev, cnt[warp]);
+    count_unit<IT>(ev, cnt[warp]);
     __syncthreads();
     // per expert: expert offset + block base, then exclusive prefix over the block's warps
     int32_t bcount_e = 0;
@@ -215,7 +222,7 @@ map_assign_kernel(const int32_t *__restrict__ te, int64_t R, int32_t E, int64_t 
     const int nbits = id_bits(E);
     int32_t *wc = cnt[warp];
 #pragma unroll
-    for (int it = 0; it < kIters; ++it) {
+    for (int it = 0; it < IT; ++it) {
         const int64_t i = base + it * 32 + lane;
         const int e = ev[it];
         const unsigned peers = same_value_lanes(e >= 0 ? (unsigned)e : (unsigned)E, nbits);
@@ -334,8 +341,41 @@ map_small_kernel(const int32_t *__restrict__ te, int64_t R, int32_t E,
 
 }  // namespace
 
+namespace {
+
+constexpr int kMinBlocks = 148;  // one block per SM of a B200
+
+// 32-route steps per warp unit of the grid path: 16 once that gives kMinBlocks blocks, else the
+// largest of 8, 4, 2 that does, else 1.
+int grid_iters(int64_t R) {
+    for (int it = kIters; it > 1; it >>= 1) {
+        const int64_t br = (int64_t)kWarpsPerBlock * 32 * it;
+        if ((R + br - 1) / br >= kMinBlocks) return it;
+    }
+    return 1;
+}
+
+int64_t grid_blocks(int64_t R) {
+    const int64_t br = (int64_t)kWarpsPerBlock * 32 * grid_iters(R);
+    return (R + br - 1) / br;
+}
+
+template <int IT>
+void launch_grid(const int32_t *te, int64_t R, int32_t E, int64_t nblk, int32_t *bcount,
+                 int32_t *totals, int32_t *counts, int32_t *offsets, int32_t *sparse_rows,
+                 int32_t *sorted_rows, unsigned *status, cudaStream_t s) {
+    map_count_kernel<IT><<<(unsigned)nblk, kWarpsPerBlock * 32, 0, s>>>(te, R, E, nblk, bcount,
+                                                                         status);
+    map_scan_kernel<<<(unsigned)E, kScanThreads, 0, s>>>(bcount, nblk, totals);
+    map_assign_kernel<IT><<<(unsigned)nblk, kWarpsPerBlock * 32, 0, s>>>(
+        te, R, E, nblk, bcount, totals, counts, offsets, sparse_rows, sorted_rows);
+}
+
+}  // namespace
+
+// (blocks + 1) x E words; blocks <= max(ceil(R / 4096), 294).
 size_t map_scratch_bytes(int64_t R, int32_t E) {
-    const int64_t nblk = (R + kBlockRoutes - 1) / kBlockRoutes;
+    const int64_t nblk = grid_blocks(R);
     return (size_t)((nblk > 0 ? nblk : 1) + 1) * (size_t)E * sizeof(int32_t);
 }
 
@@ -350,14 +390,31 @@ int launch_sparse_map(const int32_t *te, int64_t R, int32_t E, int32_t *counts, 
         return 0;
     }
     // scratch: block counts / bases [E][nblk], then the expert totals [E]
-    const int64_t nblk = (R + kBlockRoutes - 1) / kBlockRoutes;
+    const int64_t nblk = grid_blocks(R);
     int32_t *bcount = scratch;
     int32_t *totals = scratch + (int64_t)E * nblk;
-    map_count_kernel<<<(unsigned)nblk, kWarpsPerBlock * 32, 0, s>>>(te, R, E, nblk, bcount,
-                                                                     status);
-    map_scan_kernel<<<(unsigned)E, kScanThreads, 0, s>>>(bcount, nblk, totals);
-    map_assign_kernel<<<(unsigned)nblk, kWarpsPerBlock * 32, 0, s>>>(
-        te, R, E, nblk, bcount, totals, counts, offsets, sparse_rows, sorted_rows);
+    switch (grid_iters(R)) {
+        case 16:
+            launch_grid<16>(te, R, E, nblk, bcount, totals, counts, offsets, sparse_rows,
+                            sorted_rows, status, s);
+            break;
+        case 8:
+            launch_grid<8>(te, R, E, nblk, bcount, totals, counts, offsets, sparse_rows,
+                           sorted_rows, status, s);
+            break;
+        case 4:
+            launch_grid<4>(te, R, E, nblk, bcount, totals, counts, offsets, sparse_rows,
+                           sorted_rows, status, s);
+            break;
+        case 2:
+            launch_grid<2>(te, R, E, nblk, bcount, totals, counts, offsets, sparse_rows,
+                           sorted_rows, status, s);
+            break;
+        default:
+            launch_grid<1>(te, R, E, nblk, bcount, totals, counts, offsets, sparse_rows,
+                           sorted_rows, status, s);
+            break;
+    }
     if (n_launch) *n_launch += 3;
     return 0;
 }

@@ -83,6 +83,34 @@ def test_map_block_edges(oracle_lib, moe, R):
     _compare(oracle_lib, moe, te, 64)
 
 
+# Below 148 blocks of 8 x 512 routes the grid path shrinks its warp units to 256, 128, 64 or 32
+# routes (148 blocks = one per SM). Each pair straddles one switch of the unit size: the last
+# route count that keeps the smaller unit and the first that takes the larger one.
+@pytest.mark.parametrize("R", [75264, 75265, 150528, 150529, 301056, 301057, 602112, 602113])
+@pytest.mark.parametrize("E", [8, 256])
+def test_map_unit_size_switches(oracle_lib, moe, R, E):
+    te = W.make_top_experts(R, 1, E, seed=R + E, mode="any")
+    _compare(oracle_lib, moe, te, E)
+
+
+def test_map_bad_expert_id_grid_path(moe):
+    """An out-of-range id on the grid path with 64-route units (R = 98304): reported by the
+    device status, its route gets slot -1, every other route is still mapped."""
+    S, k, E = 16384, 6, 64
+    te = W.make_top_experts(S, k, E, seed=4, mode="zipf").clone()
+    te[9000, 3] = E
+    tg = te.to("cuda")
+    ws = moe.alloc_workspace(moe.workspace_size("sparse_map", S, 0, 0, E, k, 1), tg.device)
+    _, _, sparse_rows, _ = moe.sparse_map(tg, E, ws=ws)
+    with pytest.raises(moe.MoeError) as ei:
+        moe.check_device_status(ws)
+    assert ei.value.code == -5
+    sp = sparse_rows.cpu().numpy()
+    assert sp[9000 * k + 3] == -1
+    valid = np.delete(np.arange(S * k), 9000 * k + 3)
+    assert np.array_equal(np.sort(sp[valid]), np.arange(S * k - 1))
+
+
 @pytest.mark.parametrize("E,mode", [(8, "stride"), (64, "zipf"), (128, "stride"), (256, "zipf")])
 def test_map_2pow20_routes(oracle_lib, moe, E, mode):
     te = W.make_top_experts(1 << 17, 8, E, seed=E, mode=mode)
