@@ -45,6 +45,64 @@ namespace {
 
 using namespace gemm;
 
+// Router epilogue of one token row (the calling thread's TMEM lane): the K largest of
+// logit + bias over the E columns, in descending order with ties to the smaller expert id, and
+// the softmax over those K logits.
+// Each logit becomes one 64-bit key: the logit's bits in an order-preserving unsigned form above
+// the complement of the expert id. Keys then compare exactly like (logit descending, id
+// ascending) and no two are equal, so the top K is a branch-free insertion: every step keeps the
+// larger of a list entry and the carried key and carries the smaller on. NaN counts as -inf and
+// -0 as +0, as in a floating-point comparison. (A per-expert insertion that compared logits and
+// ids in branches took 23-44 us per 128-token tile, most of the router's time.)
+template <int K>
+__device__ __forceinline__ void router_row(const KParams &p, uint32_t tbase, int E, int64_t srow,
+                                           bool valid) {
+    uint64_t top[K];
+#pragma unroll
+    for (int q = 0; q < K; ++q) top[q] = 0;  // below every key (-inf maps above 0)
+    for (int c = 0; c * 32 < E; ++c) {
+        uint32_t av[32];
+        dev::tmem_ld32(tbase + c * 32, av);
+        dev::tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const int e = c * 32 + j;
+            if (e < E) {
+                float v = __uint_as_float(av[j]);
+                if (p.bias != nullptr) v += __ldg(p.bias + e);
+                if (isnan(v)) v = -INFINITY;
+                if (v == 0.0f) v = 0.0f;
+                const uint32_t u = __float_as_uint(v);
+                const uint32_t o = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+                uint64_t key = ((uint64_t)o << 32) | (uint64_t)(~(uint32_t)e);
+#pragma unroll
+                for (int q = 0; q < K; ++q) {
+                    const bool up = key > top[q];
+                    const uint64_t hi = up ? key : top[q];
+                    key = up ? top[q] : key;
+                    top[q] = hi;
+                }
+            }
+        }
+    }
+    if (!valid) return;
+    float tv[K];
+#pragma unroll
+    for (int q = 0; q < K; ++q) {
+        const uint32_t o = (uint32_t)(top[q] >> 32);
+        tv[q] = __uint_as_float((o & 0x80000000u) ? (o & 0x7FFFFFFFu) : ~o);
+    }
+    const float m = tv[0];
+    float den = 0.f;
+#pragma unroll
+    for (int q = 0; q < K; ++q) den += expf(tv[q] - m);
+#pragma unroll
+    for (int q = 0; q < K; ++q) {
+        p.top_e[srow * K + q] = (int32_t)(~(uint32_t)top[q]);
+        p.top_w[srow * K + q] = expf(tv[q] - m) / den;
+    }
+}
+
 template <bool BF16, bool GATHER, bool GLU, bool SCATTER, bool ROUTER, bool BKM, bool GBWD>
 __global__ void __launch_bounds__(GATHER ? THREADS + GATHER_THREADS : THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
@@ -354,53 +412,15 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             const int n0 = ti.n_idx * OUT_COLS;
             const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + b * BN;
             if constexpr (ROUTER) {
-                // thread = token row: running top-8 of (logit + bias) over the E columns, in
-                // increasing expert order; ties keep the smaller expert id first
-                float tv[8];
-                int tix[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    tv[j] = -INFINITY;
-                    tix[j] = 0x7fffffff;
-                }
-                for (int c = 0; c * 32 < E; ++c) {
-                    uint32_t av[32];
-                    dev::tmem_ld32(tbase + c * 32, av);
-                    dev::tmem_ld_wait();
-#pragma unroll 4
-                    for (int j = 0; j < 32; ++j) {
-                        int e = c * 32 + j;
-                        if (e >= E) break;
-                        float v = __uint_as_float(av[j]);
-                        if (p.bias != nullptr) v += __ldg(p.bias + e);
-                        if (isnan(v)) v = -INFINITY;
-#pragma unroll
-                        for (int q2 = 0; q2 < 8; ++q2) {
-                            if (v > tv[q2] || (v == tv[q2] && e < tix[q2])) {
-                                const float tf = tv[q2];
-                                const int ti2 = tix[q2];
-                                tv[q2] = v;
-                                tix[q2] = e;
-                                v = tf;
-                                e = ti2;
-                            }
-                        }
-                    }
-                }
-                if (r < ti.rows) {
-                    const int64_t srow = ti.row_begin + r;
-                    const float m = tv[0];
-                    float den = 0.f;
-#pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        if (j < p.k) den += expf(tv[j] - m);
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        if (j < p.k) {
-                            p.top_e[srow * p.k + j] = tix[j];
-                            p.top_w[srow * p.k + j] = expf(tv[j] - m) / den;
-                        }
-                    }
+                switch (p.k) {
+                    case 1: router_row<1>(p, tbase, E, ti.row_begin + r, r < ti.rows); break;
+                    case 2: router_row<2>(p, tbase, E, ti.row_begin + r, r < ti.rows); break;
+                    case 3: router_row<3>(p, tbase, E, ti.row_begin + r, r < ti.rows); break;
+                    case 4: router_row<4>(p, tbase, E, ti.row_begin + r, r < ti.rows); break;
+                    case 5: router_row<5>(p, tbase, E, ti.row_begin + r, r < ti.rows); break;
+                    case 6: router_row<6>(p, tbase, E, ti.row_begin + r, r < ti.rows); break;
+                    case 7: router_row<7>(p, tbase, E, ti.row_begin + r, r < ti.rows); break;
+                    default: router_row<8>(p, tbase, E, ti.row_begin + r, r < ti.rows); break;
                 }
             } else if constexpr (GBWD) {
                 const int64_t route = valid ? (int64_t)__ldg(p.sorted_rows + prow) : 0;

@@ -84,3 +84,35 @@ def test_route_eight_experts_exact_ties(moe):
     te, tw = moe.route_topk(x, wg, 3)
     assert torch.equal(te.cpu(), torch.tensor([[0, 1, 2]] * 3000, dtype=torch.int32))
     assert torch.allclose(tw.cpu(), torch.full((3000, 3), 1 / 3))
+
+
+def test_route_tensor_core_exact_ties(moe):
+    """The tensor-core router (bf16, E > 64): all logits equal, so experts 0..k-1 in order with
+    weight 1/k. x = -0.0 makes some logits -0 and others +0; they compare equal as numbers and
+    must tie like the +0 logits of x = +0.0."""
+    for zero in (0.0, -0.0):
+        x = torch.full((300, 136), zero, dtype=torch.bfloat16, device="cuda")
+        wg = torch.randn(136, 128, generator=torch.Generator().manual_seed(5)).to(
+            torch.bfloat16).cuda()
+        te, tw = moe.route_topk(x, wg, 4)
+        assert torch.equal(te.cpu(), torch.tensor([[0, 1, 2, 3]] * 300, dtype=torch.int32))
+        assert torch.allclose(tw.cpu(), torch.full((300, 4), 0.25))
+
+
+def test_route_tensor_core_infinite_logits(moe):
+    """x[5, 0] = +inf gives row 5 logits of +inf (W_gate[0, e] > 0), -inf (< 0) or NaN (= 0,
+    counted as -inf): its experts are the k smallest ids with W_gate[0, e] > 0, tied at +inf. The
+    other rows are unaffected."""
+    E, k = 128, 5
+    g = torch.Generator().manual_seed(11)
+    x = torch.randn(300, 136, generator=g).to(torch.bfloat16)
+    wg = torch.randn(136, E, generator=g).to(torch.bfloat16)
+    wg[0, 3] = 0.0
+    x[5, 0] = float("inf")
+    te, tw = moe.route_topk(x.cuda(), wg.cuda(), k)
+    te = te.cpu()
+    pos = [e for e in range(E) if float(wg[0, e]) > 0][:k]
+    assert te[5].tolist() == pos
+    ref_te, _ = moe.route_topk(x[6:].cuda(), wg.cuda(), k)  # rows without inf, routed alone
+    assert torch.equal(te[6:], ref_te.cpu())
+    assert bool(torch.isfinite(tw[6:]).all())
