@@ -67,6 +67,10 @@ WORKLOADS = {
 PROFILE_WORKLOADS = {
     "prefill_profile": Workload("prefill_profile", S=2048, D=4096, F=7168, E=8, k=2,
                                 dtype="bf16", router_std="0.02"),
+    # the 128-expert layer's tiles (about 256 rows per expert, D = F = 2880, one-CTA GEMMs) with
+    # a quarter of its experts and tokens: 1.6 GB of weights
+    "e128_profile": Workload("e128_profile", S=2048, D=2880, F=2880, E=32, k=4, dtype="bf16",
+                             router_std="1/sqrt(D)"),
 }
 
 
