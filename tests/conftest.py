@@ -38,6 +38,6 @@ def pytest_collection_modifyitems(config, items):
 
 @pytest.fixture(scope="session")
 def moe():
-    """The CUDA library binding; on a GPU machine a missing library is an error, never a skip."""
+    """The CUDA library binding; with a GPU present a missing library is an error, never a skip."""
     import sparse_mixture_experts_02_b200 as m
     return m
