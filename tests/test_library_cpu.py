@@ -67,6 +67,19 @@ def test_workspace_sizes(moe):
     assert moe.workspace_view("bogus", S, D, F, E, k, 1) == -1
 
 
+@pytest.mark.parametrize("R", [16385, 32768, 75264, 75265, 98304, 300000, 602112, 602113,
+                               1 << 22, (1 << 22) + 1])
+@pytest.mark.parametrize("E", [8, 256])
+def test_sparse_map_workspace_bound(moe, R, E):
+    """The grid map keeps (blocks + 1) x E int32 counters. Blocks: ceil(R / 4096) from 148 such
+    blocks up (602,113 routes); below that the warp units shrink, with at most 294 blocks."""
+    got = moe.workspace_size("sparse_map", R, 0, 0, E, 1, 1)
+    bound = 256 + (max(-(-R // 4096), 294) + 1) * E * 4
+    assert 256 < got <= bound + 255
+    if R > 602112:
+        assert got >= 256 + (-(-R // 4096) + 1) * E * 4
+
+
 def test_host_argument_errors_before_any_launch(moe):
     lib = moe.lib
     P = ctypes.c_void_p
