@@ -1,8 +1,7 @@
 // Internal declarations and sm_100a device helpers of the MoE library.
 //
-// The inline PTX here follows the public PTX ISA (mbarrier, cp.async.bulk.tensor incl. the
-// tile::gather4 mode, tcgen05.alloc / mma / commit / ld / fence). No helper here is shared with
-// the CPU oracle.
+// The inline PTX here follows the public PTX ISA (mbarrier, cp.async, cp.async.bulk.tensor,
+// tcgen05.alloc / mma / commit / ld / st / fence). No helper here is shared with the CPU oracle.
 #pragma once
 
 #include <cuda.h>

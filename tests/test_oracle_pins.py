@@ -93,6 +93,67 @@ def test_route_bruteforce_with_ties(oracle_lib, E, k):
         assert np.all(np.diff(tw[s]) <= 0)
 
 
+def test_router_absdot_magnitude_sum(oracle_lib):
+    """The magnitude sum a[s,e] = sum_d |x[s,d] W_gate[d,e]| that sets the GPU routing tie band
+    equals |x| @ |W_gate| in float64 (every term is non-negative, so any summation order agrees to
+    a few ulps), with and without a bias (the bias is not part of the dot product) and on a token
+    subset. Dropping the absolute value, summing |x_d| alone or adding the bias fails this."""
+    gen = torch.Generator().manual_seed(7)
+    S, D, E = 40, 96, 12
+    x = (torch.randn((S, D), generator=gen)).to(torch.bfloat16).float()
+    wg = (0.05 * torch.randn((D, E), generator=gen)).to(torch.bfloat16).float()
+    bias = torch.randn(E, generator=gen)
+    ref = np.abs(_np(x)) @ np.abs(_np(wg))
+    for b in (None, bias):
+        _, a = oracle_lib.router_logits(x, wg, bias=b)
+        assert np.allclose(a, ref, rtol=1e-13, atol=0)
+    toks = np.array([39, 0, 17, 17, 5], dtype=np.int32)
+    _, a = oracle_lib.router_logits(x, wg, bias=bias, tokens=toks)
+    assert np.allclose(a, ref[toks], rtol=1e-13, atol=0)
+    # integer inputs with mixed signs: exact, and different from |sum| and from sum |x_d|
+    xi = torch.randint(-3, 4, (9, 5), generator=gen).float()
+    wi = torch.randint(-3, 4, (5, 4), generator=gen).float()
+    l, a = oracle_lib.router_logits(xi, wi)
+    assert np.array_equal(a, np.abs(_np(xi)) @ np.abs(_np(wi)))
+    assert np.all(a >= np.abs(l))
+    assert np.any(a > np.abs(l))
+
+
+def test_router_absdot_closed_form(oracle_lib):
+    # x_d = (-1)^d and W[d, e] = (e + 1) (-1)^(d + e): every product is (e + 1) (-1)^e in
+    # magnitude e + 1, so a[s, e] = D (e + 1) while the logit is D (e + 1) (-1)^e.
+    D, E = 10, 5
+    x = np.array([[(-1.0) ** d for d in range(D)]], np.float32)
+    wg = np.array([[(e + 1) * (-1.0) ** (d + e) for e in range(E)] for d in range(D)], np.float32)
+    l, a = oracle_lib.router_logits(x, wg)
+    assert a[0].tolist() == [D * (e + 1.0) for e in range(E)]
+    assert l[0].tolist() == [D * (e + 1.0) * (-1.0) ** e for e in range(E)]
+
+
+def test_router_tie_band_bounds_fp32_logits(oracle_lib):
+    """The tie band built from the magnitude sum (Higham's bound gamma_D * a for a float32 dot
+    product of exact inputs) contains the float32 logits that torch computes on the CPU, in two
+    summation orders, at the Mixtral width D = 4096 and the 128-expert width D = 2880."""
+    import sys
+    sys.path.insert(0, os.path.dirname(__file__))
+    from parity import fp32_dot_bound
+    for D, E, seed in ((4096, 8, 1), (2880, 16, 2)):
+        gen = torch.Generator().manual_seed(seed)
+        x = (torch.randn((64, D), generator=gen)).to(torch.bfloat16).float()
+        wg = (torch.randn((D, E), generator=gen) / math.sqrt(D)).to(torch.bfloat16).float()
+        l, a = oracle_lib.router_logits(x, wg)
+        band = fp32_dot_bound(D, a)
+        l32 = (x @ wg).double().numpy()
+        l32_seq = torch.zeros((64, E))
+        for d0 in range(0, D, 512):  # a blocked order: partial sums of 512 added in sequence
+            l32_seq += x[:, d0:d0 + 512] @ wg[d0:d0 + 512]
+        for got in (l32, l32_seq.double().numpy()):
+            assert np.all(np.abs(got - l) <= band)
+        # the band is not vacuous: a few percent of the logits' spread (a worst-case bound, so
+        # wider than the errors themselves)
+        assert np.median(band) < 0.05 * np.std(l)
+
+
 def test_route_bias_forces_expert(oracle_lib):
     w = W.custom("b", S=64, D=32, F=16, E=6, k=2, dtype="f32")
     inp = W.make_inputs(w)
