@@ -7,12 +7,24 @@ batch of seeded synthetic inputs. Default workload: the Mixtral-8x7B-shaped pref
 (S=4096, D=4096, F=14336, E=8, top-2, bf16). With N > 1 (launched by torch.distributed.run) every
 rank runs its own replica on its own batch (weak scaling, no data-path collective); the timed
 region is bracketed by a barrier and device synchronisation, and the max over ranks is reported.
-`--impl reference` times the CPU oracle instead (rank 0 only), on a bounded token sample.
+At N = 1 the line also carries a `workloads` object: every other configuration (the fp32 tiny
+layer, Mixtral decode, the 128-expert layer and the Zipf-skewed layer), each timed the same way
+with its own clocks and its own roofline. `--impl reference` times the CPU oracle instead (rank 0
+only), on a bounded token sample.
+
+`python bench.py --record-traffic LAUNCHES.csv --workload NAME` reads an ncu CSV of
+`dram__bytes_read.sum`, `dram__bytes_write.sum` and `gpu__time_duration.sum` per launch and
+records the DRAM bytes per launch of each kernel class in profiles/dram_traffic.json, with a hash
+of the sources that define that kernel; the bench reports a recorded figure only while those
+sources are unchanged.
 """
 from __future__ import annotations
 
 import argparse
+import csv
+import datetime
 import hashlib
+import io
 import json
 import math
 import os
@@ -33,6 +45,22 @@ import moe_workloads as W  # noqa: E402
 METRIC = "MoE-layer fwd tokens/s and TFLOP/s (bf16) as % of B200 peak; sparse-map GB/s"
 NOMINAL_TFLOPS = {"bf16": 2250.0, "f32": 1125.0}   # dense bf16; tf32 for fp32 inputs
 NOMINAL_HBM_GBS = 8000.0
+L2_BYTES = 126 * 1000 * 1000
+TRAFFIC_JSON = os.path.join(ROOT, "profiles", "dram_traffic.json")
+CSRC = os.path.join(ROOT, "sparse_mixture_experts_02_b200", "csrc")
+# sources that define each kernel class (a recorded DRAM figure is void once any of them changes)
+KERNEL_SOURCES = {
+    "gemm1": ("grouped_gemm.cu", "grouped_gemm_2sm.cu", "gemm_common.cuh", "moe_internal.cuh"),
+    "gemm2": ("grouped_gemm.cu", "grouped_gemm_2sm.cu", "gemm_common.cuh", "moe_internal.cuh"),
+    "router": ("route.cu", "grouped_gemm.cu", "gemm_common.cuh", "moe_internal.cuh"),
+    "sparse_map": ("sparse_map.cu", "moe_internal.cuh"),
+}
+# forward stages in the order the library records its events
+STAGES = ("route", "sparse_map", "gemm1", "gemm2")
+
+
+def elt_bytes(w: W.Workload) -> int:
+    return 2 if w.dtype == "bf16" else 4
 
 
 def flops_of(w: W.Workload) -> dict:
@@ -42,6 +70,28 @@ def flops_of(w: W.Workload) -> dict:
         "gemm1": 4.0 * R * w.D * w.F,
         "gemm2": 2.0 * R * w.F * w.D,
     }
+
+
+def bytes_of(w: W.Workload, e_act: int) -> dict:
+    """Algorithmic DRAM bytes of each stage: what the method must move, once. e_act = experts with
+    at least one route (only their weights stream)."""
+    b = elt_bytes(w)
+    R = w.R
+    return {
+        # x read, W_gate read, top experts and weights written
+        "router": w.S * w.D * b + w.D * w.E * b + 8 * R,
+        # routes read, slots and inverse permutation written, counts and offsets written
+        "sparse_map": 12 * R + (2 * w.E + 1) * 4,
+        # x read, gate and up weights of active experts read, h written, out zeroed
+        "gemm1": w.S * w.D * b + 2 * e_act * w.D * w.F * b + R * w.F * b + w.S * w.D * 4,
+        # h read, down weights of active experts read, out read and written by the reductions
+        "gemm2": R * w.F * b + e_act * w.F * w.D * b + 2 * w.S * w.D * 4,
+    }
+
+
+def input_bytes(w: W.Workload) -> int:
+    b = elt_bytes(w)
+    return w.S * w.D * b + w.D * w.E * b + 3 * w.E * w.D * w.F * b
 
 
 def peaks():
@@ -54,30 +104,109 @@ def peaks():
             "fallback"
 
 
-def gemm_source_hash() -> str:
-    """Hash of the sources that define the grouped GEMM kernels (a recorded DRAM traffic figure is
-    only reported while they are unchanged)."""
+def tensor_peak(dtype: str, clocks, timed_s):
+    """The dense tensor peak that matches the timed region: the burst figure when the SM clock
+    stayed within 5% of its maximum (or, without clock samples, when the region lasted under a
+    second), else the sustained figure (measured over seconds under the power cap). fp32 inputs
+    run as tf32: the bf16 figure times the nominal tf32 / bf16 ratio (1/2)."""
+    pk, pk_kind = peaks()
+    ratio = 1.0 if dtype == "bf16" else NOMINAL_TFLOPS["f32"] / NOMINAL_TFLOPS["bf16"]
+    if clocks and clocks.get("sm_mhz") and clocks.get("sm_max_mhz"):
+        burst = clocks["sm_mhz"] >= 0.95 * clocks["sm_max_mhz"]
+        why = f"median SM clock {clocks['sm_mhz']:.0f} of max {clocks['sm_max_mhz']:.0f} MHz"
+    else:
+        burst = timed_s < 1.0
+        why = f"no clock samples; timed region {timed_s:.2f} s"
+    kind = "burst" if burst else "sustained"
+    value = (pk["bf16_tflops"] if burst else pk["bf16_tflops_sustained"]) * ratio
+    label = f"{pk_kind} {kind} bf16" + ("" if ratio == 1.0 else " x tf32/bf16 nominal ratio")
+    return value, f"{label} ({why})"
+
+
+def source_hash(kernel: str) -> str:
     h = hashlib.sha256()
-    for name in ("grouped_gemm.cu", "grouped_gemm_2sm.cu", "gemm_common.cuh", "moe_internal.cuh"):
-        with open(os.path.join(ROOT, "sparse_mixture_experts_02_b200", "csrc", name), "rb") as f:
+    for name in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(CSRC, name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(kernel_key: str):
-    """DRAM bytes per launch of `kernel_key` from the committed ncu summary, if the kernel source
-    is unchanged since it was captured (the summary records the source hash)."""
-    path = os.path.join(ROOT, "profiles", "dram_traffic.md")
+def recorded_traffic(kernel: str, workload: str, path: str = TRAFFIC_JSON):
+    """DRAM bytes per launch of `kernel` on `workload` from profiles/dram_traffic.json, if the
+    sources that define the kernel are unchanged since the capture; else None."""
     try:
-        text = open(path).read()
-        sha = gemm_source_hash()
-    except OSError:
+        with open(path) as f:
+            rec = json.load(f)["entries"][f"{kernel}@{workload}"]
+    except (OSError, KeyError, ValueError):
         return None
-    m = re.search(r"^\|\s*" + re.escape(kernel_key) + r"\s*\|\s*([0-9]+)\s*\|\s*([0-9a-f]+)\s*\|",
-                  text, re.M)
-    if not m or m.group(2) != sha:
+    if rec.get("sources_sha16") != source_hash(kernel):
         return None
-    return int(m.group(1))
+    return int(rec["dram_bytes_per_launch"])
+
+
+def kernel_class(name: str):
+    """Kernel class of an ncu kernel name (template arguments print as 0/1)."""
+    m = re.search(r"(grouped_gemm_2sm_kernel|grouped_gemm_kernel)<([^>]*)>", name)
+    if m:
+        a = [int(v) for v in re.findall(r"-?\d+", m.group(2))]
+        gather, glu, scatter = a[1], a[2], a[3]
+        router = m.group(1) == "grouped_gemm_kernel" and len(a) > 4 and a[4] == 1
+        if router:
+            return "router"
+        if gather and glu and not scatter:
+            return "gemm1"
+        if scatter and not gather and not glu:
+            return "gemm2"
+        return None
+    if re.search(r"\broute\w*_kernel", name):
+        return "router"
+    if re.search(r"\bmap_\w+_kernel", name):
+        return "sparse_map"
+    return None
+
+
+def record_traffic(csv_path: str, workload: str, command: str, path: str = TRAFFIC_JSON):
+    """Writes the mean DRAM bytes (read + write) per launch of each kernel class found in an ncu
+    CSV into profiles/dram_traffic.json (entries keyed "<class>@<workload>")."""
+    text = open(csv_path).read()
+    start = text.find('"ID"')
+    rows = csv.DictReader(io.StringIO(text[start:]))
+    launches = {}
+    for r in rows:
+        d = launches.setdefault(r["ID"], {"name": r["Kernel Name"]})
+        v = r["Metric Value"].replace(",", "")
+        d[r["Metric Name"]] = float(v)
+    per = {}
+    for d in launches.values():
+        c = kernel_class(d["name"])
+        if c is None or "dram__bytes_read.sum" not in d:
+            continue
+        per.setdefault(c, []).append(d)
+    try:
+        with open(path) as f:
+            doc = json.load(f)
+    except (OSError, ValueError):
+        doc = {"about": "DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum), "
+                        "mean over the captured launches of each kernel class; written by "
+                        "`bench.py --record-traffic`", "entries": {}}
+    out = {}
+    for c, ds in per.items():
+        rd = statistics.mean(d["dram__bytes_read.sum"] for d in ds)
+        wr = statistics.mean(d["dram__bytes_write.sum"] for d in ds)
+        ent = {"dram_bytes_per_launch": int(round(rd + wr)), "dram_bytes_read": int(round(rd)),
+               "dram_bytes_write": int(round(wr)), "launches": len(ds),
+               "kernel_names": sorted({d["name"].split("(")[0] for d in ds}),
+               "sources_sha16": source_hash(c), "command": command,
+               "recorded": datetime.date.today().isoformat()}
+        if all("gpu__time_duration.sum" in d for d in ds):
+            ent["ncu_duration_us_mean"] = statistics.mean(
+                d["gpu__time_duration.sum"] for d in ds) / 1e3
+        doc["entries"][f"{c}@{workload}"] = ent
+        out[c] = ent
+    with open(path, "w") as f:
+        json.dump(doc, f, indent=1, sort_keys=True)
+        f.write("\n")
+    return out
 
 
 class ClockSampler:
@@ -171,13 +300,37 @@ def dist_setup():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if ws > 1:
-        import datetime
         torch.cuda.set_device(local)
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local))
     elif torch.cuda.is_available():
         torch.cuda.set_device(local)
     return ws, rank, local
+
+
+def n_x_buffers(w: W.Workload) -> int:
+    """Copies of x the timed loop rotates through so that the router reads x from DRAM: enough
+    that the copies together exceed the L2 (the weights, streamed every step, evict them too)."""
+    xb = w.S * w.D * elt_bytes(w)
+    return int(min(1024, max(2, math.ceil(1.25 * L2_BYTES / max(xb, 1)))))
+
+
+def flush_l2_each_step(w: W.Workload) -> bool:
+    """Workloads whose inputs fit in the L2 are timed step by step with an L2 flush in between."""
+    return input_bytes(w) < 2 * L2_BYTES
+
+
+def workload_config(w: W.Workload, ws: int) -> dict:
+    """The `config` object of a bench line (the same for the GPU arm and the oracle arm)."""
+    if flush_l2_each_step(w):
+        l2 = ("inputs smaller than L2: a 256 MiB write flushes L2 before every step; steps timed "
+              "one by one with CUDA events, flushes excluded")
+    else:
+        l2 = (f"inputs larger than L2 (all expert weights streamed every step); x rotated over "
+              f"{n_x_buffers(w)} device copies")
+    return {"workload": w.name, **{k: getattr(w, k) for k in "SDFEk"},
+            "router": w.router_std, "zipf_s": w.zipf_s, "seed": "rank",
+            "parallelism": f"replicas{ws}", "l2": l2}
 
 
 def bench_reference(args, w, ws, rank):
@@ -203,8 +356,8 @@ def bench_reference(args, w, ws, rank):
         "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1000.0 * t_total / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, **{k: getattr(w, k) for k in "SDFEk"},
-                   "input_dtype": w.dtype},
+        "config": workload_config(w, ws),
+        "input_dtype": w.dtype,
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                          "sample": f"{per_step} seeded tokens of {w.S} per step"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -214,29 +367,55 @@ def bench_reference(args, w, ws, rank):
     return line
 
 
-def bench_ours(args, w, ws, rank, local):
-    import sparse_mixture_experts_02_b200 as moe
+def roofline(w: W.Workload, stage_ms: dict, e_act: int, clocks, timed_s: float):
+    """Roofline of the dominant kernel, GEMM1 (gathered x, fused gate+up, SwiGLU: two thirds of
+    the FLOPs and of the weight bytes). Both ceilings are computed; `bound` is the one whose
+    minimum time is longer at the measured peaks (the other is reported under `other`)."""
+    pk, pk_kind = peaks()
+    t = stage_ms["gemm1"] / 1000.0
+    flop = flops_of(w)["gemm1"]
+    nbytes = bytes_of(w, e_act)["gemm1"]
+    tf_peak, tf_kind = tensor_peak(w.dtype, clocks, timed_s)
+    tensor = {"bound": "tensor", "achieved": flop / t / 1e12, "peak": tf_peak,
+              "unit": "TFLOP/s", "frac": flop / t / 1e12 / tf_peak, "peak_kind": tf_kind}
+    hbm = {"bound": "hbm", "achieved": nbytes / t / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s",
+           "frac": nbytes / t / 1e9 / pk["hbm_gbs"], "peak_kind": f"{pk_kind} copy bandwidth"}
+    t_tensor = flop / (tf_peak * 1e12)
+    t_hbm = nbytes / (pk["hbm_gbs"] * 1e9)
+    main, other = (hbm, tensor) if t_hbm > t_tensor else (tensor, hbm)
+    return {"kernel": "gemm1_gateup_swiglu", **main,
+            "traffic": recorded_traffic("gemm1", w.name),
+            "algorithmic_bytes": nbytes, "flop": flop, "launch_ms": stage_ms["gemm1"],
+            "other": other}
 
-    dev = torch.device("cuda", local)
-    seed = rank  # every rank its own batch; rank 0 is the N=1 workload
+
+def time_forward(moe, w, steps, warmup, dev, ws=1, seed=0):
+    """Times `steps` forwards of workload w after `warmup` untimed ones. Returns the inputs, the
+    workspace, the output buffer and the measurements. Inputs larger than the L2 are timed as one
+    bracket of K steps (barrier + device sync on both sides, x rotated over several copies);
+    smaller ones step by step with an L2 flush before each step."""
     inp = W.make_inputs(w, device=dev, seed=seed)
     wsp = moe.ForwardWorkspace(w.S, w.D, w.F, w.E, w.k, inp["x"].dtype, dev)
     out = torch.empty((w.S, w.D), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
+    flush = flush_l2_each_step(w)
+    nx = 1 if flush else n_x_buffers(w)
+    xs = [inp["x"]] + [inp["x"].clone() for _ in range(nx - 1)]
+    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if flush else None
 
-    def step(events=None):
+    def step(i, events=None):
         if events is not None:
             moe.profile_events(events)
-        moe.mlp_forward(inp["x"], inp["w_gate"], inp["w_gate_e"], inp["w_up"], inp["w_down"],
+        moe.mlp_forward(xs[i % nx], inp["w_gate"], inp["w_gate_e"], inp["w_up"], inp["w_down"],
                         w.k, logit_bias=inp["logit_bias"], out=out, ws=wsp)
 
-    for _ in range(args.warmup):
-        step()
+    for i in range(warmup):
+        step(i)
     moe.check_device_status(wsp)
     launches_per_step = moe.last_launch_count()
 
     # events for the per-stage breakdown, 5 per step, created and recorded once up front
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
     for row in evs:
         for e in row:
             e.record(stream)
@@ -248,31 +427,60 @@ def bench_ours(args, w, ws, rank, local):
         if ws > 1:
             torch.distributed.barrier()
         torch.cuda.synchronize(dev)
-        t0.record(stream)
-        for i in range(args.steps):
-            step(evs[i])
-        t1.record(stream)
-        torch.cuda.synchronize(dev)
+        if flush:
+            ms_total = 0.0
+            for i in range(steps):
+                flush_buf.zero_()
+                step(i, evs[i])
+            torch.cuda.synchronize(dev)
+            ms_total = sum(r[0].elapsed_time(r[4]) for r in evs)
+        else:
+            t0.record(stream)
+            for i in range(steps):
+                step(i, evs[i])
+            t1.record(stream)
+            torch.cuda.synchronize(dev)
+            ms_total = t0.elapsed_time(t1)
         if ws > 1:
             torch.distributed.barrier()
-    ms_total = t0.elapsed_time(t1)
     moe.check_device_status(wsp)
     if ws > 1:
         t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         ms_total = float(t.item())
-    stage = {"route": [], "sparse_map": [], "gemm1": [], "gemm2": []}
-    for row in evs:
-        stage["route"].append(row[0].elapsed_time(row[1]))
-        stage["sparse_map"].append(row[1].elapsed_time(row[2]))
-        stage["gemm1"].append(row[2].elapsed_time(row[3]))
-        stage["gemm2"].append(row[3].elapsed_time(row[4]))
-    stage_ms = {k: sum(v) / len(v) for k, v in stage.items()}
+    stage_ms = {n: sum(r[q].elapsed_time(r[q + 1]) for r in evs) / steps
+                for q, n in enumerate(STAGES)}
+    counts = wsp.view("expert_counts").cpu()
+    e_act = int((counts > 0).sum())
+    hist = {"max": int(counts.max()) if w.E else 0, "min": int(counts.min()) if w.E else 0,
+            "empty": int((counts == 0).sum()), "mean": float(counts.float().mean())}
+    clocks = clk.summary()
+    s_per_step = ms_total / 1000.0 / steps
+    fl = flops_of(w)
+    by = bytes_of(w, e_act)
+    meas = {
+        "ms_per_step": ms_total / steps,
+        "tokens_per_s": w.S * ws / s_per_step,
+        "tflops": sum(fl.values()) / s_per_step / 1e12,
+        "gbs": sum(by.values()) / s_per_step / 1e9,
+        "stage_ms": stage_ms,
+        "stage_gbs": {n: by[n] / (stage_ms[n] / 1000.0) / 1e9 for n in STAGES if stage_ms[n] > 0},
+        "expert_hist": hist,
+        "roofline": roofline(w, stage_ms, e_act, clocks, ms_total / 1000.0),
+        "clocks": clocks,
+        "gpu_launches": launches_per_step * steps,
+        "x_buffers": nx,
+        "timed_s": ms_total / 1000.0,
+    }
+    return inp, wsp, out, meas
 
-    # End to end: every step copies its x in from pinned host memory and its fp32 out back to
-    # pinned host memory, inside the timed region. The copies run on two side streams with two
-    # device buffers each, so step i's forward overlaps step i+1's input copy and step i-1's
-    # output copy (a pipelined caller); the timed region ends when the last output has landed.
+
+def e2e_measure(moe, w, inp, wsp, out, steps, warmup, dev, ws=1):
+    """End to end: every step copies its x in from pinned host memory and its fp32 out back to
+    pinned host memory, inside the timed region. The copies run on two side streams with two
+    device buffers each, so step i's forward overlaps step i+1's input copy and step i-1's output
+    copy (a pipelined caller); the timed region ends when the last output has landed."""
+    stream = torch.cuda.current_stream(dev)
     x_host = inp["x"].cpu().pin_memory()
     out_host = [torch.empty((w.S, w.D), dtype=torch.float32).pin_memory() for _ in range(2)]
     x_dev = [torch.empty_like(inp["x"]) for _ in range(2)]
@@ -303,7 +511,7 @@ def bench_ours(args, w, ws, rank, local):
             out_read[b] = torch.cuda.Event()
             out_read[b].record(d2h)
 
-    for i in range(args.warmup):
+    for i in range(warmup):
         e2e_step(i)
     torch.cuda.synchronize(dev)
     e0 = torch.cuda.Event(enable_timing=True)
@@ -313,9 +521,9 @@ def bench_ours(args, w, ws, rank, local):
     torch.cuda.synchronize(dev)
     e0.record(stream)
     h2d.wait_event(e0)
-    for i in range(args.steps):
+    for i in range(steps):
         e2e_step(i)
-    stream.wait_event(out_read[(args.steps - 1) & 1])
+    stream.wait_event(out_read[(steps - 1) & 1])
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1)
@@ -324,59 +532,76 @@ def bench_ours(args, w, ws, rank, local):
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         e2e_ms = float(t.item())
     # the pipelined copies must reproduce the device result of the same input
-    b_last = (args.steps - 1) & 1
+    b_last = (steps - 1) & 1
     torch.testing.assert_close(out_host[b_last], out_dev[b_last].cpu(), rtol=0, atol=0)
+    return {"value": w.S * ws / (e2e_ms / 1000.0 / steps), "unit": "tokens/s",
+            "copies": "pinned host, two side streams, double-buffered, overlapping the forwards",
+            "h2d_bytes_per_step": w.S * w.D * inp["x"].element_size(),
+            "d2h_bytes_per_step": w.S * w.D * 4}
 
-    counts = wsp.view("expert_counts").cpu()
-    hist = {"max": int(counts.max()), "min": int(counts.min()),
-            "empty": int((counts == 0).sum()), "mean": float(counts.float().mean())}
 
+def workload_entry(w, meas):
+    """One entry of the `workloads` object: the measurements plus the fractions of peak."""
+    pk, pk_kind = peaks()
+    tf_peak, tf_kind = tensor_peak(w.dtype, meas["clocks"], meas["timed_s"])
+    return {"config": {k: getattr(w, k) for k in ("S", "D", "F", "E", "k", "dtype",
+                                                   "router_std", "zipf_s")},
+            "ms_per_step": meas["ms_per_step"], "tokens_per_s": meas["tokens_per_s"],
+            "tflops": meas["tflops"], "gbs": meas["gbs"],
+            "tflops_frac": {"of_measured_peak": meas["tflops"] / tf_peak, "peak_kind": tf_kind,
+                            "of_nominal": meas["tflops"] / NOMINAL_TFLOPS[w.dtype]},
+            "gbs_frac": {"of_measured": meas["gbs"] / pk["hbm_gbs"],
+                         "of_nominal": meas["gbs"] / NOMINAL_HBM_GBS},
+            "stage_ms": meas["stage_ms"], "stage_gbs": meas["stage_gbs"],
+            "expert_hist": meas["expert_hist"], "roofline": meas["roofline"],
+            "clocks": meas["clocks"], "gpu_launches": meas["gpu_launches"],
+            "l2": workload_config(w, 1)["l2"]}
+
+
+def bench_ours(args, w, ws, rank, local):
+    import sparse_mixture_experts_02_b200 as moe
+
+    dev = torch.device("cuda", local)
+    seed = rank  # every rank its own batch; rank 0 is the N=1 workload
+    inp, wsp, out, meas = time_forward(moe, w, args.steps, args.warmup, dev, ws=ws, seed=seed)
+    e2e = e2e_measure(moe, w, inp, wsp, out, args.steps, args.warmup, dev, ws=ws)
     if rank != 0:
         return None
-
-    fl = flops_of(w)
-    flop_step = sum(fl.values())
-    s_per_step = ms_total / 1000.0 / args.steps
-    tokens_per_s = w.S * ws / s_per_step
-    tflops = flop_step / s_per_step / 1e12
     pk, pk_kind = peaks()
-    dt = w.dtype
-    ratio = 1.0 if dt == "bf16" else NOMINAL_TFLOPS["f32"] / NOMINAL_TFLOPS["bf16"]
-    peak_burst = pk["bf16_tflops"] * ratio
-    peak_sust = pk["bf16_tflops_sustained"] * ratio
-    map_bytes = w.R * 4 + 2 * w.R * 4 + (2 * w.E + 1) * 4
-    g1_tflops = fl["gemm1"] / (stage_ms["gemm1"] / 1000.0) / 1e12
-    key = f"gemm1_gateup_swiglu@{w.name}"
+    tf_peak, tf_kind = tensor_peak(w.dtype, meas["clocks"], meas["timed_s"])
     line = {
-        "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": ws,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_total / args.steps,
+        "metric": METRIC, "value": meas["tokens_per_s"], "unit": "tokens/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": meas["ms_per_step"],
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": dt, "data": "synthetic",
-        "config": {"workload": w.name, **{k: getattr(w, k) for k in "SDFEk"},
-                   "router": w.router_std, "zipf_s": w.zipf_s, "seed": "rank",
-                   "parallelism": f"replicas{ws}",
-                   "l2": "inputs larger than L2 (all expert weights streamed every step)"},
-        "tflops": tflops,
-        "tflops_frac": {"of_measured_sustained": tflops / peak_sust,
-                        "of_measured_burst": tflops / peak_burst,
-                        "of_nominal": tflops / NOMINAL_TFLOPS[dt], "peaks": pk_kind},
-        "stage_ms": stage_ms,
-        "sparse_map_gbs": map_bytes / (stage_ms["sparse_map"] / 1000.0) / 1e9,
-        "expert_hist": hist,
-        "roofline": {"kernel": "gemm1_gateup_swiglu", "bound": "tensor", "achieved": g1_tflops,
-                     "peak": peak_sust, "unit": "TFLOP/s", "frac": g1_tflops / peak_sust,
-                     "peak_kind": f"{pk_kind} sustained bf16"
-                                  + ("" if dt == "bf16" else " x tf32/bf16 nominal ratio"),
-                     "traffic": recorded_traffic(key)},
-        "e2e": {"value": w.S * ws / (e2e_ms / 1000.0 / args.steps), "unit": "tokens/s",
-                "copies": "pinned host, two side streams, double-buffered, overlapping the forwards",
-                "h2d_bytes_per_step": w.S * w.D * inp["x"].element_size(),
-                "d2h_bytes_per_step": w.S * w.D * 4},
-        "gpu_launches": launches_per_step * args.steps,
-        "clocks": clk.summary(),
+        "dtype": w.dtype, "data": "synthetic",
+        "config": workload_config(w, ws),
+        "tflops": meas["tflops"],
+        "tflops_frac": {"of_measured_peak": meas["tflops"] / tf_peak, "peak_kind": tf_kind,
+                        "of_nominal": meas["tflops"] / NOMINAL_TFLOPS[w.dtype]},
+        "gbs": meas["gbs"],
+        "stage_ms": meas["stage_ms"], "stage_gbs": meas["stage_gbs"],
+        "sparse_map_gbs": meas["stage_gbs"].get("sparse_map"),
+        "expert_hist": meas["expert_hist"],
+        "roofline": meas["roofline"],
+        "e2e": e2e,
+        "gpu_launches": meas["gpu_launches"],
+        "clocks": meas["clocks"],
     }
+    del inp, wsp, out
+    if ws == 1 and not args.no_workloads:
+        # every other configuration, timed the same way (one GPU; parity cases, not bench lines)
+        others = {}
+        for name in W.WORKLOADS:
+            if name == w.name:
+                continue
+            wl = W.WORKLOADS[name]
+            i2, ws2, o2, m2 = time_forward(moe, wl, args.steps, args.warmup, dev)
+            others[name] = workload_entry(wl, m2)
+            del i2, ws2, o2
+            torch.cuda.empty_cache()
+        line["workloads"] = others
     if ws == 1 and not args.no_cpu_baseline:
-        inp_cpu = host_inputs(inp)
+        inp_cpu = host_inputs(W.make_inputs(w, device=dev, seed=0))
         n = calibrate_oracle(w, inp_cpu, args.cpu_budget_s)
         t, ntok, cores = run_oracle_sample(w, inp_cpu, n)
         line["cpu_baseline"] = {"value": ntok / t, "unit": "tokens/s", "cores": cores,
@@ -482,7 +707,8 @@ def backward_bench(args, w):
              for q, n in enumerate(names)}
     R = w.S * w.k
     flop = 12.0 * R * w.D * w.F + 2.0 * w.S * w.D * w.E + 2.0 * w.S * w.k * w.D
-    pk, pk_kind = peaks()
+    clocks = clk.summary()
+    tf_peak, tf_kind = tensor_peak(w.dtype, clocks, ms * args.steps / 1e3)
     tflops = flop / (ms * 1e-3) / 1e12
     return {"metric": "MoE-layer backward tokens/s and TFLOP/s (bf16)", "value": w.S / (ms * 1e-3),
             "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
@@ -490,20 +716,19 @@ def backward_bench(args, w):
             "config": {"workload": w.name, "S": w.S, "D": w.D, "F": w.F, "E": w.E, "k": w.k,
                        "l2": "inputs larger than L2 (all expert weights streamed every step)"},
             "tflops": tflops, "flop_per_step": flop,
-            "tflops_frac": {"of_measured_sustained": tflops / pk["bf16_tflops_sustained"],
-                            "of_nominal": tflops / 2250.0, "peaks": pk_kind},
+            "tflops_frac": {"of_measured_peak": tflops / tf_peak, "peak_kind": tf_kind,
+                            "of_nominal": tflops / 2250.0},
             "extra_flop_recompute": 4.0 * R * w.D * w.F, "stage_ms": stage,
             # dominant stage: the weight gradients of the gate and up projections (two grouped
             # weight-gradient GEMMs, 2 R D F FLOPs each)
             "roofline": {"kernel": "dW_gate_e_and_dW_up (grouped_wgrad_kernel x2)",
                          "bound": "tensor",
                          "achieved": 4.0 * R * w.D * w.F / (stage["dW_gate_e_and_dW_up"] * 1e-3) / 1e12,
-                         "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                         "peak": tf_peak, "unit": "TFLOP/s",
                          "frac": 4.0 * R * w.D * w.F / (stage["dW_gate_e_and_dW_up"] * 1e-3) / 1e12
-                         / pk["bf16_tflops_sustained"],
-                         "peak_kind": "measured sustained bf16" if pk_kind == "measured" else pk_kind,
-                         "traffic": None},
-            "gpu_launches": launches * args.steps, "clocks": clk.summary()}
+                         / tf_peak,
+                         "peak_kind": tf_kind, "traffic": None},
+            "gpu_launches": launches * args.steps, "clocks": clocks}
 
 
 def ep_bench(args, w):
@@ -570,6 +795,8 @@ def ep_bench(args, w):
             return None
         fl = flops_of(w)
         flop = ws * (fl["router"] + fl["gemm1"] + fl["gemm2"])
+        clocks = clk.summary()
+        tf_peak, tf_kind = tensor_peak(w.dtype, clocks, ms_max * args.steps / 1e3)
         return {"metric": "expert-parallel MoE-layer fwd tokens/s (bf16)",
                 "value": ws * w.S / (ms_max * 1e-3), "unit": "tokens/s", "n_gpus": ws,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
@@ -583,11 +810,10 @@ def ep_bench(args, w):
                 "roofline": {"kernel": "experts (grouped GEMMs on received rows, rank 0)",
                              "bound": "tensor",
                              "achieved": (fl["gemm1"] + fl["gemm2"]) / (stage["experts"] * 1e-3) / 1e12,
-                             "peak": peaks()[0]["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                             "peak": tf_peak, "unit": "TFLOP/s",
                              "frac": (fl["gemm1"] + fl["gemm2"]) / (stage["experts"] * 1e-3) / 1e12
-                             / peaks()[0]["bf16_tflops_sustained"],
-                             "traffic": None},
-                "clocks": clk.summary()}
+                             / tf_peak, "peak_kind": tf_kind, "traffic": None},
+                "clocks": clocks}
     finally:
         torch.distributed.destroy_process_group()
 
@@ -645,7 +871,8 @@ def moa_bench(args, w):
              for q, n in enumerate(names)}
     fl = moa_flops(w)
     flop = sum(fl.values())
-    pk, pk_kind = peaks()
+    clocks = clk.summary()
+    tf_peak, tf_kind = tensor_peak("bf16", clocks, ms * args.steps / 1e3)
     tflops = flop / (ms * 1e-3) / 1e12
     att = fl["attention"] / (stage["attention"] * 1e-3) / 1e12
     return {"metric": "MoA-layer fwd tokens/s and TFLOP/s (bf16)", "value": w.S / (ms * 1e-3),
@@ -654,12 +881,12 @@ def moa_bench(args, w):
             "config": {"workload": w.name, "S": w.S, "D": w.D, "H": w.H, "dh": w.dh, "E": w.E,
                        "k": w.k, "l2": "inputs larger than L2 (expert weights streamed)"},
             "tflops": tflops, "flop_per_step": flop, "flop_by_stage": fl,
-            "tflops_frac": {"of_measured_sustained": tflops / pk["bf16_tflops_sustained"],
-                            "of_nominal": tflops / 2250.0, "peaks": pk_kind},
+            "tflops_frac": {"of_measured_peak": tflops / tf_peak, "peak_kind": tf_kind,
+                            "of_nominal": tflops / 2250.0},
             "roofline": {"kernel": "attention core", "bound": "tensor", "achieved": att,
-                         "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-                         "frac": att / pk["bf16_tflops"], "traffic": None},
-            "stage_ms": stage, "gpu_launches": launches * args.steps, "clocks": clk.summary(),
+                         "peak": tf_peak, "unit": "TFLOP/s", "frac": att / tf_peak,
+                         "peak_kind": tf_kind, "traffic": None},
+            "stage_ms": stage, "gpu_launches": launches * args.steps, "clocks": clocks,
             "cpu_baseline": None if args.no_cpu_baseline else moa_oracle_baseline(w, inp,
                                                                                   args.cpu_budget_s)}
 
@@ -709,7 +936,18 @@ def main():
                          "split over the ranks (all-to-all dispatch and combine over NCCL)")
     ap.add_argument("--map-points", default="",
                     help="with --map-sweep: only these points, 'log2R:E,...' (e.g. 26:256)")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="headline workload only (no `workloads` object with the other configs)")
+    ap.add_argument("--record-traffic", default="", metavar="CSV",
+                    help="instead of timing: record the DRAM bytes per launch of each kernel "
+                         "class in an ncu CSV into profiles/dram_traffic.json for --workload")
+    ap.add_argument("--traffic-command", default="",
+                    help="with --record-traffic: the ncu command line that wrote the CSV")
     args = ap.parse_args()
+    if args.record_traffic:
+        out = record_traffic(args.record_traffic, args.workload, args.traffic_command)
+        print(json.dumps(out, indent=1))
+        return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.map_sweep:

@@ -110,7 +110,10 @@ int moe_sparse_map(const int32_t *top_experts, int64_t S, int32_t k, int32_t E,
  * (ceil(S*k / 4096) + 1) * E * 4 <= 1 MiB (for example S*k <= 4190208 routes at E = 256); larger
  * sizes are rejected with MOE_ERR_INVALID_ARG before any launch. The call allocates nothing.
  * The first call on a device looks up the array's device address (with that device current);
- * make that first call before any stream capture. All calls share the array, which keeps the
+ * make that first call before any stream capture. Under CUDA's lazy module loading (the default)
+ * that first call may also be what loads this library's device code on the device, and with it
+ * what reserves the fixed array in device memory: make it before a memory pool takes the rest
+ * of the device. All calls share the array, which keeps the
  * last call's contents; calls whose kernels overlap on the GPU (e.g. on two streams) race on it
  * and must be serialised by the caller. An expert id outside [0,E) is not counted and gets
  * sparse_rows[i] = -1; this call reports no device status, so such ids show as

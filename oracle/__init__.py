@@ -44,6 +44,7 @@ def lib():
         L.oracle_sparse_map.argtypes = [P, i64, i32, P, P, P, P]
         L.oracle_sparse_map.restype = ctypes.c_int
         L.oracle_expert_hidden.argtypes = [P, P, P, i64, i64, i32, i32, P]
+        L.oracle_expert_hidden_rows.argtypes = [P, P, P, i64, i64, P, P, i64, P]
         L.oracle_mlp_forward.argtypes = [P, P, P, P, P, P, i64, i64, i32, i32, P, i64, P, P, P, P]
         L.oracle_scatter_linear.argtypes = [P, P, i64, i64, i64, i32, i32, P, P, P, ctypes.c_int,
                                             ctypes.c_int, P]
@@ -140,6 +141,19 @@ def expert_hidden(x, w_gate_e, w_up, token, expert):
     F = wge.shape[2]
     h = np.zeros(F, dtype=np.float64)
     lib().oracle_expert_hidden(_p(x), _p(wge), _p(wu), D, F, int(token), int(expert), _p(h))
+    return h
+
+
+def expert_hidden_rows(x, w_gate_e, w_up, tokens, experts):
+    """expert_hidden for n (token, expert) pairs at once (rows in parallel): h [n, F]."""
+    x, wge, wu = _f32(x), _f32(w_gate_e), _f32(w_up)
+    tokens, experts = _i32(tokens).reshape(-1), _i32(experts).reshape(-1)
+    assert tokens.shape == experts.shape
+    D = x.shape[1]
+    F = wge.shape[2]
+    h = np.zeros((tokens.shape[0], F), dtype=np.float64)
+    lib().oracle_expert_hidden_rows(_p(x), _p(wge), _p(wu), D, F, _p(tokens), _p(experts),
+                                    tokens.shape[0], _p(h))
     return h
 
 

@@ -181,6 +181,15 @@ void oracle_expert_hidden(const float *x, const float *w_gate_e, const float *w_
     free(u);
 }
 
+/* The same hidden row for n (token, expert) pairs, h [n, F]; the rows are independent. */
+void oracle_expert_hidden_rows(const float *x, const float *w_gate_e, const float *w_up,
+                               int64_t D, int64_t F, const int32_t *tokens,
+                               const int32_t *experts, int64_t n, double *h) {
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t i = 0; i < n; ++i)
+        oracle_expert_hidden(x, w_gate_e, w_up, D, F, tokens[i], experts[i], h + i * F);
+}
+
 /* Forward for the listed tokens: y[s] = sum_j w_j * FFN_{J_j}(x[s]) with
  * FFN_e(v) = (silu(v W_gate_e[e]) * (v W_up[e])) W_down[e], W_down[e] of shape [F,D].
  * If given_top_experts ([S,k], indexed by token) is non-null, its experts replace the oracle's

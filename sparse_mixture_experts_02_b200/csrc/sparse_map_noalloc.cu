@@ -10,7 +10,9 @@
 // The array (kNoallocScratchBytes of map scratch plus a 256-byte status area) exists once per
 // device that loads the library and stays allocated until the process exits. Its device address
 // is looked up once per device, with that device current, on the first call on that device; make
-// that first call before any stream capture. Every call shares the one array and it keeps the
+// that first call before any stream capture. With CUDA's lazy module loading (the default), that
+// first call may be what loads this module on the device and so reserves the array: make it
+// before a memory pool reserves the rest of the device. Every call shares the one array and it keeps the
 // last call's contents: the map kernels overwrite every scratch word they later read, and the
 // status word is cleared by each call. Two calls whose kernels overlap on the GPU (for example on
 // two streams) race on the array and must be serialised by the caller.

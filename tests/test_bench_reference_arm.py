@@ -22,6 +22,11 @@ def test_reference_arm_json_line():
     assert d["value"] > 0 and d["unit"] == "tokens/s" and d["higher_is_better"] is True
     assert d["steps"] == 1 and d["warmup"] == 3 and d["n_gpus"] == 1
     assert d["config"]["workload"] == "mixtral_prefill"
+    # the same config object as the GPU arm's line, so the two lines describe one workload
+    sys.path.insert(0, ROOT)
+    import bench
+    import moe_workloads as W
+    assert d["config"] == bench.workload_config(W.WORKLOADS["mixtral_prefill"], 1)
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"]
     assert cb["sample"]

@@ -425,6 +425,12 @@ def test_expert_hidden_matches_numpy(oracle_lib):
         h = oracle_lib.expert_hidden(inp["x"], inp["w_gate_e"], inp["w_up"], s, e)
         ref = _silu_np(x[s] @ _np(inp["w_gate_e"][e])) * (x[s] @ _np(inp["w_up"][e]))
         assert np.allclose(h, ref, rtol=1e-12, atol=1e-15)
+    # the batched form returns the same rows, in the order of the pairs
+    toks, exps = np.array([4, 0, 9, 4], np.int32), np.array([1, 0, 2, 2], np.int32)
+    hb = oracle_lib.expert_hidden_rows(inp["x"], inp["w_gate_e"], inp["w_up"], toks, exps)
+    for i in range(4):
+        assert np.array_equal(hb[i], oracle_lib.expert_hidden(inp["x"], inp["w_gate_e"],
+                                                              inp["w_up"], toks[i], exps[i]))
 
 
 # ----------------------------------------------------------------------------------------------
