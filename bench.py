@@ -79,7 +79,7 @@ def bytes_of(w: W.Workload, e_act: int) -> dict:
     R = w.R
     return {
         # x read, W_gate read, top experts and weights written
-        "router": w.S * w.D * b + w.D * w.E * b + 8 * R,
+        "route": w.S * w.D * b + w.D * w.E * b + 8 * R,
         # routes read, slots and inverse permutation written, counts and offsets written
         "sparse_map": 12 * R + (2 * w.E + 1) * 4,
         # x read, gate and up weights of active experts read, h written, out zeroed
