@@ -59,7 +59,8 @@ typedef enum {
     MOE_ERR_WORKSPACE = -3,      /* ws is null, misaligned or smaller than moe_workspace_size */
     MOE_ERR_CUDA = -4,           /* a CUDA runtime / driver call failed */
     MOE_ERR_BAD_EXPERT_ID = -5,  /* device saw an expert id outside [0, E) */
-    MOE_ERR_DEVICE_TIMEOUT = -6  /* a bounded device-side wait ran out; the kernel returned */
+    MOE_ERR_DEVICE_TIMEOUT = -6, /* a bounded device-side wait ran out; the kernel returned */
+    MOE_ERR_BAD_INDEX = -7       /* debug build only: a device bounds check skipped an index */
 } moe_status;
 
 typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
@@ -314,9 +315,22 @@ const char *moe_last_error(void);
 
 /*
  * Synchronises `stream`, reads the status word in `ws` and returns MOE_OK,
- * MOE_ERR_BAD_EXPERT_ID or MOE_ERR_DEVICE_TIMEOUT (or MOE_ERR_CUDA). Off the hot path.
+ * MOE_ERR_BAD_EXPERT_ID, MOE_ERR_DEVICE_TIMEOUT or, from the debug build, MOE_ERR_BAD_INDEX
+ * (or MOE_ERR_CUDA). Off the hot path.
  */
 int moe_check_device_status(void *ws, moe_stream_t stream);
+
+/*
+ * 1 in the debug build of this library (libmoe_b200_debug.so, compiled with MOE_DEBUG=1), 0 in
+ * the release build. The debug build has the same entry points and results; in addition every
+ * index a kernel takes from its inputs before addressing memory with it (a gathered token row
+ * sorted_rows[p] / k, a slot, a route, the expert offsets behind a tile schedule) is checked
+ * against its range. An index outside it skips that access (the row is not read or written;
+ * out-of-range expert offsets empty the schedule) and sets MOE_ERR_BAD_INDEX in the status word
+ * read by moe_check_device_status. Nothing traps. This stands in for a memory sanitizer, which
+ * is not available where this library was measured. Not an operation of the pages.
+ */
+int moe_debug_build(void);
 
 /*
  * Optional per-stage timing on the calling host thread: when `events` holds n cudaEvent_t

@@ -17,18 +17,20 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "_lib", "libmoe_b200.so")
+# the same library built with MOE_DEBUG=1: device bounds checks on every index read from inputs
+DEBUG_LIB_PATH = os.path.join(_HERE, "_lib", "libmoe_b200_debug.so")
 
 MOE_F32, MOE_BF16 = 0, 1
 STATUS_NAMES = {0: "MOE_OK", -1: "MOE_ERR_INVALID_ARG", -2: "MOE_ERR_UNSUPPORTED",
                 -3: "MOE_ERR_WORKSPACE", -4: "MOE_ERR_CUDA", -5: "MOE_ERR_BAD_EXPERT_ID",
-                -6: "MOE_ERR_DEVICE_TIMEOUT"}
+                -6: "MOE_ERR_DEVICE_TIMEOUT", -7: "MOE_ERR_BAD_INDEX"}
 
 EXPORTS = ["moe_route_topk", "moe_sparse_map", "moe_sparse_map_noalloc", "moe_scatter_linear",
            "moe_scatter_linear_backward", "moe_mlp_forward", "moe_mlp_backward",
            "moe_moa_forward", "moe_ep_dispatch", "moe_expert_mlp_forward", "moe_ep_combine",
            "moe_cast_bf16", "moe_workspace_size", "moe_workspace_view", "moe_last_error",
            "moe_check_device_status", "moe_profile_events", "moe_debug_wait_timeout",
-           "moe_last_launch_count"]
+           "moe_last_launch_count", "moe_debug_build"]
 
 
 class MoeError(RuntimeError):
@@ -37,12 +39,13 @@ class MoeError(RuntimeError):
         self.code = code
 
 
-def _load():
-    if not os.path.exists(LIB_PATH):
+def _load(path: str = None):
+    path = path or LIB_PATH
+    if not os.path.exists(path):
         raise ImportError(
-            f"{LIB_PATH} is missing: build it with `python -m sparse_mixture_experts_02_b200.build`"
+            f"{path} is missing: build it with `python -m sparse_mixture_experts_02_b200.build`"
             " (the library has no fallback path)")
-    lib = ctypes.CDLL(LIB_PATH)
+    lib = ctypes.CDLL(path)
     P, i64, i32, c_int = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int
     lib.moe_route_topk.argtypes = [P, P, P, i64, i64, i32, i32, c_int, P, P, P]
     lib.moe_sparse_map.argtypes = [P, i64, i32, i32, P, P, P, P, P, ctypes.c_size_t, P]
@@ -76,9 +79,17 @@ def _load():
                  "moe_mlp_backward", "moe_moa_forward", "moe_ep_dispatch",
                  "moe_expert_mlp_forward", "moe_ep_combine", "moe_cast_bf16",
                  "moe_check_device_status", "moe_profile_events", "moe_debug_wait_timeout",
-                 "moe_last_launch_count"):
+                 "moe_last_launch_count", "moe_debug_build"):
         getattr(lib, name).restype = c_int
     return lib
+
+
+def debug_lib():
+    """The debug build (libmoe_b200_debug.so) as a separate ctypes handle with the same entry
+    points: every index its kernels read from their inputs is bounds-checked on the device, and
+    one outside its range is skipped and reported as MOE_ERR_BAD_INDEX by
+    moe_check_device_status. The module's own calls keep using the release build."""
+    return _load(DEBUG_LIB_PATH)
 
 
 _LIB = None

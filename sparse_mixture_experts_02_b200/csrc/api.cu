@@ -479,11 +479,11 @@ int moe_scatter_linear_backward(const void *X, const void *W, const void *dY, in
     if (dW != nullptr) {
         // B: the gated dY rows in the padded layout; A: the input rows in slot order
         launch_gate_rows(dY, !scatter_out, sorted_rows, top_weights, k, R, Dout, scatter_out != 0,
-                         at<void>(ws, L.dv), expert_offsets, E, s);
+                         at<void>(ws, L.dv), expert_offsets, E, status, s);
         launch_zero_pad_rows(at<void>(ws, L.dv), Dout, Dout, expert_offsets, E, s);
         const void *As = X;
         if (gather_in) {
-            launch_gather_rows(X, sorted_rows, k, R, Din, at<void>(ws, L.xs), s);
+            launch_gather_rows(X, sorted_rows, k, R, Din, at<void>(ws, L.xs), status, s);
             As = at<void>(ws, L.xs);
             ++n;
         }
@@ -518,7 +518,7 @@ int moe_scatter_linear_backward(const void *X, const void *W, const void *dY, in
             return rc;
         launch_zero_f32(dgates, R, nullptr, s);
         launch_rowdot(dY, !scatter_out, at<void>(ws, L.v), sorted_rows, k, R, Dout,
-                      scatter_out != 0, dgates, s);
+                      scatter_out != 0, dgates, status, s);
         n += 3;
     }
     g_launches = n;
@@ -643,8 +643,13 @@ int moe_check_device_status(void *ws, moe_stream_t stream) {
         return set_error(MOE_ERR_DEVICE_TIMEOUT, "a device wait ran out (kernel id %u)", (v >> 8) & 0xFFu);
     if (v & kStatusBadExpert)
         return set_error(MOE_ERR_BAD_EXPERT_ID, "an expert id outside [0, E) was seen");
+    if (v & kStatusBadIndex)
+        return set_error(MOE_ERR_BAD_INDEX,
+                         "a device bounds check skipped an index outside its range");
     return MOE_OK;
 }
+
+int moe_debug_build(void) { return kDebugChecks ? 1 : 0; }
 
 int moe_debug_wait_timeout(int64_t limit_ns, void *ws, size_t ws_bytes, moe_stream_t stream) {
     g_launches = 0;
@@ -777,7 +782,7 @@ extern "C" int moe_mlp_backward(const void *x, const void *w_gate, const void *w
     n += 3;
     record_prof(2, s);
     // dW_down[e] = sum over e's slots of h_p^T (w_i dout[s])
-    launch_gate_rows(dout, false, sorted_rows, top_w, k, R, D, true, dv, offsets, E, s);
+    launch_gate_rows(dout, false, sorted_rows, top_w, k, R, D, true, dv, offsets, E, status, s);
     launch_zero_pad_rows(dv, D, D, offsets, E, s);
     {
         WgradArgs w{};
@@ -817,7 +822,7 @@ extern "C" int moe_mlp_backward(const void *x, const void *w_gate, const void *w
     record_prof(4, s);
     // dW_gate_e, dW_up from the x rows in slot order and the two halves of [da | db]
     void *xs = at<void>(ws, L.xs);
-    launch_gather_rows(x, sorted_rows, k, R, D, xs, s);
+    launch_gather_rows(x, sorted_rows, k, R, D, xs, status, s);
     ++n;
     for (int half = 0; half < 2; ++half) {
         WgradArgs w{};
@@ -1029,7 +1034,7 @@ int moe_ep_dispatch(const void *x, const int32_t *top_experts, int64_t S, int64_
     if ((rc = check_launch("sparse_map"))) return rc;
     if (R > 0) {
         launch_ep_pack(x, (size_t)D * esize(dt), top_experts, sorted_rows, expert_offsets, E, k,
-                       R, send_x, send_e, s);
+                       R, send_x, send_e, status, s);
         ++n;
     }
     g_launches = n;

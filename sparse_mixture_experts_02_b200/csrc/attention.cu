@@ -316,6 +316,9 @@ moa_attention_tc_kernel(const __grid_constant__ CUtensorMap tmKV, const Params p
         auto slot_of = [&](int64_t pair) {
             const int64_t i = (2 * pair + x) * BM + row;
             const int32_t sl = i < p.R ? __ldg(p.sparse_rows + i) : -1;
+            // -1 marks a route without a slot (its expert id was out of range); debug builds flag
+            // any other slot outside [0, R)
+            if (sl != -1 && !dev::debug_in_range(sl, p.R, p.status)) return (int64_t)-1;
             return (sl >= 0 && sl < p.R) ? (int64_t)sl : (int64_t)-1;
         };
         // this thread's row of Q for (pair, head) -> this group's Q tile (zeros without a slot)

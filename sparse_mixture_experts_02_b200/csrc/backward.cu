@@ -73,11 +73,12 @@ __global__ void __launch_bounds__(kWarps * 32)
 gate_rows_kernel(const void *__restrict__ dY, bool dy_bf16, const int32_t *__restrict__ sorted_rows,
                  const float *__restrict__ gates, int32_t k, int64_t R, int64_t Dout,
                  bool by_token, __nv_bfloat16 *__restrict__ dv,
-                 const int32_t *__restrict__ pad_offsets, int32_t E) {
+                 const int32_t *__restrict__ pad_offsets, int32_t E, unsigned *status) {
     const int lane = threadIdx.x & 31;
     const int64_t wstride = (int64_t)gridDim.x * kWarps;
     for (int64_t p = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5); p < R; p += wstride) {
         const int32_t i = __ldg(sorted_rows + p);
+        if (!dev::debug_in_range(i, R, lane == 0 ? status : nullptr)) continue;
         const float g = gates != nullptr ? __ldg(gates + i) : 1.0f;
         const int64_t row = by_token ? (int64_t)(i / k) : p;
         const uint8_t *src = static_cast<const uint8_t *>(dY) + row * Dout * (dy_bf16 ? 2 : 4);
@@ -96,11 +97,12 @@ gate_rows_kernel(const void *__restrict__ dY, bool dy_bf16, const int32_t *__res
 __global__ void __launch_bounds__(kWarps * 32)
 rowdot_kernel(const void *__restrict__ dY, bool dy_bf16, const __nv_bfloat16 *__restrict__ v,
               const int32_t *__restrict__ sorted_rows, int32_t k, int64_t R, int64_t Dout,
-              bool by_token, float *__restrict__ dg) {
+              bool by_token, float *__restrict__ dg, unsigned *status) {
     const int lane = threadIdx.x & 31;
     const int64_t wstride = (int64_t)gridDim.x * kWarps;
     for (int64_t p = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5); p < R; p += wstride) {
         const int32_t i = __ldg(sorted_rows + p);
+        if (!dev::debug_in_range(i, R, lane == 0 ? status : nullptr)) continue;
         const int64_t row = by_token ? (int64_t)(i / k) : p;
         const uint8_t *src = static_cast<const uint8_t *>(dY) + row * Dout * (dy_bf16 ? 2 : 4);
         float acc = 0.f;
@@ -178,11 +180,13 @@ __global__ void zero_pad_rows_kernel(uint4 *__restrict__ rows, int64_t ld16, int
 // xs[p] = x[sorted_rows[p] / k], bf16 rows of D elements, one warp per slot.
 __global__ void __launch_bounds__(kWarps * 32)
 gather_rows_kernel(const uint4 *__restrict__ x, const int32_t *__restrict__ sorted_rows, int32_t k,
-                   int64_t R, int64_t d16, uint4 *__restrict__ xs) {
+                   int64_t R, int64_t d16, uint4 *__restrict__ xs, unsigned *status) {
     const int lane = threadIdx.x & 31;
     const int64_t wstride = (int64_t)gridDim.x * kWarps;
     for (int64_t p = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5); p < R; p += wstride) {
-        const int64_t s = __ldg(sorted_rows + p) / k;
+        const int32_t i = __ldg(sorted_rows + p);
+        if (!dev::debug_in_range(i, R, lane == 0 ? status : nullptr)) continue;
+        const int64_t s = i / k;
         for (int64_t c = lane; c < d16; c += 32) xs[p * d16 + c] = __ldg(x + s * d16 + c);
     }
 }
@@ -234,11 +238,11 @@ void launch_cast_bf16(const float *src, void *dst, int64_t n, cudaStream_t s) {
 
 void launch_gate_rows(const void *dY, bool dy_bf16, const int32_t *sorted_rows, const float *gates,
                       int32_t k, int64_t R, int64_t Dout, bool by_token, void *dv,
-                      const int32_t *pad_offsets, int32_t E, cudaStream_t s) {
+                      const int32_t *pad_offsets, int32_t E, unsigned *status, cudaStream_t s) {
     gate_rows_kernel<<<warp_grid(R), kWarps * 32, 0, s>>>(dY, dy_bf16, sorted_rows, gates, k, R,
                                                           Dout, by_token,
                                                           static_cast<__nv_bfloat16 *>(dv),
-                                                          pad_offsets, E);
+                                                          pad_offsets, E, status);
 }
 
 void launch_zero_pad_rows(void *rows, int64_t ld, int64_t cols, const int32_t *offsets, int32_t E,
@@ -253,17 +257,19 @@ void launch_zero_pad_rows(void *rows, int64_t ld, int64_t cols, const int32_t *o
 }
 
 void launch_gather_rows(const void *x, const int32_t *sorted_rows, int32_t k, int64_t R, int64_t D,
-                        void *xs, cudaStream_t s) {
+                        void *xs, unsigned *status, cudaStream_t s) {
     gather_rows_kernel<<<warp_grid(R), kWarps * 32, 0, s>>>(static_cast<const uint4 *>(x),
                                                             sorted_rows, k, R, D / 8,
-                                                            static_cast<uint4 *>(xs));
+                                                            static_cast<uint4 *>(xs), status);
 }
 
 void launch_rowdot(const void *dY, bool dy_bf16, const void *v, const int32_t *sorted_rows,
-                   int32_t k, int64_t R, int64_t Dout, bool by_token, float *dg, cudaStream_t s) {
+                   int32_t k, int64_t R, int64_t Dout, bool by_token, float *dg, unsigned *status,
+                   cudaStream_t s) {
     rowdot_kernel<<<warp_grid(R), kWarps * 32, 0, s>>>(dY, dy_bf16,
                                                        static_cast<const __nv_bfloat16 *>(v),
-                                                       sorted_rows, k, R, Dout, by_token, dg);
+                                                       sorted_rows, k, R, Dout, by_token, dg,
+                                                       status);
 }
 
 void launch_router_bwd(const int32_t *top_e, const float *top_w, const float *dw,

@@ -27,12 +27,13 @@ __global__ void __launch_bounds__(kWarps * 32)
 ep_pack_kernel(const uint4 *__restrict__ x, const int32_t *__restrict__ top_e,
                const int32_t *__restrict__ sorted_rows, const int32_t *__restrict__ offsets,
                int32_t E, int32_t k, int64_t R, int64_t u16, uint4 *__restrict__ send,
-               int32_t *__restrict__ send_e) {
+               int32_t *__restrict__ send_e, unsigned *status) {
     const int lane = threadIdx.x & 31;
     const int64_t valid = min(R, (int64_t)__ldg(offsets + E));
     const int64_t wstride = (int64_t)gridDim.x * kWarps;
     for (int64_t p = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5); p < valid; p += wstride) {
         const int64_t i = __ldg(sorted_rows + p);
+        if (!dev::debug_in_range(i, R, lane == 0 ? status : nullptr)) continue;
         const int64_t s = i / k;
         for (int64_t c = lane; c < u16; c += 32) send[p * u16 + c] = __ldg(x + s * u16 + c);
         if (lane == 0) send_e[p] = __ldg(top_e + i);
@@ -76,10 +77,10 @@ ep_combine_kernel(const float4 *__restrict__ ret, const int32_t *__restrict__ sp
 
 void launch_ep_pack(const void *x, size_t row_bytes, const int32_t *top_e,
                     const int32_t *sorted_rows, const int32_t *offsets, int32_t E, int32_t k,
-                    int64_t R, void *send, int32_t *send_e, cudaStream_t s) {
+                    int64_t R, void *send, int32_t *send_e, unsigned *status, cudaStream_t s) {
     ep_pack_kernel<<<warp_grid(R), kWarps * 32, 0, s>>>(
         static_cast<const uint4 *>(x), top_e, sorted_rows, offsets, E, k, R,
-        (int64_t)(row_bytes / 16), static_cast<uint4 *>(send), send_e);
+        (int64_t)(row_bytes / 16), static_cast<uint4 *>(send), send_e, status);
 }
 
 void launch_local_ids(const int32_t *ids, int32_t base, int64_t R, int32_t *local,

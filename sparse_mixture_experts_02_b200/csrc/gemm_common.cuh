@@ -88,6 +88,22 @@ __device__ __forceinline__ void build_schedule(const int32_t *off, int32_t *tsta
     tstart[E] = run;
 }
 
+// Debug builds: the expert offsets behind a schedule must start at 0 or above, never decrease and
+// end at or below the slot count R; otherwise the status word records kStatusBadIndex and the
+// schedule is emptied (no tile reads a slot index derived from them). Release builds trust the
+// offsets, which the sparse map produced.
+__device__ __forceinline__ void debug_check_offsets(const int32_t *off, int32_t *tstart, int E,
+                                                    int64_t R, unsigned *status) {
+    if constexpr (kDebugChecks) {
+        bool ok = off[0] >= 0 && (int64_t)off[E] <= R;
+        for (int e = 0; e < E; ++e) ok = ok && off[e] <= off[e + 1];
+        if (!ok) {
+            if (status != nullptr) atomicOr(status, kStatusBadIndex);
+            for (int e = 0; e <= E; ++e) tstart[e] = 0;
+        }
+    }
+}
+
 template <int TM>
 __device__ __forceinline__ TileInfo decode_tile(int t, const int32_t *off, const int32_t *tstart,
                                                 int E) {

@@ -176,7 +176,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     } else {
         for (int e = threadIdx.x; e <= E; e += blockDim.x) st.off[e] = __ldg(p.offsets + e);
         __syncthreads();
-        if (threadIdx.x == 0) build_schedule<BM>(st.off, st.tstart, E, p.n_tiles);
+        if (threadIdx.x == 0) {
+            build_schedule<BM>(st.off, st.tstart, E, p.n_tiles);
+            debug_check_offsets(st.off, st.tstart, E, p.R, p.status);
+        }
         __syncthreads();
     }
     dev::tc_fence_after();
@@ -322,7 +325,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         auto row_ptrs = [&](int t, const int *ent, const uint8_t **src) {
             const TileInfo ti = decode_tile<BM>(t, st.off, st.tstart, E_sched);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) src[i] = xa + (int64_t)(ent[i] / p.k) * row_bytes;
+            for (int i = 0; i < 8; ++i) {
+                // debug builds: a route outside [0, S*k) reads row 0 instead (and is flagged)
+                const int en = dev::debug_in_range(ent[i], (int64_t)p.S * p.k, p.status) ? ent[i] : 0;
+                src[i] = xa + (int64_t)(en / p.k) * row_bytes;
+            }
             return ti.rows;
         };
         // Shared memory is saturated by the tensor core, so a tile's schedule lookups, index
@@ -407,7 +414,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                 if (SCATTER) orow = i / p.k;
                 if (p.gates != nullptr && i >= 0 && i < p.R) g = __ldg(p.gates + i);
                 // a slot whose route is outside [0, R) is skipped rather than written anywhere
-                if (i < 0 || i >= p.R) valid = false;
+                if (!dev::debug_in_range(i, p.R, p.status) || i < 0 || i >= p.R) valid = false;
             }
             const int n0 = ti.n_idx * OUT_COLS;
             const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + b * BN;

@@ -130,7 +130,10 @@ grouped_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
     }
     for (int e = threadIdx.x; e <= E; e += blockDim.x) st.off[e] = __ldg(p.offsets + e);
     __syncthreads();
-    if (threadIdx.x == 0) build_schedule<TM2>(st.off, st.tstart, E, p.n_tiles);
+    if (threadIdx.x == 0) {
+        build_schedule<TM2>(st.off, st.tstart, E, p.n_tiles);
+        debug_check_offsets(st.off, st.tstart, E, p.R, p.status);
+    }
     // both CTAs' barriers are initialised before either CTA touches the other's
     dev::cluster_sync();
     dev::tc_fence_after();
@@ -284,8 +287,12 @@ grouped_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
             const TileInfo ti = decode_tile<TM2>(t, st.off, st.tstart, E);
             const int rows = min(128, ti.rows - 128 * (int)rank);
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-                src[i] = rows > 0 ? xa + (int64_t)(ent[i] / p.k) * row_bytes : xa;
+            for (int i = 0; i < 8; ++i) {
+                // debug builds: a route outside [0, S*k) reads row 0 instead (and is flagged)
+                const int en = rows > 0 && dev::debug_in_range(ent[i], (int64_t)p.S * p.k, p.status)
+                                   ? ent[i] : 0;
+                src[i] = xa + (int64_t)(en / p.k) * row_bytes;
+            }
             return rows;
         };
         // Shared memory is saturated by the tensor core, so a tile's schedule lookups, index
@@ -368,7 +375,7 @@ grouped_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
                 const int i = __ldg(p.sorted_rows + prow);
                 if (SCATTER) orow = i / p.k;
                 if (p.gates != nullptr && i >= 0 && i < p.R) g = __ldg(p.gates + i);
-                if (i < 0 || i >= p.R) valid = false;
+                if (!dev::debug_in_range(i, p.R, p.status) || i < 0 || i >= p.R) valid = false;
             }
             const int n0 = ti.n_idx * OUT_COLS;
             const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + b * BN;

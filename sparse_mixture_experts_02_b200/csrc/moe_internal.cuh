@@ -17,10 +17,21 @@ namespace moe {
 enum : unsigned {
     kStatusBadExpert = 1u << 0,
     kStatusTimeout = 1u << 1,
+    kStatusBadIndex = 1u << 2,  // debug builds: a bounds check skipped an out-of-range index
     // bits 8..15: id of the first kernel whose wait ran out
     kKernelGemm = 1u, kKernelDebugWait = 2u, kKernelAttention = 3u,
 };
 constexpr size_t kStatusBytes = 256;
+
+// Debug builds (compiled with -DMOE_DEBUG=1, libmoe_b200_debug.so) check every index that a
+// kernel reads from its inputs before using it as an address: a gathered token row, a slot, a
+// route, the expert offsets behind a tile schedule. An index outside its range sets
+// kStatusBadIndex in the status word and the access is skipped; nothing traps. Release builds
+// compile the checks away.
+#ifndef MOE_DEBUG
+#define MOE_DEBUG 0
+#endif
+constexpr bool kDebugChecks = MOE_DEBUG != 0;
 
 // Default bound of every device-side wait (ns). Kernels here finish in milliseconds; a wait that
 // lasts this long means a protocol fault, and the kernel returns instead of hanging the GPU.
@@ -106,7 +117,7 @@ void launch_cast_bf16(const float *src, void *dst, int64_t n, cudaStream_t s);
 // is given (the weight gradient's padded layout), else p' = p.
 void launch_gate_rows(const void *dY, bool dy_bf16, const int32_t *sorted_rows, const float *gates,
                       int32_t k, int64_t R, int64_t Dout, bool by_token, void *dv,
-                      const int32_t *pad_offsets, int32_t E, cudaStream_t s);
+                      const int32_t *pad_offsets, int32_t E, unsigned *status, cudaStream_t s);
 // Zeroes, for every expert, the padding rows after its rows in the padded layout (bf16 rows of
 // `cols` elements, row stride ld).
 void launch_zero_pad_rows(void *rows, int64_t ld, int64_t cols, const int32_t *offsets, int32_t E,
@@ -114,9 +125,10 @@ void launch_zero_pad_rows(void *rows, int64_t ld, int64_t cols, const int32_t *o
 // xs[p] = x[sorted_rows[p] / k] (bf16 rows of D elements): the slot-ordered rows the weight
 // gradient reads by TMA.
 void launch_gather_rows(const void *x, const int32_t *sorted_rows, int32_t k, int64_t R, int64_t D,
-                        void *xs, cudaStream_t s);
+                        void *xs, unsigned *status, cudaStream_t s);
 void launch_rowdot(const void *dY, bool dy_bf16, const void *v, const int32_t *sorted_rows,
-                   int32_t k, int64_t R, int64_t Dout, bool by_token, float *dg, cudaStream_t s);
+                   int32_t k, int64_t R, int64_t Dout, bool by_token, float *dg, unsigned *status,
+                   cudaStream_t s);
 // (two launches: W_gate^T into w_gate_t [E, D], then the per-token router backward)
 void launch_router_bwd(const int32_t *top_e, const float *top_w, const float *dw,
                        const void *w_gate, void *w_gate_t, int64_t S, int64_t D, int32_t E,
@@ -137,7 +149,7 @@ int launch_moa_attention(const void *q, const void *kv, const int32_t *sparse_ro
 // status word); combine returned fp32 rows per token with the router weights (D % 4 == 0).
 void launch_ep_pack(const void *x, size_t row_bytes, const int32_t *top_e,
                     const int32_t *sorted_rows, const int32_t *offsets, int32_t E, int32_t k,
-                    int64_t R, void *send, int32_t *send_e, cudaStream_t s);
+                    int64_t R, void *send, int32_t *send_e, unsigned *status, cudaStream_t s);
 void launch_local_ids(const int32_t *ids, int32_t base, int64_t R, int32_t *local,
                       unsigned *status, cudaStream_t s);
 void launch_ep_combine(const float *ret, const int32_t *sparse_rows, const float *w, int64_t S,
@@ -167,6 +179,19 @@ namespace dev {
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// Debug builds: true when 0 <= v < n; otherwise records kStatusBadIndex and returns false.
+// Release builds: always true (the check compiles away).
+template <typename T>
+__device__ __forceinline__ bool debug_in_range(T v, int64_t n, unsigned *status) {
+    if constexpr (!kDebugChecks) {
+        return true;
+    } else {
+        if (v >= 0 && (int64_t)v < n) return true;
+        if (status != nullptr) atomicOr(status, kStatusBadIndex);
+        return false;
+    }
 }
 
 __device__ __forceinline__ uint64_t globaltimer() {

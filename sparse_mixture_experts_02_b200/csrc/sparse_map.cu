@@ -161,7 +161,8 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, 4)
 map_assign_kernel(const int32_t *__restrict__ te, int64_t R, int32_t E, int64_t nblk,
                   const int32_t *__restrict__ bbase, const int32_t *__restrict__ totals,
                   int32_t *__restrict__ counts, int32_t *__restrict__ offsets,
-                  int32_t *__restrict__ sparse_rows, int32_t *__restrict__ sorted_rows) {
+                  int32_t *__restrict__ sparse_rows, int32_t *__restrict__ sorted_rows,
+                  unsigned *status) {
     constexpr int NT = kWarpsPerBlock * 32;
     constexpr int UNIT = 32 * IT, BLOCK_ROUTES = UNIT * kWarpsPerBlock;
     static_assert(NT == kMaxE, "one thread per expert");
@@ -236,9 +237,11 @@ map_assign_kernel(const int32_t *__restrict__ te, int64_t R, int32_t E, int64_t 
             if (slot >= 0) {
                 if (staged) {
                     const int32_t local = s_pre[e] + (slot - s_first[e]);
-                    stage_r[local] = (int32_t)i;
-                    stage_e[local] = (uint8_t)e;
-                } else {
+                    if (dev::debug_in_range(local, BLOCK_ROUTES, status)) {
+                        stage_r[local] = (int32_t)i;
+                        stage_e[local] = (uint8_t)e;
+                    }
+                } else if (dev::debug_in_range(slot, R, status)) {
                     sorted_rows[slot] = (int32_t)i;
                 }
             }
@@ -249,7 +252,8 @@ map_assign_kernel(const int32_t *__restrict__ te, int64_t R, int32_t E, int64_t 
     // sorted_rows: consecutive threads write consecutive slots of one expert's range
     for (int j = threadIdx.x; j < btotal; j += NT) {
         const int e = stage_e[j];
-        sorted_rows[s_first[e] + (j - s_pre[e])] = stage_r[j];
+        const int64_t slot = (int64_t)s_first[e] + (j - s_pre[e]);
+        if (dev::debug_in_range(slot, R, status)) sorted_rows[slot] = stage_r[j];
     }
 }
 
@@ -334,7 +338,7 @@ map_small_kernel(const int32_t *__restrict__ te, int64_t R, int32_t E,
         __syncwarp();
         if (i < R) {
             sparse_rows[i] = slot;
-            if (slot >= 0) sorted_rows[slot] = (int32_t)i;
+            if (slot >= 0 && dev::debug_in_range(slot, R, status)) sorted_rows[slot] = (int32_t)i;
         }
     }
 }
@@ -368,7 +372,7 @@ void launch_grid(const int32_t *te, int64_t R, int32_t E, int64_t nblk, int32_t 
                                                                          status);
     map_scan_kernel<<<(unsigned)E, kScanThreads, 0, s>>>(bcount, nblk, totals);
     map_assign_kernel<IT><<<(unsigned)nblk, kWarpsPerBlock * 32, 0, s>>>(
-        te, R, E, nblk, bcount, totals, counts, offsets, sparse_rows, sorted_rows);
+        te, R, E, nblk, bcount, totals, counts, offsets, sparse_rows, sorted_rows, status);
 }
 
 }  // namespace

@@ -75,6 +75,33 @@ def test_expert_mlp_forward(oracle_lib, moe, monkeypatch, cta, dtype):
     assert rel_frob(got, ref) < REL_FROB
 
 
+EDGE_COUNTS = [1, 64, 65, 128, 129, 256, 257, 384, 385, 0]
+
+
+@pytest.mark.parametrize("cta", ["0", "1"])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_expert_mlp_forward_tile_edges(oracle_lib, moe, monkeypatch, cta, dtype):
+    """The fused gate+up GEMM (SwiGLU epilogue) and the scatter GEMM with experts whose row
+    counts sit on every tile edge: 64 and 128 (an M=64 one-CTA tile, an M=128 pair tile), 256 (a
+    full pair tile), one past each, 384 = 256 + an M=128 pair tile, and an empty expert. F = 328
+    gives a ragged last N tile, so a half pair tile's second CTA sees only out-of-range columns."""
+    monkeypatch.setenv("MOE_GEMM_2SM", cta)
+    D, F, E, base = 136, 328, len(EDGE_COUNTS), 3
+    owners = np.repeat(np.arange(E, dtype=np.int32), EDGE_COUNTS)
+    owners = owners[np.random.default_rng(5).permutation(len(owners))]
+    R = len(owners)
+    w = W.custom("ep_edges", S=R, D=D, F=F, E=E, k=1,
+                 dtype="bf16" if dtype == torch.bfloat16 else "f32")
+    inp = {n: (t.cuda() if t is not None else None) for n, t in W.make_inputs(w).items()}
+    ids = torch.from_numpy(owners + base).cuda()
+    y = moe.expert_mlp_forward(inp["x"], ids, base, inp["w_gate_e"], inp["w_up"], inp["w_down"])
+    ref = _expert_ref(oracle_lib, inp["x"], ids, base, inp["w_gate_e"], inp["w_up"],
+                      inp["w_down"])
+    got = y.cpu().numpy()
+    assert np.abs(got - ref).max() < MAX_ABS
+    assert rel_frob(got, ref) < REL_FROB
+
+
 def test_expert_mlp_forward_bad_id(moe):
     R, D, F, E = 64, 64, 64, 4
     w = W.custom("ep_bad", S=R, D=D, F=F, E=E, k=1)

@@ -104,12 +104,15 @@ def test_scatter_linear_all_routes_one_expert(oracle_lib, moe, gemm_kernel):
 EDGE_COUNTS = [1, 64, 65, 128, 129, 256, 257, 384, 385]
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
 @pytest.mark.parametrize("gather_in,scatter_out", [(True, True), (False, True), (True, False),
                                                    (False, False)])
-def test_scatter_linear_tile_edges(oracle_lib, moe, gemm_kernel, gather_in, scatter_out):
-    # experts whose row counts sit on every tile edge: 64 (an M=64 / half pair-tile share),
-    # 128 (a one-CTA tile, a half pair tile), 256 (a pair tile) and one past each
+def test_scatter_linear_tile_edges(oracle_lib, moe, gemm_kernel, gather_in, scatter_out, dtype):
+    # experts whose row counts sit on every tile edge: 64 (an M=64 one-CTA tile), 128 (a one-CTA
+    # tile, an M=128 pair tile), 256 (a pair tile), 384 (a pair tile + an M=128 pair tile) and
+    # one past each
     k, Din, Dout = 1, 96, 264
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
     E = len(EDGE_COUNTS)
     owners = np.repeat(np.arange(E, dtype=np.int32), EDGE_COUNTS)
     perm = np.random.default_rng(7).permutation(len(owners))
@@ -118,8 +121,8 @@ def test_scatter_linear_tile_edges(oracle_lib, moe, gemm_kernel, gather_in, scat
     counts, offsets, _, sorted_rows = oracle_lib.sparse_map(te.numpy(), E)
     assert list(counts) == EDGE_COUNTS
     gen = torch.Generator().manual_seed(11)
-    X = torch.randn(S, Din, generator=gen).to(torch.bfloat16)
-    Wt = (torch.randn(E, Din, Dout, generator=gen) * 0.05).to(torch.bfloat16)
+    X = torch.randn(S, Din, generator=gen).to(tdt)
+    Wt = (torch.randn(E, Din, Dout, generator=gen) * 0.05).to(tdt)
     g = torch.rand(S * k, generator=gen)
     ref = oracle_lib.scatter_linear(X, Wt, k, sorted_rows, offsets, g, gather_in=gather_in,
                                     scatter_out=scatter_out, S=S)
@@ -128,6 +131,6 @@ def test_scatter_linear_tile_edges(oracle_lib, moe, gemm_kernel, gather_in, scat
                            scatter_out=scatter_out, S=S)
     torch.cuda.synchronize()
     got = Y.float().cpu().numpy()
-    assert rel_frob(got, ref) < _tol("bf16", scatter_out)
+    assert rel_frob(got, ref) < _tol(dtype, scatter_out)
     scale = np.abs(ref).max()
-    assert np.abs(got - ref).max() / scale < 10 * _tol("bf16", scatter_out)
+    assert np.abs(got - ref).max() / scale < 10 * _tol(dtype, scatter_out)

@@ -31,6 +31,17 @@ def test_header_symbols_exported(moe):
     assert sorted(moe.EXPORTS) == names
 
 
+def test_debug_library_exports_the_same_symbols(moe):
+    """The MOE_DEBUG build (device bounds checks) has every entry point of the release build and
+    says which build it is."""
+    names = _header_functions()
+    dbg = moe.debug_lib()
+    for n in names:
+        assert hasattr(dbg, n), n
+    assert dbg.moe_debug_build() == 1
+    assert moe.lib.moe_debug_build() == 0
+
+
 def test_library_targets_sm100a_only():
     from sparse_mixture_experts_02_b200 import build
     assert "arch=compute_100a,code=sm_100a" in " ".join(build.ARCH)
