@@ -71,6 +71,12 @@ PROFILE_WORKLOADS = {
     # a quarter of its experts and tokens: 1.6 GB of weights
     "e128_profile": Workload("e128_profile", S=2048, D=2880, F=2880, E=32, k=4, dtype="bf16",
                              router_std="1/sqrt(D)"),
+    # the routers and sparse maps of the Mixtral prefill and the 128-expert layers (same S, D, E,
+    # k, so the same kernels and launch shapes) with a small F: 50 MB and 566 MB of weights
+    "router_e8_profile": Workload("router_e8_profile", S=4096, D=4096, F=256, E=8, k=2,
+                                  dtype="bf16", router_std="0.02"),
+    "router_e128_profile": Workload("router_e128_profile", S=8192, D=2880, F=256, E=128, k=4,
+                                    dtype="bf16", router_std="1/sqrt(D)"),
 }
 
 

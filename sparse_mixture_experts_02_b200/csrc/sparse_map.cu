@@ -27,6 +27,8 @@
 // scratch is E x (blocks + 1) words, one eighth of a per-warp layout.
 #include "moe_internal.cuh"
 
+#include <algorithm>
+
 namespace moe {
 namespace {
 
@@ -257,11 +259,16 @@ map_assign_kernel(const int32_t *__restrict__ te, int64_t R, int32_t E, int64_t 
     }
 }
 
-// The whole map in one block when the routes fit 32 units (R <= 16384): warp w counts unit w
-// into cnt[w][e]; the per-expert exclusive prefix over the 32 warps plus the expert offset turns
-// cnt into bases; the warps walk their units again and assign stable slots. Same results as the
-// three-kernel path, one launch instead of three (the decode and Mixtral-prefill route counts).
+// The whole map in one block when the routes fit 32 units of 512 (R <= 16384). The block has
+// just as many warps as the routes need: w = ceil(R / (32 IT)) <= 32 warps of IT steps of 32
+// routes, IT the smallest power of two that keeps w <= 32 (a decode batch of 256 routes runs 8
+// warps of one step; 32 warps of 16 steps ran every step of every warp, with barriers and
+// __match_any_sync, for 10 us). Warp w counts its routes into cnt[w][e]; the per-expert
+// exclusive prefix over the warps plus the expert offset turns cnt into bases; the warps walk
+// their routes again and assign stable slots. Same results as the three-kernel path, one launch
+// instead of three (the decode and Mixtral-prefill route counts).
 constexpr int kSmallUnits = 32;
+template <int IT>
 __global__ void __launch_bounds__(kSmallUnits * 32)
 map_small_kernel(const int32_t *__restrict__ te, int64_t R, int32_t E,
                  int32_t *__restrict__ counts, int32_t *__restrict__ offsets,
@@ -270,14 +277,15 @@ map_small_kernel(const int32_t *__restrict__ te, int64_t R, int32_t E,
     __shared__ int32_t cnt[kSmallUnits][kMaxE];
     __shared__ int32_t eoff[kMaxE];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nw = blockDim.x >> 5;
     for (int e = lane; e < E; e += 32) cnt[warp][e] = 0;
     __syncwarp();
-    const int64_t base = (int64_t)warp * kUnit;
-    // all of this lane's routes at once: kIters independent loads instead of a dependent chain
-    int ev[kIters];
+    const int64_t base = (int64_t)warp * (32 * IT);
+    // all of this lane's routes at once: IT independent loads instead of a dependent chain
+    int ev[IT];
     bool bad = false;
 #pragma unroll
-    for (int it = 0; it < kIters; ++it) {
+    for (int it = 0; it < IT; ++it) {
         const int64_t i = base + it * 32 + lane;
         int e = -1;
         if (i < R) {
@@ -292,7 +300,7 @@ map_small_kernel(const int32_t *__restrict__ te, int64_t R, int32_t E,
     // one block, latency-bound: warp-aggregated counting with __match_any_sync measured faster
     // here than shared atomics or ballots (the grid path's choices)
 #pragma unroll
-    for (int it = 0; it < kIters; ++it) {
+    for (int it = 0; it < IT; ++it) {
         const int e = ev[it];
         const unsigned peers = __match_any_sync(0xffffffffu, e);
         if (e >= 0 && lane == __ffs(peers) - 1) cnt[warp][e] += __popc(peers);
@@ -303,7 +311,7 @@ map_small_kernel(const int32_t *__restrict__ te, int64_t R, int32_t E,
     // per expert: exclusive prefix over the warps (in place) and the total
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         int32_t run = 0;
-        for (int w = 0; w < kSmallUnits; ++w) {
+        for (int w = 0; w < nw; ++w) {
             const int32_t c = cnt[w][e];
             cnt[w][e] = run;
             run += c;
@@ -311,23 +319,33 @@ map_small_kernel(const int32_t *__restrict__ te, int64_t R, int32_t E,
         eoff[e] = run;
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-        int32_t run = 0;
-        for (int e = 0; e < E; ++e) {
-            const int32_t c = eoff[e];
-            counts[e] = c;
-            offsets[e] = run;
-            eoff[e] = run;
-            run += c;
+    // expert offsets: exclusive prefix of the totals, 32 experts at a time by warp 0
+    if (warp == 0) {
+        int32_t carry = 0;
+        for (int e0 = 0; e0 < E; e0 += 32) {
+            const int e = e0 + lane;
+            const int32_t c = e < E ? eoff[e] : 0;
+            int32_t incl = c;
+#pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const int32_t v = __shfl_up_sync(0xffffffffu, incl, d);
+                if (lane >= d) incl += v;
+            }
+            if (e < E) {
+                counts[e] = c;
+                offsets[e] = carry + incl - c;
+                eoff[e] = carry + incl - c;
+            }
+            carry += __shfl_sync(0xffffffffu, incl, 31);
         }
-        offsets[E] = run;
+        if (lane == 0) offsets[E] = carry;
     }
     __syncthreads();
     for (int e = lane; e < E; e += 32) cnt[warp][e] += eoff[e];
     __syncwarp();
     const unsigned lower = (1u << lane) - 1u;
 #pragma unroll
-    for (int it = 0; it < kIters; ++it) {
+    for (int it = 0; it < IT; ++it) {
         const int64_t i = base + it * 32 + lane;
         const int e = ev[it];
         const unsigned peers = __match_any_sync(0xffffffffu, e);
@@ -388,8 +406,19 @@ int launch_sparse_map(const int32_t *te, int64_t R, int32_t E, int32_t *counts, 
                       unsigned *status, cudaStream_t s, int *n_launch) {
     const int64_t units = (R + kUnit - 1) / kUnit;
     if (units <= kSmallUnits) {
-        map_small_kernel<<<1, kSmallUnits * 32, 0, s>>>(te, R, E, counts, offsets, sparse_rows,
-                                                         sorted_rows, status);
+        // steps per warp: the fewest that keep the warps at or below 32
+        int it = 1;
+        while (it < kIters && (R + 32 * it - 1) / (32 * it) > kSmallUnits) it *= 2;
+        const int warps = (int)std::max<int64_t>(1, (R + 32 * it - 1) / (32 * it));
+        auto k = map_small_kernel<16>;
+        switch (it) {
+            case 1: k = map_small_kernel<1>; break;
+            case 2: k = map_small_kernel<2>; break;
+            case 4: k = map_small_kernel<4>; break;
+            case 8: k = map_small_kernel<8>; break;
+            default: break;
+        }
+        k<<<1, warps * 32, 0, s>>>(te, R, E, counts, offsets, sparse_rows, sorted_rows, status);
         if (n_launch) *n_launch += 1;
         return 0;
     }

@@ -61,6 +61,15 @@ def test_map_edges(oracle_lib, moe, S, k, E):
     _compare(oracle_lib, moe, te, E)
 
 
+# One-block path: the block runs ceil(R / (32 IT)) warps of IT steps, IT the smallest power of two
+# that keeps the warps at or below 32. Each pair straddles a switch of IT (1, 2, 4, 8, 16).
+@pytest.mark.parametrize("R", [1, 31, 33, 1024, 1025, 2048, 2049, 4096, 4097, 8192, 8193, 16384])
+@pytest.mark.parametrize("E", [8, 256])
+def test_map_one_block_step_switches(oracle_lib, moe, R, E):
+    te = W.make_top_experts(R, 1, E, seed=R * 3 + E, mode="any")
+    _compare(oracle_lib, moe, te, E)
+
+
 def test_map_all_one_expert_and_empty(oracle_lib, moe):
     te = W.make_top_experts(5000, 4, 32, mode="one")
     counts, offsets, _, _ = _compare(oracle_lib, moe, te, 32)

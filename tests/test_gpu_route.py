@@ -43,6 +43,14 @@ def test_route_small(oracle_lib, moe, dtype, E, k):
     _route_and_check(oracle_lib, moe, W.make_inputs(w, seed=E * 31 + k), k)
 
 
+@pytest.mark.parametrize("S", [1, 7, 128, 2048, 2049, 5000])
+def test_route_eight_experts_every_batch_size(oracle_lib, moe, S):
+    # bf16 with eight experts: a block per token up to 2048 tokens, the shared-memory W_gate
+    # router with four tokens per warp above (and its ragged last group at 2049 and 5000)
+    w = W.custom("r8", S=S, D=4096, F=8, E=8, k=2, dtype="bf16")
+    _route_and_check(oracle_lib, moe, W.make_inputs(w, seed=S), 2)
+
+
 def test_route_bias_zipf(oracle_lib, moe):
     w = W.custom("z", S=2000, D=256, F=8, E=64, k=6, router_std="1/sqrt(D)", zipf_s=1.2)
     te, _ = _route_and_check(oracle_lib, moe, W.make_inputs(w), 6)
