@@ -192,11 +192,13 @@ route_e8_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__rest
     for (int64_t g = (int64_t)blockIdx.x * kWarps + warp; g < groups;
          g += (int64_t)gridDim.x * kWarps) {
         const int64_t s0 = g * T;
-        float acc[T][NE];
+        // experts (2j, 2j+1) of token t accumulate as one float2: a packed two-wide FMA rounds
+        // each half exactly like fmaf, so the sums are the same as with scalar FMAs
+        float2 acc2[T][NE / 2];
 #pragma unroll
         for (int t = 0; t < T; ++t)
 #pragma unroll
-            for (int e = 0; e < NE; ++e) acc[t][e] = 0.f;
+            for (int j = 0; j < NE / 2; ++j) acc2[t][j] = make_float2(0.f, 0.f);
         // B pieces of each of the T rows are loaded before any is used, so their latencies
         // overlap; a token past S reads zeros
         for (int64_t c0 = lane; c0 < pieces; c0 += 32 * B) {
@@ -229,23 +231,29 @@ route_e8_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__rest
                         const int u = 2 * h + q;
                         const uint4 wv = wrow[base + (u ^ sw)];
                         const __nv_bfloat162 *wp = reinterpret_cast<const __nv_bfloat162 *>(&wv);
-                        float wf[NE];
+                        float2 w2[NE / 2];
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const float2 f = __bfloat1622float2(wp[j]);
-                            wf[2 * j] = f.x;
-                            wf[2 * j + 1] = f.y;
-                        }
+                        for (int j = 0; j < NE / 2; ++j) w2[j] = __bfloat1622float2(wp[j]);
 #pragma unroll
                         for (int t = 0; t < T; ++t) {
                             const float xu = q == 0 ? xf[t].x : xf[t].y;
+                            const float2 xx = make_float2(xu, xu);
 #pragma unroll
-                            for (int e = 0; e < NE; ++e) acc[t][e] = fmaf(xu, wf[e], acc[t][e]);
+                            for (int j = 0; j < NE / 2; ++j)
+                                acc2[t][j] = __ffma2_rn(xx, w2[j], acc2[t][j]);
                         }
                     }
                 }
             }
         }
+        float acc[T][NE];
+#pragma unroll
+        for (int t = 0; t < T; ++t)
+#pragma unroll
+            for (int j = 0; j < NE / 2; ++j) {
+                acc[t][2 * j] = acc2[t][j].x;
+                acc[t][2 * j + 1] = acc2[t][j].y;
+            }
 #pragma unroll
         for (int t = 0; t < T; ++t)
 #pragma unroll
