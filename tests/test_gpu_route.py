@@ -51,6 +51,14 @@ def test_route_eight_experts_every_batch_size(oracle_lib, moe, S):
     _route_and_check(oracle_lib, moe, W.make_inputs(w, seed=S), 2)
 
 
+@pytest.mark.parametrize("S,E,k", [(40000, 128, 4), (20000, 256, 8), (19000, 64, 6)])
+def test_route_tensor_core_several_tiles_per_cta(oracle_lib, moe, S, E, k):
+    # more 128-token tiles than SMs: each CTA of the tensor-core router runs two or three tiles
+    # through its two TMEM accumulators
+    w = W.custom("rt", S=S, D=64, F=8, E=E, k=k, dtype="bf16", router_std="1/sqrt(D)")
+    _route_and_check(oracle_lib, moe, W.make_inputs(w, seed=S + E), k)
+
+
 def test_route_bias_zipf(oracle_lib, moe):
     w = W.custom("z", S=2000, D=256, F=8, E=64, k=6, router_std="1/sqrt(D)", zipf_s=1.2)
     te, _ = _route_and_check(oracle_lib, moe, W.make_inputs(w), 6)
