@@ -54,6 +54,8 @@ def lib():
                                           P, P, P]
         L.oracle_moa_forward.argtypes = [P, P, P, P, P, P, P, i64, i64, i32, i32, i32, i32, P, P,
                                          P, P]
+        L.oracle_moa_forward_tokens.argtypes = [P, P, P, P, P, P, P, i64, i64, i32, i32, i32, i32,
+                                                P, P, i64, P, P, P]
     return _lib
 
 
@@ -238,15 +240,28 @@ def mlp_backward(x, w_gate, w_gate_e, w_up, w_down, dout, k, bias=None, given_to
     return out
 
 
-def moa_forward(x, w_gate, w_q, w_k, w_v, w_o, k, heads, bias=None, given_top_experts=None):
+def moa_forward(x, w_gate, w_q, w_k, w_v, w_o, k, heads, bias=None, given_top_experts=None,
+                tokens=None):
     """Mixture of Attention forward in fp64: (out [S, D], top_experts [S, k], top_weights [S, k]).
-    w_q [E, D, H*dh], w_k and w_v [D, H*dh], w_o [E, H*dh, D]; causal attention per head."""
+    w_q [E, D, H*dh], w_k and w_v [D, H*dh], w_o [E, H*dh, D]; causal attention per head. With
+    `tokens`, only those query tokens (rows of the results in list order; keys and values of every
+    token up to the largest listed one)."""
     x, wg, wq, wk, wv, wo = (_f32(a) for a in (x, w_gate, w_q, w_k, w_v, w_o))
     bias = _f32(bias)
     S, D = x.shape
     E, _, HD = wq.shape
     dh = HD // heads
     given = _i32(given_top_experts) if given_top_experts is not None else None
+    if tokens is not None:
+        tok = _i32(tokens).reshape(-1)
+        n = tok.shape[0]
+        out = np.zeros((n, D))
+        te = np.zeros((n, k), dtype=np.int32)
+        tw = np.zeros((n, k))
+        lib().oracle_moa_forward_tokens(_p(x), _p(wg), _p(bias), _p(wq), _p(wk), _p(wv), _p(wo),
+                                        S, D, heads, dh, E, k, _p(given), _p(tok), n, _p(out),
+                                        _p(te), _p(tw))
+        return out, te, tw
     out = np.zeros((S, D))
     te = np.zeros((S, k), dtype=np.int32)
     tw = np.zeros((S, k))

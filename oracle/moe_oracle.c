@@ -482,16 +482,24 @@ void oracle_mlp_backward(const float *x, const float *w_gate, const float *bias,
  *   y_s += w_j * (o W_o[e]).
  * fp64; routing given ([S, k]) or the oracle's own. Outputs out [S, D] and, nullable, the
  * routing top_experts_out [S, k] / top_weights_out [S, k]. */
-void oracle_moa_forward(const float *x, const float *w_gate, const float *bias, const float *w_q,
-                        const float *w_k, const float *w_v, const float *w_o, int64_t S, int64_t D,
-                        int32_t H, int32_t dh, int32_t E, int32_t k,
-                        const int32_t *given_top_experts, double *out, int32_t *top_experts_out,
-                        double *top_weights_out) {
+/* Mixture of Attention for the query tokens `tokens` (n of them; every token 0..S-1 when tokens
+ * is NULL). Keys and values are computed for every token up to the largest query token, so a
+ * query's output is the same whichever other tokens are listed. out, top_experts_out and
+ * top_weights_out are indexed by list position; given_top_experts by token. */
+static void moa_forward_tokens(const float *x, const float *w_gate, const float *bias,
+                               const float *w_q, const float *w_k, const float *w_v,
+                               const float *w_o, int64_t S, int64_t D, int32_t H, int32_t dh,
+                               int32_t E, int32_t k, const int32_t *given_top_experts,
+                               const int32_t *tokens, int64_t n, double *out,
+                               int32_t *top_experts_out, double *top_weights_out) {
     const int64_t HD = (int64_t)H * dh;
-    double *K = (double *)calloc((size_t)S * (size_t)HD, sizeof(double));
-    double *V = (double *)calloc((size_t)S * (size_t)HD, sizeof(double));
+    int64_t S_kv = tokens ? 0 : S;
+    for (int64_t i = 0; tokens && i < n; ++i)
+        if ((int64_t)tokens[i] + 1 > S_kv) S_kv = (int64_t)tokens[i] + 1;
+    double *K = (double *)calloc((size_t)(S_kv > 0 ? S_kv : 1) * (size_t)HD, sizeof(double));
+    double *V = (double *)calloc((size_t)(S_kv > 0 ? S_kv : 1) * (size_t)HD, sizeof(double));
     #pragma omp parallel for schedule(static)
-    for (int64_t t = 0; t < S; ++t) {
+    for (int64_t t = 0; t < S_kv; ++t) {
         for (int64_t d = 0; d < D; ++d) {
             const double xv = (double)x[t * D + d];
             for (int64_t c = 0; c < HD; ++c) {
@@ -510,7 +518,8 @@ void oracle_moa_forward(const float *x, const float *w_gate, const float *bias, 
         int32_t J[64];
         double w[64];
         #pragma omp for schedule(dynamic, 1)
-        for (int64_t s = 0; s < S; ++s) {
+        for (int64_t i = 0; i < n; ++i) {
+            const int64_t s = tokens ? (int64_t)tokens[i] : i;
             const float *xs = x + s * D;
             logits_one(xs, w_gate, bias, D, E, l, NULL);
             if (given_top_experts) {
@@ -519,7 +528,7 @@ void oracle_moa_forward(const float *x, const float *w_gate, const float *bias, 
             } else {
                 topk_one(l, E, k, J, w);
             }
-            double *y = out + s * D;
+            double *y = out + i * D;
             for (int64_t d = 0; d < D; ++d) y[d] = 0.0;
             for (int32_t j = 0; j < k; ++j) {
                 const int64_t e = J[j];
@@ -556,12 +565,32 @@ void oracle_moa_forward(const float *x, const float *w_gate, const float *bias, 
                 }
             }
             if (top_experts_out)
-                for (int32_t j = 0; j < k; ++j) top_experts_out[s * k + j] = J[j];
+                for (int32_t j = 0; j < k; ++j) top_experts_out[i * k + j] = J[j];
             if (top_weights_out)
-                for (int32_t j = 0; j < k; ++j) top_weights_out[s * k + j] = w[j];
+                for (int32_t j = 0; j < k; ++j) top_weights_out[i * k + j] = w[j];
         }
         free(l); free(q); free(o); free(sc);
     }
     free(K);
     free(V);
+}
+
+void oracle_moa_forward(const float *x, const float *w_gate, const float *bias, const float *w_q,
+                        const float *w_k, const float *w_v, const float *w_o, int64_t S, int64_t D,
+                        int32_t H, int32_t dh, int32_t E, int32_t k,
+                        const int32_t *given_top_experts, double *out, int32_t *top_experts_out,
+                        double *top_weights_out) {
+    moa_forward_tokens(x, w_gate, bias, w_q, w_k, w_v, w_o, S, D, H, dh, E, k, given_top_experts,
+                       NULL, S, out, top_experts_out, top_weights_out);
+}
+
+/* The same for a list of query tokens (outputs [n, D], [n, k] by list position). */
+void oracle_moa_forward_tokens(const float *x, const float *w_gate, const float *bias,
+                               const float *w_q, const float *w_k, const float *w_v,
+                               const float *w_o, int64_t S, int64_t D, int32_t H, int32_t dh,
+                               int32_t E, int32_t k, const int32_t *given_top_experts,
+                               const int32_t *tokens, int64_t n, double *out,
+                               int32_t *top_experts_out, double *top_weights_out) {
+    moa_forward_tokens(x, w_gate, bias, w_q, w_k, w_v, w_o, S, D, H, dh, E, k, given_top_experts,
+                       tokens, n, out, top_experts_out, top_weights_out);
 }

@@ -8,7 +8,8 @@ Every case checks, in order:
     relative Frobenius 1e-2.
 The MoA output of token s depends only on tokens 0..s (causal attention), so at the full
 Mixtral-shaped size the first tokens of the GPU's output are checked against the oracle run on
-that prefix of the sequence.
+that prefix of the sequence, and 48 tokens spread over the whole sequence (key-block edges, the
+last token, seeded random ones) against the oracle's forward for that list of query tokens.
 
 Tolerance: q, K, V, the softmax weights and the attention output are each rounded once to bf16
 (relative 2^-9). The output projection sums H*dh such terms with random signs, so the error is of
@@ -126,7 +127,8 @@ def test_moa_unsupported_forms(moe):
 @pytest.mark.parametrize("name", list(W.MOA_WORKLOADS))
 def test_moa_full_workload_prefix(oracle_lib, moe, name):
     """The launch configuration the bench times; tokens [0, 40) checked against the oracle run on
-    that prefix (causality makes them independent of the later tokens)."""
+    that prefix (causality makes them independent of the later tokens), then 48 tokens spread over
+    the whole sequence, the last one included, whose attention spans run up to every key."""
     w = W.MOA_WORKLOADS[name]
     inp = W.make_moa_inputs(w, device="cuda")
     out, v = _run(moe, w, inp)
@@ -137,3 +139,24 @@ def test_moa_full_workload_prefix(oracle_lib, moe, name):
     S0 = 40
     _check(oracle_lib, w, out, v, _host(inp, S=S0), S0)
     assert bool(torch.isfinite(out).all())
+    # sampled tokens across the sequence: block edges (multiples of 128 and one past), the last
+    # token and seeded random ones; the oracle computes keys and values of every token
+    rng = np.random.default_rng(3)
+    toks = np.unique(np.concatenate([
+        [127, 128, 129, 1023, 1024, 2047, 2048, w.S - 2, w.S - 1],
+        rng.choice(w.S, size=39, replace=False)])).astype(np.int32)
+    cpu = _host(inp)
+    te = v["top_experts"]
+    logits, absdot = oracle_lib.router_logits(cpu["x"], cpu["w_gate"], cpu["logit_bias"],
+                                              tokens=toks)
+    ote, _ = oracle_lib.topk_softmax(logits, w.k)
+    check_routing(te[toks], ote, logits, absdot, w.D)
+    HD = w.HD
+    y_ref, _, tw_ref = oracle_lib.moa_forward(cpu["x"], cpu["w_gate"], cpu["w_q"],
+                                              cpu["w_kv"][:, :HD], cpu["w_kv"][:, HD:],
+                                              cpu["w_o"], w.k, w.H, bias=cpu["logit_bias"],
+                                              given_top_experts=te, tokens=toks)
+    np.testing.assert_allclose(v["top_weights"][toks], tw_ref, atol=1e-5)
+    y = out.cpu().numpy()[toks]
+    assert np.abs(y - y_ref).max() < MAX_ABS
+    assert rel_frob(y, y_ref) < REL_FROB

@@ -77,3 +77,20 @@ def test_moa_one_expert_is_causal_attention(oracle_lib):
     O = torch.nn.functional.scaled_dot_product_attention(Q, K, V, is_causal=True)
     ref = (O.transpose(0, 1).reshape(S, H * dh) @ wo[0].double()).numpy()
     np.testing.assert_allclose(out, ref, rtol=1e-11, atol=1e-12)
+
+
+def test_moa_query_token_subset_matches_full(oracle_lib):
+    """A list of query tokens gives exactly the rows of the full forward, in list order (keys and
+    values of every earlier token are still used), with and without a given routing."""
+    S, D, H, dh, E, k = 23, 16, 2, 8, 4, 2
+    x, wg, wq, wk, wv, wo = _inputs(S, D, H, dh, E, seed=12)
+    full, te, tw = oracle_lib.moa_forward(x, wg, wq, wk, wv, wo, k, H)
+    toks = np.array([22, 0, 7, 7, 15], dtype=np.int32)
+    sub, tes, tws = oracle_lib.moa_forward(x, wg, wq, wk, wv, wo, k, H, tokens=toks)
+    assert np.array_equal(sub, full[toks]) and np.array_equal(tes, te[toks])
+    assert np.array_equal(tws, tw[toks])
+    given = np.roll(te, 1, axis=1).astype(np.int32)
+    full_g, _, _ = oracle_lib.moa_forward(x, wg, wq, wk, wv, wo, k, H, given_top_experts=given)
+    sub_g, tes_g, _ = oracle_lib.moa_forward(x, wg, wq, wk, wv, wo, k, H, given_top_experts=given,
+                                             tokens=toks)
+    assert np.array_equal(sub_g, full_g[toks]) and np.array_equal(tes_g, given[toks])
