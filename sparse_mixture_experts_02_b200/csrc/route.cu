@@ -21,9 +21,7 @@ namespace {
 constexpr int kTokPerWarp = 8;
 constexpr int kWarps = 8;
 constexpr int kChunk = 64;
-constexpr int kRouteE8MaxSmem = 96 * 1024;  // W_gate rows of the eight-expert router: D <= 6144
-constexpr int kE8Batch = 16;                // x pieces a lane has in flight in that router
-constexpr int kE8Tokens = 4;                // tokens per warp task of that router
+constexpr int kRouteE8MaxSmem = 200 * 1024;  // eight-expert router: padded W_gate, D <= 9792
 
 template <bool BF16>
 __device__ __forceinline__ float ld_elem(const void *p, int64_t i) {
@@ -152,150 +150,144 @@ route_kernel(const void *__restrict__ x, const void *__restrict__ w_gate,
     }
 }
 
-// Router for E = 8 experts (bf16) at large batches. Persistent blocks stage W_gate [D, 8] (bf16
-// rows of 16 bytes) in shared memory once; a warp owns T consecutive tokens at a time, lane l
-// reads the 16-byte pieces c = l + 32 j of their x rows (8 consecutive d each, coalesced across
-// the warp; kE8Batch pieces in flight over the T rows) and accumulates the T x 8 dot products in
-// fp32, ascending d within the lane. Each W_gate row is read from shared memory and widened to
-// fp32 once per piece and used for all T tokens. Row d sits at slot d ^ ((d >> 3) & 7): the rows
-// of a piece keep their 128 bytes, permuted so that, for a given row offset, the eight lanes of a
-// quarter-warp read eight different 16-byte bank groups. The lanes' sums are added by a
-// butterfly, after which lane t takes the top-k and the softmax of token t.
-template <int T>
-__global__ void __launch_bounds__(kWarps * 32)
+// Router for E = 8 experts (bf16) at large batches, on warp-level tensor-core MMAs
+// (mma.sync m16n8k16, bf16 inputs, fp32 accumulation): the router streams x once from HBM, and an
+// MMA turns 16 tokens x 16 d x 8 experts of products into one instruction, where fp32 FMAs need
+// 64 (the CUDA-core form of this kernel issued ~6 M warp instructions at S = D = 4096 and ran at
+// a fifth of HBM bandwidth). A block of 8 warps routes 16 tokens; warp w takes the d range
+// [w P / 8, (w + 1) P / 8) of the P = ceil(D / 32) groups of 32 d.
+//
+// The d order inside one MMA is free (a dot product is a sum), so the fragments come straight
+// from coalesced 16-byte loads: lane (g = lane / 4, q = lane % 4) loads d = 32 p + 8 q .. + 7 of
+// tokens g and g + 8, and MMA j (0, 1) of group p sums, for that lane's k slots {2q, 2q+1} and
+// {2q+8, 2q+9}, the d = 32 p + 8 q + 4 j + {0, 1} and + {2, 3}. The B fragments (W_gate column
+// g at the same d) of both MMAs come from one ldmatrix.x4.trans over W_gate rows (16 bytes: the 8
+// experts of one d) staged by cp.async in shared memory: each lane names the row of the d its
+// k slot stands for, and row d sits at slot d + 2 (d / 8), which puts the 8 rows of every 8 x 8
+// matrix on 8 different 16-byte bank groups. Rows past D are zero. The warps' partial logits are
+// added in warp order, then one thread per token takes the top-k and the softmax.
+constexpr int kE8MmaTokens = 16;
+constexpr int kE8MmaUnroll = 8;  // groups of 32 d whose x a lane has in flight
+
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1,
+                                               uint32_t a2, uint32_t a3, uint32_t b0,
+                                               uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+        "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Shared memory of the eight-expert router: W_gate rows of the ceil(D / 32) groups of 32 d at
+// slot d + 2 (d / 8) (40 slots of 16 bytes per group), then the warps' partial logits.
+__host__ __device__ constexpr size_t route_e8_smem(int64_t D) {
+    return (size_t)((D + 31) / 32) * 40 * 16 + (size_t)kWarps * kE8MmaTokens * 8 * sizeof(float);
+}
+
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr)
+                 : "memory");
+}
+
+__global__ void __launch_bounds__(kWarps * 32, 2)
 route_e8_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ w_gate,
                 const float *__restrict__ bias, int64_t S, int64_t D, int32_t k,
                 int32_t *__restrict__ top_e, float *__restrict__ top_w, unsigned *status) {
-    constexpr int NE = 8;
-    constexpr int B = kE8Batch / T;  // pieces in flight per token row
-    static_assert(B * T == kE8Batch && T <= 32, "token group");
-    extern __shared__ __align__(16) uint4 wrow[];  // D rows of 8 bf16
+    constexpr int U = kE8MmaUnroll;
+    extern __shared__ __align__(16) uint8_t e8_smem[];
+    const int Di = (int)D;
+    const int P = (Di + 31) / 32;
+    float *part = reinterpret_cast<float *>(e8_smem + (size_t)P * 40 * 16);
     if (status != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *status = 0u;  // first kernel
-    const uint4 *wg = reinterpret_cast<const uint4 *>(w_gate);
-    for (int64_t d0 = threadIdx.x; d0 < D; d0 += 8 * (int64_t)blockDim.x) {
-        uint4 r[8];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, q = lane & 3;
+    const int64_t t0 = (int64_t)blockIdx.x * kE8MmaTokens;
+    const int p0 = warp * P / kWarps, p1 = (warp + 1) * P / kWarps;
+    const bool r0 = t0 + g < S, r1 = t0 + g + 8 < S;
+    const uint4 *x0 = reinterpret_cast<const uint4 *>(x + (r0 ? t0 + g : 0) * D);
+    const uint4 *x1 = reinterpret_cast<const uint4 *>(x + (r1 ? t0 + g + 8 : 0) * D);
+    uint4 xa[U], xb[U];
+    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+    auto load = [&](int p) {
 #pragma unroll
-        for (int b = 0; b < 8; ++b) {
-            const int64_t d = d0 + (int64_t)b * blockDim.x;
-            if (d < D) r[b] = __ldg(wg + d);
+        for (int u = 0; u < U; ++u) {
+            const int c = 4 * (p + u) + q;  // 16-byte piece: d = 8 c .. 8 c + 7
+            const bool ok = p + u < p1 && 8 * c < Di;
+            xa[u] = ok && r0 ? __ldg(x0 + c) : z;
+            xb[u] = ok && r1 ? __ldg(x1 + c) : z;
         }
+    };
+    // W_gate rows by cp.async (no registers held), then the first x batch: both in flight at once
+    const uint32_t wbase = dev::smem_u32(e8_smem);
+    const uint4 *wg = reinterpret_cast<const uint4 *>(w_gate);
+    for (int d = threadIdx.x; d < 32 * P; d += blockDim.x) {
+        const uint32_t dst = wbase + (uint32_t)(d + 2 * (d >> 3)) * 16u;
+        dev::cp_async16(dst, d < Di ? wg + d : wg, d < Di ? 16u : 0u);  // rows past D: zeros
+    }
+    load(p0);
+    dev::cp_async_wait_all();
+    __syncthreads();
+    // ldmatrix row of this lane: matrix m = lane / 8 (MMA j = m / 2, k half m % 2), row r = lane % 8
+    const int lm = lane >> 3, lr = lane & 7;
+    const int drow = 8 * (lr >> 1) + 4 * (lm >> 1) + 2 * (lm & 1) + (lr & 1);  // d within a group
+    float c[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int p = p0; p < p1; p += U) {
+        if (p != p0) load(p);
 #pragma unroll
-        for (int b = 0; b < 8; ++b) {
-            const int64_t d = d0 + (int64_t)b * blockDim.x;
-            if (d < D) wrow[d ^ ((d >> 3) & 7)] = r[b];
+        for (int u = 0; u < U; ++u) {
+            if (p + u >= p1) break;
+            const int d = 32 * (p + u) + drow;
+            uint32_t bw[4];
+            ldmatrix_x4_trans(wbase + (uint32_t)(d + 2 * (d >> 3)) * 16u, bw);
+            mma_bf16_16816(c, xa[u].x, xb[u].x, xa[u].y, xb[u].y, bw[0], bw[1]);
+            mma_bf16_16816(c, xa[u].z, xb[u].z, xa[u].w, xb[u].w, bw[2], bw[3]);
         }
     }
+    // c[0], c[1]: token g, experts 2q, 2q+1; c[2], c[3]: token g + 8
+    float *pw = part + (size_t)warp * kE8MmaTokens * 8;
+    pw[g * 8 + 2 * q] = c[0];
+    pw[g * 8 + 2 * q + 1] = c[1];
+    pw[(g + 8) * 8 + 2 * q] = c[2];
+    pw[(g + 8) * 8 + 2 * q + 1] = c[3];
     __syncthreads();
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t pieces = D / 8;
-    const int64_t groups = (S + T - 1) / T;
-    for (int64_t g = (int64_t)blockIdx.x * kWarps + warp; g < groups;
-         g += (int64_t)gridDim.x * kWarps) {
-        const int64_t s0 = g * T;
-        // experts (2j, 2j+1) of token t accumulate as one float2: a packed two-wide FMA rounds
-        // each half exactly like fmaf, so the sums are the same as with scalar FMAs
-        float2 acc2[T][NE / 2];
+    if (threadIdx.x < kE8MmaTokens) {
+        const int r = threadIdx.x;
+        const int64_t s = t0 + r;
+        if (s < S) {
+            float v[8];
 #pragma unroll
-        for (int t = 0; t < T; ++t)
+            for (int e = 0; e < 8; ++e) {
+                float l = part[r * 8 + e];
 #pragma unroll
-            for (int j = 0; j < NE / 2; ++j) acc2[t][j] = make_float2(0.f, 0.f);
-        // B pieces of each of the T rows are loaded before any is used, so their latencies
-        // overlap; a token past S reads zeros
-        for (int64_t c0 = lane; c0 < pieces; c0 += 32 * B) {
-            uint4 xv[T][B];
-#pragma unroll
-            for (int t = 0; t < T; ++t) {
-                const uint4 *xr = reinterpret_cast<const uint4 *>(x + (s0 + t) * D);
-#pragma unroll
-                for (int b = 0; b < B; ++b) {
-                    const int64_t c = c0 + 32 * b;
-                    xv[t][b] = (c < pieces && s0 + t < S) ? __ldg(xr + c)
-                                                          : make_uint4(0u, 0u, 0u, 0u);
-                }
+                for (int w = 1; w < kWarps; ++w) l += part[(w * kE8MmaTokens + r) * 8 + e];
+                if (bias != nullptr) l += __ldg(bias + e);
+                v[e] = isnan(l) ? -INFINITY : l;
             }
-#pragma unroll
-            for (int b = 0; b < B; ++b) {
-                const int64_t c = c0 + 32 * b;
-                if (c >= pieces) break;
-                const int64_t base = 8 * c;
-                const int sw = (int)(c & 7);
-#pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                    float2 xf[T];
-#pragma unroll
-                    for (int t = 0; t < T; ++t)
-                        xf[t] = __bfloat1622float2(
-                            reinterpret_cast<const __nv_bfloat162 *>(&xv[t][b])[h]);
-#pragma unroll
-                    for (int q = 0; q < 2; ++q) {
-                        const int u = 2 * h + q;
-                        const uint4 wv = wrow[base + (u ^ sw)];
-                        const __nv_bfloat162 *wp = reinterpret_cast<const __nv_bfloat162 *>(&wv);
-                        float2 w2[NE / 2];
-#pragma unroll
-                        for (int j = 0; j < NE / 2; ++j) w2[j] = __bfloat1622float2(wp[j]);
-#pragma unroll
-                        for (int t = 0; t < T; ++t) {
-                            const float xu = q == 0 ? xf[t].x : xf[t].y;
-                            const float2 xx = make_float2(xu, xu);
-#pragma unroll
-                            for (int j = 0; j < NE / 2; ++j)
-                                acc2[t][j] = __ffma2_rn(xx, w2[j], acc2[t][j]);
-                        }
-                    }
-                }
-            }
-        }
-        float acc[T][NE];
-#pragma unroll
-        for (int t = 0; t < T; ++t)
-#pragma unroll
-            for (int j = 0; j < NE / 2; ++j) {
-                acc[t][2 * j] = acc2[t][j].x;
-                acc[t][2 * j + 1] = acc2[t][j].y;
-            }
-#pragma unroll
-        for (int t = 0; t < T; ++t)
-#pragma unroll
-            for (int e = 0; e < NE; ++e)
-#pragma unroll
-                for (int off = 16; off > 0; off >>= 1)
-                    acc[t][e] += __shfl_xor_sync(0xffffffffu, acc[t][e], off);
-        // lane t < T finishes token s0 + t (every lane holds every sum after the butterfly)
-        float v[NE];
-#pragma unroll
-        for (int e = 0; e < NE; ++e) {
-            float l = acc[0][e];
-#pragma unroll
-            for (int t = 1; t < T; ++t)
-                if (lane == t) l = acc[t][e];
-            if (bias != nullptr) l += __ldg(bias + e);
-            v[e] = isnan(l) ? -INFINITY : l;
-        }
-        const int64_t s = s0 + lane;
-        if (lane < T && s < S) {
             unsigned taken = 0;
             float sel_v[8];
             int sel_i[8];
-            for (int r = 0; r < k; ++r) {
+            for (int rr = 0; rr < k; ++rr) {
                 float bv = -INFINITY;
                 int bi = 0x7fffffff;
 #pragma unroll
-                for (int e = 0; e < NE; ++e)
+                for (int e = 0; e < 8; ++e)
                     if (!(taken & (1u << e)) && better(v[e], e, bv, bi)) {
                         bv = v[e];
                         bi = e;
                     }
                 taken |= 1u << bi;
-                sel_v[r] = bv;
-                sel_i[r] = bi;
+                sel_v[rr] = bv;
+                sel_i[rr] = bi;
             }
             const float m = sel_v[0];
             float den = 0.f;
-            for (int r = 0; r < k; ++r) den += expf(sel_v[r] - m);
-            for (int r = 0; r < k; ++r) {
-                top_e[s * k + r] = sel_i[r];
-                top_w[s * k + r] = expf(sel_v[r] - m) / den;
+            for (int rr = 0; rr < k; ++rr) den += expf(sel_v[rr] - m);
+            for (int rr = 0; rr < k; ++rr) {
+                top_e[s * k + rr] = sel_i[rr];
+                top_w[s * k + rr] = expf(sel_v[rr] - m) / den;
             }
         }
     }
@@ -466,14 +458,13 @@ int launch_route(const void *x, const void *w_gate, const float *bias, int64_t S
                  int32_t E, int32_t k, bool bf16, int32_t *top_e, float *top_w, unsigned *status,
                  cudaStream_t s) {
     if (S == 0) return 0;
-    // Eight experts (bf16), a batch too large for one block per token: W_gate fits in shared
-    // memory and every SM streams x rows (measured 20 us with x in L2, against 29 us for the
-    // tensor-core router, at S = 4096, D = 4096).
-    if (bf16 && E == 8 && S > 2048 && D * 16 <= kRouteE8MaxSmem) {
+    // Eight experts (bf16), a batch too large for one block per token: 16 tokens per block on
+    // warp-level MMAs, W_gate in shared memory, every SM streaming x rows.
+    if (bf16 && E == 8 && S > 2048 && route_e8_smem(D) <= (size_t)kRouteE8MaxSmem) {
         static std::once_flag once;
         static cudaError_t attr_err = cudaSuccess;
         std::call_once(once, [] {
-            attr_err = cudaFuncSetAttribute(route_e8_kernel<kE8Tokens>,
+            attr_err = cudaFuncSetAttribute(route_e8_kernel,
                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             kRouteE8MaxSmem);
         });
@@ -481,9 +472,8 @@ int launch_route(const void *x, const void *w_gate, const float *bias, int64_t S
             set_error(MOE_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(attr_err));
             return -1;
         }
-        const int64_t want = (S + kE8Tokens * kWarps - 1) / (kE8Tokens * kWarps);
-        const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(want, 2LL * num_sms()));
-        route_e8_kernel<kE8Tokens><<<(unsigned)blocks, kWarps * 32, (size_t)(D * 16), s>>>(
+        const int64_t blocks = (S + kE8MmaTokens - 1) / kE8MmaTokens;
+        route_e8_kernel<<<(unsigned)blocks, kWarps * 32, route_e8_smem(D), s>>>(
             static_cast<const __nv_bfloat16 *>(x), static_cast<const __nv_bfloat16 *>(w_gate),
             bias, S, D, k, top_e, top_w, status);
         return 1;

@@ -45,10 +45,18 @@ def test_route_small(oracle_lib, moe, dtype, E, k):
 
 @pytest.mark.parametrize("S", [1, 7, 128, 2048, 2049, 5000])
 def test_route_eight_experts_every_batch_size(oracle_lib, moe, S):
-    # bf16 with eight experts: a block per token up to 2048 tokens, the shared-memory W_gate
-    # router with four tokens per warp above (and its ragged last group at 2049 and 5000)
+    # bf16 with eight experts: a block per token up to 2048 tokens, the warp-MMA router with 16
+    # tokens per block above (and its ragged last block at 2049 and 5000)
     w = W.custom("r8", S=S, D=4096, F=8, E=8, k=2, dtype="bf16")
     _route_and_check(oracle_lib, moe, W.make_inputs(w, seed=S), 2)
+
+
+@pytest.mark.parametrize("D", [8, 200, 2880, 6144, 9792])
+def test_route_eight_experts_feature_sizes(oracle_lib, moe, D):
+    # the warp-MMA router's d split: D not a multiple of 32 (zero rows past D in the last group),
+    # fewer groups of 32 d than warps (D = 8, 200), one block per SM at the largest sizes
+    w = W.custom("r8d", S=2100, D=D, F=8, E=8, k=3, dtype="bf16", router_std="1/sqrt(D)")
+    _route_and_check(oracle_lib, moe, W.make_inputs(w, seed=D), 3)
 
 
 @pytest.mark.parametrize("S,E,k", [(40000, 128, 4), (20000, 256, 8), (19000, 64, 6)])
