@@ -610,6 +610,32 @@ def bench_ours(args, w, ws, rank, local):
     return line
 
 
+def torch_map_reference_ms(te, E, flush, warmup, reps):
+    """The same map from library calls, as a reference timing for the sweep: a stable radix sort
+    of the expert ids (sorted_rows), their histogram and its exclusive prefix (counts, offsets) and
+    the inverse permutation (sparse_rows). Median CUDA-event time, L2 flushed before every call."""
+    flat = te.reshape(-1)
+    R = flat.numel()
+    ar = torch.arange(R, dtype=torch.int64, device=flat.device)
+    times = []
+    for i in range(warmup + reps):
+        flush.zero_()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        _, sorted_rows = torch.sort(flat, stable=True)
+        counts = torch.bincount(flat, minlength=E)
+        offsets = torch.cumsum(counts, 0) - counts
+        sparse_rows = torch.empty_like(sorted_rows)
+        sparse_rows.scatter_(0, sorted_rows, ar)
+        e1.record()
+        torch.cuda.synchronize(flat.device)
+        if i >= warmup:
+            times.append(e0.elapsed_time(e1))
+    del offsets
+    return sorted(times)[len(times) // 2]
+
+
 def map_sweep(args):
     """Sparse-map bandwidth over route counts 2^20..2^26 and E in {8, 64, 128, 256} (k = 8,
     distinct experts per token, uniform marginals). Each point is the median of CUDA-event-timed
@@ -648,8 +674,11 @@ def map_sweep(args):
         t_ms = sorted(times)[len(times) // 2]
         nbytes = 4 * R + 8 * R + (2 * E + 1) * 4
         gbs = nbytes / (t_ms * 1e-3) / 1e9
-        points.append({"R": R, "E": E, "us": round(t_ms * 1e3, 2), "GB/s": round(gbs, 1),
-                       "frac_of_hbm_peak": round(gbs / pk["hbm_gbs"], 3)})
+        pt = {"R": R, "E": E, "us": round(t_ms * 1e3, 2), "GB/s": round(gbs, 1),
+              "frac_of_hbm_peak": round(gbs / pk["hbm_gbs"], 3)}
+        if args.map_torch_ref:
+            pt["torch_ref_us"] = round(torch_map_reference_ms(te, E, flush, args.warmup, reps) * 1e3, 2)
+        points.append(pt)
         del te, wsp
     return {"metric": "sparse-map GB/s sweep", "unit": "GB/s", "n_gpus": 1,
             "data": "synthetic (seeded stride routing: k = 8 distinct experts per token)",
@@ -927,6 +956,9 @@ def main():
     ap.add_argument("--ref-step-s", type=float, default=None)
     ap.add_argument("--map-sweep", action="store_true",
                     help="instead of the forward: sparse-map GB/s over R = 2^20..2^26 routes")
+    ap.add_argument("--map-torch-ref", action="store_true",
+                    help="with --map-sweep: also time the same map built from torch calls "
+                         "(stable sort, bincount, cumsum, scatter) at every point")
     ap.add_argument("--backward", action="store_true",
                     help="instead of the forward: time moe_mlp_backward on --workload")
     ap.add_argument("--moa", action="store_true",
