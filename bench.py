@@ -636,6 +636,88 @@ def torch_map_reference_ms(te, E, flush, warmup, reps):
     return sorted(times)[len(times) // 2]
 
 
+def forward_torch_reference(args):
+    """The expert-MLP forward built from torch calls (a cuBLAS GEMM per expert: gather, x W_gate_e,
+    x W_up, SwiGLU, h W_down, router weight, index_add into the output), timed beside
+    moe_mlp_forward on the same inputs and the library's routing, for every workload; also the
+    reference's GEMMs alone on pre-gathered rows. Median of CUDA-event-timed calls, L2 flushed
+    (a 256 MiB write) before each. A context measurement: the product path is the library."""
+    import sparse_mixture_experts_02_b200 as moe
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def timed(fn):
+        ts = []
+        for i in range(args.warmup + args.steps):
+            flush.zero_()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize(dev)
+            if i >= args.warmup:
+                ts.append(e0.elapsed_time(e1))
+        return sorted(ts)[len(ts) // 2]
+
+    results = {}
+    for name in ("mixtral_prefill", "mixtral_decode", "e128", "zipf64"):
+        w = W.WORKLOADS[name]
+        inp = W.make_inputs(w, device=dev, seed=0)
+        ws = moe.ForwardWorkspace(w.S, w.D, w.F, w.E, w.k, inp["x"].dtype, dev)
+        out = torch.empty((w.S, w.D), dtype=torch.float32, device=dev)
+        t_lib = timed(lambda: moe.mlp_forward(inp["x"], inp["w_gate"], inp["w_gate_e"], inp["w_up"],
+                                              inp["w_down"], w.k, logit_bias=inp["logit_bias"],
+                                              out=out, ws=ws))
+        # the reference is handed the library's routing (its top-k is not timed)
+        flat = ws.view("top_experts").reshape(-1).long()
+        order = torch.sort(flat, stable=True).indices
+        counts = ws.view("expert_counts").cpu().tolist()
+        offs = [0]
+        for c in counts:
+            offs.append(offs[-1] + c)
+        tok = order // w.k
+        gates = ws.view("top_weights").reshape(-1)[order]
+        x, wg, wu, wd = inp["x"], inp["w_gate_e"], inp["w_up"], inp["w_down"]
+
+        def ref():
+            y = torch.zeros((w.S, w.D), dtype=torch.float32, device=dev)
+            for e in range(w.E):
+                a, b = offs[e], offs[e + 1]
+                if a == b:
+                    continue
+                t = tok[a:b]
+                xe = x.index_select(0, t)
+                h = torch.nn.functional.silu(xe @ wg[e]) * (xe @ wu[e])
+                y.index_add_(0, t, (h @ wd[e]).float() * gates[a:b, None])
+            return y
+
+        t_ref = timed(ref)
+        xs = [x.index_select(0, tok[offs[e]:offs[e + 1]]) for e in range(w.E)]
+        hs = [torch.empty((counts[e], w.F), dtype=x.dtype, device=dev) for e in range(w.E)]
+
+        def gemms():
+            for e in range(w.E):
+                if counts[e]:
+                    xs[e] @ wg[e]
+                    xs[e] @ wu[e]
+                    hs[e] @ wd[e]
+
+        t_gemm = timed(gemms)
+        fl = 6.0 * w.S * w.k * w.D * w.F
+        results[name] = {"library_ms": round(t_lib, 4), "torch_forward_ms": round(t_ref, 4),
+                         "torch_gemms_only_ms": round(t_gemm, 4),
+                         "library_tflops": round(fl / t_lib / 1e9, 1),
+                         "torch_gemms_only_tflops": round(fl / t_gemm / 1e9, 1)}
+        del inp, ws, out, xs, hs
+        torch.cuda.empty_cache()
+    return {"metric": "expert-MLP forward: library against a torch per-expert (cuBLAS) forward",
+            "unit": "ms", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "data": "synthetic", "l2": "flushed before every call", "workloads": results}
+
+
 def map_sweep(args):
     """Sparse-map bandwidth over route counts 2^20..2^26 and E in {8, 64, 128, 256} (k = 8,
     distinct experts per token, uniform marginals). Each point is the median of CUDA-event-timed
@@ -956,6 +1038,9 @@ def main():
     ap.add_argument("--ref-step-s", type=float, default=None)
     ap.add_argument("--map-sweep", action="store_true",
                     help="instead of the forward: sparse-map GB/s over R = 2^20..2^26 routes")
+    ap.add_argument("--forward-torch-ref", action="store_true",
+                    help="instead of the forward: time moe_mlp_forward beside a torch per-expert "
+                         "(cuBLAS) forward on every workload")
     ap.add_argument("--map-torch-ref", action="store_true",
                     help="with --map-sweep: also time the same map built from torch calls "
                          "(stable sort, bincount, cumsum, scatter) at every point")
@@ -984,6 +1069,9 @@ def main():
         ap.error("--warmup must be >= 3")
     if args.map_sweep:
         print(json.dumps(map_sweep(args)), flush=True)
+        return
+    if args.forward_torch_ref:
+        print(json.dumps(forward_torch_reference(args)), flush=True)
         return
     if args.ep:
         wl = {**W.WORKLOADS, **W.PROFILE_WORKLOADS}[args.workload]
