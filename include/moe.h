@@ -175,6 +175,10 @@ int moe_scatter_linear_backward(const void *X, const void *W, const void *dY, in
  * with (e_j, w_j) from moe_route_topk. Steps on `stream`: zero out, route, sparse map, GEMM1
  * (gathered x rows, fused gate+up, SwiGLU in registers, h in slot order), GEMM2 (h rows,
  * W_down, router weight, scatter-add into out). No host synchronisation.
+ *   For bf16 with experts of 384 or more rows on average (S*k / E >= 384) and F >= 2048, GEMM1
+ *   does not gather on load: one more kernel first copies the x rows to slot order inside the
+ *   workspace ("x_sorted"), and GEMM1 reads them by TMA (set the environment variable
+ *   MOE_PREGATHER=0 to gather on load instead; the workspace size does not change).
  *   x [S,D], w_gate [D,E], w_gate_e [E,D,F], w_up [E,D,F], w_down [E,F,D]: dt
  *   logit_bias [E] float32 nullable;  out [S,D] float32 (overwritten).
  *   ws: moe_workspace_size("mlp_forward", S, D, F, E, k, dt) bytes; after the call it holds the
@@ -305,7 +309,9 @@ size_t moe_workspace_size(const char *op, int64_t S, int64_t D, int64_t F, int32
  * Byte offsets inside an "mlp_forward" workspace of the intermediate results the forward leaves
  * there (for inspection and tests): which = "top_experts" [S*k] int32, "top_weights" [S*k] f32,
  * "expert_counts" [E], "expert_offsets" [E+1], "sparse_rows" [S*k], "sorted_rows" [S*k] int32,
- * "h" [S*k, F] (bf16 for bf16, f32 for f32). Returns -1 for an unknown name.
+ * "h" [S*k, F] (bf16 for bf16, f32 for f32), "x_sorted" [S*k, D] (the x rows in slot order, only
+ * in workspaces of shapes whose forward copies them, see moe_mlp_forward; -1 otherwise). Returns
+ * -1 for an unknown name.
  */
 int64_t moe_workspace_view(const char *which, int64_t S, int64_t D, int64_t F, int32_t E,
                            int32_t k, moe_dtype dt);

@@ -313,6 +313,7 @@ class ForwardWorkspace:
             "sparse_rows": (R, torch.int32, (R,)),
             "sorted_rows": (R, torch.int32, (R,)),
             "h": (R * F, self.dtype, (R, F)),
+            "x_sorted": (R * D, self.dtype, (R, D)),
         }[which]
         nbytes = n * torch.empty(0, dtype=dt).element_size()
         return self.buf[off:off + nbytes].view(dt).view(shape)

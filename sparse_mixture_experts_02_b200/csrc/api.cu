@@ -25,6 +25,12 @@ int set_error(int code, const char *fmt, ...) {
     return code;
 }
 
+// True when the environment variable is set to "0" (switches for tests and paired timings).
+bool env_off(const char *name) {
+    const char *v = getenv(name);
+    return v != nullptr && v[0] == '0';
+}
+
 bool prefer_2sm(int64_t R, int32_t E) {
     const char *env = getenv("MOE_GEMM_2SM");
     if (env != nullptr && (env[0] == '0' || env[0] == '1')) return env[0] == '1';
@@ -109,10 +115,23 @@ size_t esize(moe_dtype dt) { return dt == MOE_BF16 ? 2 : 4; }
 
 // ---- workspace layout ------------------------------------------------------------------------
 struct MlpLayout {
-    size_t status, top_e, top_w, counts, offsets, sparse_rows, sorted_rows, scratch, h, total;
+    size_t status, top_e, top_w, counts, offsets, sparse_rows, sorted_rows, scratch, h, xs,
+        xs_bytes, total;
 };
 
-MlpLayout mlp_layout(int64_t S, int64_t F, int32_t E, int32_t k, moe_dtype dt) {
+// Whether the forward copies the x rows to slot order before GEMM1 (decided by the shapes alone,
+// so that the workspace size never depends on the environment). The copy costs 4 R D bytes of
+// HBM traffic; GEMM1 on TMA-loaded rows instead of rows gathered on load saved ~10% of its time
+// on CTA pairs (experts of >= 384 rows), which outweighs the copy once F >= 2048 (7.5% of the
+// Mixtral-shaped prefill forward, F = 14336; no gain at F = 1408).
+bool pregather_shape(int64_t R, int64_t D, int64_t F, int32_t E, moe_dtype dt) {
+    return dt == MOE_BF16 && E > 0 && D > 0 && R / E >= 384 && F >= 2048;
+}
+
+// with_xs: the MoE forward's layout (x rows in slot order after h when pregather_shape holds);
+// the expert-parallel forward, which gathers its received rows on load, has none.
+MlpLayout mlp_layout(int64_t S, int64_t D, int64_t F, int32_t E, int32_t k, moe_dtype dt,
+                     bool with_xs = true) {
     const int64_t R = S * k;
     MlpLayout L;
     size_t o = 0;
@@ -125,6 +144,8 @@ MlpLayout mlp_layout(int64_t S, int64_t F, int32_t E, int32_t k, moe_dtype dt) {
     L.sorted_rows = o; o = align_up(o + sizeof(int32_t) * (size_t)R);
     L.scratch = o; o = align_up(o + map_scratch_bytes(R, E));
     L.h = o; o = align_up(o + esize(dt) * (size_t)R * (size_t)F);
+    L.xs_bytes = with_xs && pregather_shape(R, D, F, E, dt) ? esize(dt) * (size_t)R * (size_t)D : 0;
+    L.xs = o; o = align_up(o + L.xs_bytes);
     L.total = o;
     return L;
 }
@@ -141,7 +162,7 @@ struct MoaLayout {
 MoaLayout moa_layout(int64_t S, int64_t HD, int32_t E, int32_t k) {
     const int64_t R = S * k;
     MoaLayout L;
-    L.base = mlp_layout(S, 0, E, k, MOE_BF16);
+    L.base = mlp_layout(S, 0, 0, E, k, MOE_BF16);
     size_t o = L.base.total;
     L.kv_off = o; o = align_up(o + 2 * sizeof(int32_t));
     L.kv = o; o = align_up(o + 2 * (size_t)S * 2 * (size_t)HD);
@@ -273,20 +294,19 @@ size_t moe_workspace_size(const char *op, int64_t S, int64_t D, int64_t F, int32
     if (strcmp(op, "ep_dispatch") == 0) return map_ws_bytes(S, E, k);
     if (strcmp(op, "expert_mlp_forward") == 0) {  // S = rows, k = 1
         if (F <= 0 || k != 1 || (dt != MOE_F32 && dt != MOE_BF16)) return 0;
-        return mlp_layout(S, F, E, 1, dt).total;
+        return mlp_layout(S, D, F, E, 1, dt, false).total;
     }
     if (strcmp(op, "mlp_forward") == 0) {
         if (F <= 0 || (dt != MOE_F32 && dt != MOE_BF16)) return 0;
-        return mlp_layout(S, F, E, k, dt).total;
+        return mlp_layout(S, D, F, E, k, dt).total;
     }
     return 0;
 }
 
 int64_t moe_workspace_view(const char *which, int64_t S, int64_t D, int64_t F, int32_t E,
                            int32_t k, moe_dtype dt) {
-    (void)D;
     if (which == nullptr) return -1;
-    const MlpLayout L = mlp_layout(S, F, E, k, dt);
+    const MlpLayout L = mlp_layout(S, D, F, E, k, dt);
     if (!strcmp(which, "top_experts")) return (int64_t)L.top_e;
     if (!strcmp(which, "top_weights")) return (int64_t)L.top_w;
     if (!strcmp(which, "expert_counts")) return (int64_t)L.counts;
@@ -294,6 +314,7 @@ int64_t moe_workspace_view(const char *which, int64_t S, int64_t D, int64_t F, i
     if (!strcmp(which, "sparse_rows")) return (int64_t)L.sparse_rows;
     if (!strcmp(which, "sorted_rows")) return (int64_t)L.sorted_rows;
     if (!strcmp(which, "h")) return (int64_t)L.h;
+    if (!strcmp(which, "x_sorted")) return L.xs_bytes > 0 ? (int64_t)L.xs : -1;
     return -1;
 }
 
@@ -539,7 +560,7 @@ int moe_mlp_forward(const void *x, const void *w_gate, const float *logit_bias,
         (rc = check_ptr("w_gate_e", w_gate_e, 16)) || (rc = check_ptr("w_up", w_up, 16)) ||
         (rc = check_ptr("w_down", w_down, 16)) || (rc = check_ptr("out", out, 16, S == 0)))
         return rc;
-    const MlpLayout L = mlp_layout(S, F, E, k, dt);
+    const MlpLayout L = mlp_layout(S, D, F, E, k, dt);
     if ((rc = check_ws(ws, ws_bytes, L.total))) return rc;
     if ((rc = check_device())) return rc;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -575,9 +596,18 @@ int moe_mlp_forward(const void *x, const void *w_gate, const float *logit_bias,
     if ((rc = check_launch("sparse_map"))) return rc;
     record_prof(2, s);
     if (R > 0) {
+        // x rows copied to slot order first (the gather's own kernel), so that GEMM1 loads them
+        // by TMA like GEMM2's h rows; otherwise GEMM1 gathers them on load
+        const bool pregather = L.xs_bytes > 0 && !env_off("MOE_PREGATHER");
+        void *xs = at<void>(ws, L.xs);
+        if (pregather) {
+            launch_gather_rows(x, sorted_rows, k, R, D, xs, status, s);
+            if ((rc = check_launch("gather_rows"))) return rc;
+            ++n;
+        }
         GemmArgs a{};
-        a.A = x;
-        a.a_rows = S;
+        a.A = pregather ? xs : x;
+        a.a_rows = pregather ? R : S;
         a.B0 = w_gate_e;
         a.B1 = w_up;
         a.offsets = offsets;
@@ -591,7 +621,7 @@ int moe_mlp_forward(const void *x, const void *w_gate, const float *logit_bias,
         a.K = D;
         a.N = F;
         a.bf16 = dt == MOE_BF16;
-        a.gather = true;
+        a.gather = !pregather;
         a.glu = true;
         a.scatter = false;
         a.zero_ptr = out;   // zeroed by GEMM1's epilogue warps before GEMM2 adds into it
@@ -694,7 +724,7 @@ extern "C" int moe_mlp_backward(const void *x, const void *w_gate, const void *w
         (rc = check_ptr("dw_gate_e", dw_gate_e, 16)) || (rc = check_ptr("dw_up", dw_up, 16)) ||
         (rc = check_ptr("dw_down", dw_down, 16)))
         return rc;
-    const MlpLayout FL = mlp_layout(S, F, E, k, dt);
+    const MlpLayout FL = mlp_layout(S, D, F, E, k, dt);
     if (fwd_ws == nullptr || fwd_ws_bytes < FL.total)
         return set_error(MOE_ERR_WORKSPACE, "the forward's workspace is missing or too small");
     const MlpBwdLayout L = mlp_bwd_layout(S, D, F, E, k);
@@ -1056,7 +1086,7 @@ int moe_expert_mlp_forward(const void *x_rows, const int32_t *expert_ids, int32_
         (rc = check_ptr("w_down", w_down, 16)) || (rc = check_ptr("y", y, 16, R == 0)))
         return rc;
     // the forward's layout with one route per row: top_e holds the local ids
-    const MlpLayout L = mlp_layout(R, F, E, 1, dt);
+    const MlpLayout L = mlp_layout(R, D, F, E, 1, dt, false);
     if ((rc = check_ws(ws, ws_bytes, L.total))) return rc;
     if ((rc = check_device())) return rc;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

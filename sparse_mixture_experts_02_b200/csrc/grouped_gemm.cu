@@ -608,7 +608,7 @@ int launch_t(const GemmArgs &a, cudaStream_t s) {
 
 int launch_grouped_gemm(const GemmArgs &a, cudaStream_t s) {
     // instantiated forms: (gather, glu, scatter) in {(1,1,0), (0,0,1), (1,0,0), (1,0,1),
-    // (0,0,0)} x {bf16, f32}
+    // (0,0,0)} x {bf16, f32}, and (0,1,0) in bf16 (SwiGLU on x rows copied to slot order)
     // GLU backward epilogue (bf16, gathered x, fused gate+up): the MLP backward's recompute
     if (a.glu_bwd) {
         if (a.bf16 && a.gather && a.glu && !a.scatter && !a.b_kmajor)
@@ -628,6 +628,7 @@ int launch_grouped_gemm(const GemmArgs &a, cudaStream_t s) {
     MOE_DISPATCH_KM(false, false)
 #undef MOE_DISPATCH_KM
     MOE_DISPATCH(true, true, true, false)
+    MOE_DISPATCH(true, false, true, false)
     MOE_DISPATCH(true, false, false, true)
     MOE_DISPATCH(true, true, false, false)
     MOE_DISPATCH(true, true, false, true)

@@ -500,6 +500,7 @@ int launch_grouped_gemm_2sm(const GemmArgs &a, cudaStream_t s) {
     if (a.bf16 == BF && a.gather == G && a.glu == L && a.scatter == SC)                     \
         return launch_2sm_t<BF, G, L, SC>(a, s, pairs);
     MOE_DISPATCH2(true, true, true, false)
+    MOE_DISPATCH2(true, false, true, false)
     MOE_DISPATCH2(true, false, false, true)
     MOE_DISPATCH2(true, true, false, false)
     MOE_DISPATCH2(true, true, false, true)

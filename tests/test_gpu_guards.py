@@ -39,6 +39,8 @@ CASES = {
     "few_routes": W.custom("few_routes", S=3, D=72, F=64, E=4, k=1, dtype="bf16"),
     # fp32 (tf32 MMAs), several tiles per expert with a short last tile
     "tails_f32": W.custom("tails_f32", S=700, D=200, F=328, E=3, k=2, dtype="f32"),
+    # x rows copied to slot order before GEMM1 (experts of >= 384 rows, F >= 2048); ragged tiles
+    "pregather": W.custom("pregather", S=1000, D=136, F=2056, E=2, k=1, dtype="bf16"),
 }
 
 
@@ -90,6 +92,8 @@ def _check_forward_guards(moe, w, ws, ws_big, out_big):
                 ("expert_offsets", (E + 1) * 4), ("sparse_rows", R * 4), ("sorted_rows", R * 4),
                 ("h", R * F * hb)]
     code = moe.MOE_BF16 if w.dtype == "bf16" else moe.MOE_F32
+    if moe.workspace_view("x_sorted", S, D, F, E, k, code) >= 0:
+        sections.append(("x_sorted", R * D * hb))
     spans = sorted((moe.workspace_view(n, S, D, F, E, k, code), sz, n) for n, sz in sections)
     for (off, sz, name), nxt in zip(spans, spans[1:] + [(n_ws, 0, "end")]):
         if name == "sorted_rows":

@@ -31,6 +31,8 @@ SMALL = {
     "one_token": W.custom("one_token", S=1, D=128, F=256, E=8, k=8, dtype="bf16"),
     "e256": W.custom("e256", S=600, D=96, F=64, E=256, k=8, dtype="bf16",
                      router_std="1/sqrt(D)"),
+    # 600 rows an expert, F = 2048: GEMM1 reads x rows copied to slot order (a K tail: D = 72)
+    "pregather": W.custom("pregather", S=1200, D=72, F=2048, E=2, k=1, dtype="bf16"),
 }
 
 FULL_WORKLOADS = ["mixtral_prefill", "mixtral_decode", "e128", "zipf64"]
@@ -97,6 +99,24 @@ def test_mlp_small_all_tokens(oracle_lib, moe, monkeypatch, name, cta):
     w = SMALL[name]
     inp = {k: (t.cuda() if t is not None else None) for k, t in W.make_inputs(w).items()}
     _check_case(oracle_lib, moe, w, inp, np.arange(w.S, dtype=np.int32))
+
+
+@pytest.mark.parametrize("cta", ["0", "1"])
+def test_mlp_slot_ordered_x_matches_gather_on_load(moe, monkeypatch, cta):
+    """GEMM1 on x rows copied to slot order runs the same MMAs in the same K order as GEMM1
+    gathering them on load: h and the output are bit-identical (MOE_PREGATHER=0 turns the copy
+    off), and the copy is the x rows in slot order."""
+    monkeypatch.setenv("MOE_GEMM_2SM", cta)
+    w = SMALL["pregather"]
+    inp = {k: (t.cuda() if t is not None else None) for k, t in W.make_inputs(w).items()}
+    out1, ws1, v1 = _forward(moe, inp, w)
+    xs = ws1.view("x_sorted")
+    routes = torch.from_numpy(v1["sorted_rows"].astype(np.int64)).cuda()
+    assert torch.equal(xs, inp["x"][routes // w.k])
+    monkeypatch.setenv("MOE_PREGATHER", "0")
+    out0, ws0, v0 = _forward(moe, inp, w)
+    assert torch.equal(ws0.view("h"), ws1.view("h"))
+    assert torch.equal(out0, out1)
 
 
 def test_mlp_empty_batch(moe):

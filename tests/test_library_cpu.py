@@ -78,6 +78,30 @@ def test_workspace_sizes(moe):
     assert moe.workspace_view("bogus", S, D, F, E, k, 1) == -1
 
 
+def test_forward_workspace_slot_ordered_x(moe):
+    # bf16 forwards with experts of >= 384 rows on average and F >= 2048 copy x to slot order
+    # before GEMM1: their workspace carries an "x_sorted" region [S*k, D] after h
+    def size_view(S, D, F, E, k, dt):
+        return (moe.workspace_size("mlp_forward", S, D, F, E, k, dt),
+                moe.workspace_view("x_sorted", S, D, F, E, k, dt),
+                moe.workspace_view("h", S, D, F, E, k, dt))
+    S, D, F, E, k = 4096, 4096, 14336, 8, 2          # the Mixtral-shaped prefill layer
+    total, xs, h = size_view(S, D, F, E, k, moe.MOE_BF16)
+    R = S * k
+    assert xs >= h + R * F * 2 and xs % 256 == 0 and xs + R * D * 2 <= total
+    # the same layer without the copy is that region smaller, everything before it unchanged
+    for S2, F2, E2, dt in [(192 * 8 - 1, F, E, moe.MOE_BF16),   # R / E = 383
+                           (S, 2040, E, moe.MOE_BF16),          # F < 2048
+                           (S, F, E, moe.MOE_F32)]:             # fp32
+        t2, x2, h2 = size_view(S2, D, F2, E2, k, dt)
+        assert x2 == -1
+    t_edge, x_edge, _ = size_view(192 * 8, D, 2048, E, k, moe.MOE_BF16)  # R / E = 384, F = 2048
+    assert x_edge > 0 and x_edge + 192 * 8 * k * D * 2 <= t_edge
+    # the expert-parallel forward gathers its rows on load and has no such region
+    t_ep = moe.workspace_size("expert_mlp_forward", R, D, F, E, 1, moe.MOE_BF16)
+    assert t_ep < total
+
+
 @pytest.mark.parametrize("R", [16385, 32768, 75264, 75265, 98304, 300000, 602112, 602113,
                                1 << 22, (1 << 22) + 1])
 @pytest.mark.parametrize("E", [8, 256])
