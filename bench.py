@@ -50,13 +50,15 @@ TRAFFIC_JSON = os.path.join(ROOT, "profiles", "dram_traffic.json")
 CSRC = os.path.join(ROOT, "sparse_mixture_experts_02_b200", "csrc")
 # sources that define each kernel class (a recorded DRAM figure is void once any of them changes)
 KERNEL_SOURCES = {
+    "x_copy": ("backward.cu", "moe_internal.cuh"),
     "gemm1": ("grouped_gemm.cu", "grouped_gemm_2sm.cu", "gemm_common.cuh", "moe_internal.cuh"),
     "gemm2": ("grouped_gemm.cu", "grouped_gemm_2sm.cu", "gemm_common.cuh", "moe_internal.cuh"),
     "router": ("route.cu", "grouped_gemm.cu", "gemm_common.cuh", "moe_internal.cuh"),
     "sparse_map": ("sparse_map.cu", "moe_internal.cuh"),
 }
-# forward stages in the order the library records its events
-STAGES = ("route", "sparse_map", "gemm1", "gemm2")
+# forward stages in the order the library records its events; x_copy (the x rows copied to slot
+# order before GEMM1, for large experts and F >= 2048) takes no time when the forward makes none
+STAGES = ("route", "sparse_map", "x_copy", "gemm1", "gemm2")
 
 
 def elt_bytes(w: W.Workload) -> int:
@@ -82,6 +84,8 @@ def bytes_of(w: W.Workload, e_act: int) -> dict:
         "route": w.S * w.D * b + w.D * w.E * b + 8 * R,
         # routes read, slots and inverse permutation written, counts and offsets written
         "sparse_map": 12 * R + (2 * w.E + 1) * 4,
+        # an implementation step, not the method's: its 4 R D bytes are not algorithmic
+        "x_copy": 0,
         # x read, gate and up weights of active experts read, h written, out zeroed
         "gemm1": w.S * w.D * b + 2 * e_act * w.D * w.F * b + R * w.F * b + w.S * w.D * 4,
         # h read, down weights of active experts read, out read and written by the reductions
@@ -153,7 +157,7 @@ def kernel_class(name: str):
         router = m.group(1) == "grouped_gemm_kernel" and len(a) > 4 and a[4] == 1
         if router:
             return "router"
-        if gather and glu and not scatter:
+        if glu and not scatter:  # x rows gathered on load or copied to slot order first
             return "gemm1"
         if scatter and not gather and not glu:
             return "gemm2"
@@ -162,6 +166,8 @@ def kernel_class(name: str):
         return "router"
     if re.search(r"\bmap_\w+_kernel", name):
         return "sparse_map"
+    if re.search(r"\bgather_rows_kernel", name):
+        return "x_copy"
     return None
 
 
@@ -414,8 +420,10 @@ def time_forward(moe, w, steps, warmup, dev, ws=1, seed=0):
     moe.check_device_status(wsp)
     launches_per_step = moe.last_launch_count()
 
-    # events for the per-stage breakdown, 5 per step, created and recorded once up front
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+    # events for the per-stage breakdown, one more than the stages per step, created and
+    # recorded once up front
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(STAGES) + 1)]
+           for _ in range(steps)]
     for row in evs:
         for e in row:
             e.record(stream)
@@ -433,7 +441,7 @@ def time_forward(moe, w, steps, warmup, dev, ws=1, seed=0):
                 flush_buf.zero_()
                 step(i, evs[i])
             torch.cuda.synchronize(dev)
-            ms_total = sum(r[0].elapsed_time(r[4]) for r in evs)
+            ms_total = sum(r[0].elapsed_time(r[len(STAGES)]) for r in evs)
         else:
             t0.record(stream)
             for i in range(steps):
@@ -464,7 +472,8 @@ def time_forward(moe, w, steps, warmup, dev, ws=1, seed=0):
         "tflops": sum(fl.values()) / s_per_step / 1e12,
         "gbs": sum(by.values()) / s_per_step / 1e9,
         "stage_ms": stage_ms,
-        "stage_gbs": {n: by[n] / (stage_ms[n] / 1000.0) / 1e9 for n in STAGES if stage_ms[n] > 0},
+        "stage_gbs": {n: by[n] / (stage_ms[n] / 1000.0) / 1e9 for n in STAGES
+                      if stage_ms[n] > 0 and by[n] > 0},
         "expert_hist": hist,
         "roofline": roofline(w, stage_ms, e_act, clocks, ms_total / 1000.0),
         "clocks": clocks,

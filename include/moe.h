@@ -342,7 +342,8 @@ int moe_debug_build(void);
  * Optional per-stage timing on the calling host thread: when `events` holds n cudaEvent_t
  * handles (n <= 8), the next moe_mlp_forward, moe_mlp_backward or moe_moa_forward records the
  * first n of its stage events on its stream; then the registration clears.
- *   moe_mlp_forward (5): start, after route, after the sparse map, after GEMM1, after GEMM2.
+ *   moe_mlp_forward (6): start, after route, after the sparse map, after the copy of the x rows
+ *     to slot order (recorded at once when the forward makes none), after GEMM1, after GEMM2.
  *   moe_mlp_backward (7): start, after dh, after the recomputed GEMM1 with the SwiGLU backward,
  *     after dW_down, after dx, after dW_gate_e and dW_up, after the router backward.
  *   moe_moa_forward (7): start, after route, after the sparse map, after the key/value

@@ -605,6 +605,7 @@ int moe_mlp_forward(const void *x, const void *w_gate, const float *logit_bias,
             if ((rc = check_launch("gather_rows"))) return rc;
             ++n;
         }
+        record_prof(3, s);
         GemmArgs a{};
         a.A = pregather ? xs : x;
         a.a_rows = pregather ? R : S;
@@ -632,7 +633,7 @@ int moe_mlp_forward(const void *x, const void *w_gate, const float *logit_bias,
             return rc;
         if ((rc = check_launch("gemm1"))) return rc;
         ++n;
-        record_prof(3, s);
+        record_prof(4, s);
         GemmArgs b = a;
         b.zero_ptr = nullptr;
         b.zero_n = 0;
@@ -651,10 +652,11 @@ int moe_mlp_forward(const void *x, const void *w_gate, const float *logit_bias,
             return rc;
         if ((rc = check_launch("gemm2"))) return rc;
         ++n;
-        record_prof(4, s);
+        record_prof(5, s);
     } else {
         record_prof(3, s);
         record_prof(4, s);
+        record_prof(5, s);
     }
     g_prof_n = 0;
     g_launches = n;

@@ -65,6 +65,10 @@ def test_kernel_names_are_classified():
     assert c("void unnamed>::grouped_gemm_kernel<1, 0, 0, 0, 1>(CUtensorMap_st, ...)") == "router"
     assert c("void unnamed>::grouped_gemm_2sm_kernel<1, 1, 1, 0>(CUtensorMap_st, ...)") == "gemm1"
     assert c("void unnamed>::grouped_gemm_2sm_kernel<1, 0, 0, 1>(CUtensorMap_st, ...)") == "gemm2"
+    # GEMM1 on x rows copied to slot order, and that copy
+    assert c("void unnamed>::grouped_gemm_2sm_kernel<1, 0, 1, 0>(CUtensorMap_st, ...)") == "gemm1"
+    assert c("void unnamed>::grouped_gemm_kernel<1, 0, 1, 0, 0, 0, 0>(CUtensorMap_st, ...)") == "gemm1"
+    assert c("moe::<unnamed>::gather_rows_kernel(const uint4 *, const int *, int, ...)") == "x_copy"
     assert c("void moe::route_e8_kernel<2>(const __nv_bfloat16 *, ...)") == "router"
     assert c("void moe::map_small_kernel(const int *, long, int, ...)") == "sparse_map"
     assert c("void at::native::vectorized_elementwise_kernel<4, ...>") is None
