@@ -205,7 +205,7 @@ int32_t router_chunks(int64_t S, int64_t D) {
 
 // MLP backward scratch (the forward's workspace supplies routing, map and h).
 struct MlpBwdLayout {
-    size_t status, dyb, dhp, dpre, dw, dv, dl, xs, off1, partial, wgt, total;
+    size_t status, dhp, dpre, dw, dv, dl, xs, off1, partial, wgt, total;
 };
 
 MlpBwdLayout mlp_bwd_layout(int64_t S, int64_t D, int64_t F, int32_t E, int32_t k) {
@@ -213,7 +213,6 @@ MlpBwdLayout mlp_bwd_layout(int64_t S, int64_t D, int64_t F, int32_t E, int32_t 
     MlpBwdLayout L;
     size_t o = 0;
     L.status = o; o += kStatusBytes;
-    L.dyb = o; o = align_up(o + 2 * (size_t)S * (size_t)D);
     L.dhp = o; o = align_up(o + 2 * (size_t)R * (size_t)F);
     // [da | db], the gated dout rows and the router's dl in the weight gradient's padded layout
     const int64_t Rp = R + (int64_t)kWgradPad * E;
@@ -756,13 +755,21 @@ extern "C" int moe_mlp_backward(const void *x, const void *w_gate, const void *w
     // profile events (moe_profile_events): 0 start, 1 after dh, 2 after the GEMM1 recompute with
     // the SwiGLU backward, 3 after dW_down, 4 after dx, 5 after dW_gate_e/dW_up, 6 end
     record_prof(0, s);
-    void *dyb = at<void>(ws, L.dyb), *dhp = at<void>(ws, L.dhp);
+    void *dhp = at<void>(ws, L.dhp);
     void *dpre = at<void>(ws, L.dpre), *dv = at<void>(ws, L.dv);
     void *dl = at<void>(ws, L.dl);
     float *dwr = at<float>(ws, L.dw);
     int32_t *off1 = at<int32_t>(ws, L.off1);
-    launch_cast_bf16(dout, dyb, S * D, s);
+    // dout rows (bf16, ungated) in slot order, in the padded layout of dv (the weight gradient
+    // refills dv with the gated rows below); dh then reads them by TMA instead of gathering them
+    launch_gate_rows(dout, false, sorted_rows, nullptr, k, R, D, true, dv, offsets, E, status, s);
     ++n;
+    // x rows in slot order: read by TMA in the GEMM1 recompute, then by the W_gate_e / W_up
+    // weight gradient
+    void *xs = at<void>(ws, L.xs);
+    launch_gather_rows(x, sorted_rows, k, R, D, xs, status, s);
+    ++n;
+    const int64_t Rp = R + (int64_t)kWgradPad * E;
     GemmArgs g{};
     g.offsets = offsets;
     g.sorted_rows = sorted_rows;
@@ -776,33 +783,33 @@ extern "C" int moe_mlp_backward(const void *x, const void *w_gate, const void *w
     // GEMM2 backward, ungated: dhp[p] = dout[s] . W_down[e]^T (W_down [E, F, D] read K-major)
     {
         GemmArgs a = g;
-        a.A = dyb;
-        a.a_rows = S;
+        a.A = dv;
+        a.a_rows = Rp;
+        a.a_row_pad = kWgradPad;
         a.B0 = w_down;
         a.b_kmajor = true;
         a.out = dhp;
         a.K = D;
         a.N = F;
-        a.gather = true;
+        a.gather = false;
         if ((rc = launch_grouped_gemm(a, s))) return rc;
         ++n;
     }
     record_prof(1, s);
-    // GEMM1 recomputed (fused gate+up, gathered x) with the SwiGLU backward in its epilogue: the
+    // GEMM1 recomputed (fused gate+up, slot-ordered x) with the SwiGLU backward in its epilogue: the
     // route-weight gradient dh_u . h (atomically per N tile) and [da | db] in the padded layout
-    const int64_t Rp = R + (int64_t)kWgradPad * E;
     launch_zero_f32(dwr, R, nullptr, s);
     {
         GemmArgs a = g;
-        a.A = x;
-        a.a_rows = S;
+        a.A = xs;
+        a.a_rows = R;
         a.B0 = w_gate_e;
         a.B1 = w_up;
         a.gates = top_w;
         a.out = dpre;
         a.K = D;
         a.N = F;
-        a.gather = true;
+        a.gather = false;
         a.glu = true;
         a.glu_bwd = true;
         a.bwd_dh = dhp;
@@ -853,9 +860,6 @@ extern "C" int moe_mlp_backward(const void *x, const void *w_gate, const void *w
     }
     record_prof(4, s);
     // dW_gate_e, dW_up from the x rows in slot order and the two halves of [da | db]
-    void *xs = at<void>(ws, L.xs);
-    launch_gather_rows(x, sorted_rows, k, R, D, xs, status, s);
-    ++n;
     for (int half = 0; half < 2; ++half) {
         WgradArgs w{};
         w.A = xs;

@@ -609,10 +609,13 @@ int launch_t(const GemmArgs &a, cudaStream_t s) {
 int launch_grouped_gemm(const GemmArgs &a, cudaStream_t s) {
     // instantiated forms: (gather, glu, scatter) in {(1,1,0), (0,0,1), (1,0,0), (1,0,1),
     // (0,0,0)} x {bf16, f32}, and (0,1,0) in bf16 (SwiGLU on x rows copied to slot order)
-    // GLU backward epilogue (bf16, gathered x, fused gate+up): the MLP backward's recompute
+    // GLU backward epilogue (bf16, gathered or slot-ordered x, fused gate+up): the MLP backward's
+    // recompute
     if (a.glu_bwd) {
-        if (a.bf16 && a.gather && a.glu && !a.scatter && !a.b_kmajor)
-            return launch_t<true, true, true, false, false, false, true>(a, s);
+        if (a.bf16 && a.glu && !a.scatter && !a.b_kmajor) {
+            if (a.gather) return launch_t<true, true, true, false, false, false, true>(a, s);
+            return launch_t<true, false, true, false, false, false, true>(a, s);  // slot-ordered x
+        }
         return set_error(MOE_ERR_UNSUPPORTED, "GLU backward epilogue form not built");
     }
 #define MOE_DISPATCH(BF, G, L, SC)                                                          \
