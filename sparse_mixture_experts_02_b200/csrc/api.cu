@@ -792,7 +792,8 @@ extern "C" int moe_mlp_backward(const void *x, const void *w_gate, const void *w
         a.K = D;
         a.N = F;
         a.gather = false;
-        if ((rc = launch_grouped_gemm(a, s))) return rc;
+        if ((rc = prefer_2sm(R, E) ? launch_grouped_gemm_2sm(a, s) : launch_grouped_gemm(a, s)))
+            return rc;
         ++n;
     }
     record_prof(1, s);
@@ -815,7 +816,8 @@ extern "C" int moe_mlp_backward(const void *x, const void *w_gate, const void *w
         a.bwd_dh = dhp;
         a.bwd_dw = dwr;
         a.out_row_pad = kWgradPad;
-        if ((rc = launch_grouped_gemm(a, s))) return rc;
+        if ((rc = prefer_2sm(R, E) ? launch_grouped_gemm_2sm(a, s) : launch_grouped_gemm(a, s)))
+            return rc;
     }
     launch_zero_pad_rows(dpre, 2 * F, 2 * F, offsets, E, s);
     n += 3;
@@ -855,7 +857,8 @@ extern "C" int moe_mlp_backward(const void *x, const void *w_gate, const void *w
         a.N = D;
         a.gather = false;
         a.scatter = true;
-        if ((rc = launch_grouped_gemm(a, s))) return rc;
+        if ((rc = prefer_2sm(R, E) ? launch_grouped_gemm_2sm(a, s) : launch_grouped_gemm(a, s)))
+            return rc;
         ++n;
     }
     record_prof(4, s);

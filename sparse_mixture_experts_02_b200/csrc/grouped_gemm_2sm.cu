@@ -68,7 +68,12 @@ constexpr size_t smem2_bytes() {
 static_assert(smem2_bytes<true>() <= 232448 && smem2_bytes<false>() <= 232448,
               "dynamic shared memory per CTA");
 
-template <bool BF16, bool GATHER, bool GLU, bool SCATTER>
+// BKM: the weights read K-major ([E, N, K], a weight [E, K, N] of the forward read as its
+// transpose, optionally split over two tensor maps at K = k_split), one 64 x 128 box per CTA and
+// stage, and slot-ordered A rows in the padded layout (row p of expert e at p + a_row_pad * e):
+// the input-gradient GEMMs of the MLP backward. GBWD: the SwiGLU-backward epilogue of the
+// recomputed GEMM1 (glu_bwd_row). Both are compile-time forms; the forward's are untouched.
+template <bool BF16, bool GATHER, bool GLU, bool SCATTER, bool BKM = false, bool GBWD = false>
 __global__ void __cluster_dims__(2, 1, 1)
 __launch_bounds__(GATHER ? GATHER_BLOCK : THREADS, 1)
 grouped_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
@@ -81,7 +86,9 @@ grouped_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
     constexpr int CHUNK = BK * KBYTES;
     constexpr int B_KSTEP = (32 / EB) * KBYTES;
     constexpr int OUT_COLS = GLU ? BN / 2 : BN;
-    constexpr uint32_t IDESC = dev::idesc_f32acc(BF16, 256, BN, true);
+    static_assert(!BKM || (BF16 && !GLU && !GATHER), "K-major weights: plain bf16 forms");
+    static_assert(!GBWD || (BF16 && GLU && !SCATTER && !GATHER), "SwiGLU-backward form");
+    constexpr uint32_t IDESC = dev::idesc_f32acc(BF16, 256, BN, !BKM);
     constexpr uint32_t B_LAYOUT = BF16 ? dev::kLayoutSw128 : dev::kLayoutSw128Base32;
     constexpr uint32_t B_SBO = BF16 ? 1024 : 512;
     static_assert(NCH * CHUNK == B2_BYTES, "B half size");
@@ -121,7 +128,7 @@ grouped_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
     if (warp == 0 && lane == 0) {
         dev::prefetch_tmap(&tmA);
         dev::prefetch_tmap(&tmB0);
-        if (GLU) dev::prefetch_tmap(&tmB1);
+        if (GLU || BKM) dev::prefetch_tmap(&tmB1);
     }
     if (warp == 1) {
         dev::tmem_alloc_cg2(&st.tmem_base, TMEM_COLS);
@@ -166,16 +173,25 @@ grouped_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
                     const uint32_t full0 = dev::mapa_shared(dev::smem_u32(&st.full[s]), 0);
                     if (leader) dev::mbar_arrive_expect_tx(&st.full[s], tx);
                     const int kc = kb * BK;
-                    if (!GATHER)
-                        dev::tma_load_2d_cg2(sA, &tmA, full0, kc, ti.row_begin + 128 * (int)rank);
+                    if (!GATHER) {
+                        int arow = ti.row_begin + 128 * (int)rank;
+                        if constexpr (BKM) arow += p.a_row_pad * ti.e;
+                        dev::tma_load_2d_cg2(sA, &tmA, full0, kc, arow);
+                    }
+                    if constexpr (BKM) {
+                        const bool hi = kc >= p.k_split;
+                        dev::tma_load_3d_cg2(sB, hi ? &tmB1 : &tmB0, full0,
+                                             hi ? kc - p.k_split : kc, n0 + 128 * (int)rank, ti.e);
+                    } else {
 #pragma unroll
-                    for (int c = 0; c < NCH; ++c) {
-                        if (GLU) {
-                            dev::tma_load_3d_cg2(sB + c * CHUNK, leader ? &tmB0 : &tmB1, full0,
-                                                 n0 + c * CW, kc, ti.e);
-                        } else {
-                            dev::tma_load_3d_cg2(sB + c * CHUNK, &tmB0, full0,
-                                                 n0 + 128 * (int)rank + c * CW, kc, ti.e);
+                        for (int c = 0; c < NCH; ++c) {
+                            if (GLU) {
+                                dev::tma_load_3d_cg2(sB + c * CHUNK, leader ? &tmB0 : &tmB1, full0,
+                                                     n0 + c * CW, kc, ti.e);
+                            } else {
+                                dev::tma_load_3d_cg2(sB + c * CHUNK, &tmB0, full0,
+                                                     n0 + 128 * (int)rank + c * CW, kc, ti.e);
+                            }
                         }
                     }
                 }
@@ -222,7 +238,9 @@ grouped_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
                     for (int kk = 0; kk < KBYTES / 32; ++kk) {
                         const uint64_t ad =
                             dev::sdesc(sA + kk * 32, 16, 1024, dev::kLayoutSw128);
-                        const uint64_t bd = dev::sdesc(sB + kk * B_KSTEP, CHUNK, B_SBO, B_LAYOUT);
+                        const uint64_t bd =
+                            BKM ? dev::sdesc(sB + kk * 32, 16, 1024, dev::kLayoutSw128)
+                                : dev::sdesc(sB + kk * B_KSTEP, CHUNK, B_SBO, B_LAYOUT);
                         if (BF16) dev::mma_bf16_cg2(d_tmem, ad, bd, IDESC, (kb | kk) != 0);
                         else dev::mma_tf32_cg2(d_tmem, ad, bd, IDESC, (kb | kk) != 0);
                     }
@@ -379,10 +397,15 @@ grouped_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
             }
             const int n0 = ti.n_idx * OUT_COLS;
             const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + b * BN;
-            if constexpr (GLU)
+            if constexpr (GBWD) {
+                const int64_t route = valid ? (int64_t)__ldg(p.sorted_rows + prow) : 0;
+                glu_bwd_row(p, tbase, valid, prow, route, g,
+                            prow + (int64_t)p.out_row_pad * ti.e, n0);
+            } else if constexpr (GLU) {
                 epilogue_row<BF16, GLU, SCATTER>(p, tbase, valid, orow, g, n0, nullptr);
-            else
+            } else {
                 epilogue_row<BF16, GLU, SCATTER>(p, tbase, valid, orow, g, n0, st.stage[q]);
+            }
             dev::tc_fence_before();
             __syncwarp();
             if (lane == 0) dev::mbar_arrive_cluster(tempty0_base + b * (uint32_t)sizeof(uint64_t));
@@ -397,12 +420,12 @@ grouped_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
     }
 }
 
-template <bool BF16, bool GATHER, bool GLU, bool SCATTER>
+template <bool BF16, bool GATHER, bool GLU, bool SCATTER, bool BKM = false, bool GBWD = false>
 int launch_2sm_t(const GemmArgs &a, cudaStream_t s, int n_pairs) {
     constexpr int EB = BF16 ? 2 : 4;
     constexpr int BK = KBYTES / EB;
     constexpr int CW = KBYTES / EB;
-    auto kern = grouped_gemm_2sm_kernel<BF16, GATHER, GLU, SCATTER>;
+    auto kern = grouped_gemm_2sm_kernel<BF16, GATHER, GLU, SCATTER, BKM, GBWD>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [&] {
@@ -419,7 +442,26 @@ int launch_2sm_t(const GemmArgs &a, cudaStream_t s, int n_pairs) {
         int rc = encode_tmap(&mA, BF16, 2, a.A, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
         if (rc) return rc;
     }
-    {
+    if (BKM) {
+        // [E, N, K0] and [E, N, K - K0] with K contiguous, one (BK x 128) box per CTA and stage
+        const int64_t k0 = a.B1 != nullptr ? a.k_split : a.K;
+        if (a.B1 != nullptr && (k0 <= 0 || k0 >= a.K || k0 % BK != 0))
+            return set_error(MOE_ERR_UNSUPPORTED, "K split %lld is not a positive multiple of %d "
+                             "below K=%lld", (long long)k0, BK, (long long)a.K);
+        const uint32_t box[3] = {(uint32_t)BK, 128u, 1u};
+        const uint64_t dims0[3] = {(uint64_t)k0, (uint64_t)a.N, (uint64_t)a.E};
+        const uint64_t str0[2] = {(uint64_t)k0 * EB, (uint64_t)a.N * k0 * EB};
+        int rc = encode_tmap(&mB0, BF16, 3, a.B0, dims0, str0, box, CU_TENSOR_MAP_SWIZZLE_128B);
+        if (rc) return rc;
+        if (a.B1 != nullptr) {
+            const uint64_t dims1[3] = {(uint64_t)(a.K - k0), (uint64_t)a.N, (uint64_t)a.E};
+            const uint64_t str1[2] = {(uint64_t)(a.K - k0) * EB, (uint64_t)a.N * (a.K - k0) * EB};
+            rc = encode_tmap(&mB1, BF16, 3, a.B1, dims1, str1, box, CU_TENSOR_MAP_SWIZZLE_128B);
+            if (rc) return rc;
+        } else {
+            mB1 = mB0;
+        }
+    } else {
         const uint64_t dims[3] = {(uint64_t)a.N, (uint64_t)a.K, (uint64_t)a.E};
         const uint64_t str[2] = {(uint64_t)a.N * EB, (uint64_t)a.N * a.K * EB};
         const uint32_t box[3] = {(uint32_t)CW, (uint32_t)BK, 1u};
@@ -453,6 +495,11 @@ int launch_2sm_t(const GemmArgs &a, cudaStream_t s, int n_pairs) {
     kp.zero_n4 = a.zero_n / 4;
     kp.status = a.status;
     kp.wait_limit_ns = a.wait_limit_ns;
+    kp.k_split = (int32_t)(BKM && a.B1 != nullptr ? a.k_split : a.K + BK);
+    kp.a_row_pad = BKM ? a.a_row_pad : 0;
+    kp.out_row_pad = a.out_row_pad;
+    kp.bwd_dh = a.bwd_dh;
+    kp.bwd_dw = a.bwd_dw;
     kern<<<2 * n_pairs, GATHER ? GATHER_BLOCK : THREADS, smem2_bytes<GLU>(), s>>>(mA, mB0, mB1,
                                                                               kp);
     return MOE_OK;
@@ -492,10 +539,22 @@ int max_pairs() {
 }  // namespace
 
 int launch_grouped_gemm_2sm(const GemmArgs &a, cudaStream_t s) {
-    if (a.b_kmajor || a.a_row_pad != 0 || a.glu_bwd)
-        return set_error(MOE_ERR_UNSUPPORTED,
-                         "two-CTA grouped GEMM: K-major B / padded A / GLU backward not built");
     const int pairs = max_pairs();
+    // the MLP backward's forms: SwiGLU-backward epilogue on slot-ordered x; K-major weights on
+    // slot-ordered (padded) rows, into slot order or scatter-added into tokens
+    if (a.glu_bwd) {
+        if (a.bf16 && !a.gather && a.glu && !a.scatter && !a.b_kmajor && a.a_row_pad == 0)
+            return launch_2sm_t<true, false, true, false, false, true>(a, s, pairs);
+        return set_error(MOE_ERR_UNSUPPORTED, "two-CTA GLU backward form not built");
+    }
+    if (a.b_kmajor) {
+        if (a.bf16 && !a.gather && !a.glu)
+            return a.scatter ? launch_2sm_t<true, false, false, true, true, false>(a, s, pairs)
+                             : launch_2sm_t<true, false, false, false, true, false>(a, s, pairs);
+        return set_error(MOE_ERR_UNSUPPORTED, "two-CTA K-major B form not built");
+    }
+    if (a.a_row_pad != 0)
+        return set_error(MOE_ERR_UNSUPPORTED, "two-CTA grouped GEMM: padded A without K-major B");
 #define MOE_DISPATCH2(BF, G, L, SC)                                                         \
     if (a.bf16 == BF && a.gather == G && a.glu == L && a.scatter == SC)                     \
         return launch_2sm_t<BF, G, L, SC>(a, s, pairs);
