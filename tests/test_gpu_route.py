@@ -59,6 +59,15 @@ def test_route_eight_experts_feature_sizes(oracle_lib, moe, D):
     _route_and_check(oracle_lib, moe, W.make_inputs(w, seed=D), 3)
 
 
+@pytest.mark.parametrize("E,k,D", [(16, 2, 200), (24, 3, 2880), (64, 6, 2048), (72, 8, 136),
+                                   (120, 4, 520), (128, 4, 2880)])
+def test_route_many_experts_tensor_cores(oracle_lib, moe, E, k, D):
+    # bf16, 16-128 experts and S > 2048: the tensor-core router, 17 tiles of 128 tokens (a ragged
+    # last one at S = 2100), D in 64-wide stages with a ragged last one, E not a power of two
+    w = W.custom("rm", S=2100, D=D, F=8, E=E, k=k, dtype="bf16", router_std="1/sqrt(D)")
+    _route_and_check(oracle_lib, moe, W.make_inputs(w, seed=E * 7 + D), k)
+
+
 @pytest.mark.parametrize("S,E,k", [(40000, 128, 4), (20000, 256, 8), (19000, 64, 6)])
 def test_route_tensor_core_several_tiles_per_cta(oracle_lib, moe, S, E, k):
     # more 128-token tiles than SMs: each CTA of the tensor-core router runs two or three tiles
