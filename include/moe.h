@@ -198,10 +198,10 @@ int moe_mlp_forward(const void *x, const void *w_gate, const float *logit_bias,
  *   dx [S, D], dw_gate [D, E], dw_gate_e [E, D, F], dw_up [E, D, F], dw_down [E, F, D].
  * The selection of the top-k experts has no derivative; the weights are the softmax over the
  * selected logits, differentiated through it. Steps on `stream`:
- *   1. dout -> bf16.
+ *   1. dout rows (bf16) and x rows copied to slot order.
  *   2. dh = dout[s] . W_down[e]^T per slot (the forward's grouped GEMM, W_down read K-major).
- *   3. The fused gate+up GEMM recomputed, with the SwiGLU backward in its epilogue: the
- *      route-weight gradient dh . h, then da and db.
+ *   3. The fused gate+up GEMM recomputed on the slot-ordered x rows, with the SwiGLU backward in
+ *      its epilogue: the route-weight gradient dh . h, then da and db.
  *   4. dW_down (weight-gradient GEMM over each expert's slots).
  *   5. dx += [da | db] . [W_gate_e ; W_up]^T (scatter-added into tokens).
  *   6. dW_gate_e and dW_up.
