@@ -45,8 +45,8 @@ def test_route_small(oracle_lib, moe, dtype, E, k):
 
 @pytest.mark.parametrize("S", [1, 7, 128, 2048, 2049, 5000])
 def test_route_eight_experts_every_batch_size(oracle_lib, moe, S):
-    # bf16 with eight experts: a block per token up to 2048 tokens, the warp-MMA router with 16
-    # tokens per block above (and its ragged last block at 2049 and 5000)
+    # bf16 with eight experts: the warp-MMA router at every batch size, 16 tokens per block (one
+    # partly filled block at S = 1 and 7, ragged last blocks at 2049 and 5000)
     w = W.custom("r8", S=S, D=4096, F=8, E=8, k=2, dtype="bf16")
     _route_and_check(oracle_lib, moe, W.make_inputs(w, seed=S), 2)
 
