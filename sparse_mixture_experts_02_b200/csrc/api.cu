@@ -40,6 +40,15 @@ bool prefer_2sm(int64_t R, int32_t E) {
     return E > 0 && R / E >= 384;
 }
 
+// The same choice for the scatter-add forms (h rows by TMA, fp32 reductions into tokens): pairs
+// pay off from fewer rows an expert there (measured at ~256 rows: GEMM2 0.730 -> 0.686 ms on
+// pairs, where the fused gate+up GEMM1 loses 7%; at ~32 rows both lose).
+bool prefer_2sm_scatter(int64_t R, int32_t E) {
+    const char *env = getenv("MOE_GEMM_2SM");
+    if (env != nullptr && (env[0] == '0' || env[0] == '1')) return env[0] == '1';
+    return E > 0 && R / E >= 192;
+}
+
 int num_sms() {
     int dev = 0, n = 0;
     cudaGetDevice(&dev);
@@ -647,7 +656,7 @@ int moe_mlp_forward(const void *x, const void *w_gate, const float *logit_bias,
         b.gather = false;
         b.glu = false;
         b.scatter = true;
-        if ((rc = prefer_2sm(R, E) ? launch_grouped_gemm_2sm(b, s) : launch_grouped_gemm(b, s)))
+        if ((rc = prefer_2sm_scatter(R, E) ? launch_grouped_gemm_2sm(b, s) : launch_grouped_gemm(b, s)))
             return rc;
         if ((rc = check_launch("gemm2"))) return rc;
         ++n;
@@ -1030,7 +1039,7 @@ int moe_moa_forward(const void *x, const void *w_gate, const float *logit_bias, 
         c.N = D;
         c.gather = false;
         c.scatter = true;
-        if ((rc = prefer_2sm(R, E) ? launch_grouped_gemm_2sm(c, s) : launch_grouped_gemm(c, s)))
+        if ((rc = prefer_2sm_scatter(R, E) ? launch_grouped_gemm_2sm(c, s) : launch_grouped_gemm(c, s)))
             return rc;
         if ((rc = check_launch("o projection"))) return rc;
         ++n;
@@ -1151,7 +1160,7 @@ int moe_expert_mlp_forward(const void *x_rows, const int32_t *expert_ids, int32_
     b.gather = false;
     b.glu = false;
     b.scatter = true;
-    if ((rc = prefer_2sm(R, E) ? launch_grouped_gemm_2sm(b, s) : launch_grouped_gemm(b, s)))
+    if ((rc = prefer_2sm_scatter(R, E) ? launch_grouped_gemm_2sm(b, s) : launch_grouped_gemm(b, s)))
         return rc;
     n += 2;
     g_launches = n;

@@ -91,6 +91,9 @@ int launch_grouped_gemm_2sm(const GemmArgs &a, cudaStream_t s);
 // Picks the two-CTA kernel when experts hold >= 384 rows on average (256-row
 // pair tiles waste little there); the environment variable MOE_GEMM_2SM=0/1 forces either kernel.
 bool prefer_2sm(int64_t R, int32_t E);
+// The choice for the scatter-add forms (GEMM2, the MoA output projection): pairs from 192 rows an
+// expert on average.
+bool prefer_2sm_scatter(int64_t R, int32_t E);
 int launch_debug_wait(int64_t limit_ns, unsigned *status, cudaStream_t s);
 // Weight gradient of ParallelLinear: dW[e] = sum over the slots p of expert e of A_p^T (x) dv_p,
 // A [a_rows, Din] the source rows in slot order (row stride a_ld elements, 0: Din), dv the
