@@ -159,3 +159,41 @@ def test_map_bad_expert_id_is_reported(moe):
     # the status clears on the next call
     moe.sparse_map(W.make_top_experts(100, 2, 8, seed=2).to("cuda"), 8, ws=ws)
     moe.check_device_status(ws)
+
+
+@pytest.mark.parametrize("E", [8, 256])
+def test_map_unaligned_buffers(oracle_lib, moe, E):
+    """top_experts and the two row arrays starting 4 bytes past a 16-byte boundary (the grid path's
+    vector loads and stores then take their one-route-at-a-time form): same map as the oracle."""
+    S, k = 40001, 4
+    te_cpu = W.make_top_experts(S, k, E, seed=E + 1, mode="stride")
+    R = S * k
+    te_buf = torch.empty(R + 1, dtype=torch.int32, device="cuda")
+    te_buf[1:] = te_cpu.reshape(-1).to("cuda")
+    te = te_buf[1:]
+    assert te.data_ptr() % 16 == 4
+    rows = torch.empty(2 * (R + 1), dtype=torch.int32, device="cuda")
+    sparse_rows, sorted_rows = rows[1:R + 1], rows[R + 2:]
+    counts = torch.empty(E, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    need = moe.workspace_size("sparse_map", S, 0, 0, E, k, 1)
+    ws = moe.alloc_workspace(need, te.device)
+    lib = moe.lib
+    rc = lib.moe_sparse_map(te.data_ptr(), S, k, E, counts.data_ptr(), offsets.data_ptr(),
+                            sparse_rows.data_ptr(), sorted_rows.data_ptr(), ws.data_ptr(),
+                            ws.numel(), torch.cuda.current_stream().cuda_stream)
+    assert rc == 0
+    moe.check_device_status(ws)
+    got = [t.cpu().numpy() for t in (counts, offsets, sparse_rows, sorted_rows)]
+    ref = oracle_lib.sparse_map(te_cpu.numpy(), E)
+    for name, a, b in zip(("counts", "offsets", "sparse_rows", "sorted_rows"), got, ref):
+        assert np.array_equal(a, b), name
+
+
+@pytest.mark.parametrize("E", [8, 200])
+def test_map_past_2pow23_routes(oracle_lib, moe, E):
+    """2050 map blocks of 4096 routes: the scan of the block counts takes its row form (more than
+    2048 blocks); eight experts assign with a lane per run of routes, 200 with a lane per route."""
+    S = (2050 * 4096 - 3000) // 8
+    te = W.make_top_experts(S, 8, E, seed=E + 5, mode="stride")
+    _compare(oracle_lib, moe, te, E)
