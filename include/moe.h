@@ -22,8 +22,13 @@
  *    these calls: scratch space comes from the caller's workspace `ws` (size from
  *    moe_workspace_size, alignment 256 bytes).
  *  - Environment: MOE_GEMM_2SM=1 (or 0) forces the grouped GEMMs onto CTA pairs (or single CTAs)
- *    instead of the library's choice by rows per expert; results are the same either way (the
- *    parity tests run both). No other environment variable is read.
+ *    instead of the library's choice by rows per expert; MOE_PREGATHER=0 keeps moe_mlp_forward's
+ *    first GEMM gathering x rows on load where it would copy them to slot order first. Results
+ *    are the same either way (the parity tests run both). No other environment variable is read.
+ *  - One device per process: the first call that launches a kernel needing more than 48 KB of
+ *    shared memory raises that kernel's limit (cudaFuncSetAttribute) once, for the device current
+ *    at that call. A process that then calls on another device gets MOE_ERR_CUDA from those
+ *    launches. Run one process per GPU, as the bench and the expert-parallel path do.
  *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy default stream) and
  *    never synchronise the host. Argument errors are detected on the host and returned before any
  *    launch. Errors the device detects (an expert id outside [0,E), a bounded wait that ran out)
