@@ -71,6 +71,11 @@ def test_kernel_names_are_classified():
     assert c("moe::<unnamed>::gather_rows_kernel(const uint4 *, const int *, int, ...)") == "x_copy"
     assert c("void moe::route_e8_kernel<2>(const __nv_bfloat16 *, ...)") == "router"
     assert c("void moe::map_small_kernel(const int *, long, int, ...)") == "sparse_map"
+    # the grid map's passes: both assign forms and both scans
+    assert c("void unnamed>::map_assign_lane_kernel<16>(const int *, long, ...)") == "sparse_map"
+    assert c("void unnamed>::map_assign_warp_kernel<1>(const int *, long, ...)") == "sparse_map"
+    assert c("unnamed>::map_scan_rows_kernel(int *, long, int *)") == "sparse_map"
+    assert c("unnamed>::map_scan_kernel(int *, long, int *)") == "sparse_map"
     assert c("void at::native::vectorized_elementwise_kernel<4, ...>") is None
 
 
